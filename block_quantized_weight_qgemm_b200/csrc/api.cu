@@ -1,0 +1,444 @@
+// api.cu -- the C ABI of libqgemm (declared in include/qgemm.h): argument checks, the fixed
+// K-split rule, per-call tile configuration, workspace layout, TMA descriptors, launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/qgemm.h"
+#include "common.cuh"
+
+namespace qg {
+cudaError_t launch_prep(const PrepParams& pp, cudaStream_t stream);
+cudaError_t launch_tc(int fmt, bool bf16op, const GemmParams& p, size_t smem_bytes, int grid,
+                      const CUtensorMap* maps, cudaStream_t stream);
+cudaError_t launch_pack(int fmt, const float* W, int64_t N, int64_t K, void* codes, void* scales,
+                        float* tensor_scale, cudaStream_t stream);
+int* device_error_word();
+}  // namespace qg
+
+using namespace qg;
+
+namespace {
+
+thread_local char g_last_cuda_error[256] = "";
+thread_local cudaEvent_t g_prof_begin = nullptr;
+thread_local cudaEvent_t g_prof_end = nullptr;
+
+int cuda_fail(cudaError_t e, const char* where) {
+  snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", where, cudaGetErrorString(e));
+  return QGEMM_ERR_CUDA;
+}
+
+// ---- driver entry point for TMA descriptor encoding (no link-time libcuda dependency) ----
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D map over a row-major [rows][inner] array with the given row pitch (bytes).
+bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int esize, const void* base, uint64_t inner,
+              uint64_t rows, uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_rows,
+              CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {pitch_bytes};
+  const cuuint32_t box[2] = {box_inner, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  (void)esize;
+  CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_fmt_shape(int fmt, int64_t N, int64_t K) {
+  if (fmt != FMT_Q8_0 && fmt != FMT_NVFP4 && fmt != FMT_MXFP4) return QGEMM_ERR_FORMAT;
+  if (N < 1 || K < 1 || N > 0x7FFFFFFF || K > 0x7FFFFFFF) return QGEMM_ERR_SHAPE;
+  if (K % block_k(fmt) != 0) return QGEMM_ERR_K_BLOCK;
+  return QGEMM_OK;
+}
+
+int device_ok() {
+  static int ok = -1;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    int dev = 0, major = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+      ok = 0;
+    else
+      ok = (major == 10) ? 1 : 0;
+  });
+  return ok;
+}
+
+constexpr int kSMs = 148;  // fixed: the K split must not depend on the device or the width
+
+// The K split used for widths 1..256: a function of (fmt, N, K, nmat) only.  It picks the S
+// that best fills kSMs CTAs when each CTA holds 4 weight subtiles (the decode tiling),
+// preferring smaller S on ties.
+int split_for(int fmt, int64_t N, int64_t K, int nmat) {
+  const int64_t chunks = (K + chunk_k(fmt) - 1) / chunk_k(fmt);
+  const int64_t tiles = (N + kTileRows - 1) / kTileRows;
+  const int64_t per_group = 4 / nmat;
+  const int64_t groups = (tiles + per_group - 1) / per_group;
+  int best = 1;
+  double best_eff = -1.0;
+  const int64_t smax = std::min<int64_t>(16, chunks);
+  for (int64_t S = 1; S <= smax; ++S) {
+    const int64_t units = groups * S;
+    const int64_t waves = (units + kSMs - 1) / kSMs;
+    const double fill = double(units) / double(waves * kSMs);
+    const int64_t cmax = (chunks + S - 1) / S;
+    const double bal = (double(chunks) / double(S)) / double(cmax);
+    const double eff = fill * bal;
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best = (int)S;
+    }
+  }
+  return best;
+}
+
+struct Plan {
+  bool f16ops;  // widths <= 256
+  int NB, R, NMAT, S, n_groups, b_tiles, chunks, XS, WS, AS, tmem_cols;
+  size_t smem_bytes;
+  uint32_t smem_x, smem_w, smem_bar;
+  // workspace layout (bytes)
+  size_t off_xh, off_exp, off_cnt, off_ws, ws_total;
+};
+
+int next_pow2_cols(int c) {
+  int p = 32;
+  while (p < c) p <<= 1;
+  return p;
+}
+
+// Chooses the tiling for one call.  Only S (and the operand type, by width class) affects
+// the arithmetic; NB, R and the ring depths are scheduling choices.
+bool make_plan(int fmt, int64_t N, int64_t K, int64_t B, int nmat, Plan* pl) {
+  Plan p{};
+  p.NMAT = nmat;
+  p.f16ops = (B <= 256);
+  p.chunks = (int)((K + chunk_k(fmt) - 1) / chunk_k(fmt));
+  const int J = chunk_k(fmt) / kSubK;
+  const int64_t tiles = (N + kTileRows - 1) / kTileRows;
+  if (p.f16ops) {
+    p.S = split_for(fmt, N, K, nmat);
+    const int nb_cap = (nmat == 2) ? 128 : 256;
+    int nb = (int)std::min<int64_t>(((B + 15) / 16) * 16, nb_cap);
+    if (nmat == 2 && B > 128) nb = (int)(((B + 1) / 2 + 15) / 16 * 16);
+    p.NB = nb;
+  } else {
+    p.S = 1;
+    p.NB = (nmat == 2) ? 128 : 256;
+  }
+  p.b_tiles = (int)((B + p.NB - 1) / p.NB);
+  // subtiles per unit: TMEM holds R*NB accumulator columns plus an A ring of >= 2 stages
+  int rmax = std::min(4, (512 - 2 * kAColsPerStage) / p.NB);
+  rmax = rmax / nmat * nmat;
+  if (rmax < nmat) return false;
+  int bestR = nmat;
+  int64_t best_cost = -1;
+  for (int R = nmat; R <= rmax; R += nmat) {
+    const int64_t groups = (tiles + (R / nmat) - 1) / (R / nmat);
+    const int64_t units = groups * p.b_tiles * p.S;
+    const int64_t cost = ((units + kSMs - 1) / kSMs) * R;
+    if (best_cost < 0 || cost <= best_cost) {
+      best_cost = cost;
+      bestR = R;
+    }
+  }
+  p.R = bestR;
+  p.n_groups = (int)((tiles + (p.R / nmat) - 1) / (p.R / nmat));
+  p.AS = std::min(kMaxAStages, (512 - p.R * p.NB) / kAColsPerStage);
+  if (p.AS < 2) return false;
+  p.tmem_cols = next_pow2_cols(p.R * p.NB + p.AS * kAColsPerStage);
+  if (p.tmem_cols > 512) return false;
+  // shared memory: x ring, weight ring (gets the rest, up to 8 stages), barriers, control
+  const size_t xstage = (size_t)p.NB * 128;
+  const size_t misc = 8 * (2 * 16 + 2 * 8 + 2 * kMaxAStages + 1) + 16 + 4 * kMaxNB + 64;
+  const size_t budget = kSmemLimit - 1024 - misc;
+  // with several subtiles the x stages of a chunk stay resident until its last subtile
+  int XS = (p.R > 1) ? 2 * J : 4;
+  while (XS > J && XS * xstage + 2 * (size_t)kWStageBytes > budget) --XS;
+  if (XS * xstage + 2 * (size_t)kWStageBytes > budget) return false;
+  const int WS = (int)std::min<size_t>(8, (budget - XS * xstage) / kWStageBytes);
+  p.XS = XS;
+  p.WS = WS;
+  p.smem_x = 0;
+  p.smem_w = (uint32_t)(XS * xstage);
+  p.smem_bar = p.smem_w + (uint32_t)(WS * kWStageBytes);
+  const size_t bar_bytes = 8 * (2 * XS + 2 * WS + 2 * p.AS + 1);
+  p.smem_bytes = 1024 + p.smem_bar + bar_bytes + 16 + 4 * p.NB + 64;
+  // workspace: [xh f16 B*K][x_exp B][counters][split partials S*NMAT*B*N fp32]
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += (bytes + 255) / 256 * 256;
+    return o;
+  };
+  p.off_xh = p.f16ops ? take((size_t)B * K * 2) : 0;
+  p.off_exp = p.f16ops ? take((size_t)B * 4) : 0;
+  const size_t ncnt = (size_t)p.n_groups * p.b_tiles;
+  p.off_cnt = (p.S > 1) ? take(ncnt * 4) : 0;
+  p.off_ws = (p.S > 1) ? take((size_t)p.S * nmat * B * N * 4) : 0;
+  p.ws_total = off;
+  *pl = p;
+  return true;
+}
+
+int run_impl(int fmt, const void* x, int64_t B, int64_t K, const void* const* codes,
+             const void* const* scales, const float* const* ts, int nmat, int64_t N, void* out,
+             int out_bf16, void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  Plan pl;
+  if (!make_plan(fmt, N, K, B, nmat, &pl)) return QGEMM_ERR_SHAPE;
+  if (pl.ws_total > 0 && (workspace == nullptr || ws_bytes < pl.ws_total)) return QGEMM_ERR_WORKSPACE;
+  if (workspace && !aligned16(workspace)) return QGEMM_ERR_ALIGN;
+  int* dev_err = device_error_word();
+  if (!dev_err) return cuda_fail(cudaGetLastError(), "cudaGetSymbolAddress");
+  uint8_t* wsb = static_cast<uint8_t*>(workspace);
+
+  GemmParams p{};
+  p.N = (int)N;
+  p.K = (int)K;
+  p.B = (int)B;
+  p.NB = pl.NB;
+  p.R = pl.R;
+  p.NMAT = nmat;
+  p.S = pl.S;
+  p.n_groups = pl.n_groups;
+  p.b_tiles = pl.b_tiles;
+  p.chunks = pl.chunks;
+  p.XS = pl.XS;
+  p.WS = pl.WS;
+  p.AS = pl.AS;
+  p.tmem_cols = pl.tmem_cols;
+  p.smem_x = pl.smem_x;
+  p.smem_w = pl.smem_w;
+  p.smem_bar = pl.smem_bar;
+  p.spitch = scale_pitch(fmt, K);
+  for (int m = 0; m < 2; ++m) {
+    const int mm = (m < nmat) ? m : 0;
+    p.ts[m] = ts[mm];
+    p.scales[m] = static_cast<const uint8_t*>(scales[mm]);
+  }
+  p.x_exp = pl.f16ops ? reinterpret_cast<const int*>(wsb + pl.off_exp) : nullptr;
+  p.ws = (pl.S > 1) ? reinterpret_cast<float*>(wsb + pl.off_ws) : nullptr;
+  p.counters = (pl.S > 1) ? reinterpret_cast<int*>(wsb + pl.off_cnt) : nullptr;
+  p.out = out;
+  p.out_bf16 = out_bf16;
+  p.dev_err = dev_err;
+
+  const void* xop = x;
+  if (pl.f16ops) {
+    PrepParams pp{};
+    pp.x = static_cast<const uint16_t*>(x);
+    pp.xh = reinterpret_cast<uint16_t*>(wsb + pl.off_xh);
+    pp.x_exp = reinterpret_cast<int*>(wsb + pl.off_exp);
+    pp.B = (int)B;
+    pp.K = (int)K;
+    pp.counters = p.counters;
+    pp.n_counters = (pl.S > 1) ? pl.n_groups * pl.b_tiles : 0;
+    cudaError_t e = launch_prep(pp, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "prep kernel launch");
+    xop = pp.xh;
+  }
+
+  CUtensorMap maps[5];
+  const CUtensorMapDataType xdt =
+      pl.f16ops ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  bool ok = make_map(&maps[0], xdt, 2, xop, (uint64_t)K, (uint64_t)B, (uint64_t)K * 2, kSubK,
+                     (uint32_t)pl.NB, CU_TENSOR_MAP_SWIZZLE_128B);
+  const uint64_t code_bytes = (fmt == FMT_Q8_0) ? (uint64_t)K : (uint64_t)K / 2;
+  const uint64_t scale_bytes = (fmt == FMT_Q8_0) ? (uint64_t)K / 16
+                               : (fmt == FMT_NVFP4) ? (uint64_t)K / 16
+                                                    : (uint64_t)K / 32;
+  for (int m = 0; m < 2 && ok; ++m) {
+    const int mm = (m < nmat) ? m : 0;
+    ok = ok && make_map(&maps[1 + 2 * m], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, codes[mm], code_bytes,
+                        (uint64_t)N, (uint64_t)code_pitch(fmt, K), kWRowBytes, kTileRows,
+                        CU_TENSOR_MAP_SWIZZLE_128B);
+    ok = ok && make_map(&maps[2 + 2 * m], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, scales[mm], scale_bytes,
+                        (uint64_t)N, (uint64_t)scale_pitch(fmt, K), kScaleRowBytes, kTileRows,
+                        CU_TENSOR_MAP_SWIZZLE_NONE);
+  }
+  if (!ok) {
+    snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled failed");
+    return QGEMM_ERR_CUDA;
+  }
+  const int grid = pl.n_groups * pl.b_tiles * pl.S;
+  if (g_prof_begin) cudaEventRecord(g_prof_begin, stream);
+  cudaError_t e = launch_tc(fmt, !pl.f16ops, p, pl.smem_bytes, grid, maps, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "gemm kernel launch");
+  if (g_prof_end) cudaEventRecord(g_prof_end, stream);
+  return QGEMM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int qgemm_packed_size(int fmt, int64_t N, int64_t K, size_t* code_bytes, size_t* scale_bytes) {
+  const int st = check_fmt_shape(fmt, N, K);
+  if (st != QGEMM_OK) return st;
+  if (!code_bytes || !scale_bytes) return QGEMM_ERR_NULL;
+  *code_bytes = (size_t)(N * code_pitch(fmt, K));
+  *scale_bytes = (size_t)(N * scale_pitch(fmt, K));
+  return QGEMM_OK;
+}
+
+int qgemm_row_pitches(int fmt, int64_t K, int64_t* cp, int64_t* sp) {
+  const int st = check_fmt_shape(fmt, 1, K);
+  if (st != QGEMM_OK) return st;
+  if (!cp || !sp) return QGEMM_ERR_NULL;
+  *cp = code_pitch(fmt, K);
+  *sp = scale_pitch(fmt, K);
+  return QGEMM_OK;
+}
+
+int qgemm_pack(int fmt, const float* W, int64_t N, int64_t K, void* codes, void* scales,
+               float* tensor_scale, void* stream) {
+  const int st = check_fmt_shape(fmt, N, K);
+  if (st != QGEMM_OK) return st;
+  if (!W || !codes || !scales || (fmt == FMT_NVFP4 && !tensor_scale)) return QGEMM_ERR_NULL;
+  if (!aligned16(W) || !aligned16(codes) || !aligned16(scales)) return QGEMM_ERR_ALIGN;
+  if (fmt == FMT_NVFP4 && (reinterpret_cast<uintptr_t>(tensor_scale) & 3u)) return QGEMM_ERR_ALIGN;
+  if (!device_ok()) return QGEMM_ERR_DEVICE;
+  cudaError_t e = launch_pack(fmt, W, N, K, codes, scales, tensor_scale,
+                              static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "pack kernel launch");
+  return QGEMM_OK;
+}
+
+int qgemm_split_k(int fmt, int64_t N, int64_t K, int* splits) {
+  const int st = check_fmt_shape(fmt, N, K);
+  if (st != QGEMM_OK) return st;
+  if (!splits) return QGEMM_ERR_NULL;
+  *splits = split_for(fmt, N, K, 1);
+  return QGEMM_OK;
+}
+
+int qgemm_workspace_size(int fmt, int64_t N, int64_t K, int64_t B, size_t* bytes) {
+  int st = check_fmt_shape(fmt, N, K);
+  if (st != QGEMM_OK) return st;
+  if (B < 1 || B > 0x7FFFFFFF) return QGEMM_ERR_SHAPE;
+  if (!bytes) return QGEMM_ERR_NULL;
+  Plan pl;
+  if (!make_plan(fmt, N, K, B, 1, &pl)) return QGEMM_ERR_SHAPE;
+  *bytes = pl.ws_total;
+  return QGEMM_OK;
+}
+
+int qgemm_ffn_workspace_size(int fmt, int64_t N, int64_t K, int64_t M, size_t* bytes) {
+  int st = check_fmt_shape(fmt, N, K);
+  if (st != QGEMM_OK) return st;
+  if (M < 1 || M > 0x7FFFFFFF) return QGEMM_ERR_SHAPE;
+  if (!bytes) return QGEMM_ERR_NULL;
+  Plan pl;
+  if (!make_plan(fmt, N, K, M, 2, &pl)) return QGEMM_ERR_SHAPE;
+  *bytes = pl.ws_total;
+  return QGEMM_OK;
+}
+
+int qgemm_run(int fmt, const void* x, int64_t B, int64_t K, const void* codes, const void* scales,
+              const float* tensor_scale, int64_t N, void* y, int y_dtype, void* workspace,
+              size_t workspace_bytes, void* stream) {
+  int st = check_fmt_shape(fmt, N, K);
+  if (st != QGEMM_OK) return st;
+  if (B < 1 || B > 0x7FFFFFFF) return QGEMM_ERR_SHAPE;
+  if (y_dtype != QGEMM_Y_F32 && y_dtype != QGEMM_Y_BF16) return QGEMM_ERR_FORMAT;
+  if (!x || !codes || !scales || !y || (fmt == FMT_NVFP4 && !tensor_scale)) return QGEMM_ERR_NULL;
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || !aligned16(y))
+    return QGEMM_ERR_ALIGN;
+  if (!device_ok()) return QGEMM_ERR_DEVICE;
+  const void* cs[1] = {codes};
+  const void* ss[1] = {scales};
+  const float* tss[1] = {tensor_scale};
+  return run_impl(fmt, x, B, K, cs, ss, tss, 1, N, y, y_dtype == QGEMM_Y_BF16, workspace,
+                  workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int qgemm_ffn_gate_up(int fmt, const void* x, int64_t M, int64_t K, const void* g_codes,
+                      const void* g_scales, const float* g_ts, const void* u_codes,
+                      const void* u_scales, const float* u_ts, int64_t N, void* h,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+  int st = check_fmt_shape(fmt, N, K);
+  if (st != QGEMM_OK) return st;
+  if (M < 1 || M > 0x7FFFFFFF) return QGEMM_ERR_SHAPE;
+  if (!x || !g_codes || !g_scales || !u_codes || !u_scales || !h) return QGEMM_ERR_NULL;
+  if (fmt == FMT_NVFP4 && (!g_ts || !u_ts)) return QGEMM_ERR_NULL;
+  if (!aligned16(x) || !aligned16(g_codes) || !aligned16(g_scales) || !aligned16(u_codes) ||
+      !aligned16(u_scales) || !aligned16(h))
+    return QGEMM_ERR_ALIGN;
+  if (!device_ok()) return QGEMM_ERR_DEVICE;
+  const void* cs[2] = {g_codes, u_codes};
+  const void* ss[2] = {g_scales, u_scales};
+  const float* tss[2] = {g_ts, u_ts};
+  return run_impl(fmt, x, M, K, cs, ss, tss, 2, N, h, 1, workspace, workspace_bytes,
+                  static_cast<cudaStream_t>(stream));
+}
+
+int qgemm_device_status(int reset) {
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+  int* w = device_error_word();
+  if (!w) return cuda_fail(cudaGetLastError(), "cudaGetSymbolAddress");
+  int v = 0;
+  e = cudaMemcpy(&v, w, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy");
+  if (reset && v) {
+    const int z = 0;
+    e = cudaMemcpy(w, &z, sizeof(int), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy");
+  }
+  return v ? QGEMM_ERR_DEVICE_TIMEOUT : QGEMM_OK;
+}
+
+const char* qgemm_status_str(int status) {
+  switch (status) {
+    case QGEMM_OK: return "ok";
+    case QGEMM_ERR_FORMAT: return "unknown weight format or output dtype";
+    case QGEMM_ERR_SHAPE: return "invalid shape (N, K or B < 1, or too large)";
+    case QGEMM_ERR_K_BLOCK: return "K is not a multiple of the format's block size";
+    case QGEMM_ERR_NULL: return "a required pointer is NULL";
+    case QGEMM_ERR_ALIGN: return "a device pointer is not 16-byte aligned";
+    case QGEMM_ERR_WORKSPACE: return "workspace missing or too small";
+    case QGEMM_ERR_CUDA: return "a CUDA call or kernel launch failed";
+    case QGEMM_ERR_DEVICE: return "the current device is not an sm_100 GPU";
+    case QGEMM_ERR_DEVICE_TIMEOUT: return "a kernel wait hit its time limit";
+    default: return "unknown status";
+  }
+}
+
+const char* qgemm_last_cuda_error(void) { return g_last_cuda_error; }
+
+int qgemm_profile_events(void* begin_event, void* end_event) {
+  g_prof_begin = static_cast<cudaEvent_t>(begin_event);
+  g_prof_end = static_cast<cudaEvent_t>(end_event);
+  return QGEMM_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,709 @@
+// gemm.cu -- the block-quantized-weight GEMM kernels of libqgemm (sm_100a).
+//
+// y[b][n] = sum_k x[b][k] * dequant(W)[n][k]     (hipfire PR "fix(mtp): chunk scalar Q8
+// batched GEMM above 64 rows"; Atlas issue "Qwen3.8-27B on Strix Halo: prefill 2.4x gap",
+// kernel ranking and exact-F16-dequant sections)
+//
+// Design (swap-AB on the 5th-generation tensor cores):
+//   * Weights are the MMA M operand: one subtile = 128 weight rows, held in tensor memory
+//     (TMEM) as 16-bit values that dequant warps write with tcgen05.st.
+//   * Activations are the MMA N operand: NB <= 256 batch rows of x, loaded by TMA into
+//     128-byte-swizzled shared memory and read by the MMA through a smem descriptor.
+//   * Accumulators live in TMEM (fp32), one NB-column block per weight subtile.
+//   * Warp roles: warp 0 issues TMA loads, warp 1 allocates TMEM and issues tcgen05.mma,
+//     warps 2..9 dequantize packed weights from the smem ring into the TMEM A ring and then
+//     run the epilogue.
+//   * K is split into S contiguous ranges (S fixed by format, N, K); partials are summed in
+//     the fixed order s = 0..S-1 by whichever CTA of a tile arrives last.  Nothing in the
+//     arithmetic depends on the batch width, so row b of y is bit-identical for B <= 256.
+//   * Widths 1..256 use f16 operands: x rows are rescaled by a power of two chosen from the
+//     row's own maximum (exact), then rounded to f16 (exact for every bf16 value within
+//     2^-38 of the row maximum), and the power of two is restored in the epilogue.  The
+//     dequantized weights are exact in f16 for NVFP4 (E2M1 x E4M3 has <= 6 significant bits,
+//     range [2^-10, 2688]) and for MXFP4 (after a per-row power-of-two rebase of the E8M0
+//     exponents); Q8_0 products q*d are rounded once.
+//   * Widths above 256 (prefill) use bf16 operands straight from the caller's x, no split.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp4.h>
+#include <cuda_fp8.h>
+
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace qg {
+
+// The library's device error word (bounded waits that ran out write kErrTimeout).
+__device__ int g_dev_err = 0;
+
+// ---------------------------------------------------------------------------------------
+// Small bit helpers
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t h2u(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+__device__ __forceinline__ __half2 u2h(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
+__device__ __forceinline__ uint32_t b2u(__nv_bfloat162 h) {
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ __nv_bfloat162 u2b(uint32_t u) {
+  return *reinterpret_cast<__nv_bfloat162*>(&u);
+}
+
+__device__ __forceinline__ __half2 half2_bcast(uint16_t bits) {
+  const uint32_t u = (uint32_t)bits | ((uint32_t)bits << 16);
+  return u2h(u);
+}
+
+// f16 bit pattern of 2^ex, or 0 below the f16 subnormal range.  ex <= 15.
+__device__ __forceinline__ uint16_t f16_pow2_bits(int ex) {
+  if (ex >= -14) return (uint16_t)((ex + 15) << 10);
+  if (ex >= -24) return (uint16_t)(1u << (ex + 24));
+  return 0;
+}
+
+// Load a 16-byte chunk `ci` (0..7) of a 128-byte row stored with the 128-byte TMA swizzle.
+__device__ __forceinline__ uint4 ld_sw128(const uint8_t* row_base, int row, int ci) {
+  return *reinterpret_cast<const uint4*>(row_base + ((ci ^ (row & 7)) << 4));
+}
+
+// ---------------------------------------------------------------------------------------
+// Dequantisation of 32 consecutive K elements of one weight row into 16 packed words
+// (element 2i in the low half of word i), the layout of an A row in TMEM.
+//   crow: the row's 128 code bytes in the weight stage (swizzled); srow: its 16 scale bytes.
+//   c: chunk index (selects the half of a scale line shared by two chunks);
+//   e0: first element within the chunk (multiple of 32).
+// ---------------------------------------------------------------------------------------
+template <int FMT, bool BF16OP>
+struct Dequant;
+
+// Q8_0 -> f16: q + 1152 built as f16 from the byte (0x64XX = 1024 + XX with XX = q ^ 0x80),
+// minus 1152 gives q exactly; one rounding in q * d.
+template <>
+struct Dequant<FMT_Q8_0, false> {
+  __device__ __forceinline__ static void run(const uint8_t* crow, int row, const uint8_t* srow,
+                                             int c, int e0, int /*ex*/, uint32_t (&v)[16]) {
+    const uint4 a = ld_sw128(crow, row, e0 >> 4);
+    const uint4 b = ld_sw128(crow, row, (e0 >> 4) + 1);
+    const uint16_t dbits =
+        *reinterpret_cast<const uint16_t*>(srow + 2 * (((c & 1) << 2) + (e0 >> 5)));
+    const __half2 d2 = half2_bcast(dbits);
+    const __half2 off = half2_bcast(0x6480);  // 1152.0
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t t = w[i] ^ 0x80808080u;
+      const uint32_t lo = prmt(t, 0x64646464u, 0x4140u);
+      const uint32_t hi = prmt(t, 0x64646464u, 0x4342u);
+      v[2 * i] = h2u(__hmul2(__hsub2(u2h(lo), off), d2));
+      v[2 * i + 1] = h2u(__hmul2(__hsub2(u2h(hi), off), d2));
+    }
+  }
+};
+
+// Q8_0 -> bf16: q (sign-extended) + 1.5*2^23 as fp32 bits, fma with d and -1.5*2^23*d gives
+// q*d exactly in fp32; one rounding to bf16.
+template <>
+struct Dequant<FMT_Q8_0, true> {
+  __device__ __forceinline__ static void run(const uint8_t* crow, int row, const uint8_t* srow,
+                                             int c, int e0, int /*ex*/, uint32_t (&v)[16]) {
+    const uint4 a = ld_sw128(crow, row, e0 >> 4);
+    const uint4 b = ld_sw128(crow, row, (e0 >> 4) + 1);
+    const uint16_t dbits =
+        *reinterpret_cast<const uint16_t*>(srow + 2 * (((c & 1) << 2) + (e0 >> 5)));
+    const float d = __half2float(__ushort_as_half(dbits));
+    const float nd = -12582912.0f * d;
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float f[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        int q;
+        asm("bfe.s32 %0, %1, %2, 8;" : "=r"(q) : "r"(w[i]), "r"(8 * j));
+        f[j] = __fmaf_rn(__int_as_float(0x4B400000 + q), d, nd);
+      }
+      v[2 * i] = b2u(__floats2bfloat162_rn(f[0], f[1]));
+      v[2 * i + 1] = b2u(__floats2bfloat162_rn(f[2], f[3]));
+    }
+  }
+};
+
+// E2M1 byte pair -> f16x2 (hardware conversion), times a broadcast f16 scale (exact).
+__device__ __forceinline__ uint32_t e2m1x2_f16(uint32_t byte, __half2 s) {
+  const __half2_raw r = __nv_cvt_fp4x2_to_halfraw2((__nv_fp4x2_storage_t)byte, __NV_E2M1);
+  __half2 h;
+  *reinterpret_cast<__half2_raw*>(&h) = r;
+  return h2u(__hmul2(h, s));
+}
+
+template <>
+struct Dequant<FMT_NVFP4, false> {
+  __device__ __forceinline__ static void run(const uint8_t* crow, int row, const uint8_t* srow,
+                                             int /*c*/, int e0, int /*ex*/, uint32_t (&v)[16]) {
+    const uint4 a = ld_sw128(crow, row, e0 >> 5);
+    const uint16_t sb = *reinterpret_cast<const uint16_t*>(srow + (e0 >> 4));
+    const __half2_raw sr = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)sb, __NV_E4M3);
+    const __half2 s0 = half2_bcast(sr.x), s1 = half2_bcast(sr.y);
+    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) v[4 * i + j] = e2m1x2_f16((w[i] >> (8 * j)) & 0xFFu, i < 2 ? s0 : s1);
+    }
+  }
+};
+
+template <>
+struct Dequant<FMT_MXFP4, false> {
+  // ex = E - Emax_row, the exponent of this block relative to the row's largest block;
+  // the f16 scale is 2^(ex + 13) so the largest block's values stay below 2^16.
+  __device__ __forceinline__ static void run(const uint8_t* crow, int row, const uint8_t* srow,
+                                             int c, int e0, int emax, uint32_t (&v)[16]) {
+    const uint4 a = ld_sw128(crow, row, e0 >> 5);
+    const int e = srow[((c & 1) << 3) + (e0 >> 5)];
+    const __half2 s = half2_bcast(f16_pow2_bits(e - emax + 13));
+    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) v[4 * i + j] = e2m1x2_f16((w[i] >> (8 * j)) & 0xFFu, s);
+    }
+  }
+};
+
+// E2M1 -> bf16 for 8 codes in one word (two prmt byte tables for the magnitude, prmt sign
+// replication for the sign bits), times a broadcast bf16 scale (exact).
+__device__ __forceinline__ void e2m1x8_bf16(uint32_t w, __nv_bfloat162 s, uint32_t* out) {
+  // bf16 high / low bytes of the magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6} by code 0..7
+  constexpr uint32_t HI0 = 0x3F3F3F00u, HI1 = 0x40404040u;
+  constexpr uint32_t LO0 = 0xC0800000u, LO1 = 0xC0804000u;
+  const uint32_t m = w & 0x77777777u;
+  const uint32_t m2 = m >> 16;
+  const uint32_t w4 = w << 4;  // byte i's msb = sign of the even code 2i; w's = odd code 2i+1
+  const uint32_t H = prmt(HI0, HI1, m), L = prmt(LO0, LO1, m);
+  const uint32_t H2 = prmt(HI0, HI1, m2), L2 = prmt(LO0, LO1, m2);
+  uint32_t o[4];
+  o[0] = prmt(L, H, 0x5140u);
+  o[1] = prmt(L, H, 0x7362u);
+  o[2] = prmt(L2, H2, 0x5140u);
+  o[3] = prmt(L2, H2, 0x7362u);
+  const uint32_t sel[4] = {0xC080u, 0xD090u, 0xE0A0u, 0xF0B0u};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t sg;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(sg) : "r"(w4), "r"(w), "r"(sel[i]));
+    const uint32_t val = (o[i] & 0x7FFF7FFFu) | (sg & 0x80008000u);
+    out[i] = b2u(__hmul2(u2b(val), s));
+  }
+}
+
+template <>
+struct Dequant<FMT_NVFP4, true> {
+  __device__ __forceinline__ static void run(const uint8_t* crow, int row, const uint8_t* srow,
+                                             int /*c*/, int e0, int /*ex*/, uint32_t (&v)[16]) {
+    const uint4 a = ld_sw128(crow, row, e0 >> 5);
+    const uint16_t sb = *reinterpret_cast<const uint16_t*>(srow + (e0 >> 4));
+    const __half2_raw sr = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)sb, __NV_E4M3);
+    const __nv_bfloat16 b0 = __float2bfloat16_rn(__half2float(__ushort_as_half(sr.x)));
+    const __nv_bfloat16 b1 = __float2bfloat16_rn(__half2float(__ushort_as_half(sr.y)));
+    const __nv_bfloat162 s0 = __halves2bfloat162(b0, b0), s1 = __halves2bfloat162(b1, b1);
+    e2m1x8_bf16(a.x, s0, &v[0]);
+    e2m1x8_bf16(a.y, s0, &v[4]);
+    e2m1x8_bf16(a.z, s1, &v[8]);
+    e2m1x8_bf16(a.w, s1, &v[12]);
+  }
+};
+
+template <>
+struct Dequant<FMT_MXFP4, true> {
+  __device__ __forceinline__ static void run(const uint8_t* crow, int row, const uint8_t* srow,
+                                             int c, int e0, int /*ex*/, uint32_t (&v)[16]) {
+    const uint4 a = ld_sw128(crow, row, e0 >> 5);
+    const uint32_t e = srow[((c & 1) << 3) + (e0 >> 5)];
+    const uint32_t bits = e ? (e << 7) : 0x0040u;  // 2^(e-127) as bf16 (e = 0: subnormal)
+    const __nv_bfloat162 s = u2b(bits | (bits << 16));
+    e2m1x8_bf16(a.x, s, &v[0]);
+    e2m1x8_bf16(a.y, s, &v[4]);
+    e2m1x8_bf16(a.z, s, &v[8]);
+    e2m1x8_bf16(a.w, s, &v[12]);
+  }
+};
+
+// ---------------------------------------------------------------------------------------
+// x preparation for the f16 path: per row, e = floor(log2 amax) - 14, xh = f16(x * 2^-e).
+// Also clears the split-K arrival counters of the GEMM that follows on the stream.
+// ---------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) qgemm_prep_x_kernel(const PrepParams p) {
+  const int b = blockIdx.x;
+  const uint16_t* xr = p.x + (size_t)b * p.K;
+  __shared__ float red[8];
+  float amax = 0.f;
+  for (int k = threadIdx.x * 8; k < p.K; k += blockDim.x * 8) {
+    const uint4 v = *reinterpret_cast<const uint4*>(xr + k);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      amax = fmaxf(amax, fabsf(__uint_as_float(w[i] << 16)));
+      amax = fmaxf(amax, fabsf(__uint_as_float(w[i] & 0xFFFF0000u)));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  amax = red[0];
+  for (int i = 1; i < (int)(blockDim.x >> 5); ++i) amax = fmaxf(amax, red[i]);
+  int e = 0;
+  if (amax > 0.f && amax <= 3.4e38f) {
+    int ex;
+    (void)frexpf(amax, &ex);  // amax = f * 2^ex, f in [0.5, 1)
+    e = (ex - 1) - 14;        // amax * 2^-e in [2^14, 2^15)
+  }
+  const float sc = ldexpf(1.0f, -e);
+  uint16_t* xo = p.xh + (size_t)b * p.K;
+  for (int k = threadIdx.x * 8; k < p.K; k += blockDim.x * 8) {
+    const uint4 v = *reinterpret_cast<const uint4*>(xr + k);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __half lo = __float2half_rn(__uint_as_float(w[i] << 16) * sc);
+      const __half hi = __float2half_rn(__uint_as_float(w[i] & 0xFFFF0000u) * sc);
+      o[i] = (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
+    }
+    *reinterpret_cast<uint4*>(xo + k) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+  if (threadIdx.x == 0) p.x_exp[b] = e;
+  if (b == 0)
+    for (int i = threadIdx.x; i < p.n_counters; i += blockDim.x) p.counters[i] = 0;
+}
+
+// ---------------------------------------------------------------------------------------
+// Epilogue helpers
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ void store_y(const GemmParams& p, int b, int n, float v) {
+  if (p.out_bf16)
+    reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)b * p.N + n] = __float2bfloat16_rn(v);
+  else
+    reinterpret_cast<float*>(p.out)[(size_t)b * p.N + n] = v;
+}
+
+__device__ __forceinline__ void store_h(const GemmParams& p, int b, int n, float g, float u) {
+  const float silu = g / (1.0f + expf(-g));
+  reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)b * p.N + n] = __float2bfloat16_rn(silu * u);
+}
+
+__device__ __forceinline__ void named_bar_epilogue() {
+  asm volatile("bar.sync 1, %0;" ::"r"(kDequantWarps * 32) : "memory");
+}
+
+// ---------------------------------------------------------------------------------------
+// The GEMM kernel.  One CTA = one work unit (row group g, batch tile bt, K split s).
+// ---------------------------------------------------------------------------------------
+template <int FMT, bool BF16OP>
+__global__ void __launch_bounds__(kThreads, 1)
+    qgemm_tc_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ CUtensorMap tm_x,
+                    const __grid_constant__ CUtensorMap tm_c0,
+                    const __grid_constant__ CUtensorMap tm_s0,
+                    const __grid_constant__ CUtensorMap tm_c1,
+                    const __grid_constant__ CUtensorMap tm_s1) {
+  constexpr int KW = chunk_k(FMT);
+  constexpr int J = KW / kSubK;       // x stages per chunk
+  constexpr int JA = KW / kAStageK;   // A stages per chunk
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t sx = sbase + p.smem_x;
+  const uint32_t sw = sbase + p.smem_w;
+  const int XS = p.XS, WS = p.WS;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.smem_bar);
+  const uint32_t bar_x_full = smem_u32(bars);
+  const uint32_t bar_x_empty = bar_x_full + 8 * XS;
+  const uint32_t bar_w_full = bar_x_empty + 8 * XS;
+  const uint32_t bar_w_empty = bar_w_full + 8 * WS;
+  const uint32_t bar_a_full = bar_w_empty + 8 * WS;
+  const int AS = p.AS;
+  const uint32_t bar_a_empty = bar_a_full + 8 * AS;
+  const uint32_t bar_acc = bar_a_empty + 8 * AS;
+  int* ctl = reinterpret_cast<int*>(bars + 2 * XS + 2 * WS + 2 * AS + 1);
+  volatile int* abort_flag = ctl + 1;
+  float* col_fac = reinterpret_cast<float*>(ctl + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int u = blockIdx.x;
+  const int g = u % p.n_groups;
+  u /= p.n_groups;
+  const int bt = u % p.b_tiles;
+  const int s = u / p.b_tiles;
+  const int c0 = (int)((int64_t)s * p.chunks / p.S);
+  const int c1 = (int)((int64_t)(s + 1) * p.chunks / p.S);
+  const int tiles_per_group = p.R / p.NMAT;
+  const uint32_t a_col0 = (uint32_t)(p.R * p.NB);
+
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tm_x);
+    prefetch_tmap(&tm_c0);
+    prefetch_tmap(&tm_s0);
+    if (p.NMAT == 2) {
+      prefetch_tmap(&tm_c1);
+      prefetch_tmap(&tm_s1);
+    }
+    for (int i = 0; i < XS; ++i) {
+      mbar_init(bar_x_full + 8 * i, 1);
+      mbar_init(bar_x_empty + 8 * i, 1);
+    }
+    for (int i = 0; i < WS; ++i) {
+      mbar_init(bar_w_full + 8 * i, 1);
+      mbar_init(bar_w_empty + 8 * i, kDequantWarps);
+    }
+    for (int i = 0; i < AS; ++i) {
+      mbar_init(bar_a_full + 8 * i, kDequantWarps);
+      mbar_init(bar_a_empty + 8 * i, 1);
+    }
+    mbar_init(bar_acc, 1);
+    ctl[1] = 0;
+    ctl[2] = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(ctl), (uint32_t)p.tmem_cols);
+    tmem_relinquish();
+  }
+  if (warp >= 2) {
+    for (int i = threadIdx.x - 64; i < p.NB; i += kDequantWarps * 32) {
+      const int b = bt * p.NB + i;
+      col_fac[i] = (b < p.B) ? (p.x_exp ? ldexpf(1.0f, p.x_exp[b]) : 1.0f) : 0.0f;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = static_cast<uint32_t>(ctl[0]);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_x = policy_evict_last();
+      int xi = 0, wi = 0;
+      bool ok = true;
+      for (int c = c0; c < c1 && ok; ++c) {
+        for (int step = 0; step < p.R + J && ok; ++step) {
+          // order per chunk: W(c,0), x(c,0..J-1), W(c,1..R-1)
+          const bool is_w = (step == 0) || (step > J);
+          if (is_w) {
+            const int r = (step == 0) ? 0 : step - J;
+            const int slot = wi % WS;
+            if (wi >= WS && !mbar_wait(bar_w_empty + 8 * slot, ((wi / WS) & 1) ^ 1, abort_flag,
+                                       p.dev_err, kErrTimeout)) {
+              ok = false;
+              break;
+            }
+            const uint32_t fb = bar_w_full + 8 * slot;
+            mbar_arrive_expect_tx(fb, kWStageBytes);
+            const int m = r % p.NMAT;
+            const int t = g * tiles_per_group + r / p.NMAT;
+            const uint32_t dst = sw + slot * kWStageBytes;
+            const int sxb = (FMT == FMT_NVFP4) ? c * 16 : (c >> 1) * 16;
+            tma_load_2d(dst, m ? &tm_c1 : &tm_c0, fb, c * kWRowBytes, t * kTileRows, pol_w);
+            tma_load_2d(dst + kWCodeBytes, m ? &tm_s1 : &tm_s0, fb, sxb, t * kTileRows, pol_w);
+            ++wi;
+          } else {
+            const int j = step - 1;
+            const int slot = xi % XS;
+            if (xi >= XS && !mbar_wait(bar_x_empty + 8 * slot, ((xi / XS) & 1) ^ 1, abort_flag,
+                                       p.dev_err, kErrTimeout)) {
+              ok = false;
+              break;
+            }
+            const uint32_t fb = bar_x_full + 8 * slot;
+            mbar_arrive_expect_tx(fb, (uint32_t)p.NB * 128u);
+            tma_load_2d(sx + slot * p.NB * 128, &tm_x, fb, c * KW + j * kSubK, bt * p.NB, pol_x);
+            ++xi;
+          }
+        }
+      }
+      if (!ok) {
+        // let every load already issued land before the CTA leaves
+        for (int k = (xi > XS ? xi - XS : 0); k < xi; ++k) {
+          const uint32_t bar = bar_x_full + 8 * (k % XS);
+          const uint64_t t0 = globaltimer_ns();
+          while (!mbar_try_wait(bar, (k / XS) & 1) && globaltimer_ns() - t0 < kWaitLimitNs) {
+          }
+        }
+        for (int k = (wi > WS ? wi - WS : 0); k < wi; ++k) {
+          const uint32_t bar = bar_w_full + 8 * (k % WS);
+          const uint64_t t0 = globaltimer_ns();
+          while (!mbar_try_wait(bar, (k / WS) & 1) && globaltimer_ns() - t0 < kWaitLimitNs) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_f16(BF16OP, (uint32_t)p.NB);
+      int xi = 0, ai = 0;
+      bool ok = true;
+      for (int c = c0; c < c1 && ok; ++c) {
+        for (int r = 0; r < p.R && ok; ++r) {
+          for (int ja = 0; ja < JA && ok; ++ja) {
+            const int aslot = ai % AS;
+            if (!mbar_wait(bar_a_full + 8 * aslot, (ai / AS) & 1, abort_flag, p.dev_err,
+                           kErrTimeout)) {
+              ok = false;
+              break;
+            }
+            const uint32_t d = tmem + (uint32_t)(r * p.NB);
+            const uint32_t a = tmem + a_col0 + (uint32_t)(aslot * kAColsPerStage);
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+              const int xk = xi + ja * 2 + jj;
+              const int xslot = xk % XS;
+              if (r == 0 && !mbar_wait(bar_x_full + 8 * xslot, (xk / XS) & 1, abort_flag,
+                                       p.dev_err, kErrTimeout)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const uint32_t bx = sx + (uint32_t)(xslot * p.NB * 128);
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint32_t acc = (c > c0 || ja > 0 || jj > 0 || kk > 0) ? 1u : 0u;
+                mma_f16_ts(d, a + (uint32_t)(jj * 32 + kk * 8), smem_desc_sw128(bx + kk * 32),
+                           idesc, acc);
+              }
+              if (r == p.R - 1) mma_commit(bar_x_empty + 8 * xslot);
+            }
+            mma_commit(bar_a_empty + 8 * aslot);
+            ++ai;
+          }
+        }
+        xi += J;
+      }
+      mma_commit(bar_acc);
+    }
+  } else {
+    // ------------------------------------------------------------ dequant + epilogue
+    const int dw = warp - 2;
+    const int q = warp & 3;       // TMEM lane quarter this warp may access
+    const int h = dw >> 2;        // which 64-element half of each 128-element A stage
+    const int row = q * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+
+    // MXFP4 on f16 operands: largest block exponent of this row within the split
+    int emax[4] = {0, 0, 0, 0};
+    if (FMT == FMT_MXFP4 && !BF16OP) {
+      const int kb0 = c0 * (KW / 32);
+      const int kb1 = min(c1 * (KW / 32), p.K / 32);
+      for (int r = 0; r < p.R; ++r) {
+        const int n = (g * tiles_per_group + r / p.NMAT) * kTileRows + row;
+        int mx = 0;
+        if (n < p.N) {
+          const uint8_t* sr = p.scales[r % p.NMAT] + (size_t)n * p.spitch;
+          for (int kb = kb0; kb < kb1; ++kb) mx = max(mx, (int)__ldg(sr + kb));
+        }
+        emax[r] = mx;
+      }
+    }
+
+    int wi = 0, ai = 0;
+    bool ok = true;
+    for (int c = c0; c < c1 && ok; ++c) {
+      for (int r = 0; r < p.R && ok; ++r) {
+        const int wslot = wi % WS;
+        ok = mbar_wait(bar_w_full + 8 * wslot, (wi / WS) & 1, abort_flag, p.dev_err, kErrTimeout);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        const uint8_t* stage = smem + p.smem_w + wslot * kWStageBytes;
+        const uint8_t* crow = stage + row * kWRowBytes;
+        const uint8_t* srow = stage + kWCodeBytes + row * kScaleRowBytes;
+        const int ex = emax[r & 3];
+        for (int ja = 0; ja < JA; ++ja) {
+          const int aslot = ai % AS;
+          if (ai >= AS) {
+            ok = mbar_wait(bar_a_empty + 8 * aslot, ((ai / AS) & 1) ^ 1, abort_flag, p.dev_err,
+                           kErrTimeout);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+          }
+          tc_fence_after();
+          // this warp's 64 elements of the 128-element A stage, as two independent halves
+          const int e0 = ja * kAStageK + h * 64;
+          uint32_t v[32];
+          Dequant<FMT, BF16OP>::run(crow, row, srow, c, e0, ex,
+                                    *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
+          Dequant<FMT, BF16OP>::run(crow, row, srow, c, e0 + 32, ex,
+                                    *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
+          tmem_st32(tmem + lane_base + a_col0 + (uint32_t)(aslot * kAColsPerStage + h * 32), v);
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_a_full + 8 * aslot);
+          ++ai;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_w_empty + 8 * wslot);
+        ++wi;
+      }
+    }
+
+    if (ok) {
+      ok = mbar_wait(bar_acc, 0, abort_flag, p.dev_err, kErrTimeout);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    tc_fence_after();
+    const int half_cols = p.NB >> 1;
+    const int cb0 = h * half_cols;
+    const size_t BN = (size_t)p.B * p.N;
+    float ts[2] = {1.0f, 1.0f};
+    if (FMT == FMT_NVFP4) {
+      ts[0] = __ldg(p.ts[0]);
+      if (p.NMAT == 2) ts[1] = __ldg(p.ts[1]);
+    }
+    float rowfac[4] = {1.0f, 1.0f, 1.0f, 1.0f};
+    if (FMT == FMT_MXFP4 && !BF16OP)
+      for (int r = 0; r < p.R; ++r) rowfac[r & 3] = ldexpf(1.0f, emax[r & 3] - 140);
+    if (ok) {
+      // pass 1: scale the accumulators; store finals (S == 1) or partials (S > 1)
+      for (int t2 = 0; t2 < tiles_per_group; ++t2) {
+        const int n = (g * tiles_per_group + t2) * kTileRows + row;
+        for (int cb = cb0; cb < cb0 + half_cols; cb += 8) {
+          uint32_t va[8], vb[8];
+          tmem_ld8(tmem + lane_base + (uint32_t)(t2 * p.NMAT * p.NB + cb), va);
+          if (p.NMAT == 2) tmem_ld8(tmem + lane_base + (uint32_t)((t2 * 2 + 1) * p.NB + cb), vb);
+          tmem_ld_wait();
+          if (n < p.N) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int b = bt * p.NB + cb + i;
+              if (b >= p.B) break;
+              const float cf = col_fac[cb + i];
+              const float ga = __uint_as_float(va[i]) * cf * rowfac[(t2 * p.NMAT) & 3];
+              if (p.NMAT == 1) {
+                if (p.S > 1) p.ws[(size_t)s * BN + (size_t)b * p.N + n] = ga;
+                else store_y(p, b, n, ga * ts[0]);
+              } else {
+                const float ua = __uint_as_float(vb[i]) * cf * rowfac[(t2 * 2 + 1) & 3];
+                if (p.S > 1) {
+                  p.ws[(size_t)(2 * s) * BN + (size_t)b * p.N + n] = ga;
+                  p.ws[(size_t)(2 * s + 1) * BN + (size_t)b * p.N + n] = ua;
+                } else {
+                  store_h(p, b, n, ga * ts[0], ua * ts[1]);
+                }
+              }
+            }
+          }
+        }
+      }
+    }
+    // pass 2 (split K): the last CTA of this tile sums the S partials in order s = 0..S-1.
+    // Every epilogue warp reaches both barriers, whatever its own status.
+    if (p.S > 1) {
+      {
+        __threadfence();
+        named_bar_epilogue();
+        if (threadIdx.x == 64) {
+          int last = 0;
+          if (!*abort_flag) {
+            int* cnt = p.counters + (g * p.b_tiles + bt);
+            const int old = atomicAdd(cnt, 1);
+            last = (old == p.S - 1);
+            if (last) *cnt = 0;
+          }
+          ctl[2] = last;
+        }
+        named_bar_epilogue();
+        if (ok && ctl[2]) {
+          __threadfence();
+          for (int t2 = 0; t2 < tiles_per_group; ++t2) {
+            const int n = (g * tiles_per_group + t2) * kTileRows + row;
+            if (n >= p.N) continue;
+            for (int cb = cb0; cb < cb0 + half_cols; ++cb) {
+              const int b = bt * p.NB + cb;
+              if (b >= p.B) break;
+              const size_t off = (size_t)b * p.N + n;
+              if (p.NMAT == 1) {
+                float acc = 0.0f;
+                for (int s2 = 0; s2 < p.S; ++s2) acc += __ldcg(p.ws + (size_t)s2 * BN + off);
+                store_y(p, b, n, acc * ts[0]);
+              } else {
+                float ga = 0.0f, ua = 0.0f;
+                for (int s2 = 0; s2 < p.S; ++s2) {
+                  ga += __ldcg(p.ws + (size_t)(2 * s2) * BN + off);
+                  ua += __ldcg(p.ws + (size_t)(2 * s2 + 1) * BN + off);
+                }
+                store_h(p, b, n, ga * ts[0], ua * ts[1]);
+              }
+            }
+          }
+        }
+      }
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    if (lane == 0 && *abort_flag) {
+      // the final commit arrives once every MMA issued by this CTA has completed
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(bar_acc, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+      }
+    }
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, (uint32_t)p.tmem_cols);
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Host-side launchers (called by the C-ABI layer)
+// ---------------------------------------------------------------------------------------
+int* device_error_word() {
+  void* ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_dev_err) != cudaSuccess) return nullptr;
+  return static_cast<int*>(ptr);
+}
+
+cudaError_t launch_prep(const PrepParams& pp, cudaStream_t stream) {
+  qgemm_prep_x_kernel<<<pp.B, 256, 0, stream>>>(pp);
+  return cudaGetLastError();
+}
+
+template <int FMT, bool BF16OP>
+static cudaError_t launch_tc_impl(const GemmParams& p, size_t smem_bytes, int grid,
+                                  const CUtensorMap* maps, cudaStream_t stream) {
+  auto kern = qgemm_tc_kernel<FMT, BF16OP>;
+  static size_t configured = 0;  // per instantiation: largest dynamic smem granted so far
+  if (smem_bytes > configured) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem_bytes));
+    if (e != cudaSuccess) return e;
+    configured = smem_bytes;
+  }
+  kern<<<grid, kThreads, smem_bytes, stream>>>(p, maps[0], maps[1], maps[2], maps[3], maps[4]);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tc(int fmt, bool bf16op, const GemmParams& p, size_t smem_bytes, int grid,
+                      const CUtensorMap* maps, cudaStream_t stream) {
+  switch (fmt * 2 + (bf16op ? 1 : 0)) {
+    case FMT_Q8_0 * 2: return launch_tc_impl<FMT_Q8_0, false>(p, smem_bytes, grid, maps, stream);
+    case FMT_Q8_0 * 2 + 1: return launch_tc_impl<FMT_Q8_0, true>(p, smem_bytes, grid, maps, stream);
+    case FMT_NVFP4 * 2: return launch_tc_impl<FMT_NVFP4, false>(p, smem_bytes, grid, maps, stream);
+    case FMT_NVFP4 * 2 + 1: return launch_tc_impl<FMT_NVFP4, true>(p, smem_bytes, grid, maps, stream);
+    case FMT_MXFP4 * 2: return launch_tc_impl<FMT_MXFP4, false>(p, smem_bytes, grid, maps, stream);
+    case FMT_MXFP4 * 2 + 1: return launch_tc_impl<FMT_MXFP4, true>(p, smem_bytes, grid, maps, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace qg

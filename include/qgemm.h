@@ -1,0 +1,168 @@
+/*
+ * qgemm.h -- C ABI of libqgemm: bf16 activations x block-quantized weights on NVIDIA B200.
+ *
+ *   y[b][n] = sum_k x[b][k] * dequant(W)[n][k]        b < B, n < N, k < K
+ *
+ * Operation.  The batched quantized-weight GEMM behind the pages' `gemm_q8_0_batched`
+ * (hipfire PR "fix(mtp): chunk scalar Q8 batched GEMM above 64 rows", section "Root
+ * cause and fix") and the W4A16 prefill GEMMs (Atlas issue "Qwen3.8-27B on Strix Halo:
+ * prefill 2.4x gap + DP4A verify tiers", section "Kernel ranking ...").  Unlike the
+ * fixed MAX_BATCH=64 scalar kernel there, every width B >= 1 is accepted in one call,
+ * and for 1 <= B <= 256 row b of y is bit-identical whatever the width of the call it
+ * belongs to (the PR's chunked-vs-unchunked bit-exactness, generalised).
+ *
+ * Weight formats (the pages name them; their bit layouts are fixed here):
+ *   QGEMM_FMT_Q8_0  int8 codes; one IEEE fp16 scale per 32 consecutive k:  w = q * d.
+ *   QGEMM_FMT_NVFP4 E2M1 codes; one E4M3 scale per 16 consecutive k; one fp32 tensor
+ *                   scale ts:  w = e2m1 * e4m3 * ts  (ts applied in the epilogue, as on
+ *                   the Atlas issue's exact-F16-dequant section).
+ *   QGEMM_FMT_MXFP4 E2M1 codes; one E8M0 scale per 32 consecutive k (the MXFP4 model
+ *                   card's format, OCP MX v1.0):  w = e2m1 * 2^(e-127).
+ *
+ * Packed layout (row-major, every row starts 16-byte aligned):
+ *   codes  [N][code_pitch] bytes.  Q8_0: byte k is int8 q_k, code_pitch = roundup(K,16).
+ *          FP4: byte k/2 holds element k, the even element in the low nibble,
+ *          code_pitch = roundup(K/2,16).
+ *   scales [N][scale_pitch] bytes.  Q8_0: little-endian fp16 per 32-block,
+ *          scale_pitch = roundup(K/16,16).  NVFP4: E4M3 byte per 16-block,
+ *          scale_pitch = roundup(K/16,16).  MXFP4: E8M0 byte per 32-block,
+ *          scale_pitch = roundup(K/32,16).
+ *
+ * Conventions for every entry point:
+ *   - Pointers named *_dev are device pointers; the caller owns every buffer and the
+ *     stream.  `stream` is a cudaStream_t (NULL = legacy default stream).
+ *   - Calls are asynchronous on `stream` and return a status immediately; they never
+ *     abort or exit the process.  A status other than QGEMM_OK means nothing was
+ *     launched (argument errors) or a launch failed (QGEMM_ERR_CUDA).
+ *   - Device pointers must be 16-byte aligned (TMA); x, y and h must be contiguous.
+ *   - The library keeps no device state between calls except a small cache of
+ *     TMA descriptors and a device error word read by qgemm_device_status().
+ *   - Calls that overlap on the device may share nothing writable: each needs its own
+ *     workspace.
+ */
+#ifndef QGEMM_H
+#define QGEMM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Weight formats. */
+#define QGEMM_FMT_Q8_0 0
+#define QGEMM_FMT_NVFP4 1
+#define QGEMM_FMT_MXFP4 2
+
+/* Output element types of qgemm_run. */
+#define QGEMM_Y_F32 0
+#define QGEMM_Y_BF16 1
+
+/* Status codes. */
+#define QGEMM_OK 0
+#define QGEMM_ERR_FORMAT 1         /* unknown format or output dtype                     */
+#define QGEMM_ERR_SHAPE 2          /* N, K or B < 1, or a dimension above 2^31-1        */
+#define QGEMM_ERR_K_BLOCK 3        /* K not a multiple of the format's block size       */
+#define QGEMM_ERR_NULL 4           /* a required pointer is NULL                         */
+#define QGEMM_ERR_ALIGN 5          /* a device pointer is not 16-byte aligned            */
+#define QGEMM_ERR_WORKSPACE 6      /* workspace NULL or smaller than the required size   */
+#define QGEMM_ERR_CUDA 7           /* a CUDA call or kernel launch failed                */
+#define QGEMM_ERR_DEVICE 8         /* the current device is not an sm_100 part           */
+#define QGEMM_ERR_DEVICE_TIMEOUT 9 /* a kernel's bounded wait ran out (see device_status) */
+
+/*
+ * Sizes of the packed buffers for an N x K weight matrix.  No device work.
+ * Returns QGEMM_ERR_FORMAT / _SHAPE / _K_BLOCK / _NULL.
+ */
+int qgemm_packed_size(int fmt, int64_t N, int64_t K, size_t* code_bytes, size_t* scale_bytes);
+
+/* Row pitches in bytes of the packed codes and scales (see the layout above). */
+int qgemm_row_pitches(int fmt, int64_t K, int64_t* code_pitch, int64_t* scale_pitch);
+
+/*
+ * Quantize W_dev (fp32, row-major [N][K], contiguous) into the packed layout.
+ *   Q8_0 : d = fp16_RNE(max|w|/127) (kept finite), q = clamp(RNE(w/d), -127, 127);
+ *          a block whose d is 0 gets q = 0.
+ *   NVFP4: ts = fp32_RNE(max|W|/(6*448)); per 16-block s = E4M3_RNE_sat(amax/(6*ts));
+ *          code = E2M1_RNE_sat(w/(e4m3(s)*ts)); an all-zero block (or a scale that
+ *          rounds to 0) gets scale 0 and codes 0.  Writes ts to *tensor_scale_dev.
+ *   MXFP4: e = clamp(floor(log2 amax) - 2 + 127, 0, 254); code = E2M1_RNE_sat(w/2^(e-127));
+ *          an all-zero block gets e = 0 and codes 0.
+ * Ties round to even.  A negative element whose magnitude rounds to 0 keeps its sign bit.
+ * codes_dev / scales_dev: qgemm_packed_size() bytes each, 16-byte aligned.
+ * tensor_scale_dev: one float (NVFP4 only; must be NULL or ignored otherwise).
+ * Not performance critical (uses fp64 for exact tie decisions).
+ */
+int qgemm_pack(int fmt, const float* W_dev, int64_t N, int64_t K, void* codes_dev,
+               void* scales_dev, float* tensor_scale_dev, void* stream);
+
+/*
+ * Bytes of device workspace qgemm_run needs for (fmt, N, K, B).  May be 0.
+ */
+int qgemm_workspace_size(int fmt, int64_t N, int64_t K, int64_t B, size_t* bytes);
+
+/*
+ * y_dev[B][N] = x_dev[B][K] (bf16) * dequant(W)^T, W given by codes_dev / scales_dev
+ * (packed as above) and, for NVFP4, the fp32 tensor scale at *tensor_scale_dev.
+ *   y_dtype    : QGEMM_Y_F32 (fp32) or QGEMM_Y_BF16 (bf16, round to nearest even).
+ *   workspace  : qgemm_workspace_size() bytes of device memory (may be NULL if that
+ *                size is 0).  Its contents need no initialisation.
+ * Any B >= 1.  For B <= 256 the result row b depends only on x row b, W, and (N, K):
+ * the split of K, the order of every sum and the arithmetic do not depend on B.
+ * Accuracy: fp32 accumulation of exactly dequantized weights (Q8_0 products are rounded
+ * once to the 16-bit operand type); see the project notes for the bound.
+ */
+int qgemm_run(int fmt, const void* x_dev, int64_t B, int64_t K, const void* codes_dev,
+              const void* scales_dev, const float* tensor_scale_dev, int64_t N, void* y_dev,
+              int y_dtype, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of device workspace qgemm_ffn_gate_up needs for (fmt, N, K, M). */
+int qgemm_ffn_workspace_size(int fmt, int64_t N, int64_t K, int64_t M, size_t* bytes);
+
+/*
+ * Fused gate+up projection with a SiLU(gate)*up epilogue (Atlas issue, "fused gate+up
+ * with dual accumulators ... gate/up are never written to global"):
+ *   g = x Wg^T, u = x Wu^T (fp32 accumulators, never stored);
+ *   h_dev[M][N] = bf16_RNE( g / (1 + exp(-g)) * u ).
+ * Both matrices use the same format and shape [N][K]; x_dev is bf16 [M][K].
+ * g_ts_dev / u_ts_dev: NVFP4 tensor scales (NULL for the other formats).
+ * For M <= 256 row m of h depends only on x row m (as for qgemm_run).
+ */
+int qgemm_ffn_gate_up(int fmt, const void* x_dev, int64_t M, int64_t K, const void* g_codes_dev,
+                      const void* g_scales_dev, const float* g_ts_dev, const void* u_codes_dev,
+                      const void* u_scales_dev, const float* u_ts_dev, int64_t N, void* h_dev,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Number of K splits qgemm_run uses for 1 <= B <= 256 (a function of fmt, N, K only).
+ */
+int qgemm_split_k(int fmt, int64_t N, int64_t K, int* splits);
+
+/*
+ * Synchronizes the current device and reports whether any kernel of this library hit a
+ * bounded-wait limit since the last reset (QGEMM_ERR_DEVICE_TIMEOUT), else QGEMM_OK or
+ * QGEMM_ERR_CUDA.  reset != 0 clears the flag.
+ */
+int qgemm_device_status(int reset);
+
+/*
+ * Instrumentation: when begin_event / end_event are non-NULL (cudaEvent_t handles created by
+ * the caller), the next qgemm_run / qgemm_ffn_gate_up calls made by this thread record them
+ * on their stream immediately before and after the GEMM kernel (excluding the small x
+ * preparation kernel that widths <= 256 run first).  Pass NULL, NULL to stop.  Returns
+ * QGEMM_OK.
+ */
+int qgemm_profile_events(void* begin_event, void* end_event);
+
+/* Static, human-readable text for a status code. */
+const char* qgemm_status_str(int status);
+
+/* Text of the last CUDA error seen by this library in the calling thread ("" if none). */
+const char* qgemm_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QGEMM_H */

@@ -1,0 +1,105 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry point the header
+declares, and its host-side logic (validation, sizes, the K-split rule) behaves as documented.
+No compute is launched."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+from block_quantized_weight_qgemm_b200 import build as qbuild
+from block_quantized_weight_qgemm_b200 import qgemm
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qgemm.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    qbuild.build()
+    return qgemm.lib()
+
+
+def header_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(qgemm_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = header_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), n
+    # and the binding covers exactly the header's entry points
+    assert sorted(n for n, _, _ in qgemm.SIGNATURES) == names
+
+
+def test_status_strings(lib):
+    for code in range(10):
+        s = lib.qgemm_status_str(code).decode()
+        assert s and s != "unknown status"
+    assert lib.qgemm_status_str(99).decode() == "unknown status"
+    assert lib.qgemm_last_cuda_error().decode() == ""
+
+
+@pytest.mark.parametrize("fmt", ["q8_0", "nvfp4", "mxfp4"])
+@pytest.mark.parametrize("K", [32, 64, 96, 1024, 5120, 17408])
+def test_pitches_match_layout_spec(lib, fmt, K):
+    if fmt != "nvfp4" and K % 32:
+        pytest.skip("K must be a multiple of 32")
+    cp, sp = qgemm.row_pitches(fmt, K)
+    assert (cp, sp) == (oracle.code_pitch(fmt, K), oracle.scale_pitch(fmt, K))
+    cb, sb = qgemm.packed_size(fmt, 7, K)
+    assert (cb, sb) == (7 * cp, 7 * sp)
+
+
+def test_argument_errors(lib):
+    sz = ctypes.c_size_t()
+    i64 = ctypes.c_int64()
+    assert lib.qgemm_packed_size(5, 4, 32, ctypes.byref(sz), ctypes.byref(sz)) == 1   # format
+    assert lib.qgemm_packed_size(0, 0, 32, ctypes.byref(sz), ctypes.byref(sz)) == 2   # N < 1
+    assert lib.qgemm_packed_size(0, 4, 0, ctypes.byref(sz), ctypes.byref(sz)) == 2    # K < 1
+    assert lib.qgemm_packed_size(0, 4, 48, ctypes.byref(sz), ctypes.byref(sz)) == 3   # K % 32
+    assert lib.qgemm_packed_size(1, 4, 40, ctypes.byref(sz), ctypes.byref(sz)) == 3   # K % 16
+    assert lib.qgemm_packed_size(1, 4, 48, ctypes.byref(sz), ctypes.byref(sz)) == 0
+    assert lib.qgemm_packed_size(0, 4, 32, None, None) == 4                           # NULL
+    assert lib.qgemm_row_pitches(2, 48, ctypes.byref(i64), ctypes.byref(i64)) == 3
+    assert lib.qgemm_workspace_size(0, 4, 32, 0, ctypes.byref(sz)) == 2               # B < 1
+    # qgemm_run: validation happens before any device work
+    assert lib.qgemm_run(0, None, 4, 64, None, None, None, 8, None, 0, None, 0, None) == 4
+    assert lib.qgemm_run(0, 16, 4, 64, 16, 16, None, 8, 16, 7, None, 0, None) == 1   # y dtype
+    assert lib.qgemm_run(1, 16, 4, 64, 16, 16, None, 8, 16, 0, None, 0, None) == 4   # NVFP4 ts
+    assert lib.qgemm_run(0, 8, 4, 64, 16, 16, None, 8, 16, 0, None, 0, None) == 5    # misaligned
+    assert lib.qgemm_run(0, 16, 0, 64, 16, 16, None, 8, 16, 0, None, 0, None) == 2   # B = 0
+    assert lib.qgemm_pack(0, None, 4, 64, None, None, None, None) == 4
+    assert lib.qgemm_ffn_gate_up(0, 16, 4, 64, 16, 16, None, None, 16, None, 8, 16, None, 0,
+                                 None) == 4
+
+
+def test_no_width_limit_in_sizes(lib):
+    # every width has a workspace size; nothing is rejected above 64 (the pages' MAX_BATCH)
+    for B in (1, 63, 64, 65, 70, 76, 255, 256, 257, 1000, 8192):
+        assert qgemm.workspace_size("q8_0", 17408, 5120, B) >= 0
+
+
+def test_split_rule_depends_only_on_shape(lib):
+    # the K split is a function of (format, N, K): pinned values for the 27B FFN shapes
+    got = {(f, N, K): qgemm.split_k(f, N, K) for f in ("q8_0", "nvfp4", "mxfp4")
+           for (N, K) in ((17408, 5120), (5120, 17408), (512, 1024))}
+    for (f, N, K), s in got.items():
+        assert 1 <= s <= 16
+    assert got[("q8_0", 17408, 5120)] == 4
+    assert got[("nvfp4", 17408, 5120)] == 4
+    assert got[("q8_0", 5120, 17408)] == 14
+    assert got[("nvfp4", 5120, 17408)] == 14
+    # workspace grows with B but the split does not
+    w64 = qgemm.workspace_size("q8_0", 17408, 5120, 64)
+    w65 = qgemm.workspace_size("q8_0", 17408, 5120, 65)
+    assert w65 > w64
+
+
+def test_prefill_path_needs_no_workspace(lib):
+    assert qgemm.workspace_size("nvfp4", 17408, 5120, 2048) == 0
+    assert qgemm.ffn_workspace_size("nvfp4", 17408, 5120, 2048) == 0
