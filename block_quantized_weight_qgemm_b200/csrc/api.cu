@@ -5,6 +5,7 @@
 
 #include <algorithm>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -17,6 +18,7 @@ cudaError_t launch_tc(int fmt, bool bf16op, const GemmParams& p, size_t smem_byt
                       const CUtensorMap* maps, cudaStream_t stream);
 cudaError_t launch_pack(int fmt, const float* W, int64_t N, int64_t K, void* codes, void* scales,
                         float* tensor_scale, cudaStream_t stream);
+cudaError_t launch_repack(const RepackParams& rp, cudaStream_t stream);
 int* device_error_word();
 }  // namespace qg
 
@@ -156,13 +158,13 @@ bool make_plan(int fmt, int64_t N, int64_t K, int64_t B, int nmat, Plan* pl) {
     p.NB = (nmat == 2) ? 128 : 256;
   }
   p.b_tiles = (int)((B + p.NB - 1) / p.NB);
-  // subtiles per unit: TMEM holds R*NB accumulator columns plus an A ring of >= 2 stages
-  int rmax = std::min(4, (512 - 2 * kAColsPerStage) / p.NB);
-  rmax = rmax / nmat * nmat;
-  if (rmax < nmat) return false;
-  int bestR = nmat;
+  // subtiles per unit: TMEM holds R*NB accumulator columns plus the A ring (kMaxAStages
+  // stages, split evenly between the R subtiles' MMA issuers, so R divides kMaxAStages)
+  const int rmax = std::min(kMaxAStages, (512 - kMaxAStages * kAColsPerStage) / p.NB);
+  int bestR = 0;
   int64_t best_cost = -1;
-  for (int R = nmat; R <= rmax; R += nmat) {
+  for (int R = nmat; R <= rmax; R *= 2) {
+    if (R % nmat) continue;
     const int64_t groups = (tiles + (R / nmat) - 1) / (R / nmat);
     const int64_t units = groups * p.b_tiles * p.S;
     const int64_t cost = ((units + kSMs - 1) / kSMs) * R;
@@ -171,10 +173,15 @@ bool make_plan(int fmt, int64_t N, int64_t K, int64_t B, int nmat, Plan* pl) {
       bestR = R;
     }
   }
+  if (bestR == 0) return false;
+  // debug override (scheduling only: R never changes the arithmetic)
+  if (const char* e = getenv("QGEMM_DEBUG_R")) {
+    const int r = atoi(e);
+    if ((r == 1 || r == 2 || r == 4) && r % nmat == 0 && r <= rmax) bestR = r;
+  }
   p.R = bestR;
   p.n_groups = (int)((tiles + (p.R / nmat) - 1) / (p.R / nmat));
-  p.AS = std::min(kMaxAStages, (512 - p.R * p.NB) / kAColsPerStage);
-  if (p.AS < 2) return false;
+  p.AS = kMaxAStages;
   p.tmem_cols = next_pow2_cols(p.R * p.NB + p.AS * kAColsPerStage);
   if (p.tmem_cols > 512) return false;
   // shared memory: x ring, weight ring (gets the rest, up to 8 stages), barriers, control
@@ -239,10 +246,10 @@ int run_impl(int fmt, const void* x, int64_t B, int64_t K, const void* const* co
   p.smem_x = pl.smem_x;
   p.smem_w = pl.smem_w;
   p.smem_bar = pl.smem_bar;
-  p.spitch = scale_pitch(fmt, K);
   for (int m = 0; m < 2; ++m) {
     const int mm = (m < nmat) ? m : 0;
     p.ts[m] = ts[mm];
+    p.codes[m] = static_cast<const uint8_t*>(codes[mm]);
     p.scales[m] = static_cast<const uint8_t*>(scales[mm]);
   }
   p.x_exp = pl.f16ops ? reinterpret_cast<const int*>(wsb + pl.off_exp) : nullptr;
@@ -267,31 +274,17 @@ int run_impl(int fmt, const void* x, int64_t B, int64_t K, const void* const* co
     xop = pp.xh;
   }
 
-  CUtensorMap maps[5];
+  CUtensorMap xmap;
   const CUtensorMapDataType xdt =
       pl.f16ops ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  bool ok = make_map(&maps[0], xdt, 2, xop, (uint64_t)K, (uint64_t)B, (uint64_t)K * 2, kSubK,
-                     (uint32_t)pl.NB, CU_TENSOR_MAP_SWIZZLE_128B);
-  const uint64_t code_bytes = (fmt == FMT_Q8_0) ? (uint64_t)K : (uint64_t)K / 2;
-  const uint64_t scale_bytes = (fmt == FMT_Q8_0) ? (uint64_t)K / 16
-                               : (fmt == FMT_NVFP4) ? (uint64_t)K / 16
-                                                    : (uint64_t)K / 32;
-  for (int m = 0; m < 2 && ok; ++m) {
-    const int mm = (m < nmat) ? m : 0;
-    ok = ok && make_map(&maps[1 + 2 * m], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, codes[mm], code_bytes,
-                        (uint64_t)N, (uint64_t)code_pitch(fmt, K), kWRowBytes, kTileRows,
-                        CU_TENSOR_MAP_SWIZZLE_128B);
-    ok = ok && make_map(&maps[2 + 2 * m], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, scales[mm], scale_bytes,
-                        (uint64_t)N, (uint64_t)scale_pitch(fmt, K), kScaleRowBytes, kTileRows,
-                        CU_TENSOR_MAP_SWIZZLE_NONE);
-  }
-  if (!ok) {
+  if (!make_map(&xmap, xdt, 2, xop, (uint64_t)K, (uint64_t)B, (uint64_t)K * 2, kSubK,
+                (uint32_t)pl.NB, CU_TENSOR_MAP_SWIZZLE_128B)) {
     snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled failed");
     return QGEMM_ERR_CUDA;
   }
   const int grid = pl.n_groups * pl.b_tiles * pl.S;
   if (g_prof_begin) cudaEventRecord(g_prof_begin, stream);
-  cudaError_t e = launch_tc(fmt, !pl.f16ops, p, pl.smem_bytes, grid, maps, stream);
+  cudaError_t e = launch_tc(fmt, !pl.f16ops, p, pl.smem_bytes, grid, &xmap, stream);
   if (e != cudaSuccess) return cuda_fail(e, "gemm kernel launch");
   if (g_prof_end) cudaEventRecord(g_prof_end, stream);
   return QGEMM_OK;
@@ -305,8 +298,20 @@ int qgemm_packed_size(int fmt, int64_t N, int64_t K, size_t* code_bytes, size_t*
   const int st = check_fmt_shape(fmt, N, K);
   if (st != QGEMM_OK) return st;
   if (!code_bytes || !scale_bytes) return QGEMM_ERR_NULL;
-  *code_bytes = (size_t)(N * code_pitch(fmt, K));
-  *scale_bytes = (size_t)(N * scale_pitch(fmt, K));
+  *code_bytes = (size_t)packed_code_bytes(fmt, N, K);
+  *scale_bytes = (size_t)packed_scale_bytes(fmt, N, K);
+  return QGEMM_OK;
+}
+
+int qgemm_packed_geometry(int fmt, int64_t N, int64_t K, int64_t* tiles, int64_t* chunks,
+                          int* chunk_elems, int* scale_bytes_per_row) {
+  const int st = check_fmt_shape(fmt, N, K);
+  if (st != QGEMM_OK) return st;
+  if (!tiles || !chunks || !chunk_elems || !scale_bytes_per_row) return QGEMM_ERR_NULL;
+  *tiles = row_tiles(N);
+  *chunks = k_chunks(fmt, K);
+  *chunk_elems = chunk_k(fmt);
+  *scale_bytes_per_row = scale_row_bytes(fmt);
   return QGEMM_OK;
 }
 
@@ -314,8 +319,33 @@ int qgemm_row_pitches(int fmt, int64_t K, int64_t* cp, int64_t* sp) {
   const int st = check_fmt_shape(fmt, 1, K);
   if (st != QGEMM_OK) return st;
   if (!cp || !sp) return QGEMM_ERR_NULL;
-  *cp = code_pitch(fmt, K);
-  *sp = scale_pitch(fmt, K);
+  *cp = rm_code_pitch(fmt, K);
+  *sp = rm_scale_pitch(fmt, K);
+  return QGEMM_OK;
+}
+
+int qgemm_repack_rowmajor(int fmt, int64_t N, int64_t K, const void* codes_rm, int64_t code_pitch,
+                          const void* scales_rm, int64_t scale_pitch, void* codes, void* scales,
+                          void* stream) {
+  const int st = check_fmt_shape(fmt, N, K);
+  if (st != QGEMM_OK) return st;
+  if (!codes_rm || !scales_rm || !codes || !scales) return QGEMM_ERR_NULL;
+  if (code_pitch < rm_code_bytes_per_row(fmt, K) || scale_pitch < rm_scale_bytes_per_row(fmt, K))
+    return QGEMM_ERR_SHAPE;
+  if (!aligned16(codes) || !aligned16(scales)) return QGEMM_ERR_ALIGN;
+  if (!device_ok()) return QGEMM_ERR_DEVICE;
+  RepackParams rp{};
+  rp.codes_rm = static_cast<const uint8_t*>(codes_rm);
+  rp.scales_rm = static_cast<const uint8_t*>(scales_rm);
+  rp.code_pitch = code_pitch;
+  rp.scale_pitch = scale_pitch;
+  rp.codes = static_cast<uint8_t*>(codes);
+  rp.scales = static_cast<uint8_t*>(scales);
+  rp.N = N;
+  rp.K = K;
+  rp.fmt = fmt;
+  cudaError_t e = launch_repack(rp, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "repack kernel launch");
   return QGEMM_OK;
 }
 

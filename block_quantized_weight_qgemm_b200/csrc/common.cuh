@@ -18,19 +18,53 @@ constexpr int kAStageK = 128;                     // K per A stage (TMEM)
 constexpr int kMaxAStages = 4;                    // A ring depth limit
 constexpr int kAColsPerStage = kAStageK / 2;      // 16-bit elements, 2 per TMEM column
 constexpr int kDequantWarps = 8;                  // 2 per TMEM lane quarter
-constexpr int kThreads = (2 + kDequantWarps) * 32;
+constexpr int kMmaWarps = 4;                      // one MMA-issuing thread per weight subtile
+constexpr int kFirstDequantWarp = 1 + kMmaWarps;  // warp 0 is the TMA producer
+constexpr int kThreads = (1 + kMmaWarps + kDequantWarps) * 32;
 constexpr int kMaxNB = 256;                       // MMA N limit
 constexpr int kSmemLimit = 227 * 1024;
 
 // K covered by one weight stage (128 code bytes per row).
 __host__ __device__ constexpr int chunk_k(int fmt) { return fmt == FMT_Q8_0 ? 128 : 256; }
 __host__ __device__ constexpr int block_k(int fmt) { return fmt == FMT_NVFP4 ? 16 : 32; }
-__host__ __device__ constexpr int64_t roundup16(int64_t v) { return (v + 15) / 16 * 16; }
-__host__ __device__ constexpr int64_t code_pitch(int fmt, int64_t K) {
-  return fmt == FMT_Q8_0 ? roundup16(K) : roundup16(K / 2);
+// scale bytes per row per chunk: Q8_0 4 x fp16, NVFP4 16 x E4M3, MXFP4 8 x E8M0
+__host__ __device__ constexpr int scale_row_bytes(int fmt) { return fmt == FMT_NVFP4 ? 16 : 8; }
+__host__ __device__ constexpr int64_t row_tiles(int64_t N) { return (N + kTileRows - 1) / kTileRows; }
+__host__ __device__ constexpr int64_t k_chunks(int fmt, int64_t K) {
+  return (K + chunk_k(fmt) - 1) / chunk_k(fmt);
 }
-__host__ __device__ constexpr int64_t scale_pitch(int fmt, int64_t K) {
-  return fmt == FMT_Q8_0 ? roundup16(K / 16) : fmt == FMT_NVFP4 ? roundup16(K / 16) : roundup16(K / 32);
+// Row-major interchange layout (qgemm_repack_rowmajor input): codes [N][code pitch],
+// scales [N][scale pitch], rows 16-byte aligned.
+__host__ __device__ constexpr int64_t roundup16(int64_t v) { return (v + 15) / 16 * 16; }
+__host__ __device__ constexpr int64_t rm_code_bytes_per_row(int fmt, int64_t K) {
+  return fmt == FMT_Q8_0 ? K : K / 2;
+}
+__host__ __device__ constexpr int64_t rm_scale_bytes_per_row(int fmt, int64_t K) {
+  return fmt == FMT_Q8_0 ? 2 * (K / 32) : fmt == FMT_NVFP4 ? K / 16 : K / 32;
+}
+__host__ __device__ constexpr int64_t rm_code_pitch(int fmt, int64_t K) {
+  return roundup16(rm_code_bytes_per_row(fmt, K));
+}
+__host__ __device__ constexpr int64_t rm_scale_pitch(int fmt, int64_t K) {
+  return roundup16(rm_scale_bytes_per_row(fmt, K));
+}
+// Tile-major packed layout: for row tile t and chunk c, one contiguous block of
+// 128 rows x 128 code bytes (16-byte groups of row r stored at group ^ (r & 7)) and one
+// contiguous block of 128 rows x scale_row_bytes.
+__host__ __device__ constexpr int64_t packed_code_bytes(int fmt, int64_t N, int64_t K) {
+  return row_tiles(N) * k_chunks(fmt, K) * kWCodeBytes;
+}
+__host__ __device__ constexpr int64_t packed_scale_bytes(int fmt, int64_t N, int64_t K) {
+  return row_tiles(N) * k_chunks(fmt, K) * kTileRows * scale_row_bytes(fmt);
+}
+// byte offset of code byte `b` (0..127) of row n, chunk c
+__host__ __device__ constexpr int64_t code_offset(int64_t C, int64_t n, int64_t c, int b) {
+  return (((n / kTileRows) * C + c) * kTileRows + (n % kTileRows)) * kWRowBytes +
+         ((((b >> 4) ^ (int)(n & 7)) << 4) | (b & 15));
+}
+// byte offset of the scale bytes of row n, chunk c
+__host__ __device__ constexpr int64_t scale_offset(int fmt, int64_t C, int64_t n, int64_t c) {
+  return (((n / kTileRows) * C + c) * kTileRows + (n % kTileRows)) * scale_row_bytes(fmt);
 }
 
 // Everything the GEMM kernel needs besides its tensor maps.
@@ -49,13 +83,24 @@ struct GemmParams {
   uint32_t smem_x, smem_w, smem_bar;  // byte offsets in the 1024-aligned dynamic smem
   const int* x_exp;          // f16 operands: x row b was scaled by 2^-x_exp[b]
   const float* ts[2];        // NVFP4 tensor scales (device), else nullptr
-  const uint8_t* scales[2];  // packed scales (MXFP4 exponent pre-pass)
-  int64_t spitch;            // scale row pitch
+  const uint8_t* codes[2];   // tile-major packed codes of each matrix
+  const uint8_t* scales[2];  // tile-major packed scales of each matrix
   float* ws;                 // split-K partials [S][NMAT][B][N]
   int* counters;             // [n_groups * b_tiles], zero on entry, left zero
   void* out;                 // y [B][N] (fp32 or bf16), or h [B][N] bf16 for NMAT == 2
   int out_bf16;
   int* dev_err;
+};
+
+// Conversion of the row-major packed layout into the tile-major one.
+struct RepackParams {
+  const uint8_t* codes_rm;
+  const uint8_t* scales_rm;
+  int64_t code_pitch, scale_pitch;  // row pitches of the row-major arrays (bytes)
+  uint8_t* codes;
+  uint8_t* scales;
+  int64_t N, K;
+  int fmt;
 };
 
 // Per-row power-of-two scaling of x before the bf16 -> f16 conversion.

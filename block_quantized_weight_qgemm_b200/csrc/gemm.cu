@@ -90,7 +90,7 @@ struct Dequant<FMT_Q8_0, false> {
     const uint4 a = ld_sw128(crow, row, e0 >> 4);
     const uint4 b = ld_sw128(crow, row, (e0 >> 4) + 1);
     const uint16_t dbits =
-        *reinterpret_cast<const uint16_t*>(srow + 2 * (((c & 1) << 2) + (e0 >> 5)));
+        *reinterpret_cast<const uint16_t*>(srow + 2 * (e0 >> 5));
     const __half2 d2 = half2_bcast(dbits);
     const __half2 off = half2_bcast(0x6480);  // 1152.0
     const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
@@ -114,7 +114,7 @@ struct Dequant<FMT_Q8_0, true> {
     const uint4 a = ld_sw128(crow, row, e0 >> 4);
     const uint4 b = ld_sw128(crow, row, (e0 >> 4) + 1);
     const uint16_t dbits =
-        *reinterpret_cast<const uint16_t*>(srow + 2 * (((c & 1) << 2) + (e0 >> 5)));
+        *reinterpret_cast<const uint16_t*>(srow + 2 * (e0 >> 5));
     const float d = __half2float(__ushort_as_half(dbits));
     const float nd = -12582912.0f * d;
     const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
@@ -165,7 +165,7 @@ struct Dequant<FMT_MXFP4, false> {
   __device__ __forceinline__ static void run(const uint8_t* crow, int row, const uint8_t* srow,
                                              int c, int e0, int emax, uint32_t (&v)[16]) {
     const uint4 a = ld_sw128(crow, row, e0 >> 5);
-    const int e = srow[((c & 1) << 3) + (e0 >> 5)];
+    const int e = srow[e0 >> 5];
     const __half2 s = half2_bcast(f16_pow2_bits(e - emax + 13));
     const uint32_t w[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
@@ -224,7 +224,7 @@ struct Dequant<FMT_MXFP4, true> {
   __device__ __forceinline__ static void run(const uint8_t* crow, int row, const uint8_t* srow,
                                              int c, int e0, int /*ex*/, uint32_t (&v)[16]) {
     const uint4 a = ld_sw128(crow, row, e0 >> 5);
-    const uint32_t e = srow[((c & 1) << 3) + (e0 >> 5)];
+    const uint32_t e = srow[e0 >> 5];
     const uint32_t bits = e ? (e << 7) : 0x0040u;  // 2^(e-127) as bf16 (e = 0: subnormal)
     const __nv_bfloat162 s = u2b(bits | (bits << 16));
     e2m1x8_bf16(a.x, s, &v[0]);
@@ -307,14 +307,11 @@ __device__ __forceinline__ void named_bar_epilogue() {
 // ---------------------------------------------------------------------------------------
 template <int FMT, bool BF16OP>
 __global__ void __launch_bounds__(kThreads, 1)
-    qgemm_tc_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ CUtensorMap tm_x,
-                    const __grid_constant__ CUtensorMap tm_c0,
-                    const __grid_constant__ CUtensorMap tm_s0,
-                    const __grid_constant__ CUtensorMap tm_c1,
-                    const __grid_constant__ CUtensorMap tm_s1) {
+    qgemm_tc_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ CUtensorMap tm_x) {
   constexpr int KW = chunk_k(FMT);
   constexpr int J = KW / kSubK;       // x stages per chunk
   constexpr int JA = KW / kAStageK;   // A stages per chunk
+  constexpr int SB = scale_row_bytes(FMT);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -344,19 +341,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int c0 = (int)((int64_t)s * p.chunks / p.S);
   const int c1 = (int)((int64_t)(s + 1) * p.chunks / p.S);
   const int tiles_per_group = p.R / p.NMAT;
+  const int64_t n_row_tiles = row_tiles(p.N);
   const uint32_t a_col0 = (uint32_t)(p.R * p.NB);
 
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tm_x);
-    prefetch_tmap(&tm_c0);
-    prefetch_tmap(&tm_s0);
-    if (p.NMAT == 2) {
-      prefetch_tmap(&tm_c1);
-      prefetch_tmap(&tm_s1);
-    }
     for (int i = 0; i < XS; ++i) {
       mbar_init(bar_x_full + 8 * i, 1);
-      mbar_init(bar_x_empty + 8 * i, 1);
+      mbar_init(bar_x_empty + 8 * i, (uint32_t)p.R);  // every MMA issuer releases each x stage
     }
     for (int i = 0; i < WS; ++i) {
       mbar_init(bar_w_full + 8 * i, 1);
@@ -366,7 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar_a_full + 8 * i, kDequantWarps);
       mbar_init(bar_a_empty + 8 * i, 1);
     }
-    mbar_init(bar_acc, 1);
+    mbar_init(bar_acc, (uint32_t)p.R);  // one commit per MMA issuer
     ctl[1] = 0;
     ctl[2] = 0;
     fence_mbar_init();
@@ -375,8 +367,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(smem_u32(ctl), (uint32_t)p.tmem_cols);
     tmem_relinquish();
   }
-  if (warp >= 2) {
-    for (int i = threadIdx.x - 64; i < p.NB; i += kDequantWarps * 32) {
+  if (warp >= kFirstDequantWarp) {
+    for (int i = threadIdx.x - kFirstDequantWarp * 32; i < p.NB; i += kDequantWarps * 32) {
       const int b = bt * p.NB + i;
       col_fac[i] = (b < p.B) ? (p.x_exp ? ldexpf(1.0f, p.x_exp[b]) : 1.0f) : 0.0f;
     }
@@ -388,110 +380,150 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
+    // Two independent streams, each limited only by its own ring: weight stages in the
+    // order (c, r) and x stages in the order (c, j).  Lane 0 polls both without blocking
+    // on either, so weight prefetch never waits behind an x slot (and vice versa).
     if (lane == 0) {
       const uint64_t pol_w = policy_evict_first();
       const uint64_t pol_x = policy_evict_last();
-      int xi = 0, wi = 0;
+      const int nchunks = c1 - c0;
+      const int w_total = nchunks * p.R, x_total = nchunks * J;
+      RingPos xp, wp;
+      int x_issued = 0, w_issued = 0;
+      int wc = c0, wr = 0;  // next weight stage (chunk, subtile)
+      int xc = c0, xj = 0;  // next x stage (chunk, slice)
       bool ok = true;
-      for (int c = c0; c < c1 && ok; ++c) {
-        for (int step = 0; step < p.R + J && ok; ++step) {
-          // order per chunk: W(c,0), x(c,0..J-1), W(c,1..R-1)
-          const bool is_w = (step == 0) || (step > J);
-          if (is_w) {
-            const int r = (step == 0) ? 0 : step - J;
-            const int slot = wi % WS;
-            if (wi >= WS && !mbar_wait(bar_w_empty + 8 * slot, ((wi / WS) & 1) ^ 1, abort_flag,
-                                       p.dev_err, kErrTimeout)) {
-              ok = false;
-              break;
-            }
-            const uint32_t fb = bar_w_full + 8 * slot;
-            mbar_arrive_expect_tx(fb, kWStageBytes);
-            const int m = r % p.NMAT;
-            const int t = g * tiles_per_group + r / p.NMAT;
-            const uint32_t dst = sw + slot * kWStageBytes;
-            const int sxb = (FMT == FMT_NVFP4) ? c * 16 : (c >> 1) * 16;
-            tma_load_2d(dst, m ? &tm_c1 : &tm_c0, fb, c * kWRowBytes, t * kTileRows, pol_w);
-            tma_load_2d(dst + kWCodeBytes, m ? &tm_s1 : &tm_s0, fb, sxb, t * kTileRows, pol_w);
-            ++wi;
+      uint64_t idle_since = 0;
+      while (ok && (w_issued < w_total || x_issued < x_total)) {
+        bool progressed = false;
+        if (w_issued < w_total &&
+            (w_issued < WS || mbar_try_wait(bar_w_empty + 8 * wp.slot, wp.phase ^ 1u))) {
+          const uint32_t fb = bar_w_full + 8 * wp.slot;
+          const int m = (p.NMAT == 2) ? (wr & 1) : 0;
+          const int64_t t = (int64_t)g * tiles_per_group + (p.NMAT == 2 ? (wr >> 1) : wr);
+          const uint32_t dst = sw + (uint32_t)(wp.slot * kWStageBytes);
+          if (t < n_row_tiles) {
+            // one contiguous block of codes and one of scales per (tile, chunk)
+            const int64_t blk = t * p.chunks + wc;
+            mbar_arrive_expect_tx(fb, (uint32_t)(kWCodeBytes + kTileRows * SB));
+            bulk_load(dst, p.codes[m] + blk * kWCodeBytes, kWCodeBytes, fb, pol_w);
+            bulk_load(dst + kWCodeBytes, p.scales[m] + blk * (kTileRows * SB),
+                      (uint32_t)(kTileRows * SB), fb, pol_w);
           } else {
-            const int j = step - 1;
-            const int slot = xi % XS;
-            if (xi >= XS && !mbar_wait(bar_x_empty + 8 * slot, ((xi / XS) & 1) ^ 1, abort_flag,
-                                       p.dev_err, kErrTimeout)) {
-              ok = false;
-              break;
-            }
-            const uint32_t fb = bar_x_full + 8 * slot;
-            mbar_arrive_expect_tx(fb, (uint32_t)p.NB * 128u);
-            tma_load_2d(sx + slot * p.NB * 128, &tm_x, fb, c * KW + j * kSubK, bt * p.NB, pol_x);
-            ++xi;
+            mbar_arrive(fb);  // a tile past the matrix: its rows are never stored
           }
+          wp.next(WS);
+          ++w_issued;
+          if (++wr == p.R) {
+            wr = 0;
+            ++wc;
+          }
+          progressed = true;
+        }
+        if (x_issued < x_total &&
+            (x_issued < XS || mbar_try_wait(bar_x_empty + 8 * xp.slot, xp.phase ^ 1u))) {
+          const uint32_t fb = bar_x_full + 8 * xp.slot;
+          mbar_arrive_expect_tx(fb, (uint32_t)p.NB * 128u);
+          tma_load_2d(sx + (uint32_t)(xp.slot * p.NB * 128), &tm_x, fb, xc * KW + xj * kSubK,
+                      bt * p.NB, pol_x);
+          xp.next(XS);
+          ++x_issued;
+          if (++xj == J) {
+            xj = 0;
+            ++xc;
+          }
+          progressed = true;
+        }
+        if (progressed) {
+          idle_since = 0;
+        } else {
+          const uint64_t now = globaltimer_ns();
+          if (idle_since == 0) idle_since = now;
+          if (*abort_flag) ok = false;
+          if (now - idle_since > kWaitLimitNs) {
+            *abort_flag = 1;
+            atomicExch(p.dev_err, kErrTimeout);
+            ok = false;
+          }
+          __nanosleep(20);
         }
       }
       if (!ok) {
-        // let every load already issued land before the CTA leaves
-        for (int k = (xi > XS ? xi - XS : 0); k < xi; ++k) {
-          const uint32_t bar = bar_x_full + 8 * (k % XS);
+        // let every load already issued land before the CTA leaves: the last use of each
+        // slot is at most one ring depth back
+        for (int k = 0; k < XS && k < x_issued; ++k) {
+          xp.slot = (xp.slot == 0) ? XS - 1 : xp.slot - 1;
+          if (xp.slot == XS - 1) xp.phase ^= 1u;
           const uint64_t t0 = globaltimer_ns();
-          while (!mbar_try_wait(bar, (k / XS) & 1) && globaltimer_ns() - t0 < kWaitLimitNs) {
+          while (!mbar_try_wait(bar_x_full + 8 * xp.slot, xp.phase) &&
+                 globaltimer_ns() - t0 < kWaitLimitNs) {
           }
         }
-        for (int k = (wi > WS ? wi - WS : 0); k < wi; ++k) {
-          const uint32_t bar = bar_w_full + 8 * (k % WS);
+        for (int k = 0; k < WS && k < w_issued; ++k) {
+          wp.slot = (wp.slot == 0) ? WS - 1 : wp.slot - 1;
+          if (wp.slot == WS - 1) wp.phase ^= 1u;
           const uint64_t t0 = globaltimer_ns();
-          while (!mbar_try_wait(bar, (k / WS) & 1) && globaltimer_ns() - t0 < kWaitLimitNs) {
+          while (!mbar_try_wait(bar_w_full + 8 * wp.slot, wp.phase) &&
+                 globaltimer_ns() - t0 < kWaitLimitNs) {
           }
         }
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    __syncwarp();
+  } else if (warp < kFirstDequantWarp) {
+    // ------------------------------------------------------------ MMA issuers
+    // One thread per weight subtile r (warp 1 + r): it owns accumulator r, so the issuers'
+    // MMAs never touch the same accumulator and each accumulator still receives its K slices
+    // in ascending order.  Several issuers keep the tensor pipe fed while one of them is busy
+    // with its waits and commits.
+    const int r = warp - 1;
+    if (lane == 0 && r < p.R) {
       const uint32_t idesc = idesc_f16(BF16OP, (uint32_t)p.NB);
-      int xi = 0, ai = 0;
+      const uint32_t xstage_bytes = (uint32_t)p.NB * 128u;
+      const uint32_t d = tmem + (uint32_t)(r * p.NB);
+      // this issuer's A slots: spr = AS / R of them, used in turn, so each slot's uses
+      // alternate phase within one thread (no parity aliasing between issuers)
+      const int spr = AS / p.R;
+      RingPos xc;  // first x stage of the current chunk
       bool ok = true;
       for (int c = c0; c < c1 && ok; ++c) {
-        for (int r = 0; r < p.R && ok; ++r) {
-          for (int ja = 0; ja < JA && ok; ++ja) {
-            const int aslot = ai % AS;
-            if (!mbar_wait(bar_a_full + 8 * aslot, (ai / AS) & 1, abort_flag, p.dev_err,
-                           kErrTimeout)) {
+        RingPos xp = xc;
+        for (int ja = 0; ja < JA && ok; ++ja) {
+          const int li = (c - c0) * JA + ja;  // this subtile's A stage count
+          const int aslot = r * spr + li % spr;
+          if (!mbar_wait(bar_a_full + 8 * aslot, (uint32_t)(li / spr) & 1u, abort_flag, p.dev_err,
+                         kErrTimeout)) {
+            ok = false;
+            break;
+          }
+          const uint32_t a = tmem + a_col0 + (uint32_t)(aslot * kAColsPerStage);
+#pragma unroll
+          for (int jj = 0; jj < 2; ++jj) {
+            if (!mbar_wait(bar_x_full + 8 * xp.slot, xp.phase, abort_flag, p.dev_err, kErrTimeout)) {
               ok = false;
               break;
             }
-            const uint32_t d = tmem + (uint32_t)(r * p.NB);
-            const uint32_t a = tmem + a_col0 + (uint32_t)(aslot * kAColsPerStage);
+            tc_fence_after();
+            const uint32_t bx = sx + (uint32_t)xp.slot * xstage_bytes;
 #pragma unroll
-            for (int jj = 0; jj < 2; ++jj) {
-              const int xk = xi + ja * 2 + jj;
-              const int xslot = xk % XS;
-              if (r == 0 && !mbar_wait(bar_x_full + 8 * xslot, (xk / XS) & 1, abort_flag,
-                                       p.dev_err, kErrTimeout)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-              const uint32_t bx = sx + (uint32_t)(xslot * p.NB * 128);
-#pragma unroll
-              for (int kk = 0; kk < 4; ++kk) {
-                const uint32_t acc = (c > c0 || ja > 0 || jj > 0 || kk > 0) ? 1u : 0u;
-                mma_f16_ts(d, a + (uint32_t)(jj * 32 + kk * 8), smem_desc_sw128(bx + kk * 32),
-                           idesc, acc);
-              }
-              if (r == p.R - 1) mma_commit(bar_x_empty + 8 * xslot);
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint32_t acc = (c > c0 || ja > 0 || jj > 0 || kk > 0) ? 1u : 0u;
+              mma_f16_ts(d, a + (uint32_t)(jj * 32 + kk * 8), smem_desc_sw128(bx + kk * 32), idesc,
+                         acc);
             }
-            mma_commit(bar_a_empty + 8 * aslot);
-            ++ai;
+            mma_commit(bar_x_empty + 8 * xp.slot);
+            xp.next(XS);
           }
+          mma_commit(bar_a_empty + 8 * aslot);
         }
-        xi += J;
+        for (int j = 0; j < J; ++j) xc.next(XS);
       }
       mma_commit(bar_acc);
     }
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ dequant + epilogue
-    const int dw = warp - 2;
+    const int dw = warp - kFirstDequantWarp;
     const int q = warp & 3;       // TMEM lane quarter this warp may access
     const int h = dw >> 2;        // which 64-element half of each 128-element A stage
     const int row = q * 32 + lane;
@@ -500,35 +532,40 @@ __global__ void __launch_bounds__(kThreads, 1)
     // MXFP4 on f16 operands: largest block exponent of this row within the split
     int emax[4] = {0, 0, 0, 0};
     if (FMT == FMT_MXFP4 && !BF16OP) {
-      const int kb0 = c0 * (KW / 32);
-      const int kb1 = min(c1 * (KW / 32), p.K / 32);
+      // (padding blocks past K are zero and cannot raise the maximum)
       for (int r = 0; r < p.R; ++r) {
-        const int n = (g * tiles_per_group + r / p.NMAT) * kTileRows + row;
-        int mx = 0;
+        const int64_t n = (int64_t)(g * tiles_per_group + r / p.NMAT) * kTileRows + row;
+        uint32_t mx = 0;
         if (n < p.N) {
-          const uint8_t* sr = p.scales[r % p.NMAT] + (size_t)n * p.spitch;
-          for (int kb = kb0; kb < kb1; ++kb) mx = max(mx, (int)__ldg(sr + kb));
+          const uint8_t* sb = p.scales[r % p.NMAT];
+          for (int c = c0; c < c1; ++c) {
+            const uint2 v = __ldg(reinterpret_cast<const uint2*>(sb + scale_offset(FMT, p.chunks, n, c)));
+            mx = __vmaxu4(mx, __vmaxu4(v.x, v.y));
+          }
         }
-        emax[r] = mx;
+        mx = max(max(mx & 0xFFu, (mx >> 8) & 0xFFu), max((mx >> 16) & 0xFFu, mx >> 24));
+        emax[r] = (int)mx;
       }
     }
 
-    int wi = 0, ai = 0;
+    RingPos wp;
+    const int spr = AS / p.R;  // A slots per subtile (see the MMA issuers)
     bool ok = true;
     for (int c = c0; c < c1 && ok; ++c) {
       for (int r = 0; r < p.R && ok; ++r) {
-        const int wslot = wi % WS;
-        ok = mbar_wait(bar_w_full + 8 * wslot, (wi / WS) & 1, abort_flag, p.dev_err, kErrTimeout);
+        ok = mbar_wait(bar_w_full + 8 * wp.slot, wp.phase, abort_flag, p.dev_err, kErrTimeout);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
-        const uint8_t* stage = smem + p.smem_w + wslot * kWStageBytes;
+        const uint8_t* stage = smem + p.smem_w + wp.slot * kWStageBytes;
         const uint8_t* crow = stage + row * kWRowBytes;
-        const uint8_t* srow = stage + kWCodeBytes + row * kScaleRowBytes;
+        const uint8_t* srow = stage + kWCodeBytes + row * SB;
         const int ex = emax[r & 3];
         for (int ja = 0; ja < JA; ++ja) {
-          const int aslot = ai % AS;
-          if (ai >= AS) {
-            ok = mbar_wait(bar_a_empty + 8 * aslot, ((ai / AS) & 1) ^ 1, abort_flag, p.dev_err,
+          const int li = (c - c0) * JA + ja;
+          const int aslot = r * spr + li % spr;
+          const int use = li / spr;
+          if (use > 0) {
+            ok = mbar_wait(bar_a_empty + 8 * aslot, (uint32_t)(use - 1) & 1u, abort_flag, p.dev_err,
                            kErrTimeout);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
@@ -546,11 +583,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(bar_a_full + 8 * aslot);
-          ++ai;
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar_w_empty + 8 * wslot);
-        ++wi;
+        if (lane == 0) mbar_arrive(bar_w_empty + 8 * wp.slot);
+        wp.next(WS);
       }
     }
 
@@ -574,23 +610,36 @@ __global__ void __launch_bounds__(kThreads, 1)
       // pass 1: scale the accumulators; store finals (S == 1) or partials (S > 1)
       for (int t2 = 0; t2 < tiles_per_group; ++t2) {
         const int n = (g * tiles_per_group + t2) * kTileRows + row;
-        for (int cb = cb0; cb < cb0 + half_cols; cb += 8) {
-          uint32_t va[8], vb[8];
-          tmem_ld8(tmem + lane_base + (uint32_t)(t2 * p.NMAT * p.NB + cb), va);
-          if (p.NMAT == 2) tmem_ld8(tmem + lane_base + (uint32_t)((t2 * 2 + 1) * p.NB + cb), vb);
+        const float rf_g = rowfac[(t2 * p.NMAT) & 3];
+        const float rf_u = rowfac[(t2 * p.NMAT + 1) & 3];
+        for (int cb = cb0; cb < cb0 + half_cols; cb += 32) {
+          const int nchunk = min(32, cb0 + half_cols - cb) >> 3;  // groups of 8 columns
+          uint32_t va[4][8], vb[4][8];
+#pragma unroll
+          for (int q8 = 0; q8 < 4; ++q8) {
+            if (q8 < nchunk) {
+              tmem_ld8(tmem + lane_base + (uint32_t)(t2 * p.NMAT * p.NB + cb + q8 * 8), va[q8]);
+              if (p.NMAT == 2)
+                tmem_ld8(tmem + lane_base + (uint32_t)((t2 * 2 + 1) * p.NB + cb + q8 * 8), vb[q8]);
+            }
+          }
           tmem_ld_wait();
-          if (n < p.N) {
+          if (n >= p.N) continue;
+#pragma unroll
+          for (int q8 = 0; q8 < 4; ++q8) {
+            if (q8 >= nchunk) break;
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-              const int b = bt * p.NB + cb + i;
+              const int col = cb + q8 * 8 + i;
+              const int b = bt * p.NB + col;
               if (b >= p.B) break;
-              const float cf = col_fac[cb + i];
-              const float ga = __uint_as_float(va[i]) * cf * rowfac[(t2 * p.NMAT) & 3];
+              const float cf = col_fac[col];
+              const float ga = __uint_as_float(va[q8][i]) * cf * rf_g;
               if (p.NMAT == 1) {
                 if (p.S > 1) p.ws[(size_t)s * BN + (size_t)b * p.N + n] = ga;
                 else store_y(p, b, n, ga * ts[0]);
               } else {
-                const float ua = __uint_as_float(vb[i]) * cf * rowfac[(t2 * 2 + 1) & 3];
+                const float ua = __uint_as_float(vb[q8][i]) * cf * rf_u;
                 if (p.S > 1) {
                   p.ws[(size_t)(2 * s) * BN + (size_t)b * p.N + n] = ga;
                   p.ws[(size_t)(2 * s + 1) * BN + (size_t)b * p.N + n] = ua;
@@ -606,41 +655,88 @@ __global__ void __launch_bounds__(kThreads, 1)
     // pass 2 (split K): the last CTA of this tile sums the S partials in order s = 0..S-1.
     // Every epilogue warp reaches both barriers, whatever its own status.
     if (p.S > 1) {
-      {
-        __threadfence();
-        named_bar_epilogue();
-        if (threadIdx.x == 64) {
-          int last = 0;
-          if (!*abort_flag) {
-            int* cnt = p.counters + (g * p.b_tiles + bt);
-            const int old = atomicAdd(cnt, 1);
-            last = (old == p.S - 1);
-            if (last) *cnt = 0;
-          }
-          ctl[2] = last;
+      __threadfence();
+      named_bar_epilogue();
+      if (threadIdx.x == kFirstDequantWarp * 32) {
+        int last = 0;
+        if (!*abort_flag) {
+          int* cnt = p.counters + (g * p.b_tiles + bt);
+          const int old = atomicAdd(cnt, 1);
+          last = (old == p.S - 1);
+          if (last) *cnt = 0;
         }
-        named_bar_epilogue();
-        if (ok && ctl[2]) {
-          __threadfence();
-          for (int t2 = 0; t2 < tiles_per_group; ++t2) {
-            const int n = (g * tiles_per_group + t2) * kTileRows + row;
-            if (n >= p.N) continue;
-            for (int cb = cb0; cb < cb0 + half_cols; ++cb) {
-              const int b = bt * p.NB + cb;
-              if (b >= p.B) break;
-              const size_t off = (size_t)b * p.N + n;
-              if (p.NMAT == 1) {
-                float acc = 0.0f;
-                for (int s2 = 0; s2 < p.S; ++s2) acc += __ldcg(p.ws + (size_t)s2 * BN + off);
-                store_y(p, b, n, acc * ts[0]);
+        ctl[2] = last;
+      }
+      named_bar_epilogue();
+      if (ok && ctl[2]) {
+        __threadfence();
+        // work items: (subtile, column, 4-row quad); 4 items per thread per round so that
+        // 4 * S independent float4 loads are in flight
+        const int ncols = min(p.NB, p.B - bt * p.NB);
+        constexpr int kQuads = kTileRows / 4;
+        const int items = tiles_per_group * ncols * kQuads;
+        const int tid = threadIdx.x - kFirstDequantWarp * 32;
+        const bool vec = (p.N & 3) == 0;
+        for (int it0 = tid; it0 < items; it0 += 4 * kDequantWarps * 32) {
+          int nn[4], bb[4];
+          bool valid[4];
+          float4 ga[4], ua[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int it = it0 + u * kDequantWarps * 32;
+            const int q4 = it % kQuads;
+            const int rest = it / kQuads;
+            const int col = rest % ncols;
+            const int t2 = rest / ncols;
+            nn[u] = (g * tiles_per_group + t2) * kTileRows + q4 * 4;
+            bb[u] = bt * p.NB + col;
+            valid[u] = (it < items) && (nn[u] < p.N);
+            ga[u] = ua[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+          for (int s2 = 0; s2 < p.S; ++s2) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              if (!valid[u]) continue;
+              const float* src = p.ws + (size_t)(s2 * p.NMAT) * BN + (size_t)bb[u] * p.N + nn[u];
+              float4 tg, tu;
+              if (vec) {
+                tg = __ldcg(reinterpret_cast<const float4*>(src));
+                if (p.NMAT == 2) tu = __ldcg(reinterpret_cast<const float4*>(src + BN));
               } else {
-                float ga = 0.0f, ua = 0.0f;
-                for (int s2 = 0; s2 < p.S; ++s2) {
-                  ga += __ldcg(p.ws + (size_t)(2 * s2) * BN + off);
-                  ua += __ldcg(p.ws + (size_t)(2 * s2 + 1) * BN + off);
+                const int lim = p.N - nn[u];
+                tg.x = __ldcg(src);
+                tg.y = lim > 1 ? __ldcg(src + 1) : 0.f;
+                tg.z = lim > 2 ? __ldcg(src + 2) : 0.f;
+                tg.w = lim > 3 ? __ldcg(src + 3) : 0.f;
+                if (p.NMAT == 2) {
+                  tu.x = __ldcg(src + BN);
+                  tu.y = lim > 1 ? __ldcg(src + BN + 1) : 0.f;
+                  tu.z = lim > 2 ? __ldcg(src + BN + 2) : 0.f;
+                  tu.w = lim > 3 ? __ldcg(src + BN + 3) : 0.f;
                 }
-                store_h(p, b, n, ga * ts[0], ua * ts[1]);
               }
+              ga[u].x += tg.x;
+              ga[u].y += tg.y;
+              ga[u].z += tg.z;
+              ga[u].w += tg.w;
+              if (p.NMAT == 2) {
+                ua[u].x += tu.x;
+                ua[u].y += tu.y;
+                ua[u].z += tu.z;
+                ua[u].w += tu.w;
+              }
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            if (!valid[u]) continue;
+            const float g4[4] = {ga[u].x, ga[u].y, ga[u].z, ga[u].w};
+            const float u4[4] = {ua[u].x, ua[u].y, ua[u].z, ua[u].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              if (nn[u] + e >= p.N) break;
+              if (p.NMAT == 1) store_y(p, bb[u], nn[u] + e, g4[e] * ts[0]);
+              else store_h(p, bb[u], nn[u] + e, g4[e] * ts[0], u4[e] * ts[1]);
             }
           }
         }
@@ -689,7 +785,7 @@ static cudaError_t launch_tc_impl(const GemmParams& p, size_t smem_bytes, int gr
     if (e != cudaSuccess) return e;
     configured = smem_bytes;
   }
-  kern<<<grid, kThreads, smem_bytes, stream>>>(p, maps[0], maps[1], maps[2], maps[3], maps[4]);
+  kern<<<grid, kThreads, smem_bytes, stream>>>(p, maps[0]);
   return cudaGetLastError();
 }
 

@@ -61,14 +61,16 @@ __global__ void pack_q8_0_kernel(const float* __restrict__ W, int64_t N, int64_t
   if (dq > 65504.0) dq = 65504.0;
   const uint16_t hb = f16_bits_rne(dq);
   const double d = (double)__half2float(__ushort_as_half(hb));
-  uint8_t* sp = scales + n * scale_pitch(FMT_Q8_0, K) + 2 * kb;
+  const int64_t C = k_chunks(FMT_Q8_0, K);
+  const int64_t k0 = kb * 32, c = k0 / 128;
+  const int b0 = (int)(k0 % 128);
+  uint8_t* sp = scales + scale_offset(FMT_Q8_0, C, n, c) + 2 * (b0 / 32);
   sp[0] = (uint8_t)(hb & 0xFF);
   sp[1] = (uint8_t)(hb >> 8);
-  int8_t* cp = reinterpret_cast<int8_t*>(codes + n * code_pitch(FMT_Q8_0, K) + kb * 32);
   for (int i = 0; i < 32; ++i) {
     double q = 0.0;
     if (d != 0.0) q = fmin(127.0, fmax(-127.0, rint((double)w[i] / d)));
-    cp[i] = (int8_t)q;
+    codes[code_offset(C, n, c, b0 + i)] = (uint8_t)(int8_t)q;
   }
 }
 
@@ -103,8 +105,10 @@ __global__ void pack_nvfp4_kernel(const float* __restrict__ W, int64_t N, int64_
     s = (uint32_t)__nv_cvt_double_to_fp8((double)ab / (6.0 * (double)ts), __NV_SATFINITE, __NV_E4M3);
   const __half_raw sr = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)s, __NV_E4M3);
   const double sv = (double)__half2float(__ushort_as_half(sr.x));
-  scales[n * scale_pitch(FMT_NVFP4, K) + kb] = (uint8_t)s;
-  uint8_t* cp = codes + n * code_pitch(FMT_NVFP4, K) + kb * 8;
+  const int64_t C = k_chunks(FMT_NVFP4, K);
+  const int64_t k0 = kb * 16, c = k0 / 256;
+  const int e0 = (int)(k0 % 256);
+  scales[scale_offset(FMT_NVFP4, C, n, c) + e0 / 16] = (uint8_t)s;
   const double den = sv * (double)ts;
   for (int i = 0; i < 8; ++i) {
     uint32_t lo = 0, hi = 0;
@@ -112,7 +116,7 @@ __global__ void pack_nvfp4_kernel(const float* __restrict__ W, int64_t N, int64_
       lo = e2m1_code((double)w[2 * i] / den);
       hi = e2m1_code((double)w[2 * i + 1] / den);
     }
-    cp[i] = (uint8_t)(lo | (hi << 4));
+    codes[code_offset(C, n, c, e0 / 2 + i)] = (uint8_t)(lo | (hi << 4));
   }
 }
 
@@ -137,26 +141,58 @@ __global__ void pack_mxfp4_kernel(const float* __restrict__ W, int64_t N, int64_
     (void)frexp((double)ab, &ex);  // floor(log2 ab) = ex - 1 exactly
     e = min(254, max(0, (ex - 1) - 2 + 127));
   }
-  scales[n * scale_pitch(FMT_MXFP4, K) + kb] = (uint8_t)e;
+  const int64_t C = k_chunks(FMT_MXFP4, K);
+  const int64_t k0 = kb * 32, c = k0 / 256;
+  const int e0 = (int)(k0 % 256);
+  scales[scale_offset(FMT_MXFP4, C, n, c) + e0 / 32] = (uint8_t)e;
   const double sc = ldexp(1.0, e - 127);
-  uint8_t* cp = codes + n * code_pitch(FMT_MXFP4, K) + kb * 16;
   for (int i = 0; i < 16; ++i) {
     uint32_t lo = 0, hi = 0;
     if (ab != 0.f) {
       lo = e2m1_code((double)w[2 * i] / sc);
       hi = e2m1_code((double)w[2 * i + 1] / sc);
     }
-    cp[i] = (uint8_t)(lo | (hi << 4));
+    codes[code_offset(C, n, c, e0 / 2 + i)] = (uint8_t)(lo | (hi << 4));
   }
+}
+
+// Row-major interchange layout -> tile-major layout.  One thread per (row, chunk); rows and
+// chunks past the matrix are written as zeros.
+__global__ void repack_kernel(const RepackParams p) {
+  const int64_t C = k_chunks(p.fmt, p.K);
+  const int64_t T = row_tiles(p.N);
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= T * kTileRows * C) return;
+  const int64_t n = idx / C, c = idx % C;
+  const int64_t row_bytes = rm_code_bytes_per_row(p.fmt, p.K);
+  const int64_t srow_bytes = rm_scale_bytes_per_row(p.fmt, p.K);
+  const int SBr = scale_row_bytes(p.fmt);
+  for (int b = 0; b < kWRowBytes; ++b) {
+    const int64_t src = c * kWRowBytes + b;
+    const uint8_t v = (n < p.N && src < row_bytes) ? p.codes_rm[n * p.code_pitch + src] : 0;
+    p.codes[code_offset(C, n, c, b)] = v;
+  }
+  for (int b = 0; b < SBr; ++b) {
+    const int64_t src = c * SBr + b;
+    const uint8_t v = (n < p.N && src < srow_bytes) ? p.scales_rm[n * p.scale_pitch + src] : 0;
+    p.scales[scale_offset(p.fmt, C, n, c) + b] = v;
+  }
+}
+
+cudaError_t launch_repack(const RepackParams& rp, cudaStream_t stream) {
+  const int64_t total = row_tiles(rp.N) * kTileRows * k_chunks(rp.fmt, rp.K);
+  const int threads = 256;
+  repack_kernel<<<(unsigned)((total + threads - 1) / threads), threads, 0, stream>>>(rp);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_pack(int fmt, const float* W, int64_t N, int64_t K, void* codes, void* scales,
                         float* tensor_scale, cudaStream_t stream) {
   cudaError_t e = cudaSuccess;
-  // padding bytes of each row are defined (zero)
-  e = cudaMemsetAsync(codes, 0, (size_t)(N * code_pitch(fmt, K)), stream);
+  // padding rows and K past the last block are zero
+  e = cudaMemsetAsync(codes, 0, (size_t)packed_code_bytes(fmt, N, K), stream);
   if (e != cudaSuccess) return e;
-  e = cudaMemsetAsync(scales, 0, (size_t)(N * scale_pitch(fmt, K)), stream);
+  e = cudaMemsetAsync(scales, 0, (size_t)packed_scale_bytes(fmt, N, K), stream);
   if (e != cudaSuccess) return e;
   const int threads = 256;
   if (fmt == FMT_Q8_0) {

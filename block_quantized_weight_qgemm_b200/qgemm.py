@@ -33,7 +33,10 @@ _lock = threading.Lock()
 _I64, _SZ, _VP, _I = ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_int
 SIGNATURES = [
     ("qgemm_packed_size", _I, [_I, _I64, _I64, ctypes.POINTER(_SZ), ctypes.POINTER(_SZ)]),
+    ("qgemm_packed_geometry", _I, [_I, _I64, _I64, ctypes.POINTER(_I64), ctypes.POINTER(_I64),
+                                   ctypes.POINTER(_I), ctypes.POINTER(_I)]),
     ("qgemm_row_pitches", _I, [_I, _I64, ctypes.POINTER(_I64), ctypes.POINTER(_I64)]),
+    ("qgemm_repack_rowmajor", _I, [_I, _I64, _I64, _VP, _I64, _VP, _I64, _VP, _VP, _VP]),
     ("qgemm_pack", _I, [_I, _VP, _I64, _I64, _VP, _VP, _VP, _VP]),
     ("qgemm_workspace_size", _I, [_I, _I64, _I64, _I64, ctypes.POINTER(_SZ)]),
     ("qgemm_run", _I, [_I, _VP, _I64, _I64, _VP, _VP, _VP, _I64, _VP, _I, _VP, _SZ, _VP]),
@@ -103,6 +106,14 @@ def packed_size(fmt, N: int, K: int):
     return cb.value, sb.value
 
 
+def packed_geometry(fmt, N: int, K: int):
+    """(row tiles T, chunks C, elements per chunk CK, scale bytes per row per chunk SB)."""
+    t, c, ck, sb = _I64(), _I64(), _I(), _I()
+    _check(lib().qgemm_packed_geometry(_fmt(fmt), N, K, ctypes.byref(t), ctypes.byref(c),
+                                       ctypes.byref(ck), ctypes.byref(sb)), "qgemm_packed_geometry")
+    return t.value, c.value, ck.value, sb.value
+
+
 def row_pitches(fmt, K: int):
     cp, sp = _I64(), _I64()
     _check(lib().qgemm_row_pitches(_fmt(fmt), K, ctypes.byref(cp), ctypes.byref(sp)),
@@ -148,9 +159,9 @@ class PackedWeight:
         self.fmt = _fmt(fmt)
         self.N, self.K = N, K
         device = device or torch.device("cuda", torch.cuda.current_device())
-        cp, sp = row_pitches(self.fmt, K)
-        self.codes = torch.empty((N, cp), dtype=torch.uint8, device=device)
-        self.scales = torch.empty((N, sp), dtype=torch.uint8, device=device)
+        cb, sb = packed_size(self.fmt, N, K)
+        self.codes = torch.empty(cb, dtype=torch.uint8, device=device)   # tile-major layout
+        self.scales = torch.empty(sb, dtype=torch.uint8, device=device)
         self.tensor_scale = (torch.empty(1, dtype=torch.float32, device=device)
                              if self.fmt == NVFP4 else None)
 
@@ -169,6 +180,17 @@ def pack(fmt, W: torch.Tensor, stream=None, out: PackedWeight | None = None) -> 
     pw = out or PackedWeight(fmt, N, K, W.device)
     _check(lib().qgemm_pack(pw.fmt, _ptr(W), N, K, _ptr(pw.codes), _ptr(pw.scales),
                             _ptr(pw.tensor_scale), None, _stream(stream)), "qgemm_pack")
+    return pw
+
+
+def repack_rowmajor(fmt, codes_rm: torch.Tensor, scales_rm: torch.Tensor, N: int, K: int,
+                    stream=None, out: PackedWeight | None = None) -> PackedWeight:
+    """qgemm_repack_rowmajor: row-major interchange layout [N, pitch] -> PackedWeight."""
+    assert codes_rm.is_cuda and scales_rm.is_cuda and codes_rm.dim() == 2 and scales_rm.dim() == 2
+    pw = out or PackedWeight(fmt, N, K, codes_rm.device)
+    _check(lib().qgemm_repack_rowmajor(pw.fmt, N, K, _ptr(codes_rm), codes_rm.stride(0),
+                                       _ptr(scales_rm), scales_rm.stride(0), _ptr(pw.codes),
+                                       _ptr(pw.scales), _stream(stream)), "qgemm_repack_rowmajor")
     return pw
 
 

@@ -19,14 +19,23 @@
  *   QGEMM_FMT_MXFP4 E2M1 codes; one E8M0 scale per 32 consecutive k (the MXFP4 model
  *                   card's format, OCP MX v1.0):  w = e2m1 * 2^(e-127).
  *
- * Packed layout (row-major, every row starts 16-byte aligned):
- *   codes  [N][code_pitch] bytes.  Q8_0: byte k is int8 q_k, code_pitch = roundup(K,16).
- *          FP4: byte k/2 holds element k, the even element in the low nibble,
- *          code_pitch = roundup(K/2,16).
- *   scales [N][scale_pitch] bytes.  Q8_0: little-endian fp16 per 32-block,
- *          scale_pitch = roundup(K/16,16).  NVFP4: E4M3 byte per 16-block,
- *          scale_pitch = roundup(K/16,16).  MXFP4: E8M0 byte per 32-block,
- *          scale_pitch = roundup(K/32,16).
+ * Packed layout (tile-major; what qgemm_pack writes and qgemm_run reads).  Rows are grouped
+ * in tiles of 128 (T = ceil(N/128)), K in chunks of CK elements (CK = 128 for Q8_0, 256 for
+ * NVFP4 and MXFP4; C = ceil(K/CK)).  Rows past N and elements past K are zero.
+ *   codes  [T][C][128 rows][128 bytes]: the row's CK elements of the chunk (Q8_0: one int8
+ *          byte each; FP4: element 2j in the low nibble of byte j), with the row's 16-byte
+ *          groups permuted: group g of row r is stored at position g ^ (r & 7).
+ *          Size T*C*16384 bytes.
+ *   scales [T][C][128 rows][SB bytes], SB = 8 (Q8_0: 4 little-endian fp16; MXFP4: 8 E8M0)
+ *          or 16 (NVFP4: 16 E4M3), the row's block scales of the chunk in K order.
+ *          Size T*C*128*SB bytes.
+ * Each (tile, chunk) is one contiguous block of codes and one of scales, so the kernel
+ * streams it with two 1-D bulk copies.
+ *
+ * Row-major interchange layout (input of qgemm_repack_rowmajor): codes [N][code pitch]
+ * (Q8_0: K bytes; FP4: K/2 bytes, element 2j in the low nibble of byte j), scales
+ * [N][scale pitch] (Q8_0: K/32 little-endian fp16; NVFP4: K/16 E4M3; MXFP4: K/32 E8M0);
+ * qgemm_row_pitches gives the smallest 16-byte-aligned pitches.
  *
  * Conventions for every entry point:
  *   - Pointers named *_dev are device pointers; the caller owns every buffer and the
@@ -72,13 +81,31 @@ extern "C" {
 #define QGEMM_ERR_DEVICE_TIMEOUT 9 /* a kernel's bounded wait ran out (see device_status) */
 
 /*
- * Sizes of the packed buffers for an N x K weight matrix.  No device work.
+ * Sizes of the tile-major packed buffers for an N x K weight matrix.  No device work.
  * Returns QGEMM_ERR_FORMAT / _SHAPE / _K_BLOCK / _NULL.
  */
 int qgemm_packed_size(int fmt, int64_t N, int64_t K, size_t* code_bytes, size_t* scale_bytes);
 
-/* Row pitches in bytes of the packed codes and scales (see the layout above). */
+/*
+ * Geometry of the tile-major layout: T row tiles, C chunks, CK elements per chunk and SB
+ * scale bytes per row per chunk.  No device work.
+ */
+int qgemm_packed_geometry(int fmt, int64_t N, int64_t K, int64_t* row_tiles, int64_t* k_chunks,
+                          int* chunk_elems, int* scale_bytes_per_row);
+
+/* Smallest 16-byte-aligned row pitches (bytes) of the row-major interchange layout. */
 int qgemm_row_pitches(int fmt, int64_t K, int64_t* code_pitch, int64_t* scale_pitch);
+
+/*
+ * Converts weights packed in the row-major interchange layout (codes_rm_dev with row pitch
+ * code_pitch, scales_rm_dev with row pitch scale_pitch, both in bytes) into the tile-major
+ * layout (codes_dev / scales_dev of qgemm_packed_size() bytes, 16-byte aligned).  A pure byte
+ * permutation; padding is written as zeros.  Asynchronous on `stream`.
+ * QGEMM_ERR_SHAPE if a pitch is smaller than the row's packed bytes.
+ */
+int qgemm_repack_rowmajor(int fmt, int64_t N, int64_t K, const void* codes_rm_dev,
+                          int64_t code_pitch, const void* scales_rm_dev, int64_t scale_pitch,
+                          void* codes_dev, void* scales_dev, void* stream);
 
 /*
  * Quantize W_dev (fp32, row-major [N][K], contiguous) into the packed layout.
@@ -90,7 +117,7 @@ int qgemm_row_pitches(int fmt, int64_t K, int64_t* code_pitch, int64_t* scale_pi
  *   MXFP4: e = clamp(floor(log2 amax) - 2 + 127, 0, 254); code = E2M1_RNE_sat(w/2^(e-127));
  *          an all-zero block gets e = 0 and codes 0.
  * Ties round to even.  A negative element whose magnitude rounds to 0 keeps its sign bit.
- * codes_dev / scales_dev: qgemm_packed_size() bytes each, 16-byte aligned.
+ * codes_dev / scales_dev: qgemm_packed_size() bytes (tile-major layout), 16-byte aligned.
  * tensor_scale_dev: one float (NVFP4 only; must be NULL or ignored otherwise).
  * Not performance critical (uses fp64 for exact tie decisions).
  */

@@ -17,10 +17,34 @@ from block_quantized_weight_qgemm_b200 import qgemm
 TOL = 1e-3  # max |y - y_ref| / (||x_b|| ||w_n||), the acceptance bound of the method
 
 
+def tile_packed(fmt, codes_rm: np.ndarray, scales_rm: np.ndarray, N: int, K: int):
+    """The tile-major layout of include/qgemm.h, built from the row-major packing with numpy
+    (a byte permutation written from the header's description, independent of the library)."""
+    f = oracle.FORMATS[fmt] if isinstance(fmt, str) else fmt
+    CK = 128 if f == oracle.Q8_0 else 256
+    SB = 16 if f == oracle.NVFP4 else 8
+    T, C = -(-N // 128), -(-K // CK)
+    row_code = K if f == oracle.Q8_0 else K // 2
+    row_scale = {oracle.Q8_0: 2 * (K // 32), oracle.NVFP4: K // 16, oracle.MXFP4: K // 32}[f]
+    cfull = np.zeros((T * 128, C * 128), dtype=np.uint8)
+    cfull[:N, :row_code] = codes_rm[:, :row_code]
+    grp = cfull.reshape(T, 128, C, 8, 16).transpose(0, 2, 1, 3, 4)  # [T][C][row][group][16]
+    out = np.empty_like(grp)
+    for r in range(128):
+        perm = [g ^ (r & 7) for g in range(8)]
+        out[:, :, r, perm, :] = grp[:, :, r, :, :]
+    sfull = np.zeros((T * 128, C * SB), dtype=np.uint8)
+    sfull[:N, :row_scale] = scales_rm[:, :row_scale]
+    st = sfull.reshape(T, 128, C, SB).transpose(0, 2, 1, 3)
+    return np.ascontiguousarray(out).reshape(-1), np.ascontiguousarray(st).reshape(-1)
+
+
 def upload_packed(fmt, codes: np.ndarray, scales: np.ndarray, ts: float, N: int, K: int):
+    """Oracle row-major packing -> tile-major device buffers (numpy permutation + copy)."""
     pw = qgemm.PackedWeight(fmt, N, K)
-    pw.codes.copy_(torch.from_numpy(codes))
-    pw.scales.copy_(torch.from_numpy(scales))
+    ct, st = tile_packed(fmt, codes, scales, N, K)
+    pw.codes.copy_(torch.from_numpy(ct))
+    pw.scales.copy_(torch.from_numpy(st))
     if pw.tensor_scale is not None:
         pw.tensor_scale.fill_(ts)
     return pw

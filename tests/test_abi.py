@@ -51,8 +51,13 @@ def test_pitches_match_layout_spec(lib, fmt, K):
         pytest.skip("K must be a multiple of 32")
     cp, sp = qgemm.row_pitches(fmt, K)
     assert (cp, sp) == (oracle.code_pitch(fmt, K), oracle.scale_pitch(fmt, K))
-    cb, sb = qgemm.packed_size(fmt, 7, K)
-    assert (cb, sb) == (7 * cp, 7 * sp)
+    T, C, CK, SB = qgemm.packed_geometry(fmt, 300, K)
+    assert T == 3 and CK == (128 if fmt == "q8_0" else 256) and C == -(-K // CK)
+    assert SB == (16 if fmt == "nvfp4" else 8)
+    cb, sb = qgemm.packed_size(fmt, 300, K)
+    assert (cb, sb) == (T * C * 128 * 128, T * C * 128 * SB)
+    # the tiled layout holds every byte of the row-major packing (plus zero padding)
+    assert cb >= 300 * (K if fmt == "q8_0" else K // 2)
 
 
 def test_argument_errors(lib):

@@ -12,7 +12,7 @@ import oracle
 from block_quantized_weight_qgemm_b200 import inputs
 from block_quantized_weight_qgemm_b200 import qgemm
 
-from gpu_helpers import TOL, Case, gpu_run, norm_err, round_bf16, round_f16, x_bits
+from gpu_helpers import TOL, Case, gpu_run, norm_err, round_bf16, round_f16, tile_packed, x_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -46,7 +46,8 @@ def _specials(N, K, seed):
 @pytest.mark.parametrize("N,K", [(300, 512), (512, 1024), (129, 2048)])
 def test_pack_byte_exact(fmt, N, K):
     W = _specials(N, K, 40 + N)
-    codes, scales, ts = oracle.pack(fmt, W)
+    codes_rm, scales_rm, ts = oracle.pack(fmt, W)
+    codes, scales = tile_packed(fmt, codes_rm, scales_rm, N, K)
     pw = qgemm.pack(fmt, torch.from_numpy(W).cuda())
     torch.cuda.synchronize()
     gc, gs = pw.codes.cpu().numpy(), pw.scales.cpu().numpy()
@@ -57,6 +58,21 @@ def test_pack_byte_exact(fmt, N, K):
     assert mism.size == 0, "scales differ at %s" % mism[:5].tolist()
     if fmt == "nvfp4":
         assert pw.tensor_scale.item() == ts
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("N,K", [(300, 512), (129, 1056)])
+def test_repack_rowmajor_matches_layout(fmt, N, K):
+    if fmt != "nvfp4" and K % 32:
+        pytest.skip("K must be a multiple of 32")
+    W = _specials(N, K, 60 + N)
+    codes_rm, scales_rm, ts = oracle.pack(fmt, W)
+    ct, st = tile_packed(fmt, codes_rm, scales_rm, N, K)
+    pw = qgemm.repack_rowmajor(fmt, torch.from_numpy(codes_rm).cuda(),
+                               torch.from_numpy(scales_rm).cuda(), N, K)
+    torch.cuda.synchronize()
+    assert np.array_equal(pw.codes.cpu().numpy(), ct)
+    assert np.array_equal(pw.scales.cpu().numpy(), st)
 
 
 # --------------------------------------------------------------------------------------
@@ -196,3 +212,37 @@ def test_errors_on_device(small_cases):
                        ws.data_ptr(), need, None)
     assert st == 5
     torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("B", [3, 300])
+def test_run_ragged_k(fmt, B):
+    # K = 1056: the last weight chunk is partial (8.25 Q8_0 chunks, 4.125 FP4 chunks); N = 200
+    case = Case(fmt, 200, 1056, seed=13)
+    x = inputs.activations(B, 1056, seed=14)
+    xb = x_bits(x)
+    y_ref = oracle.gemm(xb, case.Wd)
+    err = norm_err(gpu_run(case, x), y_ref, xb, case.Wd)
+    assert err <= TOL, err
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_subtile_count_does_not_change_results(fmt, monkeypatch):
+    # R (weight subtiles sharing each x tile, one MMA issuer each) is a scheduling choice:
+    # every R gives bit-identical results.  R = 4 with FP4 (two A stages per chunk) is the
+    # case where issuers must not share A slots.
+    case = Case(fmt, 1100, 1024, seed=15)
+    x = inputs.activations(64, 1024, seed=16)
+    xb = x_bits(x)
+    y_ref = oracle.gemm(xb, case.Wd)
+    outs = {}
+    for R in ("1", "2", "4"):
+        monkeypatch.setenv("QGEMM_DEBUG_R", R)
+        for B in (8, 64):
+            outs[(R, B)] = gpu_run(case, x[:B])
+    monkeypatch.delenv("QGEMM_DEBUG_R")
+    for B in (8, 64):
+        assert norm_err(outs[("1", B)], y_ref[:B], xb[:B], case.Wd) <= TOL
+        assert np.array_equal(outs[("1", B)], outs[("2", B)]), B
+        assert np.array_equal(outs[("1", B)], outs[("4", B)]), B
+    assert qgemm.device_status(reset=False) == qgemm.OK
