@@ -19,6 +19,7 @@ cudaError_t launch_tc(int fmt, bool bf16op, const GemmParams& p, size_t smem_byt
 cudaError_t launch_pack(int fmt, const float* W, int64_t N, int64_t K, void* codes, void* scales,
                         float* tensor_scale, cudaStream_t stream);
 cudaError_t launch_repack(const RepackParams& rp, cudaStream_t stream);
+cudaError_t launch_reduce(const ReduceParams& rp, cudaStream_t stream);
 int* device_error_word();
 }  // namespace qg
 
@@ -209,8 +210,7 @@ bool make_plan(int fmt, int64_t N, int64_t K, int64_t B, int nmat, Plan* pl) {
   };
   p.off_xh = p.f16ops ? take((size_t)B * K * 2) : 0;
   p.off_exp = p.f16ops ? take((size_t)B * 4) : 0;
-  const size_t ncnt = (size_t)p.n_groups * p.b_tiles;
-  p.off_cnt = (p.S > 1) ? take(ncnt * 4) : 0;
+  p.off_cnt = 0;
   p.off_ws = (p.S > 1) ? take((size_t)p.S * nmat * B * N * 4) : 0;
   p.ws_total = off;
   *pl = p;
@@ -254,7 +254,7 @@ int run_impl(int fmt, const void* x, int64_t B, int64_t K, const void* const* co
   }
   p.x_exp = pl.f16ops ? reinterpret_cast<const int*>(wsb + pl.off_exp) : nullptr;
   p.ws = (pl.S > 1) ? reinterpret_cast<float*>(wsb + pl.off_ws) : nullptr;
-  p.counters = (pl.S > 1) ? reinterpret_cast<int*>(wsb + pl.off_cnt) : nullptr;
+  p.counters = nullptr;
   p.out = out;
   p.out_bf16 = out_bf16;
   p.dev_err = dev_err;
@@ -267,8 +267,8 @@ int run_impl(int fmt, const void* x, int64_t B, int64_t K, const void* const* co
     pp.x_exp = reinterpret_cast<int*>(wsb + pl.off_exp);
     pp.B = (int)B;
     pp.K = (int)K;
-    pp.counters = p.counters;
-    pp.n_counters = (pl.S > 1) ? pl.n_groups * pl.b_tiles : 0;
+    pp.counters = nullptr;
+    pp.n_counters = 0;
     cudaError_t e = launch_prep(pp, stream);
     if (e != cudaSuccess) return cuda_fail(e, "prep kernel launch");
     xop = pp.xh;
@@ -287,6 +287,20 @@ int run_impl(int fmt, const void* x, int64_t B, int64_t K, const void* const* co
   cudaError_t e = launch_tc(fmt, !pl.f16ops, p, pl.smem_bytes, grid, &xmap, stream);
   if (e != cudaSuccess) return cuda_fail(e, "gemm kernel launch");
   if (g_prof_end) cudaEventRecord(g_prof_end, stream);
+  if (pl.S > 1) {
+    ReduceParams rp{};
+    rp.ws = p.ws;
+    rp.S = pl.S;
+    rp.NMAT = nmat;
+    rp.B = (int)B;
+    rp.N = (int)N;
+    rp.ts[0] = p.ts[0];
+    rp.ts[1] = (nmat == 2) ? p.ts[1] : nullptr;
+    rp.out = out;
+    rp.out_bf16 = out_bf16;
+    e = launch_reduce(rp, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "split-K reduce launch");
+  }
   return QGEMM_OK;
 }
 

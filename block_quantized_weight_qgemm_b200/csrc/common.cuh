@@ -92,6 +92,15 @@ struct GemmParams {
   int* dev_err;
 };
 
+// Fixed-order sum of the split-K partials and the output epilogue.
+struct ReduceParams {
+  const float* ws;     // partials [S][NMAT][B][N]
+  int S, NMAT, B, N;
+  const float* ts[2];  // NVFP4 tensor scales, else nullptr
+  void* out;           // y [B][N] fp32 / bf16, or h [B][N] bf16 for NMAT == 2
+  int out_bf16;
+};
+
 // Conversion of the row-major packed layout into the tile-major one.
 struct RepackParams {
   const uint8_t* codes_rm;

@@ -652,96 +652,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    // pass 2 (split K): the last CTA of this tile sums the S partials in order s = 0..S-1.
-    // Every epilogue warp reaches both barriers, whatever its own status.
-    if (p.S > 1) {
-      __threadfence();
-      named_bar_epilogue();
-      if (threadIdx.x == kFirstDequantWarp * 32) {
-        int last = 0;
-        if (!*abort_flag) {
-          int* cnt = p.counters + (g * p.b_tiles + bt);
-          const int old = atomicAdd(cnt, 1);
-          last = (old == p.S - 1);
-          if (last) *cnt = 0;
-        }
-        ctl[2] = last;
-      }
-      named_bar_epilogue();
-      if (ok && ctl[2]) {
-        __threadfence();
-        // work items: (subtile, column, 4-row quad); 4 items per thread per round so that
-        // 4 * S independent float4 loads are in flight
-        const int ncols = min(p.NB, p.B - bt * p.NB);
-        constexpr int kQuads = kTileRows / 4;
-        const int items = tiles_per_group * ncols * kQuads;
-        const int tid = threadIdx.x - kFirstDequantWarp * 32;
-        const bool vec = (p.N & 3) == 0;
-        for (int it0 = tid; it0 < items; it0 += 4 * kDequantWarps * 32) {
-          int nn[4], bb[4];
-          bool valid[4];
-          float4 ga[4], ua[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int it = it0 + u * kDequantWarps * 32;
-            const int q4 = it % kQuads;
-            const int rest = it / kQuads;
-            const int col = rest % ncols;
-            const int t2 = rest / ncols;
-            nn[u] = (g * tiles_per_group + t2) * kTileRows + q4 * 4;
-            bb[u] = bt * p.NB + col;
-            valid[u] = (it < items) && (nn[u] < p.N);
-            ga[u] = ua[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-          }
-          for (int s2 = 0; s2 < p.S; ++s2) {
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              if (!valid[u]) continue;
-              const float* src = p.ws + (size_t)(s2 * p.NMAT) * BN + (size_t)bb[u] * p.N + nn[u];
-              float4 tg, tu;
-              if (vec) {
-                tg = __ldcg(reinterpret_cast<const float4*>(src));
-                if (p.NMAT == 2) tu = __ldcg(reinterpret_cast<const float4*>(src + BN));
-              } else {
-                const int lim = p.N - nn[u];
-                tg.x = __ldcg(src);
-                tg.y = lim > 1 ? __ldcg(src + 1) : 0.f;
-                tg.z = lim > 2 ? __ldcg(src + 2) : 0.f;
-                tg.w = lim > 3 ? __ldcg(src + 3) : 0.f;
-                if (p.NMAT == 2) {
-                  tu.x = __ldcg(src + BN);
-                  tu.y = lim > 1 ? __ldcg(src + BN + 1) : 0.f;
-                  tu.z = lim > 2 ? __ldcg(src + BN + 2) : 0.f;
-                  tu.w = lim > 3 ? __ldcg(src + BN + 3) : 0.f;
-                }
-              }
-              ga[u].x += tg.x;
-              ga[u].y += tg.y;
-              ga[u].z += tg.z;
-              ga[u].w += tg.w;
-              if (p.NMAT == 2) {
-                ua[u].x += tu.x;
-                ua[u].y += tu.y;
-                ua[u].z += tu.z;
-                ua[u].w += tu.w;
-              }
-            }
-          }
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            if (!valid[u]) continue;
-            const float g4[4] = {ga[u].x, ga[u].y, ga[u].z, ga[u].w};
-            const float u4[4] = {ua[u].x, ua[u].y, ua[u].z, ua[u].w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              if (nn[u] + e >= p.N) break;
-              if (p.NMAT == 1) store_y(p, bb[u], nn[u] + e, g4[e] * ts[0]);
-              else store_h(p, bb[u], nn[u] + e, g4[e] * ts[0], u4[e] * ts[1]);
-            }
-          }
-        }
-      }
-    }
   }
 
   // ------------------------------------------------------------ teardown
@@ -761,12 +671,66 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------------------
+// Split-K reduction: out = epilogue(sum_{s=0..S-1} partial_s), in that fixed order, one
+// 4-wide column group (b, n..n+3) per thread.
+// ---------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) qgemm_splitk_reduce_kernel(const ReduceParams p) {
+  const int64_t nq = (p.N + 3) / 4;
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (int64_t)p.B * nq) return;
+  const int b = (int)(idx / nq);
+  const int n = (int)(idx % nq) * 4;
+  const size_t BN = (size_t)p.B * p.N;
+  const size_t off = (size_t)b * p.N + n;
+  const int lim = min(4, p.N - n);
+  const bool vec = ((p.N & 3) == 0);
+  float g[4] = {0.f, 0.f, 0.f, 0.f}, u[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int s = 0; s < p.S; ++s) {
+    const float* src = p.ws + (size_t)(s * p.NMAT) * BN + off;
+    if (vec) {
+      const float4 t = __ldcs(reinterpret_cast<const float4*>(src));
+      g[0] += t.x; g[1] += t.y; g[2] += t.z; g[3] += t.w;
+      if (p.NMAT == 2) {
+        const float4 v = __ldcs(reinterpret_cast<const float4*>(src + BN));
+        u[0] += v.x; u[1] += v.y; u[2] += v.z; u[3] += v.w;
+      }
+    } else {
+      for (int e = 0; e < lim; ++e) {
+        g[e] += __ldcs(src + e);
+        if (p.NMAT == 2) u[e] += __ldcs(src + BN + e);
+      }
+    }
+  }
+  const float ts0 = p.ts[0] ? __ldg(p.ts[0]) : 1.0f;
+  const float ts1 = (p.NMAT == 2 && p.ts[1]) ? __ldg(p.ts[1]) : 1.0f;
+  for (int e = 0; e < lim; ++e) {
+    if (p.NMAT == 1) {
+      const float v = g[e] * ts0;
+      if (p.out_bf16)
+        reinterpret_cast<__nv_bfloat16*>(p.out)[off + e] = __float2bfloat16_rn(v);
+      else
+        reinterpret_cast<float*>(p.out)[off + e] = v;
+    } else {
+      const float gv = g[e] * ts0, uv = u[e] * ts1;
+      reinterpret_cast<__nv_bfloat16*>(p.out)[off + e] =
+          __float2bfloat16_rn(gv / (1.0f + expf(-gv)) * uv);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------------
 // Host-side launchers (called by the C-ABI layer)
 // ---------------------------------------------------------------------------------------
 int* device_error_word() {
   void* ptr = nullptr;
   if (cudaGetSymbolAddress(&ptr, g_dev_err) != cudaSuccess) return nullptr;
   return static_cast<int*>(ptr);
+}
+
+cudaError_t launch_reduce(const ReduceParams& rp, cudaStream_t stream) {
+  const int64_t total = (int64_t)rp.B * ((rp.N + 3) / 4);
+  qgemm_splitk_reduce_kernel<<<(unsigned)((total + 255) / 256), 256, 0, stream>>>(rp);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_prep(const PrepParams& pp, cudaStream_t stream) {
