@@ -187,13 +187,13 @@ bool make_plan(int fmt, int64_t N, int64_t K, int64_t B, int nmat, Plan* pl) {
   if (p.tmem_cols > 512) return false;
   // shared memory: x ring, weight ring (gets the rest, up to 8 stages), barriers, control
   const size_t xstage = (size_t)p.NB * 128;
-  const size_t misc = 8 * (2 * 16 + 2 * 8 + 2 * kMaxAStages + 1) + 16 + 4 * kMaxNB + 64;
+  const size_t misc = 8 * (2 * 16 + 2 * kMaxWStages + 2 * kMaxAStages + 1) + 16 + 4 * kMaxNB + 64;
   const size_t budget = kSmemLimit - 1024 - misc;
   // with several subtiles the x stages of a chunk stay resident until its last subtile
   int XS = (p.R > 1) ? 2 * J : 4;
   while (XS > J && XS * xstage + 2 * (size_t)kWStageBytes > budget) --XS;
   if (XS * xstage + 2 * (size_t)kWStageBytes > budget) return false;
-  const int WS = (int)std::min<size_t>(8, (budget - XS * xstage) / kWStageBytes);
+  const int WS = (int)std::min<size_t>(kMaxWStages, (budget - XS * xstage) / kWStageBytes);
   p.XS = XS;
   p.WS = WS;
   p.smem_x = 0;

@@ -16,6 +16,7 @@ constexpr int kWStageBytes = kWCodeBytes + kTileRows * kScaleRowBytes;  // 18 KB
 constexpr int kSubK = 64;                         // K per x stage (one 128-byte swizzle atom)
 constexpr int kAStageK = 128;                     // K per A stage (TMEM)
 constexpr int kMaxAStages = 4;                    // A ring depth limit
+constexpr int kMaxWStages = 8;                    // weight ring depth limit
 constexpr int kAColsPerStage = kAStageK / 2;      // 16-bit elements, 2 per TMEM column
 constexpr int kDequantWarps = 8;                  // 2 per TMEM lane quarter
 constexpr int kMmaWarps = 4;                      // one MMA-issuing thread per weight subtile
