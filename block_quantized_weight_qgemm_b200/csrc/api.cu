@@ -25,6 +25,11 @@ int* device_error_word();
 
 using namespace qg;
 
+// Scratch of qgemm_run_noalloc: a device global sized QGEMM_NOALLOC_SCRATCH_BYTES, reserved on
+// every GPU that loads this library for as long as the process lives.  Host code never reads
+// this name as an address: it asks the runtime for the device address of the current GPU's copy.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[QGEMM_NOALLOC_SCRATCH_BYTES];
+
 namespace {
 
 thread_local char g_last_cuda_error[256] = "";
@@ -304,6 +309,29 @@ int run_impl(int fmt, const void* x, int64_t B, int64_t K, const void* const* co
   return QGEMM_OK;
 }
 
+// Device address of g_noalloc_scratch on the current device, looked up once per device (the
+// lookup may load this library's device code on that device, so it must not happen inside a
+// stream capture).
+constexpr int kMaxNoAllocDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxNoAllocDevices] = {};
+
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxNoAllocDevices) return QGEMM_ERR_DEVICE;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return QGEMM_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -423,6 +451,31 @@ int qgemm_run(int fmt, const void* x, int64_t B, int64_t K, const void* codes, c
   const float* tss[1] = {tensor_scale};
   return run_impl(fmt, x, B, K, cs, ss, tss, 1, N, y, y_dtype == QGEMM_Y_BF16, workspace,
                   workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int qgemm_run_noalloc(int fmt, const void* x, int64_t B, int64_t K, const void* codes,
+                      const void* scales, const float* tensor_scale, int64_t N, void* y,
+                      int y_dtype, void* stream) {
+  int st = check_fmt_shape(fmt, N, K);
+  if (st != QGEMM_OK) return st;
+  if (B < 1 || B > 0x7FFFFFFF) return QGEMM_ERR_SHAPE;
+  if (y_dtype != QGEMM_Y_F32 && y_dtype != QGEMM_Y_BF16) return QGEMM_ERR_FORMAT;
+  if (!x || !codes || !scales || !y || (fmt == FMT_NVFP4 && !tensor_scale)) return QGEMM_ERR_NULL;
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || !aligned16(y))
+    return QGEMM_ERR_ALIGN;
+  // the same plan qgemm_run would use; its workspace must fit the fixed scratch
+  Plan pl;
+  if (!make_plan(fmt, N, K, B, 1, &pl)) return QGEMM_ERR_SHAPE;
+  if (pl.ws_total > (size_t)QGEMM_NOALLOC_SCRATCH_BYTES) return QGEMM_ERR_WORKSPACE;
+  if (!device_ok()) return QGEMM_ERR_DEVICE;
+  void* scratch = nullptr;
+  st = noalloc_scratch(&scratch);
+  if (st != QGEMM_OK) return st;
+  const void* cs[1] = {codes};
+  const void* ss[1] = {scales};
+  const float* tss[1] = {tensor_scale};
+  return run_impl(fmt, x, B, K, cs, ss, tss, 1, N, y, y_dtype == QGEMM_Y_BF16, scratch,
+                  (size_t)QGEMM_NOALLOC_SCRATCH_BYTES, static_cast<cudaStream_t>(stream));
 }
 
 int qgemm_ffn_gate_up(int fmt, const void* x, int64_t M, int64_t K, const void* g_codes,

@@ -40,6 +40,7 @@ SIGNATURES = [
     ("qgemm_pack", _I, [_I, _VP, _I64, _I64, _VP, _VP, _VP, _VP]),
     ("qgemm_workspace_size", _I, [_I, _I64, _I64, _I64, ctypes.POINTER(_SZ)]),
     ("qgemm_run", _I, [_I, _VP, _I64, _I64, _VP, _VP, _VP, _I64, _VP, _I, _VP, _SZ, _VP]),
+    ("qgemm_run_noalloc", _I, [_I, _VP, _I64, _I64, _VP, _VP, _VP, _I64, _VP, _I, _VP]),
     ("qgemm_ffn_workspace_size", _I, [_I, _I64, _I64, _I64, ctypes.POINTER(_SZ)]),
     ("qgemm_ffn_gate_up", _I, [_I, _VP, _I64, _I64, _VP, _VP, _VP, _VP, _VP, _VP, _I64, _VP, _VP,
                                _SZ, _VP]),

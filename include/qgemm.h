@@ -144,6 +144,38 @@ int qgemm_run(int fmt, const void* x_dev, int64_t B, int64_t K, const void* code
               const void* scales_dev, const float* tensor_scale_dev, int64_t N, void* y_dev,
               int y_dtype, void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * Size in bytes of the fixed device scratch that qgemm_run_noalloc uses in place of a
+ * caller-supplied workspace (32 MiB, reserved on every GPU that loads the library).
+ */
+#define QGEMM_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/*
+ * qgemm_run without a workspace argument, for callers that cannot allocate device memory:
+ * a serving runtime whose memory pool has reserved the GPU's memory up front and forbids
+ * allocations outside it, a plugin to which the host framework hands nothing but its input
+ * and output buffers, or a latency-critical path where an allocation's cost, its implicit
+ * synchronisation or its possible failure cannot be afforded.  The paper has no counterpart;
+ * this is a deployment convenience, not part of the method.
+ *   Arguments, layouts, results and accuracy: as for qgemm_run (the same kernels run, with
+ *   the same K split, so y matches qgemm_run's y for the same inputs).
+ *   Scratch: a device global of QGEMM_NOALLOC_SCRATCH_BYTES inside the library, one per GPU.
+ *   The call allocates nothing (no cudaMalloc, no library allocator).  A shape whose
+ *   qgemm_workspace_size() exceeds QGEMM_NOALLOC_SCRATCH_BYTES is rejected with
+ *   QGEMM_ERR_WORKSPACE before any device work; use qgemm_run for it.
+ *   Set-up: the first call on each device looks up that device's scratch address (which
+ *   may load the library's device code there); make that first call outside any stream
+ *   capture, with the device current.
+ *   Sharing: every call on a device uses the same scratch, which keeps whatever the last
+ *   call left in it.  Nothing needs to start at zero (each call writes every scratch byte
+ *   before it reads it), but calls that may overlap on the GPU -- on different streams, or
+ *   from several host threads without ordering -- race on the scratch and give wrong
+ *   results.  Calls ordered on one stream are safe.
+ */
+int qgemm_run_noalloc(int fmt, const void* x_dev, int64_t B, int64_t K, const void* codes_dev,
+                      const void* scales_dev, const float* tensor_scale_dev, int64_t N,
+                      void* y_dev, int y_dtype, void* stream);
+
 /* Bytes of device workspace qgemm_ffn_gate_up needs for (fmt, N, K, M). */
 int qgemm_ffn_workspace_size(int fmt, int64_t N, int64_t K, int64_t M, size_t* bytes);
 
