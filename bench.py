@@ -182,6 +182,15 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def launches_per_call(fmt, N, K, B):
+    """Kernels one qgemm_run launches: the x conversion (widths <= 256), the GEMM, and the
+    split-K reduction when the K split is above 1."""
+    from block_quantized_weight_qgemm_b200 import qgemm
+    if B > 256:
+        return 1
+    return 2 + (1 if qgemm.split_k(fmt, N, K) > 1 else 0)
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
@@ -335,7 +344,7 @@ def main():
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": 2 * len(calls) * args.steps,
+        "gpu_launches": sum(launches_per_call(fmt, c["N"], c["K"], B) for c in calls) * args.steps,
         "clocks": clk,
         "device_status": status,
     }
