@@ -16,6 +16,8 @@ namespace qg {
 cudaError_t launch_prep(const PrepParams& pp, cudaStream_t stream);
 cudaError_t launch_tc(int fmt, bool bf16op, const GemmParams& p, size_t smem_bytes, int grid,
                       const CUtensorMap* maps, cudaStream_t stream);
+cudaError_t launch_pair(int fmt, bool bf16op, const GemmParams& p, size_t smem_bytes, int units,
+                        const CUtensorMap* maps, cudaStream_t stream);
 cudaError_t launch_pack(int fmt, const float* W, int64_t N, int64_t K, void* codes, void* scales,
                         float* tensor_scale, cudaStream_t stream);
 cudaError_t launch_repack(const RepackParams& rp, cudaStream_t stream);
@@ -78,6 +80,24 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int esize, const void* bas
   return r == CUDA_SUCCESS;
 }
 
+// 3-D map {64, rows, slices} over a row-major [rows][pitch] array of 16-bit elements whose
+// rows are read in slices of 64: box {64, box_rows, box_slices}.
+bool make_map3(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t rows,
+               uint64_t pitch_elems, uint32_t box_rows, uint32_t box_slices) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {64, rows, pitch_elems / 64};
+  const cuuint64_t strides[2] = {pitch_elems * 2, 128};
+  const cuuint32_t box[3] = {64, box_rows, box_slices};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int64_t pad64(int64_t k) { return (k + 63) / 64 * 64; }
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int check_fmt_shape(int fmt, int64_t N, int64_t K) {
@@ -129,7 +149,39 @@ int split_for(int fmt, int64_t N, int64_t K, int nmat) {
   return best;
 }
 
+// The K split of the CTA-pair kernel for widths 1..256: a function of (fmt, N, K) only.  A
+// work unit is one pair of 128-row tiles over K/S; kPairSMs units run at once.  The cost
+// model is (waves of units) x (chunks per unit) plus a small charge per split for the
+// partials the reduction reads; the smallest S of least cost wins.
+int split_for_pair(int fmt, int64_t N, int64_t K) {
+  const int64_t chunks = (K + chunk_k(fmt) - 1) / chunk_k(fmt);
+  const int64_t pairs = (row_tiles(N) + 1) / 2;
+  int best = 1;
+  double best_cost = 0.0;
+  const int64_t smax = std::min<int64_t>(16, chunks);
+  for (int64_t S = 1; S <= smax; ++S) {
+    const int64_t waves = (pairs * S + kPairSMs - 1) / kPairSMs;
+    const int64_t cmax = (chunks + S - 1) / S;
+    const double cost = double(waves * cmax) + 0.3 * double(S);
+    if (S == 1 || cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best = (int)S;
+    }
+  }
+  return best;
+}
+
+bool use_one_sm() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("QGEMM_DEBUG_ONESM");
+    v = (e && e[0] == '1') ? 1 : 0;
+  }
+  return v == 1;
+}
+
 struct Plan {
+  bool pair;    // CTA-pair kernel
   bool f16ops;  // widths <= 256
   int NB, R, NMAT, S, n_groups, b_tiles, chunks, XS, WS, AS, tmem_cols;
   size_t smem_bytes;
@@ -144,9 +196,77 @@ int next_pow2_cols(int c) {
   return p;
 }
 
+// Tiling of the CTA-pair kernel.  Only S (and the operand type, by width class) affects the
+// arithmetic; NB, R and the ring depths are scheduling choices.
+bool make_plan_pair(int fmt, int64_t N, int64_t K, int64_t B, int nmat, Plan* pl) {
+  Plan p{};
+  p.pair = true;
+  p.NMAT = nmat;
+  p.f16ops = (B <= 256);
+  p.chunks = (int)((K + chunk_k(fmt) - 1) / chunk_k(fmt));
+  const int J = chunk_k(fmt) / kSubK;
+  const int64_t pairs = (row_tiles(N) + 1) / 2;
+  if (p.f16ops) {
+    p.S = split_for_pair(fmt, N, K);
+    const int nb_cap = (nmat == 2) ? 128 : 256;
+    int nb = (int)std::min<int64_t>(((B + 15) / 16) * 16, nb_cap);
+    if (nmat == 2 && B > 128) nb = (int)(((B + 1) / 2 + 15) / 16 * 16);
+    p.NB = nb;
+  } else {
+    p.S = 1;
+    p.NB = (nmat == 2) ? 128 : 256;
+  }
+  p.b_tiles = (int)((B + p.NB - 1) / p.NB);
+  // tile pairs per unit: 1, or 2 to share each x stage between two pairs when x is wide
+  int m = 1;
+  if (p.NB >= 64 && 2 * nmat * p.NB + 2 * kPairACols <= 512) {
+    const int64_t w1 = (pairs * p.b_tiles * p.S + kPairSMs - 1) / kPairSMs;
+    const int64_t w2 = (((pairs + 1) / 2) * p.b_tiles * p.S + kPairSMs - 1) / kPairSMs;
+    if (2 * w2 <= w1 + (p.NB >= 128 ? 1 : 0)) m = 2;
+  }
+  if (const char* e = getenv("QGEMM_DEBUG_R")) {
+    const int r = atoi(e);
+    if ((r == 1 || r == 2) && r * nmat * p.NB + 2 * kPairACols <= 512) m = r;
+  }
+  p.R = m * nmat;
+  p.n_groups = (int)((pairs + m - 1) / m);
+  p.AS = std::min(4, (512 - p.R * p.NB) / kPairACols);
+  if (p.AS < 2) return false;
+  p.tmem_cols = next_pow2_cols(p.R * p.NB + p.AS * kPairACols);
+  if (p.tmem_cols > 512) return false;
+  // x ring: one stage per A slot (kPairAK / 64 slices of this CTA's NB/2 rows)
+  const size_t xstage = (size_t)(p.NB / 2) * 128 * (kPairAK / kSubK);
+  const size_t misc = 8 * (2 * 4 + 2 * kMaxWStages + 2 * 8 + 1) + 16 + 4 * kMaxNB + 64;
+  const size_t budget = kSmemLimit - 1024 - misc;
+  int XS = 4;
+  while (XS > 2 && XS * xstage + 4 * (size_t)kWStageBytes > budget) --XS;
+  if (XS * xstage + 2 * (size_t)kWStageBytes > budget) return false;
+  const int WS = (int)std::min<size_t>(kMaxWStages, (budget - XS * xstage) / kWStageBytes);
+  p.XS = XS;
+  p.WS = WS;
+  p.smem_x = 0;
+  p.smem_w = (uint32_t)(XS * xstage);
+  p.smem_bar = p.smem_w + (uint32_t)(WS * kWStageBytes);
+  const size_t bar_bytes = 8 * (2 * XS + 2 * WS + 2 * p.AS + 1);
+  p.smem_bytes = 1024 + p.smem_bar + bar_bytes + 16 + 4 * p.NB + 64;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += (bytes + 255) / 256 * 256;
+    return o;
+  };
+  p.off_xh = p.f16ops ? take((size_t)B * pad64(K) * 2) : 0;
+  p.off_exp = p.f16ops ? take((size_t)B * 4) : 0;
+  p.off_cnt = 0;
+  p.off_ws = (p.S > 1) ? take((size_t)p.S * nmat * B * N * 4) : 0;
+  p.ws_total = off;
+  *pl = p;
+  return true;
+}
+
 // Chooses the tiling for one call.  Only S (and the operand type, by width class) affects
 // the arithmetic; NB, R and the ring depths are scheduling choices.
-bool make_plan(int fmt, int64_t N, int64_t K, int64_t B, int nmat, Plan* pl) {
+bool make_plan_one_sm(int fmt, int64_t N, int64_t K, int64_t B, int nmat, Plan* pl) {
   Plan p{};
   p.NMAT = nmat;
   p.f16ops = (B <= 256);
@@ -213,13 +333,18 @@ bool make_plan(int fmt, int64_t N, int64_t K, int64_t B, int nmat, Plan* pl) {
     off += (bytes + 255) / 256 * 256;
     return o;
   };
-  p.off_xh = p.f16ops ? take((size_t)B * K * 2) : 0;
+  p.off_xh = p.f16ops ? take((size_t)B * pad64(K) * 2) : 0;
   p.off_exp = p.f16ops ? take((size_t)B * 4) : 0;
   p.off_cnt = 0;
   p.off_ws = (p.S > 1) ? take((size_t)p.S * nmat * B * N * 4) : 0;
   p.ws_total = off;
   *pl = p;
   return true;
+}
+
+bool make_plan(int fmt, int64_t N, int64_t K, int64_t B, int nmat, Plan* pl) {
+  return use_one_sm() ? make_plan_one_sm(fmt, N, K, B, nmat, pl)
+                      : make_plan_pair(fmt, N, K, B, nmat, pl);
 }
 
 int run_impl(int fmt, const void* x, int64_t B, int64_t K, const void* const* codes,
@@ -272,6 +397,7 @@ int run_impl(int fmt, const void* x, int64_t B, int64_t K, const void* const* co
     pp.x_exp = reinterpret_cast<int*>(wsb + pl.off_exp);
     pp.B = (int)B;
     pp.K = (int)K;
+    pp.Kp = (int)pad64(K);
     pp.counters = nullptr;
     pp.n_counters = 0;
     cudaError_t e = launch_prep(pp, stream);
@@ -282,14 +408,21 @@ int run_impl(int fmt, const void* x, int64_t B, int64_t K, const void* const* co
   CUtensorMap xmap;
   const CUtensorMapDataType xdt =
       pl.f16ops ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  if (!make_map(&xmap, xdt, 2, xop, (uint64_t)K, (uint64_t)B, (uint64_t)K * 2, kSubK,
-                (uint32_t)pl.NB, CU_TENSOR_MAP_SWIZZLE_128B)) {
+  const int64_t xpitch = pl.f16ops ? pad64(K) : K;  // elements per row of the x operand
+  p.x3d = (pl.pair && xpitch % 64 == 0) ? 1 : 0;
+  const bool mapped =
+      p.x3d ? make_map3(&xmap, xdt, xop, (uint64_t)B, (uint64_t)xpitch, (uint32_t)(pl.NB / 2),
+                        (uint32_t)(kPairAK / kSubK))
+            : make_map(&xmap, xdt, 2, xop, (uint64_t)K, (uint64_t)B, (uint64_t)xpitch * 2, kSubK,
+                       (uint32_t)(pl.pair ? pl.NB / 2 : pl.NB), CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!mapped) {
     snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled failed");
     return QGEMM_ERR_CUDA;
   }
   const int grid = pl.n_groups * pl.b_tiles * pl.S;
   if (g_prof_begin) cudaEventRecord(g_prof_begin, stream);
-  cudaError_t e = launch_tc(fmt, !pl.f16ops, p, pl.smem_bytes, grid, &xmap, stream);
+  cudaError_t e = pl.pair ? launch_pair(fmt, !pl.f16ops, p, pl.smem_bytes, grid, &xmap, stream)
+                          : launch_tc(fmt, !pl.f16ops, p, pl.smem_bytes, grid, &xmap, stream);
   if (e != cudaSuccess) return cuda_fail(e, "gemm kernel launch");
   if (g_prof_end) cudaEventRecord(g_prof_end, stream);
   if (pl.S > 1) {
@@ -409,7 +542,7 @@ int qgemm_split_k(int fmt, int64_t N, int64_t K, int* splits) {
   const int st = check_fmt_shape(fmt, N, K);
   if (st != QGEMM_OK) return st;
   if (!splits) return QGEMM_ERR_NULL;
-  *splits = split_for(fmt, N, K, 1);
+  *splits = use_one_sm() ? split_for(fmt, N, K, 1) : split_for_pair(fmt, N, K);
   return QGEMM_OK;
 }
 

@@ -22,6 +22,13 @@ constexpr int kDequantWarps = 8;                  // 2 per TMEM lane quarter
 constexpr int kMmaWarps = 4;                      // one MMA-issuing thread per weight subtile
 constexpr int kFirstDequantWarp = 1 + kMmaWarps;  // warp 0 is the TMA producer
 constexpr int kThreads = (1 + kMmaWarps + kDequantWarps) * 32;
+// CTA-pair kernel: warp 0 producer, warp 1 TMEM owner / pair MMA issuer, then dequant warps
+constexpr int kPairDequantWarps = 8;              // 2 per TMEM lane quarter
+constexpr int kPairFirstDequantWarp = 2;
+constexpr int kPairThreads = (kPairFirstDequantWarp + kPairDequantWarps) * 32;
+constexpr int kPairSMs = 74;                      // CTA pairs resident at once (148 SMs)
+constexpr int kPairAK = 256;                      // K per A slot of the pair kernel
+constexpr int kPairACols = kPairAK / 2;           // its TMEM columns
 constexpr int kMaxNB = 256;                       // MMA N limit
 constexpr int kSmemLimit = 227 * 1024;
 
@@ -81,6 +88,7 @@ struct GemmParams {
   int XS, WS;    // x ring and weight ring depths
   int AS;        // A ring depth (TMEM stages of kAStageK)
   int tmem_cols; // allocated TMEM columns
+  int x3d;       // pair kernel: x map is 3-D {64, B, K/64} (one TMA load per x stage)
   uint32_t smem_x, smem_w, smem_bar;  // byte offsets in the 1024-aligned dynamic smem
   const int* x_exp;          // f16 operands: x row b was scaled by 2^-x_exp[b]
   const float* ts[2];        // NVFP4 tensor scales (device), else nullptr
@@ -116,9 +124,9 @@ struct RepackParams {
 // Per-row power-of-two scaling of x before the bf16 -> f16 conversion.
 struct PrepParams {
   const uint16_t* x;  // bf16 [B][K]
-  uint16_t* xh;       // f16 [B][K]
+  uint16_t* xh;       // f16 [B][Kp], columns K..Kp-1 zero
   int* x_exp;         // [B]
-  int B, K;
+  int B, K, Kp;       // Kp: row pitch of xh in elements (K rounded up to 64)
   int* counters;      // zeroed here (split-K arrival counters of the following GEMM)
   int n_counters;
 };

@@ -1,0 +1,473 @@
+// pair.cu -- the block-quantized-weight GEMM on CTA pairs (sm_100a).
+//
+// y[b][n] = sum_k x[b][k] * dequant(W)[n][k]     (hipfire PR "fix(mtp): chunk scalar Q8
+// batched GEMM above 64 rows"; Atlas issue "Qwen3.8-27B on Strix Halo: prefill 2.4x gap",
+// kernel ranking and exact-F16-dequant sections)
+//
+// Swap-AB on the 5th-generation tensor cores, two SMs per MMA:
+//   * A cluster of two CTAs shares one tcgen05.mma.cta_group::2 stream.  The MMA M operand
+//     is 256 weight rows: the even CTA's 128 rows in its tensor memory (TMEM), the odd CTA's
+//     128 rows at the same TMEM address of its own SM.  One M=256 instruction costs the
+//     tensor pipe about what an M=128 one does on a single SM, so the pair halves the
+//     instruction count per weight byte -- the limit of the one-SM form at small widths.
+//   * The MMA N operand is NB batch rows of x: rows [0, NB/2) in the even CTA's shared
+//     memory, [NB/2, NB) in the odd CTA's, both loaded by TMA in the 128-byte swizzle.
+//     Each CTA's TMEM receives the fp32 accumulator of its own 128 rows x all NB columns.
+//   * Warp roles per CTA: warp 0 lane 0 streams packed weight stages (1-D bulk copies, the
+//     tile-major layout makes each stage contiguous) and x stages (tiled TMA whose byte
+//     count lands on the even CTA's barrier); warp 1 allocates TMEM and, in the even CTA,
+//     issues the pair MMAs; warps 2..17 dequantize weight stages from shared memory into
+//     the TMEM A ring (tcgen05.st) and run the epilogue.
+//   * K is split into S contiguous ranges, S fixed by (format, N, K).  Partials are summed
+//     in the fixed order s = 0..S-1 by the reduce kernel; nothing in the arithmetic depends
+//     on the batch width, so row b of y is bit-identical for every width up to 256.
+//   * Operand types as in the one-SM design: f16 (x rescaled per row by a power of two) for
+//     widths up to 256, bf16 straight from the caller above that.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "common.cuh"
+#include "dequant.cuh"
+#include "ptx.cuh"
+
+namespace qg {
+
+// a[i] for a runtime i in 0..3 without indexing the array dynamically (which would place
+// it in local memory)
+template <typename T>
+__device__ __forceinline__ T sel4(const T (&a)[4], int i) {
+  return i == 0 ? a[0] : i == 1 ? a[1] : i == 2 ? a[2] : a[3];
+}
+
+template <int FMT, bool BF16OP>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
+    qgemm_pair_kernel(const __grid_constant__ GemmParams p,
+                      const __grid_constant__ CUtensorMap tm_x) {
+  constexpr int KW = chunk_k(FMT);
+  constexpr int J = KW / kSubK;       // 64-element x slices per chunk
+  constexpr int CPA = kPairAK / KW;   // chunks per A slot (Q8_0: 2, FP4: 1)
+  constexpr int SB = scale_row_bytes(FMT);
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte aligned base, by pointer arithmetic on the shared array so that every access
+  // through it stays a shared-memory access (an integer round trip would make them generic)
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t sx = sbase + p.smem_x;
+  const uint32_t sw = sbase + p.smem_w;
+  const int XS = p.XS, WS = p.WS, AS = p.AS;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.smem_bar);
+  const uint32_t bar_x_full = smem_u32(bars);
+  const uint32_t bar_x_empty = bar_x_full + 8 * XS;
+  const uint32_t bar_w_full = bar_x_empty + 8 * XS;
+  const uint32_t bar_w_empty = bar_w_full + 8 * WS;
+  const uint32_t bar_a_full = bar_w_empty + 8 * WS;
+  const uint32_t bar_a_empty = bar_a_full + 8 * AS;
+  const uint32_t bar_acc = bar_a_empty + 8 * AS;
+  int* ctl = reinterpret_cast<int*>(bars + 2 * XS + 2 * WS + 2 * AS + 1);
+  volatile int* abort_flag = ctl + 1;
+  float* col_fac = reinterpret_cast<float*>(ctl + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0: even CTA (issues the MMAs), 1: odd CTA
+  int u = (int)(blockIdx.x >> 1);
+  const int g = u % p.n_groups;
+  u /= p.n_groups;
+  const int bt = u % p.b_tiles;
+  const int s = u / p.b_tiles;
+  const int c0 = (int)((int64_t)s * p.chunks / p.S);
+  const int c1 = (int)((int64_t)(s + 1) * p.chunks / p.S);
+  const int tpg = p.R / p.NMAT;  // tile pairs per group
+  const int64_t n_row_tiles = row_tiles(p.N);
+  const uint32_t a_col0 = (uint32_t)(p.R * p.NB);
+  const int half = p.NB >> 1;  // x rows (MMA N) held by each CTA
+  const uint32_t xslice = (uint32_t)half * 128u;  // one 64-element K slice of those rows
+  const uint32_t xstage = xslice * (uint32_t)(CPA * J);  // one A slot's K range
+  const int ngroups = (c1 - c0 + CPA - 1) / CPA;  // A slots per subtile in this unit
+
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tm_x);
+    for (int i = 0; i < XS; ++i) {
+      mbar_init(bar_x_full + 8 * i, 1);   // the even CTA's producer arrives (expect_tx)
+      mbar_init(bar_x_empty + 8 * i, 1);  // one pair commit per use
+    }
+    for (int i = 0; i < WS; ++i) {
+      mbar_init(bar_w_full + 8 * i, 1);
+      mbar_init(bar_w_empty + 8 * i, kPairDequantWarps / CPA);  // the warps that read it
+    }
+    for (int i = 0; i < AS; ++i) {
+      mbar_init(bar_a_full + 8 * i, 2 * kPairDequantWarps);  // both CTAs' dequant warps
+      mbar_init(bar_a_empty + 8 * i, 1);
+    }
+    mbar_init(bar_acc, 1);
+    ctl[1] = 0;
+    ctl[2] = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(ctl), (uint32_t)p.tmem_cols);
+    tmem_relinquish_pair();
+  }
+  if (warp >= kPairFirstDequantWarp) {
+    for (int i = threadIdx.x - kPairFirstDequantWarp * 32; i < p.NB; i += kPairDequantWarps * 32) {
+      const int b = bt * p.NB + i;
+      col_fac[i] = (b < p.B) ? (p.x_exp ? ldexpf(1.0f, p.x_exp[b]) : 1.0f) : 0.0f;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers are initialised before any remote arrive
+  tc_fence_after();
+  const uint32_t tmem = static_cast<uint32_t>(ctl[0]);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    // Two independent streams polled without blocking: this CTA's weight stages in the
+    // order (A slot group, subtile, chunk) into its own ring, and its half of x for each
+    // group (CPA chunks = 4 slices of 64 K elements) into the x ring.  The x bytes of both
+    // CTAs count on the even CTA's x barrier, which the even CTA's producer arms with the
+    // pair's total.
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_x = policy_evict_last();
+      const uint32_t xbar0 = mapa_shared(bar_x_full, 0);  // even CTA's x_full[0]
+      const int w_total = (c1 - c0) * p.R, x_total = ngroups;
+      RingPos xp, wp;
+      int x_issued = 0, w_issued = 0;
+      int wg = 0, wr = 0, wcc = 0;  // next weight stage (group, subtile, chunk in group)
+      bool ok = true;
+      uint64_t idle_since = 0;
+      while (ok && (w_issued < w_total || x_issued < x_total)) {
+        bool progressed = false;
+        if (w_issued < w_total &&
+            (w_issued < WS || mbar_test_wait(bar_w_empty + 8 * wp.slot, wp.phase ^ 1u))) {
+          const uint32_t fb = bar_w_full + 8 * wp.slot;
+          const int m = (p.NMAT == 2) ? (wr & 1) : 0;
+          const int64_t t = 2 * ((int64_t)g * tpg + wr / p.NMAT) + rank;
+          const int c = c0 + wg * CPA + wcc;
+          const uint32_t dst = sw + (uint32_t)(wp.slot * kWStageBytes);
+          if (t < n_row_tiles) {
+            const int64_t blk = t * p.chunks + c;
+            mbar_arrive_expect_tx(fb, (uint32_t)(kWCodeBytes + kTileRows * SB));
+            bulk_load(dst, p.codes[m] + blk * kWCodeBytes, kWCodeBytes, fb, pol_w);
+            bulk_load(dst + kWCodeBytes, p.scales[m] + blk * (kTileRows * SB),
+                      (uint32_t)(kTileRows * SB), fb, pol_w);
+          } else {
+            mbar_arrive(fb);  // a tile past the matrix: its rows are never stored
+          }
+          wp.next(WS);
+          ++w_issued;
+          const int n = min(CPA, c1 - (c0 + wg * CPA));
+          if (++wcc == n) {
+            wcc = 0;
+            if (++wr == p.R) {
+              wr = 0;
+              ++wg;
+            }
+          }
+          progressed = true;
+        }
+        if (x_issued < x_total &&
+            (x_issued < XS || mbar_test_wait(bar_x_empty + 8 * xp.slot, xp.phase ^ 1u))) {
+          const int cg = c0 + x_issued * CPA;
+          const uint32_t dst = sx + (uint32_t)xp.slot * xstage;
+          const uint32_t cbar = xbar0 + 8u * (uint32_t)xp.slot;
+          const int row0 = bt * p.NB + (int)rank * half;
+          if (p.x3d) {
+            // one box of 4 slices (slices past K read zeros from the padded rows or the
+            // out-of-range fill)
+            if (rank == 0) mbar_arrive_expect_tx(bar_x_full + 8 * xp.slot, 2u * xstage);
+            tma_load_3d_pair(dst, &tm_x, cbar, 0, row0, cg * KW / kSubK, pol_x);
+          } else {
+            const int nsl = min(CPA, c1 - cg) * J;  // slices in this group
+            if (rank == 0)
+              mbar_arrive_expect_tx(bar_x_full + 8 * xp.slot, 2u * xslice * (uint32_t)nsl);
+            for (int j = 0; j < nsl; ++j)
+              tma_load_2d_pair(dst + (uint32_t)j * xslice, &tm_x, cbar, cg * KW + j * kSubK, row0,
+                               pol_x);
+          }
+          xp.next(XS);
+          ++x_issued;
+          progressed = true;
+        }
+        if (progressed) {
+          idle_since = 0;
+        } else {
+          const uint64_t now = globaltimer_ns();
+          if (idle_since == 0) idle_since = now;
+          if (*abort_flag) ok = false;
+          if (now - idle_since > kWaitLimitNs) {
+            *abort_flag = 1;
+            atomicExch(p.dev_err, kErrTimeout);
+            ok = false;
+          }
+          __nanosleep(20);
+        }
+      }
+      if (!ok) {
+        // let this CTA's weight loads land before it leaves (their barrier is local); the
+        // x loads complete on the even CTA's barrier, so give them a fixed grace period
+        for (int k = 0; k < WS && k < w_issued; ++k) {
+          wp.slot = (wp.slot == 0) ? WS - 1 : wp.slot - 1;
+          if (wp.slot == WS - 1) wp.phase ^= 1u;
+          const uint64_t t0 = globaltimer_ns();
+          while (!mbar_try_wait(bar_w_full + 8 * wp.slot, wp.phase) &&
+                 globaltimer_ns() - t0 < kWaitLimitNs) {
+          }
+        }
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 200000) __nanosleep(1000);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ pair MMA issuer
+    // One thread of the even CTA.  For each A slot group (kPairAK elements of K): wait for
+    // the pair's x stage; then for each subtile wait until both CTAs have written the A slot
+    // (a_full counts both CTAs' dequant warps), issue its K=16 MMAs in K order and release
+    // the slot to both CTAs with a multicast commit.  The x stage is released after the
+    // group's last subtile.  Accumulator i receives its K slices in ascending order.
+    if (rank == 0 && lane == 0) {
+      const uint32_t idesc = idesc_f16_pair(BF16OP, (uint32_t)p.NB);
+      RingPos xc;  // x stage of the current group
+      RingPos ap;  // A ring
+      bool ok = true;
+      for (int gi = 0; gi < ngroups && ok; ++gi) {
+        const int ksteps = min(CPA, c1 - (c0 + gi * CPA)) * (KW / 16);
+        if (!mbar_wait_spin(bar_x_full + 8 * xc.slot, xc.phase, false, abort_flag, p.dev_err,
+                            kErrTimeout))
+          break;
+        const uint32_t xbase = sx + (uint32_t)xc.slot * xstage;
+        for (int i = 0; i < p.R; ++i) {
+          if (!mbar_wait_spin(bar_a_full + 8 * ap.slot, ap.phase, false, abort_flag, p.dev_err,
+                              kErrTimeout)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t d = tmem + (uint32_t)(i * p.NB);
+          const uint32_t a = tmem + a_col0 + (uint32_t)(ap.slot * kPairACols);
+#pragma unroll 4
+          for (int ks = 0; ks < ksteps; ++ks) {
+            const uint32_t bx = xbase + (uint32_t)(ks >> 2) * xslice + (uint32_t)((ks & 3) * 32);
+            mma_f16_ts_pair(d, a + (uint32_t)(ks * 8), smem_desc_sw128(bx), idesc,
+                            (gi > 0 || ks > 0) ? 1u : 0u);
+          }
+          mma_commit_pair(bar_a_empty + 8 * ap.slot);
+          ap.next(AS);
+        }
+        if (!ok) break;
+        mma_commit_pair(bar_x_empty + 8 * xc.slot);
+        xc.next(XS);
+      }
+      mma_commit_pair(bar_acc);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ dequant + epilogue
+    // Warp w may touch TMEM lanes 32*(w%4)..+31 (its lane quarter q); the kWPQ warps of a
+    // quarter split each A slot into parts h of EPW elements.
+    constexpr int kWPQ = kPairDequantWarps / 4;
+    constexpr int EPW = kPairAK / kWPQ;
+    const int dw = warp - kPairFirstDequantWarp;
+    const int q = warp & 3;
+    const int h = dw >> 2;
+    const int row = q * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    const uint32_t afull0 = mapa_shared(bar_a_full, 0);  // even CTA's a_full[0]
+
+    // MXFP4 on f16 operands: largest block exponent of this row within the split
+    int emax[4] = {0, 0, 0, 0};
+    if (FMT == FMT_MXFP4 && !BF16OP) {
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        if (r >= p.R) break;
+        const int64_t t = 2 * ((int64_t)g * tpg + r / p.NMAT) + rank;
+        const int64_t n = t * kTileRows + row;
+        uint32_t mx = 0;
+        if (n < p.N) {
+          const uint8_t* sb = p.scales[r % p.NMAT];
+          for (int c = c0; c < c1; ++c) {
+            const uint2 v = __ldg(reinterpret_cast<const uint2*>(sb + scale_offset(FMT, p.chunks, n, c)));
+            mx = __vmaxu4(mx, __vmaxu4(v.x, v.y));
+          }
+        }
+        mx = max(max(mx & 0xFFu, (mx >> 8) & 0xFFu), max((mx >> 16) & 0xFFu, mx >> 24));
+        emax[r] = (int)mx;
+      }
+    }
+
+    RingPos ap;  // A ring
+    int li = 0;  // A slots written so far
+    int wbase = 0;  // index of the first weight stage of the current (group, subtile)
+    // this warp's EPW elements of each A slot: chunk ccw of the group, from element eo
+    const int ccw = (h * EPW) / KW;
+    const int eo = (h * EPW) % KW;
+    bool ok = true;
+    for (int gi = 0; gi < ngroups && ok; ++gi) {
+      const int cg = c0 + gi * CPA;
+      const int n = min(CPA, c1 - cg);
+      for (int r = 0; r < p.R; ++r) {
+        if (li >= AS) {
+          // the pair MMAs of this slot's previous use have completed
+          ok = mbar_wait(bar_a_empty + 8 * ap.slot, ap.phase ^ 1u, abort_flag, p.dev_err,
+                         kErrTimeout);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+        }
+        if (ccw < n) {
+          const int wi = wbase + ccw;
+          const int wslot = wi % WS;
+          ok = mbar_wait(bar_w_full + 8 * wslot, (uint32_t)(wi / WS) & 1u, abort_flag, p.dev_err,
+                         kErrTimeout);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          const uint8_t* stage = smem + p.smem_w + wslot * kWStageBytes;
+          const uint8_t* crow = stage + row * kWRowBytes;
+          const uint8_t* srow = stage + kWCodeBytes + row * SB;
+          tc_fence_after();
+          uint32_t v[EPW / 2];
+          const int ex = sel4(emax, r);
+#pragma unroll
+          for (int i = 0; i < EPW / 32; ++i)
+            Dequant<FMT, BF16OP>::run(crow, row, srow, cg + ccw, eo + 32 * i, ex,
+                                      *reinterpret_cast<uint32_t(*)[16]>(&v[16 * i]));
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_w_empty + 8 * wslot);  // registers hold the data
+          const uint32_t ta = tmem + lane_base + a_col0 + (uint32_t)(ap.slot * kPairACols + h * (EPW / 2));
+#pragma unroll
+          for (int i = 0; i < EPW / 64; ++i)
+            tmem_st32(ta + (uint32_t)(32 * i), *reinterpret_cast<const uint32_t(*)[32]>(&v[32 * i]));
+          tmem_st_wait();
+        }
+        tc_fence_before();
+        __syncwarp();
+        // the stores above are complete (wait::st): the even CTA's warps arrive locally, the
+        // odd CTA's with a relaxed remote arrive (a cluster-scope release here would cost
+        // about a thousand cycles per slot)
+        if (lane == 0) {
+          if (rank == 0) mbar_arrive(bar_a_full + 8 * ap.slot);
+          else mbar_arrive_cluster_relaxed(afull0 + 8u * (uint32_t)ap.slot);
+        }
+        ap.next(AS);
+        ++li;
+        wbase += n;
+      }
+    }
+
+    if (ok) {
+      ok = mbar_wait(bar_acc, 0, abort_flag, p.dev_err, kErrTimeout);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    tc_fence_after();
+    const int qcols = p.NB / kWPQ;  // columns per warp of a lane quarter (multiple of 4)
+    const int cb0 = h * qcols;
+    const size_t BN = (size_t)p.B * p.N;
+    float ts[2] = {1.0f, 1.0f};
+    if (FMT == FMT_NVFP4) {
+      ts[0] = __ldg(p.ts[0]);
+      if (p.NMAT == 2) ts[1] = __ldg(p.ts[1]);
+    }
+    float rowfac[4] = {1.0f, 1.0f, 1.0f, 1.0f};
+    if (FMT == FMT_MXFP4 && !BF16OP)
+#pragma unroll
+      for (int r = 0; r < 4; ++r) rowfac[r] = ldexpf(1.0f, emax[r] - 140);
+    if (ok) {
+      // scale the accumulators; store finals (S == 1) or partials (S > 1)
+      for (int lt = 0; lt < tpg; ++lt) {
+        const int64_t t = 2 * ((int64_t)g * tpg + lt) + rank;
+        const int64_t n64 = t * kTileRows + row;
+        const int n = (int)n64;
+        const float rf_g = sel4(rowfac, lt * p.NMAT);
+        const float rf_u = sel4(rowfac, lt * p.NMAT + 1);
+        for (int cb = cb0; cb < cb0 + qcols; cb += 16) {
+          const int ngrp = min(16, cb0 + qcols - cb) >> 2;  // groups of 4 columns
+          uint32_t va[4][4], vb[4][4];
+#pragma unroll
+          for (int g4 = 0; g4 < 4; ++g4) {
+            if (g4 < ngrp) {
+              tmem_ld4(tmem + lane_base + (uint32_t)(lt * p.NMAT * p.NB + cb + g4 * 4), va[g4]);
+              if (p.NMAT == 2)
+                tmem_ld4(tmem + lane_base + (uint32_t)((lt * 2 + 1) * p.NB + cb + g4 * 4), vb[g4]);
+            }
+          }
+          tmem_ld_wait();
+          if (n64 >= p.N) continue;
+#pragma unroll
+          for (int g4 = 0; g4 < 4; ++g4) {
+            if (g4 >= ngrp) break;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int col = cb + g4 * 4 + i;
+              const int b = bt * p.NB + col;
+              if (b >= p.B) break;
+              const float cf = col_fac[col];
+              const float ga = __uint_as_float(va[g4][i]) * cf * rf_g;
+              if (p.NMAT == 1) {
+                if (p.S > 1) p.ws[(size_t)s * BN + (size_t)b * p.N + n] = ga;
+                else store_y(p, b, n, ga * ts[0]);
+              } else {
+                const float ua = __uint_as_float(vb[g4][i]) * cf * rf_u;
+                if (p.S > 1) {
+                  p.ws[(size_t)(2 * s) * BN + (size_t)b * p.N + n] = ga;
+                  p.ws[(size_t)(2 * s + 1) * BN + (size_t)b * p.N + n] = ua;
+                } else {
+                  store_h(p, b, n, ga * ts[0], ua * ts[1]);
+                }
+              }
+            }
+          }
+        }
+      }
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    if (lane == 0 && *abort_flag) {
+      // the final pair commit arrives once every MMA of the pair has completed
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(bar_acc, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+      }
+    }
+    __syncwarp();
+  }
+  // neither CTA leaves (or frees TMEM the pair MMAs write) while its peer may still use it
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, (uint32_t)p.tmem_cols);
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Launcher (grid = 2 CTAs per work unit, clusters of 2 from the kernel attribute).
+// ---------------------------------------------------------------------------------------
+template <int FMT, bool BF16OP>
+cudaError_t launch_pair_impl(const GemmParams& p, size_t smem_bytes, int units,
+                             const CUtensorMap* maps, cudaStream_t stream) {
+  auto kern = qgemm_pair_kernel<FMT, BF16OP>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem_bytes);
+  if (e != cudaSuccess) return e;
+  kern<<<2 * units, kPairThreads, smem_bytes, stream>>>(p, maps[0]);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pair(int fmt, bool bf16op, const GemmParams& p, size_t smem_bytes, int units,
+                        const CUtensorMap* maps, cudaStream_t stream) {
+  switch (fmt) {
+    case FMT_Q8_0:
+      return bf16op ? launch_pair_impl<FMT_Q8_0, true>(p, smem_bytes, units, maps, stream)
+                    : launch_pair_impl<FMT_Q8_0, false>(p, smem_bytes, units, maps, stream);
+    case FMT_NVFP4:
+      return bf16op ? launch_pair_impl<FMT_NVFP4, true>(p, smem_bytes, units, maps, stream)
+                    : launch_pair_impl<FMT_NVFP4, false>(p, smem_bytes, units, maps, stream);
+    default:
+      return bf16op ? launch_pair_impl<FMT_MXFP4, true>(p, smem_bytes, units, maps, stream)
+                    : launch_pair_impl<FMT_MXFP4, false>(p, smem_bytes, units, maps, stream);
+  }
+}
+
+}  // namespace qg

@@ -95,13 +95,13 @@ def test_split_rule_depends_only_on_shape(lib):
            for (N, K) in ((17408, 5120), (5120, 17408), (512, 1024))}
     for (f, N, K), s in got.items():
         assert 1 <= s <= 16
-    assert got[("q8_0", 17408, 5120)] == 4
-    assert got[("nvfp4", 17408, 5120)] == 4
-    assert got[("q8_0", 5120, 17408)] == 14
-    assert got[("nvfp4", 5120, 17408)] == 14
+    assert got[("q8_0", 17408, 5120)] == 1
+    assert got[("nvfp4", 17408, 5120)] == 1
+    assert got[("q8_0", 5120, 17408)] == 7
+    assert got[("nvfp4", 5120, 17408)] == 7
     # workspace grows with B but the split does not
-    w64 = qgemm.workspace_size("q8_0", 17408, 5120, 64)
-    w65 = qgemm.workspace_size("q8_0", 17408, 5120, 65)
+    w64 = qgemm.workspace_size("q8_0", 5120, 17408, 64)
+    w65 = qgemm.workspace_size("q8_0", 5120, 17408, 65)
     assert w65 > w64
 
 
