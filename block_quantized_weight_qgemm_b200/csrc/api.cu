@@ -182,6 +182,7 @@ bool use_one_sm() {
 
 struct Plan {
   bool pair;    // CTA-pair kernel
+  int NACC;     // pair kernel: accumulators per subtile
   bool f16ops;  // widths <= 256
   int NB, R, NMAT, S, n_groups, b_tiles, chunks, XS, WS, AS, tmem_cols;
   size_t smem_bytes;
@@ -204,49 +205,39 @@ bool make_plan_pair(int fmt, int64_t N, int64_t K, int64_t B, int nmat, Plan* pl
   p.NMAT = nmat;
   p.f16ops = (B <= 256);
   p.chunks = (int)((K + chunk_k(fmt) - 1) / chunk_k(fmt));
-  const int J = chunk_k(fmt) / kSubK;
   const int64_t pairs = (row_tiles(N) + 1) / 2;
   if (p.f16ops) {
+    // two accumulators per subtile (two concurrent MMA issuers), so NB <= 128 (64 fused)
     p.S = split_for_pair(fmt, N, K);
-    const int nb_cap = (nmat == 2) ? 128 : 256;
-    int nb = (int)std::min<int64_t>(((B + 15) / 16) * 16, nb_cap);
-    if (nmat == 2 && B > 128) nb = (int)(((B + 1) / 2 + 15) / 16 * 16);
-    p.NB = nb;
+    p.NACC = 2;
+    const int nb_cap = (nmat == 2) ? 64 : 128;
+    const int64_t tiles_b = (B + nb_cap - 1) / nb_cap;  // balanced batch tiles
+    p.NB = (int)std::min<int64_t>(((B + tiles_b - 1) / tiles_b + 15) / 16 * 16, nb_cap);
   } else {
     p.S = 1;
+    p.NACC = 1;
     p.NB = (nmat == 2) ? 128 : 256;
   }
   p.b_tiles = (int)((B + p.NB - 1) / p.NB);
-  // tile pairs per unit: 1, or 2 to share each x stage between two pairs when x is wide
-  int m = 1;
-  if (p.NB >= 64 && 2 * nmat * p.NB + 2 * kPairACols <= 512) {
-    const int64_t w1 = (pairs * p.b_tiles * p.S + kPairSMs - 1) / kPairSMs;
-    const int64_t w2 = (((pairs + 1) / 2) * p.b_tiles * p.S + kPairSMs - 1) / kPairSMs;
-    if (2 * w2 <= w1 + (p.NB >= 128 ? 1 : 0)) m = 2;
-  }
-  if (const char* e = getenv("QGEMM_DEBUG_R")) {
-    const int r = atoi(e);
-    if ((r == 1 || r == 2) && r * nmat * p.NB + 2 * kPairACols <= 512) m = r;
-  }
-  p.R = m * nmat;
-  p.n_groups = (int)((pairs + m - 1) / m);
-  p.AS = std::min(4, (512 - p.R * p.NB) / kPairACols);
+  p.R = nmat;
+  p.n_groups = (int)pairs;
+  p.AS = std::min(4, (512 - p.R * p.NACC * p.NB) / kPairACols);
   if (p.AS < 2) return false;
-  p.tmem_cols = next_pow2_cols(p.R * p.NB + p.AS * kPairACols);
+  p.tmem_cols = next_pow2_cols(p.R * p.NACC * p.NB + p.AS * kPairACols);
   if (p.tmem_cols > 512) return false;
-  // x ring: one stage per A slot (kPairAK / 64 slices of this CTA's NB/2 rows)
   const size_t xstage = (size_t)(p.NB / 2) * 128 * (kPairAK / kSubK);
   const size_t misc = 8 * (2 * 4 + 2 * kMaxWStages + 2 * 8 + 1) + 16 + 4 * kMaxNB + 64;
   const size_t budget = kSmemLimit - 1024 - misc;
+  const size_t wstage = (size_t)pair_wstage_bytes(fmt);
   int XS = 4;
-  while (XS > 2 && XS * xstage + 4 * (size_t)kWStageBytes > budget) --XS;
-  if (XS * xstage + 2 * (size_t)kWStageBytes > budget) return false;
-  const int WS = (int)std::min<size_t>(kMaxWStages, (budget - XS * xstage) / kWStageBytes);
+  while (XS > 2 && XS * xstage + 4 * wstage > budget) --XS;
+  if (XS * xstage + 2 * wstage > budget) return false;
+  const int WS = (int)std::min<size_t>(kMaxWStages, (budget - XS * xstage) / wstage);
   p.XS = XS;
   p.WS = WS;
   p.smem_x = 0;
   p.smem_w = (uint32_t)(XS * xstage);
-  p.smem_bar = p.smem_w + (uint32_t)(WS * kWStageBytes);
+  p.smem_bar = p.smem_w + (uint32_t)(WS * wstage);
   const size_t bar_bytes = 8 * (2 * XS + 2 * WS + 2 * p.AS + 1);
   p.smem_bytes = 1024 + p.smem_bar + bar_bytes + 16 + 4 * p.NB + 64;
   size_t off = 0;
@@ -373,6 +364,7 @@ int run_impl(int fmt, const void* x, int64_t B, int64_t K, const void* const* co
   p.WS = pl.WS;
   p.AS = pl.AS;
   p.tmem_cols = pl.tmem_cols;
+  p.NACC = pl.NACC;
   p.smem_x = pl.smem_x;
   p.smem_w = pl.smem_w;
   p.smem_bar = pl.smem_bar;

@@ -25,7 +25,8 @@ constexpr int kThreads = (1 + kMmaWarps + kDequantWarps) * 32;
 // CTA-pair kernel: warp 0 producer, warp 1 TMEM owner / pair MMA issuer, then dequant warps
 constexpr int kPairDequantWarps = 8;              // 2 per TMEM lane quarter
 constexpr int kPairFirstDequantWarp = 2;
-constexpr int kPairThreads = (kPairFirstDequantWarp + kPairDequantWarps) * 32;
+constexpr int kPairIssuer2Warp = kPairFirstDequantWarp + kPairDequantWarps;  // second MMA issuer
+constexpr int kPairThreads = (kPairIssuer2Warp + 1) * 32;
 constexpr int kPairSMs = 74;                      // CTA pairs resident at once (148 SMs)
 constexpr int kPairAK = 256;                      // K per A slot of the pair kernel
 constexpr int kPairACols = kPairAK / 2;           // its TMEM columns
@@ -40,6 +41,11 @@ __host__ __device__ constexpr int scale_row_bytes(int fmt) { return fmt == FMT_N
 __host__ __device__ constexpr int64_t row_tiles(int64_t N) { return (N + kTileRows - 1) / kTileRows; }
 __host__ __device__ constexpr int64_t k_chunks(int fmt, int64_t K) {
   return (K + chunk_k(fmt) - 1) / chunk_k(fmt);
+}
+// Weight stage of the pair kernel: one A slot of one subtile, i.e. kPairAK / chunk_k chunks
+// of a 128-row tile (contiguous in the tile-major layout): their codes, then their scales.
+__host__ __device__ constexpr int pair_wstage_bytes(int fmt) {
+  return (kPairAK / chunk_k(fmt)) * (kWCodeBytes + kTileRows * scale_row_bytes(fmt));
 }
 // Row-major interchange layout (qgemm_repack_rowmajor input): codes [N][code pitch],
 // scales [N][scale pitch], rows 16-byte aligned.
@@ -89,6 +95,7 @@ struct GemmParams {
   int AS;        // A ring depth (TMEM stages of kAStageK)
   int tmem_cols; // allocated TMEM columns
   int x3d;       // pair kernel: x map is 3-D {64, B, K/64} (one TMA load per x stage)
+  int NACC;      // pair kernel: accumulators per subtile (1, or 2 for the f16 path)
   uint32_t smem_x, smem_w, smem_bar;  // byte offsets in the 1024-aligned dynamic smem
   const int* x_exp;          // f16 operands: x row b was scaled by 2^-x_exp[b]
   const float* ts[2];        // NVFP4 tensor scales (device), else nullptr

@@ -15,9 +15,10 @@
 //     Each CTA's TMEM receives the fp32 accumulator of its own 128 rows x all NB columns.
 //   * Warp roles per CTA: warp 0 lane 0 streams packed weight stages (1-D bulk copies, the
 //     tile-major layout makes each stage contiguous) and x stages (tiled TMA whose byte
-//     count lands on the even CTA's barrier); warp 1 allocates TMEM and, in the even CTA,
-//     issues the pair MMAs; warps 2..17 dequantize weight stages from shared memory into
-//     the TMEM A ring (tcgen05.st) and run the epilogue.
+//     count lands on the even CTA's barrier); warp 1 allocates TMEM and, with warp 10, issues
+//     the pair MMAs from the even CTA (alternate A slots, one MMA order); warps 2..9
+//     dequantize weight stages from shared memory into the TMEM A ring (tcgen05.st) and run
+//     the epilogue.
 //   * K is split into S contiguous ranges, S fixed by (format, N, K).  Partials are summed
 //     in the fixed order s = 0..S-1 by the reduce kernel; nothing in the arithmetic depends
 //     on the batch width, so row b of y is bit-identical for every width up to 256.
@@ -47,6 +48,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   constexpr int J = KW / kSubK;       // 64-element x slices per chunk
   constexpr int CPA = kPairAK / KW;   // chunks per A slot (Q8_0: 2, FP4: 1)
   constexpr int SB = scale_row_bytes(FMT);
+  constexpr int WSTAGE = pair_wstage_bytes(FMT);
+  constexpr int WSCALES = (kPairAK / chunk_k(FMT)) * kWCodeBytes;  // offset of the scales in a stage
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base, by pointer arithmetic on the shared array so that every access
   // through it stays a shared-memory access (an integer round trip would make them generic)
@@ -78,7 +81,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   const int c1 = (int)((int64_t)(s + 1) * p.chunks / p.S);
   const int tpg = p.R / p.NMAT;  // tile pairs per group
   const int64_t n_row_tiles = row_tiles(p.N);
-  const uint32_t a_col0 = (uint32_t)(p.R * p.NB);
+  const uint32_t a_col0 = (uint32_t)(p.R * p.NACC * p.NB);  // accumulators, then the A ring
   const int half = p.NB >> 1;  // x rows (MMA N) held by each CTA
   const uint32_t xslice = (uint32_t)half * 128u;  // one 64-element K slice of those rows
   const uint32_t xstage = xslice * (uint32_t)(CPA * J);  // one A slot's K range
@@ -88,17 +91,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     prefetch_tmap(&tm_x);
     for (int i = 0; i < XS; ++i) {
       mbar_init(bar_x_full + 8 * i, 1);   // the even CTA's producer arrives (expect_tx)
-      mbar_init(bar_x_empty + 8 * i, 1);  // one pair commit per use
+      mbar_init(bar_x_empty + 8 * i, 1);  // the commit of the group's issuer
     }
     for (int i = 0; i < WS; ++i) {
       mbar_init(bar_w_full + 8 * i, 1);
-      mbar_init(bar_w_empty + 8 * i, kPairDequantWarps / CPA);  // the warps that read it
+      mbar_init(bar_w_empty + 8 * i, kPairDequantWarps);
     }
     for (int i = 0; i < AS; ++i) {
       mbar_init(bar_a_full + 8 * i, 2 * kPairDequantWarps);  // both CTAs' dequant warps
       mbar_init(bar_a_empty + 8 * i, 1);
     }
-    mbar_init(bar_acc, 1);
+    mbar_init(bar_acc, 2);  // one final commit per issuer
     ctl[1] = 0;
     ctl[2] = 0;
     fence_mbar_init();
@@ -107,7 +110,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     tmem_alloc_pair(smem_u32(ctl), (uint32_t)p.tmem_cols);
     tmem_relinquish_pair();
   }
-  if (warp >= kPairFirstDequantWarp) {
+  if (warp >= kPairFirstDequantWarp && warp < kPairIssuer2Warp) {
     for (int i = threadIdx.x - kPairFirstDequantWarp * 32; i < p.NB; i += kPairDequantWarps * 32) {
       const int b = bt * p.NB + i;
       col_fac[i] = (b < p.B) ? (p.x_exp ? ldexpf(1.0f, p.x_exp[b]) : 1.0f) : 0.0f;
@@ -130,39 +133,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       const uint64_t pol_w = policy_evict_first();
       const uint64_t pol_x = policy_evict_last();
       const uint32_t xbar0 = mapa_shared(bar_x_full, 0);  // even CTA's x_full[0]
-      const int w_total = (c1 - c0) * p.R, x_total = ngroups;
+      const int w_total = ngroups * p.R, x_total = ngroups;
       RingPos xp, wp;
       int x_issued = 0, w_issued = 0;
-      int wg = 0, wr = 0, wcc = 0;  // next weight stage (group, subtile, chunk in group)
+      int wg = 0, wr = 0;  // next weight stage (group, subtile)
       bool ok = true;
       uint64_t idle_since = 0;
       while (ok && (w_issued < w_total || x_issued < x_total)) {
         bool progressed = false;
         if (w_issued < w_total &&
             (w_issued < WS || mbar_test_wait(bar_w_empty + 8 * wp.slot, wp.phase ^ 1u))) {
+          // one stage: the group's n chunks of this subtile's tile, codes then scales
           const uint32_t fb = bar_w_full + 8 * wp.slot;
           const int m = (p.NMAT == 2) ? (wr & 1) : 0;
           const int64_t t = 2 * ((int64_t)g * tpg + wr / p.NMAT) + rank;
-          const int c = c0 + wg * CPA + wcc;
-          const uint32_t dst = sw + (uint32_t)(wp.slot * kWStageBytes);
+          const int cg = c0 + wg * CPA;
+          const int n = min(CPA, c1 - cg);
+          const uint32_t dst = sw + (uint32_t)(wp.slot * WSTAGE);
           if (t < n_row_tiles) {
-            const int64_t blk = t * p.chunks + c;
-            mbar_arrive_expect_tx(fb, (uint32_t)(kWCodeBytes + kTileRows * SB));
-            bulk_load(dst, p.codes[m] + blk * kWCodeBytes, kWCodeBytes, fb, pol_w);
-            bulk_load(dst + kWCodeBytes, p.scales[m] + blk * (kTileRows * SB),
-                      (uint32_t)(kTileRows * SB), fb, pol_w);
+            const int64_t blk = t * p.chunks + cg;
+            const uint32_t cbytes = (uint32_t)n * kWCodeBytes;
+            const uint32_t sbytes = (uint32_t)n * (kTileRows * SB);
+            mbar_arrive_expect_tx(fb, cbytes + sbytes);
+            bulk_load(dst, p.codes[m] + blk * kWCodeBytes, cbytes, fb, pol_w);
+            bulk_load(dst + WSCALES, p.scales[m] + blk * (kTileRows * SB), sbytes, fb, pol_w);
           } else {
             mbar_arrive(fb);  // a tile past the matrix: its rows are never stored
           }
           wp.next(WS);
           ++w_issued;
-          const int n = min(CPA, c1 - (c0 + wg * CPA));
-          if (++wcc == n) {
-            wcc = 0;
-            if (++wr == p.R) {
-              wr = 0;
-              ++wg;
-            }
+          if (++wr == p.R) {
+            wr = 0;
+            ++wg;
           }
           progressed = true;
         }
@@ -219,19 +221,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ pair MMA issuer
-    // One thread of the even CTA.  For each A slot group (kPairAK elements of K): wait for
-    // the pair's x stage; then for each subtile wait until both CTAs have written the A slot
-    // (a_full counts both CTAs' dequant warps), issue its K=16 MMAs in K order and release
-    // the slot to both CTAs with a multicast commit.  The x stage is released after the
-    // group's last subtile.  Accumulator i receives its K slices in ascending order.
-    if (rank == 0 && lane == 0) {
+  } else if (warp == 1 || warp == kPairIssuer2Warp) {
+    // ------------------------------------------------------------ pair MMA issuers
+    // One tcgen05.mma takes its issuing thread about as long as the tensor pipe needs for
+    // an N=128 tile, so at small N the issue rate, not the pipe, bounds the MMA stream.  With
+    // NACC = 2 two threads of the even CTA issue concurrently, each into its own accumulators:
+    // issuer e takes the A-slot groups gi with gi % 2 == e (every subtile of the group) and
+    // accumulates them into D[i][e]; the epilogue adds D[i][0] + D[i][1].  Within each
+    // accumulator the K slices arrive in ascending order.  For each of its groups an issuer
+    // waits for the pair's x stage, then per subtile for the A slot (a_full counts both CTAs'
+    // dequant warps), issues the slot's K=16 MMAs and releases the slot to both CTAs with a
+    // multicast commit; the x stage is released after the group's last subtile.
+    const int e = (warp == 1) ? 0 : 1;
+    if (rank == 0 && lane == 0 && e < p.NACC) {
       const uint32_t idesc = idesc_f16_pair(BF16OP, (uint32_t)p.NB);
       RingPos xc;  // x stage of the current group
       RingPos ap;  // A ring
       bool ok = true;
       for (int gi = 0; gi < ngroups && ok; ++gi) {
+        if (gi % p.NACC != e) {
+          // another issuer's group: keep the ring positions in step
+          for (int i = 0; i < p.R; ++i) ap.next(AS);
+          xc.next(XS);
+          continue;
+        }
         const int ksteps = min(CPA, c1 - (c0 + gi * CPA)) * (KW / 16);
         if (!mbar_wait_spin(bar_x_full + 8 * xc.slot, xc.phase, false, abort_flag, p.dev_err,
                             kErrTimeout))
@@ -244,13 +257,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t d = tmem + (uint32_t)(i * p.NB);
+          const uint32_t d = tmem + (uint32_t)((i * p.NACC + e) * p.NB);
           const uint32_t a = tmem + a_col0 + (uint32_t)(ap.slot * kPairACols);
+          const bool first = (gi < p.NACC);  // this accumulator's first group
 #pragma unroll 4
           for (int ks = 0; ks < ksteps; ++ks) {
             const uint32_t bx = xbase + (uint32_t)(ks >> 2) * xslice + (uint32_t)((ks & 3) * 32);
             mma_f16_ts_pair(d, a + (uint32_t)(ks * 8), smem_desc_sw128(bx), idesc,
-                            (gi > 0 || ks > 0) ? 1u : 0u);
+                            (!first || ks > 0) ? 1u : 0u);
           }
           mma_commit_pair(bar_a_empty + 8 * ap.slot);
           ap.next(AS);
@@ -259,8 +273,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         mma_commit_pair(bar_x_empty + 8 * xc.slot);
         xc.next(XS);
       }
-      mma_commit_pair(bar_acc);
     }
+    if (rank == 0 && lane == 0) mma_commit_pair(bar_acc);  // both issuers, used or not
     __syncwarp();
   } else {
     // ------------------------------------------------------------ dequant + epilogue
@@ -298,7 +312,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 
     RingPos ap;  // A ring
     int li = 0;  // A slots written so far
-    int wbase = 0;  // index of the first weight stage of the current (group, subtile)
     // this warp's EPW elements of each A slot: chunk ccw of the group, from element eo
     const int ccw = (h * EPW) / KW;
     const int eo = (h * EPW) % KW;
@@ -314,16 +327,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
         }
+        // weight stage li (one per A slot): this warp's chunk ccw of it, if the group has one
+        const int wslot = li % WS;
+        bool wdone = false;
         if (ccw < n) {
-          const int wi = wbase + ccw;
-          const int wslot = wi % WS;
-          ok = mbar_wait(bar_w_full + 8 * wslot, (uint32_t)(wi / WS) & 1u, abort_flag, p.dev_err,
+          ok = mbar_wait(bar_w_full + 8 * wslot, (uint32_t)(li / WS) & 1u, abort_flag, p.dev_err,
                          kErrTimeout);
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
-          const uint8_t* stage = smem + p.smem_w + wslot * kWStageBytes;
-          const uint8_t* crow = stage + row * kWRowBytes;
-          const uint8_t* srow = stage + kWCodeBytes + row * SB;
+          const uint8_t* stage = smem + p.smem_w + wslot * WSTAGE;
+          const uint8_t* crow = stage + ccw * kWCodeBytes + row * kWRowBytes;
+          const uint8_t* srow = stage + WSCALES + ccw * (kTileRows * SB) + row * SB;
           tc_fence_after();
           uint32_t v[EPW / 2];
           const int ex = sel4(emax, r);
@@ -333,11 +347,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                                       *reinterpret_cast<uint32_t(*)[16]>(&v[16 * i]));
           __syncwarp();
           if (lane == 0) mbar_arrive(bar_w_empty + 8 * wslot);  // registers hold the data
+          wdone = true;
           const uint32_t ta = tmem + lane_base + a_col0 + (uint32_t)(ap.slot * kPairACols + h * (EPW / 2));
 #pragma unroll
           for (int i = 0; i < EPW / 64; ++i)
             tmem_st32(ta + (uint32_t)(32 * i), *reinterpret_cast<const uint32_t(*)[32]>(&v[32 * i]));
           tmem_st_wait();
+        }
+        if (!wdone) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_w_empty + 8 * wslot);  // nothing of this stage to read
         }
         tc_fence_before();
         __syncwarp();
@@ -350,7 +369,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         }
         ap.next(AS);
         ++li;
-        wbase += n;
       }
     }
 
@@ -371,6 +389,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     if (FMT == FMT_MXFP4 && !BF16OP)
 #pragma unroll
       for (int r = 0; r < 4; ++r) rowfac[r] = ldexpf(1.0f, emax[r] - 140);
+    const bool two_acc = (p.NACC == 2 && ngroups > 1);
     if (ok) {
       // scale the accumulators; store finals (S == 1) or partials (S > 1)
       for (int lt = 0; lt < tpg; ++lt) {
@@ -382,15 +401,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         for (int cb = cb0; cb < cb0 + qcols; cb += 16) {
           const int ngrp = min(16, cb0 + qcols - cb) >> 2;  // groups of 4 columns
           uint32_t va[4][4], vb[4][4];
+          // accumulator of subtile i, issuer e: columns ((i * NACC) + e) * NB
+          const int ig = lt * p.NMAT, iu = lt * p.NMAT + 1;
 #pragma unroll
           for (int g4 = 0; g4 < 4; ++g4) {
             if (g4 < ngrp) {
-              tmem_ld4(tmem + lane_base + (uint32_t)(lt * p.NMAT * p.NB + cb + g4 * 4), va[g4]);
+              tmem_ld4(tmem + lane_base + (uint32_t)(ig * p.NACC * p.NB + cb + g4 * 4), va[g4]);
               if (p.NMAT == 2)
-                tmem_ld4(tmem + lane_base + (uint32_t)((lt * 2 + 1) * p.NB + cb + g4 * 4), vb[g4]);
+                tmem_ld4(tmem + lane_base + (uint32_t)(iu * p.NACC * p.NB + cb + g4 * 4), vb[g4]);
             }
           }
           tmem_ld_wait();
+          if (two_acc) {
+            // the odd groups' accumulators, added in the fixed order even + odd
+            uint32_t wa[4][4], wb[4][4];
+#pragma unroll
+            for (int g4 = 0; g4 < 4; ++g4) {
+              if (g4 < ngrp) {
+                tmem_ld4(tmem + lane_base + (uint32_t)((ig * p.NACC + 1) * p.NB + cb + g4 * 4), wa[g4]);
+                if (p.NMAT == 2)
+                  tmem_ld4(tmem + lane_base + (uint32_t)((iu * p.NACC + 1) * p.NB + cb + g4 * 4), wb[g4]);
+              }
+            }
+            tmem_ld_wait();
+#pragma unroll
+            for (int g4 = 0; g4 < 4; ++g4)
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                va[g4][j] = __float_as_uint(__uint_as_float(va[g4][j]) + __uint_as_float(wa[g4][j]));
+                if (p.NMAT == 2)
+                  vb[g4][j] = __float_as_uint(__uint_as_float(vb[g4][j]) + __uint_as_float(wb[g4][j]));
+              }
+          }
           if (n64 >= p.N) continue;
 #pragma unroll
           for (int g4 = 0; g4 < 4; ++g4) {
