@@ -1,7 +1,8 @@
 """Benchmark of the block-quantized-weight GEMM hot path on B200.
 
 Default workload (one "step"): the Q8_0 27B FFN at decode width B = 64 -- qgemm_run on the
-gate [17408, 5120], up [17408, 5120] and down [5120, 17408] matrices, fp32 outputs.  The
+gate [17408, 5120], up [17408, 5120] and down [5120, 17408] matrices, fp32 outputs.  Steps
+are timed as replays of a CUDA graph holding the three calls.  The
 metric is weight GB/s: packed weight bytes read per step / step time (the pages' weight-
 streaming bound for widths <= 64).  Weights cycle through a ring of distinct copies so that
 no step finds its weights in L2.
@@ -34,7 +35,7 @@ BATCH = 64
 RING = 4  # copies of each matrix: 3 x 4 x 94.7 MB = 1.14 GB of Q8_0 weights > L2
 METRIC = "qGEMM weight GB/s (B≤64) & TFLOP/s (prefill) as % of B200 roofline"
 WORKLOAD = "Q8_0 27B FFN decode step: gate+up W[17408,5120] and down W[5120,17408], B=64"
-KERNEL = "qgemm_tc_kernel<Q8_0, f16 operands>"
+KERNEL = "qgemm_pair_kernel<Q8_0, f16 operands> (CTA pairs, tcgen05.mma.cta_group::2)"
 SM_MAX_FALLBACK = 1965.0
 
 
@@ -230,28 +231,35 @@ def main():
     torch.cuda.synchronize()
     step_bytes = sum(weight_bytes(fmt, c["N"], c["K"]) for c in calls)
 
-    def step(i, events=None):
+    def step(i, events=None, stream=None):
         for j, c in enumerate(calls):
             if events is not None:
                 qgemm.profile_events(*events[j])
-            qgemm.run(c["x"], c["ring"][i % RING], y=c["y"], workspace=c["ws"])
+            qgemm.run(c["x"], c["ring"][i % RING], y=c["y"], workspace=c["ws"], stream=stream)
         if events is not None:
             qgemm.profile_events(None, None)
 
+    # one CUDA graph per weight copy of the ring: a step is the replay of graph[i % RING]
+    gstream = torch.cuda.Stream(device=dev)
+    graphs = []
+    with torch.cuda.stream(gstream):
+        for r in range(RING):
+            step(r, stream=gstream)
+        torch.cuda.synchronize()
+        for r in range(RING):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=gstream):
+                step(r, stream=gstream)
+            graphs.append(g)
+    torch.cuda.synchronize()
+
     for i in range(args.warmup):
-        step(i)
+        graphs[i % RING].replay()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
 
-    # ---- device-timed region (CUDA events on the launching stream) ----------------------
-    kev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            for _ in calls] for _ in range(args.steps)]
-    for pairs in kev:  # torch creates the CUDA events lazily, on first record
-        for a, b in pairs:
-            a.record()
-            b.record()
-    torch.cuda.synchronize()
+    # ---- device-timed region: K graph replays between CUDA events -----------------------
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
@@ -262,15 +270,26 @@ def main():
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record()
     for i in range(args.steps):
-        step(i, kev[i])
+        graphs[i % RING].replay()
     t1.record()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
     ms = t0.elapsed_time(t1) / args.steps
+
+    # ---- the dominant kernel alone: events around each GEMM launch (stream launches) ----
+    kev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in calls] for _ in range(args.steps)]
+    for pairs in kev:  # torch creates the CUDA events lazily, on first record
+        for a, b in pairs:
+            a.record()
+            b.record()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        step(i, kev[i])
+    torch.cuda.synchronize()
     kernel_ms = [[a.elapsed_time(b) for (a, b) in kev[i]] for i in range(args.steps)]
-    # dominant kernel: the GEMM kernel over all three matrices; bytes per launch = its matrix
     per_launch = []
     for i in range(args.steps):
         for j, c in enumerate(calls):
@@ -336,6 +355,8 @@ def main():
                    "weight_bytes_per_step": step_bytes,
                    "l2": "weights cycle through %d distinct copies per matrix (%.2f GB) > 126 MB L2"
                          % (RING, RING * step_bytes / 1e9),
+                   "timing": "step = CUDA-graph replay of the three qgemm_run calls; the kernel "
+                             "figure times each GEMM launch between events on its stream",
                    "parallelism": "replicas" if world > 1 else "single GPU"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,

@@ -14,10 +14,8 @@
 
 namespace qg {
 cudaError_t launch_prep(const PrepParams& pp, cudaStream_t stream);
-cudaError_t launch_tc(int fmt, bool bf16op, const GemmParams& p, size_t smem_bytes, int grid,
-                      const CUtensorMap* maps, cudaStream_t stream);
 cudaError_t launch_pair(int fmt, bool bf16op, const GemmParams& p, size_t smem_bytes, int units,
-                        const CUtensorMap* maps, cudaStream_t stream);
+                        const CUtensorMap* maps, bool pdl, cudaStream_t stream);
 cudaError_t launch_pack(int fmt, const float* W, int64_t N, int64_t K, void* codes, void* scales,
                         float* tensor_scale, cudaStream_t stream);
 cudaError_t launch_repack(const RepackParams& rp, cudaStream_t stream);
@@ -121,34 +119,6 @@ int device_ok() {
   return ok;
 }
 
-constexpr int kSMs = 148;  // fixed: the K split must not depend on the device or the width
-
-// The K split used for widths 1..256: a function of (fmt, N, K, nmat) only.  It picks the S
-// that best fills kSMs CTAs when each CTA holds 4 weight subtiles (the decode tiling),
-// preferring smaller S on ties.
-int split_for(int fmt, int64_t N, int64_t K, int nmat) {
-  const int64_t chunks = (K + chunk_k(fmt) - 1) / chunk_k(fmt);
-  const int64_t tiles = (N + kTileRows - 1) / kTileRows;
-  const int64_t per_group = 4 / nmat;
-  const int64_t groups = (tiles + per_group - 1) / per_group;
-  int best = 1;
-  double best_eff = -1.0;
-  const int64_t smax = std::min<int64_t>(16, chunks);
-  for (int64_t S = 1; S <= smax; ++S) {
-    const int64_t units = groups * S;
-    const int64_t waves = (units + kSMs - 1) / kSMs;
-    const double fill = double(units) / double(waves * kSMs);
-    const int64_t cmax = (chunks + S - 1) / S;
-    const double bal = (double(chunks) / double(S)) / double(cmax);
-    const double eff = fill * bal;
-    if (eff > best_eff + 1e-9) {
-      best_eff = eff;
-      best = (int)S;
-    }
-  }
-  return best;
-}
-
 // The K split of the CTA-pair kernel for widths 1..256: a function of (fmt, N, K) only.  A
 // work unit is one pair of 128-row tiles over K/S; kPairSMs units run at once.  The cost
 // model is (waves of units) x (chunks per unit) plus a small charge per split for the
@@ -171,17 +141,7 @@ int split_for_pair(int fmt, int64_t N, int64_t K) {
   return best;
 }
 
-bool use_one_sm() {
-  static int v = -1;
-  if (v < 0) {
-    const char* e = getenv("QGEMM_DEBUG_ONESM");
-    v = (e && e[0] == '1') ? 1 : 0;
-  }
-  return v == 1;
-}
-
 struct Plan {
-  bool pair;    // CTA-pair kernel
   int NACC;     // pair kernel: accumulators per subtile
   bool f16ops;  // widths <= 256
   int NB, R, NMAT, S, n_groups, b_tiles, chunks, XS, WS, AS, tmem_cols;
@@ -201,12 +161,15 @@ int next_pow2_cols(int c) {
 // arithmetic; NB, R and the ring depths are scheduling choices.
 bool make_plan_pair(int fmt, int64_t N, int64_t K, int64_t B, int nmat, Plan* pl) {
   Plan p{};
-  p.pair = true;
   p.NMAT = nmat;
+  // widths <= 256: f16 operands (x rescaled per row by the preparation kernel, which the GEMM
+  // overlaps as its programmatic dependent); above: bf16 straight from the caller.  f16 keeps
+  // the Q8_0 products q*d to one f16 rounding, and converts E2M1 codes in one instruction per
+  // pair (NVFP4 and MXFP4 weights are exact either way).
   p.f16ops = (B <= 256);
   p.chunks = (int)((K + chunk_k(fmt) - 1) / chunk_k(fmt));
   const int64_t pairs = (row_tiles(N) + 1) / 2;
-  if (p.f16ops) {
+  if (B <= 256) {
     // two accumulators per subtile (two concurrent MMA issuers), so NB <= 128 (64 fused)
     p.S = split_for_pair(fmt, N, K);
     p.NACC = 2;
@@ -255,87 +218,8 @@ bool make_plan_pair(int fmt, int64_t N, int64_t K, int64_t B, int nmat, Plan* pl
   return true;
 }
 
-// Chooses the tiling for one call.  Only S (and the operand type, by width class) affects
-// the arithmetic; NB, R and the ring depths are scheduling choices.
-bool make_plan_one_sm(int fmt, int64_t N, int64_t K, int64_t B, int nmat, Plan* pl) {
-  Plan p{};
-  p.NMAT = nmat;
-  p.f16ops = (B <= 256);
-  p.chunks = (int)((K + chunk_k(fmt) - 1) / chunk_k(fmt));
-  const int J = chunk_k(fmt) / kSubK;
-  const int64_t tiles = (N + kTileRows - 1) / kTileRows;
-  if (p.f16ops) {
-    p.S = split_for(fmt, N, K, nmat);
-    const int nb_cap = (nmat == 2) ? 128 : 256;
-    int nb = (int)std::min<int64_t>(((B + 15) / 16) * 16, nb_cap);
-    if (nmat == 2 && B > 128) nb = (int)(((B + 1) / 2 + 15) / 16 * 16);
-    p.NB = nb;
-  } else {
-    p.S = 1;
-    p.NB = (nmat == 2) ? 128 : 256;
-  }
-  p.b_tiles = (int)((B + p.NB - 1) / p.NB);
-  // subtiles per unit: TMEM holds R*NB accumulator columns plus the A ring (kMaxAStages
-  // stages, split evenly between the R subtiles' MMA issuers, so R divides kMaxAStages)
-  const int rmax = std::min(kMaxAStages, (512 - kMaxAStages * kAColsPerStage) / p.NB);
-  int bestR = 0;
-  int64_t best_cost = -1;
-  for (int R = nmat; R <= rmax; R *= 2) {
-    if (R % nmat) continue;
-    const int64_t groups = (tiles + (R / nmat) - 1) / (R / nmat);
-    const int64_t units = groups * p.b_tiles * p.S;
-    const int64_t cost = ((units + kSMs - 1) / kSMs) * R;
-    if (best_cost < 0 || cost <= best_cost) {
-      best_cost = cost;
-      bestR = R;
-    }
-  }
-  if (bestR == 0) return false;
-  // debug override (scheduling only: R never changes the arithmetic)
-  if (const char* e = getenv("QGEMM_DEBUG_R")) {
-    const int r = atoi(e);
-    if ((r == 1 || r == 2 || r == 4) && r % nmat == 0 && r <= rmax) bestR = r;
-  }
-  p.R = bestR;
-  p.n_groups = (int)((tiles + (p.R / nmat) - 1) / (p.R / nmat));
-  p.AS = kMaxAStages;
-  p.tmem_cols = next_pow2_cols(p.R * p.NB + p.AS * kAColsPerStage);
-  if (p.tmem_cols > 512) return false;
-  // shared memory: x ring, weight ring (gets the rest, up to 8 stages), barriers, control
-  const size_t xstage = (size_t)p.NB * 128;
-  const size_t misc = 8 * (2 * 16 + 2 * kMaxWStages + 2 * kMaxAStages + 1) + 16 + 4 * kMaxNB + 64;
-  const size_t budget = kSmemLimit - 1024 - misc;
-  // with several subtiles the x stages of a chunk stay resident until its last subtile
-  int XS = (p.R > 1) ? 2 * J : 4;
-  while (XS > J && XS * xstage + 2 * (size_t)kWStageBytes > budget) --XS;
-  if (XS * xstage + 2 * (size_t)kWStageBytes > budget) return false;
-  const int WS = (int)std::min<size_t>(kMaxWStages, (budget - XS * xstage) / kWStageBytes);
-  p.XS = XS;
-  p.WS = WS;
-  p.smem_x = 0;
-  p.smem_w = (uint32_t)(XS * xstage);
-  p.smem_bar = p.smem_w + (uint32_t)(WS * kWStageBytes);
-  const size_t bar_bytes = 8 * (2 * XS + 2 * WS + 2 * p.AS + 1);
-  p.smem_bytes = 1024 + p.smem_bar + bar_bytes + 16 + 4 * p.NB + 64;
-  // workspace: [xh f16 B*K][x_exp B][counters][split partials S*NMAT*B*N fp32]
-  size_t off = 0;
-  auto take = [&](size_t bytes) {
-    const size_t o = off;
-    off += (bytes + 255) / 256 * 256;
-    return o;
-  };
-  p.off_xh = p.f16ops ? take((size_t)B * pad64(K) * 2) : 0;
-  p.off_exp = p.f16ops ? take((size_t)B * 4) : 0;
-  p.off_cnt = 0;
-  p.off_ws = (p.S > 1) ? take((size_t)p.S * nmat * B * N * 4) : 0;
-  p.ws_total = off;
-  *pl = p;
-  return true;
-}
-
 bool make_plan(int fmt, int64_t N, int64_t K, int64_t B, int nmat, Plan* pl) {
-  return use_one_sm() ? make_plan_one_sm(fmt, N, K, B, nmat, pl)
-                      : make_plan_pair(fmt, N, K, B, nmat, pl);
+  return make_plan_pair(fmt, N, K, B, nmat, pl);
 }
 
 int run_impl(int fmt, const void* x, int64_t B, int64_t K, const void* const* codes,
@@ -376,7 +260,6 @@ int run_impl(int fmt, const void* x, int64_t B, int64_t K, const void* const* co
   }
   p.x_exp = pl.f16ops ? reinterpret_cast<const int*>(wsb + pl.off_exp) : nullptr;
   p.ws = (pl.S > 1) ? reinterpret_cast<float*>(wsb + pl.off_ws) : nullptr;
-  p.counters = nullptr;
   p.out = out;
   p.out_bf16 = out_bf16;
   p.dev_err = dev_err;
@@ -390,8 +273,6 @@ int run_impl(int fmt, const void* x, int64_t B, int64_t K, const void* const* co
     pp.B = (int)B;
     pp.K = (int)K;
     pp.Kp = (int)pad64(K);
-    pp.counters = nullptr;
-    pp.n_counters = 0;
     cudaError_t e = launch_prep(pp, stream);
     if (e != cudaSuccess) return cuda_fail(e, "prep kernel launch");
     xop = pp.xh;
@@ -401,20 +282,20 @@ int run_impl(int fmt, const void* x, int64_t B, int64_t K, const void* const* co
   const CUtensorMapDataType xdt =
       pl.f16ops ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const int64_t xpitch = pl.f16ops ? pad64(K) : K;  // elements per row of the x operand
-  p.x3d = (pl.pair && xpitch % 64 == 0) ? 1 : 0;
+  p.x3d = (xpitch % 64 == 0) ? 1 : 0;
   const bool mapped =
       p.x3d ? make_map3(&xmap, xdt, xop, (uint64_t)B, (uint64_t)xpitch, (uint32_t)(pl.NB / 2),
                         (uint32_t)(kPairAK / kSubK))
             : make_map(&xmap, xdt, 2, xop, (uint64_t)K, (uint64_t)B, (uint64_t)xpitch * 2, kSubK,
-                       (uint32_t)(pl.pair ? pl.NB / 2 : pl.NB), CU_TENSOR_MAP_SWIZZLE_128B);
+                       (uint32_t)(pl.NB / 2), CU_TENSOR_MAP_SWIZZLE_128B);
   if (!mapped) {
     snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled failed");
     return QGEMM_ERR_CUDA;
   }
   const int grid = pl.n_groups * pl.b_tiles * pl.S;
   if (g_prof_begin) cudaEventRecord(g_prof_begin, stream);
-  cudaError_t e = pl.pair ? launch_pair(fmt, !pl.f16ops, p, pl.smem_bytes, grid, &xmap, stream)
-                          : launch_tc(fmt, !pl.f16ops, p, pl.smem_bytes, grid, &xmap, stream);
+  // with f16 operands the GEMM follows the x preparation as its programmatic dependent
+  cudaError_t e = launch_pair(fmt, !pl.f16ops, p, pl.smem_bytes, grid, &xmap, pl.f16ops, stream);
   if (e != cudaSuccess) return cuda_fail(e, "gemm kernel launch");
   if (g_prof_end) cudaEventRecord(g_prof_end, stream);
   if (pl.S > 1) {
@@ -534,7 +415,7 @@ int qgemm_split_k(int fmt, int64_t N, int64_t K, int* splits) {
   const int st = check_fmt_shape(fmt, N, K);
   if (st != QGEMM_OK) return st;
   if (!splits) return QGEMM_ERR_NULL;
-  *splits = use_one_sm() ? split_for(fmt, N, K, 1) : split_for_pair(fmt, N, K);
+  *splits = split_for_pair(fmt, N, K);
   return QGEMM_OK;
 }
 

@@ -11,17 +11,8 @@ enum Fmt : int { FMT_Q8_0 = 0, FMT_NVFP4 = 1, FMT_MXFP4 = 2 };
 constexpr int kTileRows = 128;                    // weight rows per subtile (MMA M)
 constexpr int kWRowBytes = 128;                   // code bytes per row in one weight stage
 constexpr int kWCodeBytes = kTileRows * kWRowBytes;        // 16 KB, 128-byte swizzled
-constexpr int kScaleRowBytes = 16;                // scale bytes per row in one weight stage
-constexpr int kWStageBytes = kWCodeBytes + kTileRows * kScaleRowBytes;  // 18 KB
 constexpr int kSubK = 64;                         // K per x stage (one 128-byte swizzle atom)
-constexpr int kAStageK = 128;                     // K per A stage (TMEM)
-constexpr int kMaxAStages = 4;                    // A ring depth limit
 constexpr int kMaxWStages = 8;                    // weight ring depth limit
-constexpr int kAColsPerStage = kAStageK / 2;      // 16-bit elements, 2 per TMEM column
-constexpr int kDequantWarps = 8;                  // 2 per TMEM lane quarter
-constexpr int kMmaWarps = 4;                      // one MMA-issuing thread per weight subtile
-constexpr int kFirstDequantWarp = 1 + kMmaWarps;  // warp 0 is the TMA producer
-constexpr int kThreads = (1 + kMmaWarps + kDequantWarps) * 32;
 // CTA-pair kernel: warp 0 producer, warp 1 TMEM owner / pair MMA issuer, then dequant warps
 constexpr int kPairDequantWarps = 8;              // 2 per TMEM lane quarter
 constexpr int kPairFirstDequantWarp = 2;
@@ -92,7 +83,7 @@ struct GemmParams {
   int b_tiles;   // ceil(B / NB)
   int chunks;    // ceil(K / chunk_k)
   int XS, WS;    // x ring and weight ring depths
-  int AS;        // A ring depth (TMEM stages of kAStageK)
+  int AS;        // A ring depth (TMEM slots of kPairAK)
   int tmem_cols; // allocated TMEM columns
   int x3d;       // pair kernel: x map is 3-D {64, B, K/64} (one TMA load per x stage)
   int NACC;      // pair kernel: accumulators per subtile (1, or 2 for the f16 path)
@@ -102,7 +93,6 @@ struct GemmParams {
   const uint8_t* codes[2];   // tile-major packed codes of each matrix
   const uint8_t* scales[2];  // tile-major packed scales of each matrix
   float* ws;                 // split-K partials [S][NMAT][B][N]
-  int* counters;             // [n_groups * b_tiles], zero on entry, left zero
   void* out;                 // y [B][N] (fp32 or bf16), or h [B][N] bf16 for NMAT == 2
   int out_bf16;
   int* dev_err;
@@ -134,8 +124,6 @@ struct PrepParams {
   uint16_t* xh;       // f16 [B][Kp], columns K..Kp-1 zero
   int* x_exp;         // [B]
   int B, K, Kp;       // Kp: row pitch of xh in elements (K rounded up to 64)
-  int* counters;      // zeroed here (split-K arrival counters of the following GEMM)
-  int n_counters;
 };
 
 // Device error codes written to the library's error word.

@@ -225,9 +225,6 @@ __device__ __forceinline__ void store_h(const GemmParams& p, int b, int n, float
   reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)b * p.N + n] = __float2bfloat16_rn(silu * u);
 }
 
-__device__ __forceinline__ void named_bar_epilogue() {
-  asm volatile("bar.sync 1, %0;" ::"r"(kDequantWarps * 32) : "memory");
-}
 
 
 }  // namespace qg

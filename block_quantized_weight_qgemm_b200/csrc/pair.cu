@@ -110,12 +110,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     tmem_alloc_pair(smem_u32(ctl), (uint32_t)p.tmem_cols);
     tmem_relinquish_pair();
   }
-  if (warp >= kPairFirstDequantWarp && warp < kPairIssuer2Warp) {
-    for (int i = threadIdx.x - kPairFirstDequantWarp * 32; i < p.NB; i += kPairDequantWarps * 32) {
-      const int b = bt * p.NB + i;
-      col_fac[i] = (b < p.B) ? (p.x_exp ? ldexpf(1.0f, p.x_exp[b]) : 1.0f) : 0.0f;
-    }
-  }
   tc_fence_before();
   __syncthreads();
   cluster_sync_all();  // both CTAs' barriers are initialised before any remote arrive
@@ -138,6 +132,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       int x_issued = 0, w_issued = 0;
       int wg = 0, wr = 0;  // next weight stage (group, subtile)
       bool ok = true;
+      bool x_ready = false;  // the grid producing x (if any) has completed
       uint64_t idle_since = 0;
       while (ok && (w_issued < w_total || x_issued < x_total)) {
         bool progressed = false;
@@ -171,6 +166,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         if (x_issued < x_total &&
             (x_issued < XS || mbar_test_wait(bar_x_empty + 8 * xp.slot, xp.phase ^ 1u))) {
           const int cg = c0 + x_issued * CPA;
+          if (!x_ready) {
+            griddep_wait();
+            x_ready = true;
+          }
           const uint32_t dst = sx + (uint32_t)xp.slot * xstage;
           const uint32_t cbar = xbar0 + 8u * (uint32_t)xp.slot;
           const int row0 = bt * p.NB + (int)rank * half;
@@ -377,6 +376,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
     }
     tc_fence_after();
+    // the output may be read by a dependent grid only after it completes; let it launch
+    griddep_launch_dependents();
+    // per-column factors 2^x_exp[b] (f16 path) -- x_exp comes from the preceding grid
+    griddep_wait();
+    for (int i = threadIdx.x - kPairFirstDequantWarp * 32; i < p.NB; i += kPairDequantWarps * 32) {
+      const int b = bt * p.NB + i;
+      col_fac[i] = (b < p.B) ? (p.x_exp ? ldexpf(1.0f, p.x_exp[b]) : 1.0f) : 0.0f;
+    }
+    asm volatile("bar.sync 1, %0;" ::"r"(kPairDequantWarps * 32) : "memory");
     const int qcols = p.NB / kWPQ;  // columns per warp of a lane quarter (multiple of 4)
     const int cb0 = h * qcols;
     const size_t BN = (size_t)p.B * p.N;
@@ -488,27 +496,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 // ---------------------------------------------------------------------------------------
 template <int FMT, bool BF16OP>
 cudaError_t launch_pair_impl(const GemmParams& p, size_t smem_bytes, int units,
-                             const CUtensorMap* maps, cudaStream_t stream) {
+                             const CUtensorMap* maps, bool pdl, cudaStream_t stream) {
   auto kern = qgemm_pair_kernel<FMT, BF16OP>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem_bytes);
+  // raise the dynamic shared-memory limit once per instantiation (to the device maximum)
+  static int set_device = -1;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  kern<<<2 * units, kPairThreads, smem_bytes, stream>>>(p, maps[0]);
-  return cudaGetLastError();
+  if (set_device != dev) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
+    if (e != cudaSuccess) return e;
+    set_device = dev;
+  }
+  if (smem_bytes > (size_t)kSmemLimit) return cudaErrorInvalidValue;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(2 * units), 1, 1);
+  cfg.blockDim = dim3(kPairThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem_bytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, p, maps[0]);
 }
 
 cudaError_t launch_pair(int fmt, bool bf16op, const GemmParams& p, size_t smem_bytes, int units,
-                        const CUtensorMap* maps, cudaStream_t stream) {
+                        const CUtensorMap* maps, bool pdl, cudaStream_t stream) {
   switch (fmt) {
     case FMT_Q8_0:
-      return bf16op ? launch_pair_impl<FMT_Q8_0, true>(p, smem_bytes, units, maps, stream)
-                    : launch_pair_impl<FMT_Q8_0, false>(p, smem_bytes, units, maps, stream);
+      return bf16op ? launch_pair_impl<FMT_Q8_0, true>(p, smem_bytes, units, maps, pdl, stream)
+                    : launch_pair_impl<FMT_Q8_0, false>(p, smem_bytes, units, maps, pdl, stream);
     case FMT_NVFP4:
-      return bf16op ? launch_pair_impl<FMT_NVFP4, true>(p, smem_bytes, units, maps, stream)
-                    : launch_pair_impl<FMT_NVFP4, false>(p, smem_bytes, units, maps, stream);
+      return bf16op ? launch_pair_impl<FMT_NVFP4, true>(p, smem_bytes, units, maps, pdl, stream)
+                    : launch_pair_impl<FMT_NVFP4, false>(p, smem_bytes, units, maps, pdl, stream);
     default:
-      return bf16op ? launch_pair_impl<FMT_MXFP4, true>(p, smem_bytes, units, maps, stream)
-                    : launch_pair_impl<FMT_MXFP4, false>(p, smem_bytes, units, maps, stream);
+      return bf16op ? launch_pair_impl<FMT_MXFP4, true>(p, smem_bytes, units, maps, pdl, stream)
+                    : launch_pair_impl<FMT_MXFP4, false>(p, smem_bytes, units, maps, pdl, stream);
   }
 }
 

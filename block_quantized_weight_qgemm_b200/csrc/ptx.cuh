@@ -249,6 +249,17 @@ __host__ __device__ __forceinline__ uint32_t idesc_f16(bool bf16, uint32_t n) {
 }
 
 // ---------------------------------------------------------------------------------------
+// Programmatic dependent launch
+// ---------------------------------------------------------------------------------------
+// Wait until the grids this one depends on have completed and their writes are visible (a
+// no-op when the grid was launched without a programmatic dependency).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Allow the dependent grid on the stream to begin launching.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------------------
 // CTA pairs (thread-block clusters of 2) and the pair form of the tensor-core MMA
 // ---------------------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t cluster_ctarank() {

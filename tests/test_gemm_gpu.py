@@ -224,25 +224,3 @@ def test_run_ragged_k(fmt, B):
     y_ref = oracle.gemm(xb, case.Wd)
     err = norm_err(gpu_run(case, x), y_ref, xb, case.Wd)
     assert err <= TOL, err
-
-
-@pytest.mark.parametrize("fmt", FMTS)
-def test_subtile_count_does_not_change_results(fmt, monkeypatch):
-    # R (weight subtiles sharing each x tile, one MMA issuer each) is a scheduling choice:
-    # every R gives bit-identical results.  R = 4 with FP4 (two A stages per chunk) is the
-    # case where issuers must not share A slots.
-    case = Case(fmt, 1100, 1024, seed=15)
-    x = inputs.activations(64, 1024, seed=16)
-    xb = x_bits(x)
-    y_ref = oracle.gemm(xb, case.Wd)
-    outs = {}
-    for R in ("1", "2", "4"):
-        monkeypatch.setenv("QGEMM_DEBUG_R", R)
-        for B in (8, 64):
-            outs[(R, B)] = gpu_run(case, x[:B])
-    monkeypatch.delenv("QGEMM_DEBUG_R")
-    for B in (8, 64):
-        assert norm_err(outs[("1", B)], y_ref[:B], xb[:B], case.Wd) <= TOL
-        assert np.array_equal(outs[("1", B)], outs[("2", B)]), B
-        assert np.array_equal(outs[("1", B)], outs[("4", B)]), B
-    assert qgemm.device_status(reset=False) == qgemm.OK
