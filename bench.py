@@ -183,6 +183,23 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def max_over_ranks(v: float, device, world: int) -> float:
+    """The largest value of v over all ranks (every rank calls this, in the same order)."""
+    if world <= 1:
+        return float(v)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(bytes_per_rank_step: float, ms_max: float, world: int) -> float:
+    """Whole-job GB/s: every rank processes bytes_per_rank_step per step; the job's step time
+    is the slowest rank's."""
+    return world * bytes_per_rank_step / (ms_max * 1e-3) / 1e9
+
+
 def launches_per_call(fmt, N, K, B):
     """Kernels one qgemm_run launches: the x conversion (widths <= 256), the GEMM, and the
     split-K reduction when the K split is above 1."""
@@ -297,11 +314,8 @@ def main():
     k_bytes = sum(b for b, _ in per_launch) / len(per_launch)
     k_ms = sum(t for _, t in per_launch) / len(per_launch)
 
-    ms_t = torch.tensor([ms], device=dev)
-    if world > 1:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
-    value = world * step_bytes / (ms_max * 1e-3) / 1e9
+    ms_max = max_over_ranks(ms, dev, world)
+    value = job_rate(step_bytes, ms_max, world)
 
     # ---- end-to-end through the public API with host buffers ---------------------------
     hx = [c["x"].cpu().pin_memory() for c in calls]
@@ -330,10 +344,8 @@ def main():
         e2e_step(i)
     e1.record()
     torch.cuda.synchronize()
-    e_ms = torch.tensor([e0.elapsed_time(e1) / args.steps], device=dev)
-    if world > 1:
-        dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
-    e2e_value = world * step_bytes / (float(e_ms.item()) * 1e-3) / 1e9
+    e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev, world)
+    e2e_value = job_rate(step_bytes, e_ms, world)
 
     status = qgemm.device_status(reset=True)
 

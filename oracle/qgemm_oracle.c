@@ -224,8 +224,16 @@ static void put_nibble(uint8_t *row, int64_t k, unsigned code) {
     else *p = (uint8_t)((*p & 0x0Fu) | ((code & 0xFu) << 4));
 }
 
+/* ORC_MUTATE plants one known mistake (for the tests that show the pins catch it; the
+   library build never defines it): 1 nibble order, 2 dropped NVFP4 tensor scale,
+   3 dropped last term of each dot product, 4 Q8_0 scale bytes swapped. */
+#ifndef ORC_MUTATE
+#define ORC_MUTATE 0
+#endif
+
 static unsigned get_nibble(const uint8_t *row, int64_t k) {
     uint8_t b = row[k / 2];
+    if (ORC_MUTATE == 1) return (k % 2 == 0) ? (b >> 4) : (b & 0xFu);
     return (k % 2 == 0) ? (b & 0xFu) : (b >> 4);
 }
 
@@ -338,9 +346,12 @@ void orc_dequant(int fmt, const uint8_t *codes, const uint8_t *scales, float ts,
             double v;
             if (fmt == ORC_Q8_0) {
                 unsigned h = (unsigned)sr[2 * (k / 32)] | ((unsigned)sr[2 * (k / 32) + 1] << 8);
+                if (ORC_MUTATE == 4)
+                    h = (unsigned)sr[2 * (k / 32) + 1] | ((unsigned)sr[2 * (k / 32)] << 8);
                 v = (double)(int8_t)cr[k] * orc_f16(h);
             } else if (fmt == ORC_NVFP4) {
-                v = orc_e2m1(get_nibble(cr, k)) * orc_e4m3(sr[k / 16]) * (double)ts;
+                v = orc_e2m1(get_nibble(cr, k)) * orc_e4m3(sr[k / 16]) *
+                    (ORC_MUTATE == 2 ? 1.0 : (double)ts);
             } else {
                 v = orc_e2m1(get_nibble(cr, k)) * orc_e8m0(sr[k / 32]);
             }
@@ -368,7 +379,8 @@ static void *gemm_worker(void *arg) {
         for (int64_t b = 0; b < j->B; ++b) {
             const double *x = j->xd + b * j->K;
             double acc = 0.0;
-            for (int64_t k = 0; k < j->K; ++k) acc += x[k] * w[k];
+            const int64_t kend = (ORC_MUTATE == 3) ? j->K - 1 : j->K;
+            for (int64_t k = 0; k < kend; ++k) acc += x[k] * w[k];
             j->y[b * j->N + n] = acc;
         }
     }

@@ -6,6 +6,7 @@ Sources: values the pages print (golden fixtures), library float conversions
 (Q8_0 round-trip error <= scale/2).
 """
 import math
+import os
 import random
 from fractions import Fraction
 
@@ -405,3 +406,70 @@ def test_ffn_special_cases_and_rounding():
             # h is the bf16 value nearest to v: no neighbour is closer
             assert abs(Fraction(v) - hv) <= abs(Fraction(v) - Fraction(oracle.bf16(int(h[i, j]) + 1)))
             assert abs(Fraction(v) - hv) <= abs(Fraction(v) - lo)
+
+
+# --------------------------------------------------------------------------------------
+# the pins catch planted mistakes: each variant of the oracle is compiled with one known
+# error (ORC_MUTATE) and run through the same checks, which must now fail
+# --------------------------------------------------------------------------------------
+def _mutant(tmp_path, m):
+    import ctypes
+    import subprocess
+    src = os.path.join(os.path.dirname(oracle.__file__), "qgemm_oracle.c")
+    so = str(tmp_path / ("liboracle_mut%d.so" % m))
+    subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-std=c11", "-fno-fast-math",
+                           "-ffp-contract=off", "-pthread", "-DORC_MUTATE=%d" % m, src, "-o", so,
+                           "-lm"])
+    lib = ctypes.CDLL(so)
+    vp, i64 = ctypes.c_void_p, ctypes.c_int64
+    lib.orc_dequant.argtypes = [ctypes.c_int, vp, vp, ctypes.c_float, i64, i64, vp]
+    lib.orc_gemm.argtypes = [vp, i64, i64, vp, i64, vp, ctypes.c_int]
+    return lib
+
+
+def _dequant_with(lib, fmt, codes, scales, ts, N, K):
+    Wd = np.zeros((N, K), dtype=np.float64)
+    lib.orc_dequant(oracle.FORMATS[fmt], codes.ctypes.data, scales.ctypes.data, ts, N, K,
+                    Wd.ctypes.data)
+    return Wd
+
+
+def _hand_rows_hold(lib):
+    # the hand-built rows of test_dequant_hand_built_rows, through `lib`
+    K = 64
+    ok = True
+    codes = np.zeros((1, oracle.code_pitch("q8_0", K)), dtype=np.uint8)
+    scales = np.zeros((1, oracle.scale_pitch("q8_0", K)), dtype=np.uint8)
+    codes[0, 0] = 0x81
+    codes[0, 1] = 1
+    scales[0, 0:2] = [0x00, 0x3C]  # fp16 1.0
+    Wd = _dequant_with(lib, "q8_0", codes, scales, 1.0, 1, K)
+    ok &= bool(Wd[0, 0] == -127.0 and Wd[0, 1] == 1.0)
+    codes = np.zeros((1, oracle.code_pitch("nvfp4", K)), dtype=np.uint8)
+    scales = np.zeros((1, oracle.scale_pitch("nvfp4", K)), dtype=np.uint8)
+    codes[0, 0] = 0x7F
+    scales[0, 0] = 0x38
+    Wd = _dequant_with(lib, "nvfp4", codes, scales, 0.5, 1, K)
+    ok &= bool(Wd[0, 0] == -3.0 and Wd[0, 1] == 3.0)
+    return ok
+
+
+def _gemm_matches_fractions(lib):
+    N, K, B = 4, 32, 3
+    W = inputs.weights(N, K, seed=21).numpy()
+    codes, scales, ts = oracle.pack("q8_0", W)
+    Wd = oracle.dequant("q8_0", codes, scales, ts, N, K)
+    x16 = np.ascontiguousarray(inputs.bf16_bits(inputs.activations(B, K, seed=22)))
+    y = np.zeros((B, N), dtype=np.float64)
+    lib.orc_gemm(x16.ctypes.data, B, K, Wd.ctypes.data, N, y.ctypes.data, 1)
+    exact = _fraction_gemm(x16, Wd)
+    return all(abs(Fraction(float(y[b, n])) - exact[b][n]) <= Fraction(1e-12)
+               for b in range(B) for n in range(N))
+
+
+def test_pins_catch_planted_mistakes(tmp_path):
+    assert _hand_rows_hold(_mutant(tmp_path, 0)) and _gemm_matches_fractions(_mutant(tmp_path, 0))
+    assert not _hand_rows_hold(_mutant(tmp_path, 1))        # nibble order swapped
+    assert not _hand_rows_hold(_mutant(tmp_path, 2))        # NVFP4 tensor scale dropped
+    assert not _gemm_matches_fractions(_mutant(tmp_path, 3))  # last term of each sum dropped
+    assert not _hand_rows_hold(_mutant(tmp_path, 4))        # Q8_0 scale bytes swapped
