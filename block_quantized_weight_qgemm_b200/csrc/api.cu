@@ -120,19 +120,24 @@ int device_ok() {
 }
 
 // The K split of the CTA-pair kernel for widths 1..256: a function of (fmt, N, K) only.  A
-// work unit is one pair of 128-row tiles over K/S; kPairSMs units run at once.  The cost
-// model is (waves of units) x (chunks per unit) plus a small charge per split for the
-// partials the reduction reads; the smallest S of least cost wins.
+// work unit is one pair of 128-row tiles over K/S; kPairSMs units run at once.  A unit costs
+// its A slots (kPairAK elements of K each) plus a fixed cost of about kUnitOverheadSlots slots
+// (set-up, the first weight latency, the MMA tail and the epilogue, measured); the time of a
+// split is (waves of units) x (cost per unit), plus a small charge per split for the
+// partials the reduction reads.  The smallest S of least cost wins.
+constexpr int kUnitOverheadSlots = 6;
+
 int split_for_pair(int fmt, int64_t N, int64_t K) {
   const int64_t chunks = (K + chunk_k(fmt) - 1) / chunk_k(fmt);
+  const int64_t cpa = kPairAK / chunk_k(fmt);  // chunks per A slot
   const int64_t pairs = (row_tiles(N) + 1) / 2;
   int best = 1;
   double best_cost = 0.0;
   const int64_t smax = std::min<int64_t>(16, chunks);
   for (int64_t S = 1; S <= smax; ++S) {
     const int64_t waves = (pairs * S + kPairSMs - 1) / kPairSMs;
-    const int64_t cmax = (chunks + S - 1) / S;
-    const double cost = double(waves * cmax) + 0.3 * double(S);
+    const int64_t slots = ((chunks + S - 1) / S + cpa - 1) / cpa;
+    const double cost = double(waves * (slots + kUnitOverheadSlots)) + 0.3 * double(S);
     if (S == 1 || cost < best_cost - 1e-9) {
       best_cost = cost;
       best = (int)S;

@@ -97,8 +97,8 @@ def test_split_rule_depends_only_on_shape(lib):
         assert 1 <= s <= 16
     assert got[("q8_0", 17408, 5120)] == 1
     assert got[("nvfp4", 17408, 5120)] == 1
-    assert got[("q8_0", 5120, 17408)] == 7
-    assert got[("nvfp4", 5120, 17408)] == 7
+    assert got[("q8_0", 5120, 17408)] == 3
+    assert got[("nvfp4", 5120, 17408)] == 3
     # workspace grows with B but the split does not
     w64 = qgemm.workspace_size("q8_0", 5120, 17408, 64)
     w65 = qgemm.workspace_size("q8_0", 5120, 17408, 65)

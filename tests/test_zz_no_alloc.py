@@ -35,7 +35,7 @@ def _vp(t):
 
 def test_oversize_shape_is_refused_before_device_work(lib):
     # needs no GPU: the size check comes before any device call
-    fmt, N, K, B = 0, 5120, 17408, 256
+    fmt, N, K, B = 0, 8192, 65536, 256  # the f16 copy of x alone is 32 MiB
     need = qgemm.workspace_size("q8_0", N, K, B)
     assert need > SCRATCH_BYTES
     st = lib.qgemm_run_noalloc(fmt, 256, B, K, 256, 256, None, N, 256, 0, None)
