@@ -371,20 +371,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       }
     }
 
-    if (ok) {
-      ok = mbar_wait(bar_acc, 0, abort_flag, p.dev_err, kErrTimeout);
-      ok = __all_sync(0xffffffffu, ok);
-    }
-    tc_fence_after();
     // the output may be read by a dependent grid only after it completes; let it launch
     griddep_launch_dependents();
-    // per-column factors 2^x_exp[b] (f16 path) -- x_exp comes from the preceding grid
+    // per-column factors 2^x_exp[b] (f16 path); x_exp comes from the preceding grid.  Loaded
+    // before the accumulator wait so that their latency hides behind the last MMAs.
     griddep_wait();
     for (int i = threadIdx.x - kPairFirstDequantWarp * 32; i < p.NB; i += kPairDequantWarps * 32) {
       const int b = bt * p.NB + i;
       col_fac[i] = (b < p.B) ? (p.x_exp ? ldexpf(1.0f, p.x_exp[b]) : 1.0f) : 0.0f;
     }
     asm volatile("bar.sync 1, %0;" ::"r"(kPairDequantWarps * 32) : "memory");
+    if (ok) {
+      ok = mbar_wait(bar_acc, 0, abort_flag, p.dev_err, kErrTimeout);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    tc_fence_after();
     const int qcols = p.NB / kWPQ;  // columns per warp of a lane quarter (multiple of 4)
     const int cb0 = h * qcols;
     const size_t BN = (size_t)p.B * p.N;
