@@ -21,29 +21,64 @@ __device__ int g_dev_err = 0;
 // row's exponent e, which the GEMM epilogue restores.  Rows of xh are padded with zeros to
 // a multiple of 64 elements.
 // ---------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) qgemm_prep_x_kernel(const PrepParams p) {
+constexpr int kPrepThreads = 1024;  // one CTA per x row
+constexpr int kPrepRegs = 3;        // 16-byte words per thread held in registers (rows to 24576)
+
+__device__ __forceinline__ float amax8(float m, const uint4& v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    m = fmaxf(m, fabsf(__uint_as_float(w[i] << 16)));
+    m = fmaxf(m, fabsf(__uint_as_float(w[i] & 0xFFFF0000u)));
+  }
+  return m;
+}
+
+__device__ __forceinline__ uint4 to_f16x8(const uint4& v, float sc) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __half lo = __float2half_rn(__uint_as_float(w[i] << 16) * sc);
+    const __half hi = __float2half_rn(__uint_as_float(w[i] & 0xFFFF0000u) * sc);
+    o[i] = (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+__global__ void __launch_bounds__(kPrepThreads) qgemm_prep_x_kernel(const PrepParams p) {
   // the GEMM that follows may start its set-up and weight streaming now; it waits for this
   // grid before it reads xh or x_exp
   griddep_launch_dependents();
+  // x may come from the grid before this one, which may also still read xh and x_exp
+  griddep_wait();
   const int b = blockIdx.x;
   const uint16_t* xr = p.x + (size_t)b * p.K;
-  __shared__ float red[8];
+  __shared__ float red[kPrepThreads / 32];
+  // one pass over the row: the first kPrepRegs words of each thread stay in registers, any
+  // longer tail is read again for the conversion
+  uint4 v[kPrepRegs];
   float amax = 0.f;
-  for (int k = threadIdx.x * 8; k < p.K; k += blockDim.x * 8) {
-    const uint4 v = *reinterpret_cast<const uint4*>(xr + k);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      amax = fmaxf(amax, fabsf(__uint_as_float(w[i] << 16)));
-      amax = fmaxf(amax, fabsf(__uint_as_float(w[i] & 0xFFFF0000u)));
-    }
+  for (int j = 0; j < kPrepRegs; ++j) {
+    const int k = (threadIdx.x + j * kPrepThreads) * 8;
+    v[j] = (k < p.K) ? *reinterpret_cast<const uint4*>(xr + k) : make_uint4(0u, 0u, 0u, 0u);
+    amax = amax8(amax, v[j]);
   }
+  for (int k = (threadIdx.x + kPrepRegs * kPrepThreads) * 8; k < p.K; k += kPrepThreads * 8)
+    amax = amax8(amax, *reinterpret_cast<const uint4*>(xr + k));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
   __syncthreads();
+  if (threadIdx.x < 32) {
+    float m = red[threadIdx.x];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (threadIdx.x == 0) red[0] = m;
+  }
+  __syncthreads();
   amax = red[0];
-  for (int i = 1; i < (int)(blockDim.x >> 5); ++i) amax = fmaxf(amax, red[i]);
   int e = 0;
   if (amax > 0.f && amax <= 3.4e38f) {
     int ex;
@@ -52,20 +87,15 @@ __global__ void __launch_bounds__(256) qgemm_prep_x_kernel(const PrepParams p) {
   }
   const float sc = ldexpf(1.0f, -e);
   uint16_t* xo = p.xh + (size_t)b * p.Kp;
-  for (int k = p.K + threadIdx.x * 8; k < p.Kp; k += blockDim.x * 8)
-    *reinterpret_cast<uint4*>(xo + k) = make_uint4(0u, 0u, 0u, 0u);
-  for (int k = threadIdx.x * 8; k < p.K; k += blockDim.x * 8) {
-    const uint4 v = *reinterpret_cast<const uint4*>(xr + k);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    uint32_t o[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const __half lo = __float2half_rn(__uint_as_float(w[i] << 16) * sc);
-      const __half hi = __float2half_rn(__uint_as_float(w[i] & 0xFFFF0000u) * sc);
-      o[i] = (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
-    }
-    *reinterpret_cast<uint4*>(xo + k) = make_uint4(o[0], o[1], o[2], o[3]);
+  for (int j = 0; j < kPrepRegs; ++j) {
+    const int k = (threadIdx.x + j * kPrepThreads) * 8;
+    if (k < p.K) *reinterpret_cast<uint4*>(xo + k) = to_f16x8(v[j], sc);
   }
+  for (int k = (threadIdx.x + kPrepRegs * kPrepThreads) * 8; k < p.K; k += kPrepThreads * 8)
+    *reinterpret_cast<uint4*>(xo + k) = to_f16x8(*reinterpret_cast<const uint4*>(xr + k), sc);
+  for (int k = p.K + threadIdx.x * 8; k < p.Kp; k += kPrepThreads * 8)
+    *reinterpret_cast<uint4*>(xo + k) = make_uint4(0u, 0u, 0u, 0u);
   if (threadIdx.x == 0) p.x_exp[b] = e;
 }
 
@@ -74,6 +104,7 @@ __global__ void __launch_bounds__(256) qgemm_prep_x_kernel(const PrepParams p) {
 // 4-wide column group (b, n..n+3) per thread.
 // ---------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) qgemm_splitk_reduce_kernel(const ReduceParams p) {
+  griddep_launch_dependents();  // the next call's preparation may launch and wait
   griddep_wait();  // launched as a programmatic dependent of the GEMM that wrote the partials
   const int64_t nq = (p.N + 3) / 4;
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -153,8 +184,18 @@ cudaError_t launch_reduce(const ReduceParams& rp, cudaStream_t stream) {
 cudaError_t launch_prep(const PrepParams& pp, cudaStream_t stream) {
   static const bool once = (prefer_max_shared((const void*)qgemm_prep_x_kernel), true);
   (void)once;
-  qgemm_prep_x_kernel<<<pp.B, 256, 0, stream>>>(pp);
-  return cudaGetLastError();
+  // a programmatic dependent of whatever precedes it: it launches early and waits for that
+  // grid (griddepcontrol.wait) before it reads x or writes the workspace
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)pp.B, 1, 1);
+  cfg.blockDim = dim3(kPrepThreads, 1, 1);
+  cfg.stream = stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, qgemm_prep_x_kernel, pp);
 }
 
 }  // namespace qg
