@@ -17,7 +17,8 @@ constexpr int kMaxWStages = 8;                    // weight ring depth limit
 constexpr int kPairDequantWarps = 8;              // 2 per TMEM lane quarter
 constexpr int kPairFirstDequantWarp = 2;
 constexpr int kPairIssuer2Warp = kPairFirstDequantWarp + kPairDequantWarps;  // second MMA issuer
-constexpr int kPairThreads = (kPairIssuer2Warp + 1) * 32;
+constexpr int kPairXWarp = kPairIssuer2Warp + 1;  // x producer
+constexpr int kPairThreads = (kPairXWarp + 1) * 32;
 constexpr int kPairSMs = 74;                      // CTA pairs resident at once (148 SMs)
 constexpr int kPairAK = 256;                      // K per A slot of the pair kernel
 constexpr int kPairACols = kPairAK / 2;           // its TMEM columns

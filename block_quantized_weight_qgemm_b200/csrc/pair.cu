@@ -14,11 +14,11 @@
 //     memory, [NB/2, NB) in the odd CTA's, both loaded by TMA in the 128-byte swizzle.
 //     Each CTA's TMEM receives the fp32 accumulator of its own 128 rows x all NB columns.
 //   * Warp roles per CTA: warp 0 lane 0 streams packed weight stages (1-D bulk copies, the
-//     tile-major layout makes each stage contiguous) and x stages (tiled TMA whose byte
-//     count lands on the even CTA's barrier); warp 1 allocates TMEM and, with warp 10, issues
-//     the pair MMAs from the even CTA (alternate A slots, one MMA order); warps 2..9
-//     dequantize weight stages from shared memory into the TMEM A ring (tcgen05.st) and run
-//     the epilogue.
+//     tile-major layout makes each stage contiguous); warp 11 lane 0 streams x stages (tiled
+//     TMA whose byte count lands on the even CTA's barrier); warp 1 allocates TMEM and, with
+//     warp 10, issues the pair MMAs from the even CTA (two accumulators, alternate A-slot
+//     groups); warps 2..9 dequantize weight stages from shared memory into the TMEM A ring
+//     (tcgen05.st) and run the epilogue.
 //   * K is split into S contiguous ranges, S fixed by (format, N, K).  Partials are summed
 //     in the fixed order s = 0..S-1 by the reduce kernel; nothing in the arithmetic depends
 //     on the batch width, so row b of y is bit-identical for every width up to 256.
@@ -117,96 +117,49 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   const uint32_t tmem = static_cast<uint32_t>(ctl[0]);
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    // Two independent streams polled without blocking: this CTA's weight stages in the
-    // order (A slot group, subtile, chunk) into its own ring, and its half of x for each
-    // group (CPA chunks = 4 slices of 64 K elements) into the x ring.  The x bytes of both
-    // CTAs count on the even CTA's x barrier, which the even CTA's producer arms with the
-    // pair's total.
+    // ------------------------------------------------------------ weight producer
+    // This CTA's weight stages in the order (A-slot group, subtile) into its own ring: one
+    // bulk copy of the group's codes and one of its scales per stage, completing on the
+    // CTA's own barrier.  The thread does nothing else, so no other wait delays the stream.
     if (lane == 0) {
       const uint64_t pol_w = policy_evict_first();
-      const uint64_t pol_x = policy_evict_last();
-      const uint32_t xbar0 = mapa_shared(bar_x_full, 0);  // even CTA's x_full[0]
-      const int w_total = ngroups * p.R, x_total = ngroups;
-      RingPos xp, wp;
-      int x_issued = 0, w_issued = 0;
+      const int w_total = ngroups * p.R;
+      RingPos wp;
+      int w_issued = 0;
       int wg = 0, wr = 0;  // next weight stage (group, subtile)
       bool ok = true;
-      bool x_ready = false;  // the grid producing x (if any) has completed
-      uint64_t idle_since = 0;
-      while (ok && (w_issued < w_total || x_issued < x_total)) {
-        bool progressed = false;
-        if (w_issued < w_total &&
-            (w_issued < WS || mbar_test_wait(bar_w_empty + 8 * wp.slot, wp.phase ^ 1u))) {
-          // one stage: the group's n chunks of this subtile's tile, codes then scales
-          const uint32_t fb = bar_w_full + 8 * wp.slot;
-          const int m = (p.NMAT == 2) ? (wr & 1) : 0;
-          const int64_t t = 2 * ((int64_t)g * tpg + wr / p.NMAT) + rank;
-          const int cg = c0 + wg * CPA;
-          const int n = min(CPA, c1 - cg);
-          const uint32_t dst = sw + (uint32_t)(wp.slot * WSTAGE);
-          if (t < n_row_tiles) {
-            const int64_t blk = t * p.chunks + cg;
-            const uint32_t cbytes = (uint32_t)n * kWCodeBytes;
-            const uint32_t sbytes = (uint32_t)n * (kTileRows * SB);
-            mbar_arrive_expect_tx(fb, cbytes + sbytes);
-            bulk_load(dst, p.codes[m] + blk * kWCodeBytes, cbytes, fb, pol_w);
-            bulk_load(dst + WSCALES, p.scales[m] + blk * (kTileRows * SB), sbytes, fb, pol_w);
-          } else {
-            mbar_arrive(fb);  // a tile past the matrix: its rows are never stored
-          }
-          wp.next(WS);
-          ++w_issued;
-          if (++wr == p.R) {
-            wr = 0;
-            ++wg;
-          }
-          progressed = true;
+      while (w_issued < w_total) {
+        if (w_issued >= WS &&
+            !mbar_wait(bar_w_empty + 8 * wp.slot, wp.phase ^ 1u, abort_flag, p.dev_err,
+                       kErrTimeout)) {
+          ok = false;
+          break;
         }
-        if (x_issued < x_total &&
-            (x_issued < XS || mbar_test_wait(bar_x_empty + 8 * xp.slot, xp.phase ^ 1u))) {
-          const int cg = c0 + x_issued * CPA;
-          if (!x_ready) {
-            griddep_wait();
-            x_ready = true;
-          }
-          const uint32_t dst = sx + (uint32_t)xp.slot * xstage;
-          const uint32_t cbar = xbar0 + 8u * (uint32_t)xp.slot;
-          const int row0 = bt * p.NB + (int)rank * half;
-          if (p.x3d) {
-            // one box of 4 slices (slices past K read zeros from the padded rows or the
-            // out-of-range fill)
-            if (rank == 0) mbar_arrive_expect_tx(bar_x_full + 8 * xp.slot, 2u * xstage);
-            tma_load_3d_pair(dst, &tm_x, cbar, 0, row0, cg * KW / kSubK, pol_x);
-          } else {
-            const int nsl = min(CPA, c1 - cg) * J;  // slices in this group
-            if (rank == 0)
-              mbar_arrive_expect_tx(bar_x_full + 8 * xp.slot, 2u * xslice * (uint32_t)nsl);
-            for (int j = 0; j < nsl; ++j)
-              tma_load_2d_pair(dst + (uint32_t)j * xslice, &tm_x, cbar, cg * KW + j * kSubK, row0,
-                               pol_x);
-          }
-          xp.next(XS);
-          ++x_issued;
-          progressed = true;
-        }
-        if (progressed) {
-          idle_since = 0;
+        const uint32_t fb = bar_w_full + 8 * wp.slot;
+        const int m = (p.NMAT == 2) ? (wr & 1) : 0;
+        const int64_t t = 2 * ((int64_t)g * tpg + wr / p.NMAT) + rank;
+        const int cg = c0 + wg * CPA;
+        const int n = min(CPA, c1 - cg);
+        const uint32_t dst = sw + (uint32_t)(wp.slot * WSTAGE);
+        if (t < n_row_tiles) {
+          const int64_t blk = t * p.chunks + cg;
+          const uint32_t cbytes = (uint32_t)n * kWCodeBytes;
+          const uint32_t sbytes = (uint32_t)n * (kTileRows * SB);
+          mbar_arrive_expect_tx(fb, cbytes + sbytes);
+          bulk_load(dst, p.codes[m] + blk * kWCodeBytes, cbytes, fb, pol_w);
+          bulk_load(dst + WSCALES, p.scales[m] + blk * (kTileRows * SB), sbytes, fb, pol_w);
         } else {
-          const uint64_t now = globaltimer_ns();
-          if (idle_since == 0) idle_since = now;
-          if (*abort_flag) ok = false;
-          if (now - idle_since > kWaitLimitNs) {
-            *abort_flag = 1;
-            atomicExch(p.dev_err, kErrTimeout);
-            ok = false;
-          }
-          __nanosleep(20);
+          mbar_arrive(fb);  // a tile past the matrix: its rows are never stored
+        }
+        wp.next(WS);
+        ++w_issued;
+        if (++wr == p.R) {
+          wr = 0;
+          ++wg;
         }
       }
       if (!ok) {
-        // let this CTA's weight loads land before it leaves (their barrier is local); the
-        // x loads complete on the even CTA's barrier, so give them a fixed grace period
+        // let this CTA's weight loads land before it leaves (their barrier is local)
         for (int k = 0; k < WS && k < w_issued; ++k) {
           wp.slot = (wp.slot == 0) ? WS - 1 : wp.slot - 1;
           if (wp.slot == WS - 1) wp.phase ^= 1u;
@@ -215,6 +168,49 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                  globaltimer_ns() - t0 < kWaitLimitNs) {
           }
         }
+      }
+    }
+    __syncwarp();
+  } else if (warp == kPairXWarp) {
+    // ------------------------------------------------------------ x producer
+    // This CTA's half of x for each A-slot group (4 slices of 64 K elements) into the x ring.
+    // The bytes of both CTAs count on the even CTA's x barrier, which the even CTA arms with
+    // the pair's total.  x comes from the preceding grid (the preparation kernel), so the
+    // first load waits for it.
+    if (lane == 0) {
+      const uint64_t pol_x = policy_evict_last();
+      const uint32_t xbar0 = mapa_shared(bar_x_full, 0);  // even CTA's x_full[0]
+      RingPos xp;
+      bool ok = true;
+      griddep_wait();
+      for (int x_issued = 0; x_issued < ngroups; ++x_issued) {
+        if (x_issued >= XS &&
+            !mbar_wait(bar_x_empty + 8 * xp.slot, xp.phase ^ 1u, abort_flag, p.dev_err,
+                       kErrTimeout)) {
+          ok = false;
+          break;
+        }
+        const int cg = c0 + x_issued * CPA;
+        const uint32_t dst = sx + (uint32_t)xp.slot * xstage;
+        const uint32_t cbar = xbar0 + 8u * (uint32_t)xp.slot;
+        const int row0 = bt * p.NB + (int)rank * half;
+        if (p.x3d) {
+          // one box of 4 slices (slices past K read zeros from the padded rows or the
+          // out-of-range fill)
+          if (rank == 0) mbar_arrive_expect_tx(bar_x_full + 8 * xp.slot, 2u * xstage);
+          tma_load_3d_pair(dst, &tm_x, cbar, 0, row0, cg * KW / kSubK, pol_x);
+        } else {
+          const int nsl = min(CPA, c1 - cg) * J;  // slices in this group
+          if (rank == 0)
+            mbar_arrive_expect_tx(bar_x_full + 8 * xp.slot, 2u * xslice * (uint32_t)nsl);
+          for (int j = 0; j < nsl; ++j)
+            tma_load_2d_pair(dst + (uint32_t)j * xslice, &tm_x, cbar, cg * KW + j * kSubK, row0,
+                             pol_x);
+        }
+        xp.next(XS);
+      }
+      if (!ok) {
+        // the x loads complete on the even CTA's barrier: give them a fixed grace period
         const uint64_t t0 = globaltimer_ns();
         while (globaltimer_ns() - t0 < 200000) __nanosleep(1000);
       }
