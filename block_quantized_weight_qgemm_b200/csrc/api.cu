@@ -175,10 +175,11 @@ bool make_plan_pair(int fmt, int64_t N, int64_t K, int64_t B, int nmat, Plan* pl
   p.chunks = (int)((K + chunk_k(fmt) - 1) / chunk_k(fmt));
   const int64_t pairs = (row_tiles(N) + 1) / 2;
   if (B <= 256) {
-    // two accumulators per subtile (two concurrent MMA issuers), so NB <= 128 (64 fused)
+    // plain GEMM: two accumulators per subtile (two concurrent MMA issuers), so NB <= 128;
+    // fused gate+up: one accumulator per matrix, one issuer per matrix
     p.S = split_for_pair(fmt, N, K);
-    p.NACC = 2;
-    const int nb_cap = (nmat == 2) ? 64 : 128;
+    p.NACC = (nmat == 2) ? 1 : 2;
+    const int nb_cap = 128;
     const int64_t tiles_b = (B + nb_cap - 1) / nb_cap;  // balanced batch tiles
     p.NB = (int)std::min<int64_t>(((B + tiles_b - 1) / tiles_b + 15) / 16 * 16, nb_cap);
   } else {
@@ -190,7 +191,10 @@ bool make_plan_pair(int fmt, int64_t N, int64_t K, int64_t B, int nmat, Plan* pl
   p.R = nmat;
   p.n_groups = (int)pairs;
   p.AS = std::min(4, (512 - p.R * p.NACC * p.NB) / kPairACols);
-  if (p.AS < 2) return false;
+  // an issuer's consecutive A slots lie at most 2 apart in the ring (plain GEMM with two
+  // accumulators: alternate groups of one slot; fused: alternate slots), so AS >= 2 keeps a
+  // slot's previous use complete before its issuer waits for it
+  if (p.AS < 2 || (nmat == 1 && p.NACC == 2 && p.R != 1)) return false;
   p.tmem_cols = next_pow2_cols(p.R * p.NACC * p.NB + p.AS * kPairACols);
   if (p.tmem_cols > 512) return false;
   const size_t xstage = (size_t)(p.NB / 2) * 128 * (kPairAK / kSubK);

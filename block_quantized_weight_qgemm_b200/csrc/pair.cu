@@ -91,7 +91,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     prefetch_tmap(&tm_x);
     for (int i = 0; i < XS; ++i) {
       mbar_init(bar_x_full + 8 * i, 1);   // the even CTA's producer arrives (expect_tx)
-      mbar_init(bar_x_empty + 8 * i, 1);  // the commit of the group's issuer
+      mbar_init(bar_x_empty + 8 * i, (p.NMAT == 2) ? 2u : 1u);  // each issuer using the group
     }
     for (int i = 0; i < WS; ++i) {
       mbar_init(bar_w_full + 8 * i, 1);
@@ -219,22 +219,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   } else if (warp == 1 || warp == kPairIssuer2Warp) {
     // ------------------------------------------------------------ pair MMA issuers
     // One tcgen05.mma takes its issuing thread about as long as the tensor pipe needs for
-    // an N=128 tile, so at small N the issue rate, not the pipe, bounds the MMA stream.  With
-    // NACC = 2 two threads of the even CTA issue concurrently, each into its own accumulators:
-    // issuer e takes the A-slot groups gi with gi % 2 == e (every subtile of the group) and
-    // accumulates them into D[i][e]; the epilogue adds D[i][0] + D[i][1].  Within each
-    // accumulator the K slices arrive in ascending order.  For each of its groups an issuer
-    // waits for the pair's x stage, then per subtile for the A slot (a_full counts both CTAs'
-    // dequant warps), issues the slot's K=16 MMAs and releases the slot to both CTAs with a
-    // multicast commit; the x stage is released after the group's last subtile.
+    // an N=128 tile, so at small N the issue rate, not the pipe, bounds the MMA stream.  Two
+    // threads of the even CTA therefore issue concurrently, each into its own accumulators:
+    //   * plain GEMM, NACC = 2: issuer e takes the A-slot groups gi with gi % 2 == e and
+    //     accumulates them into D[i][e]; the epilogue adds D[i][0] + D[i][1];
+    //   * fused gate+up (NMAT = 2, NACC = 1): issuer e takes matrix e's subtiles (gate or up),
+    //     one accumulator each;
+    //   * NACC = 1 plain GEMM (widths > 256): issuer 0 alone.
+    // An issuer's consecutive slots are at most AS apart in the A ring (AS >= 2 for the
+    // first two; the planner checks), so a slot's previous use has always completed when
+    // its issuer waits for it.  Within each accumulator the K slices arrive in ascending
+    // order.  Per slot: wait for the A slot (a_full counts both CTAs' dequant warps), issue
+    // its K=16 MMAs, release it to both CTAs with a multicast commit; per group: wait for
+    // the pair's x stage first and release it after the issuer's last slot of the group.
     const int e = (warp == 1) ? 0 : 1;
-    if (rank == 0 && lane == 0 && e < p.NACC) {
+    const bool by_matrix = (p.NMAT == 2);
+    if (rank == 0 && lane == 0 && (by_matrix || e < p.NACC)) {
       const uint32_t idesc = idesc_f16_pair(BF16OP, (uint32_t)p.NB);
       RingPos xc;  // x stage of the current group
       RingPos ap;  // A ring
       bool ok = true;
       for (int gi = 0; gi < ngroups && ok; ++gi) {
-        if (gi % p.NACC != e) {
+        if (!by_matrix && gi % p.NACC != e) {
           // another issuer's group: keep the ring positions in step
           for (int i = 0; i < p.R; ++i) ap.next(AS);
           xc.next(XS);
@@ -246,15 +252,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           break;
         const uint32_t xbase = sx + (uint32_t)xc.slot * xstage;
         for (int i = 0; i < p.R; ++i) {
+          if (by_matrix && (i & 1) != e) {  // the other matrix's slot
+            ap.next(AS);
+            continue;
+          }
           if (!mbar_wait_spin(bar_a_full + 8 * ap.slot, ap.phase, false, abort_flag, p.dev_err,
                               kErrTimeout)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t d = tmem + (uint32_t)((i * p.NACC + e) * p.NB);
+          const int acc_i = by_matrix ? i : i * p.NACC + e;
+          const uint32_t d = tmem + (uint32_t)(acc_i * p.NB);
           const uint32_t a = tmem + a_col0 + (uint32_t)(ap.slot * kPairACols);
-          const bool first = (gi < p.NACC);  // this accumulator's first group
+          const bool first = by_matrix ? (gi == 0) : (gi < p.NACC);  // accumulator's first group
 #pragma unroll 4
           for (int ks = 0; ks < ksteps; ++ks) {
             const uint32_t bx = xbase + (uint32_t)(ks >> 2) * xslice + (uint32_t)((ks & 3) * 32);

@@ -129,3 +129,23 @@ def test_mxfp4_serving_mix():
         rows = inputs.sample_rows(8192)
         _check_rows(case, yp, inputs.bf16_bits(xp.cpu()), rows)
         del case
+
+
+@pytest.mark.parametrize("fmt", ["q8_0", "nvfp4"])
+def test_ffn_gate_up_decode_widths_27b(fmt):
+    """The fused gate+up at the 27B gate/up shape and decode widths: every unit holds many
+    A-slot groups, so both MMA issuers alternate through the A ring many times."""
+    cg = Case(fmt, INTER, HIDDEN, seed=inputs.W_SEED)
+    cu = Case(fmt, INTER, HIDDEN, seed=inputs.W2_SEED)
+    x = inputs.activations(65, HIDDEN, seed=inputs.X_SEED).cuda()
+    full = bf16_bits_of(qgemm.ffn_gate_up(x, cg.pw, cu.pw))
+    torch.cuda.synchronize()
+    assert qgemm.device_status(reset=False) == qgemm.OK
+    rows = [0, 1, 15, 16, 63, 64]
+    xb = inputs.bf16_bits(x.cpu())[rows]
+    g, u, _ = oracle.ffn_gate_up(xb, cg.Wd, cu.Wd)
+    bad, worst = h_bound_violations(full[rows], g, u, xb, cg.Wd, cu.Wd)
+    assert bad == 0, "%d outputs outside the bound (worst ratio %.3g)" % (bad, worst)
+    for M in (1, 16, 64):
+        h = bf16_bits_of(qgemm.ffn_gate_up(x[:M], cg.pw, cu.pw))
+        assert np.array_equal(h, full[:M]), "width %d differs from width 65" % M
