@@ -1,11 +1,11 @@
 """Benchmark of the block-quantized-weight GEMM hot path on B200.
 
-Default workload (one "step"): the Q8_0 27B FFN at decode width B = 64 -- qgemm_run on the
-gate [17408, 5120], up [17408, 5120] and down [5120, 17408] matrices, fp32 outputs.  Steps
-are timed as replays of a CUDA graph holding the three calls.  The
-metric is weight GB/s: packed weight bytes read per step / step time (the pages' weight-
-streaming bound for widths <= 64).  Weights cycle through a ring of distinct copies so that
-no step finds its weights in L2.
+Default workload (one "step"): the Q8_0 27B FFN at decode width B = 64 -- h = bf16(SiLU(x Wg^T)
+* (x Wu^T)) with qgemm_ffn_gate_up on the gate and up [17408, 5120] matrices, then
+y = h Wd^T (fp32) with qgemm_run on the down [5120, 17408] matrix.  Steps are timed as replays
+of a CUDA graph holding the two calls.  The metric is weight GB/s: packed weight bytes read
+per step / step time (the pages' weight-streaming bound for widths <= 64).  Weights cycle
+through a ring of distinct copies so that no step finds its weights in L2.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -34,7 +34,8 @@ FMT = "q8_0"
 BATCH = 64
 RING = 4  # copies of each matrix: 3 x 4 x 94.7 MB = 1.14 GB of Q8_0 weights > L2
 METRIC = "qGEMM weight GB/s (B≤64) & TFLOP/s (prefill) as % of B200 roofline"
-WORKLOAD = "Q8_0 27B FFN decode step: gate+up W[17408,5120] and down W[5120,17408], B=64"
+WORKLOAD = ("Q8_0 27B FFN decode step, B=64: h = SiLU(x Wg^T)*(x Wu^T) with gate/up W[17408,5120] "
+            "(qgemm_ffn_gate_up), then y = h Wd^T with down W[5120,17408] (qgemm_run)")
 KERNEL = "qgemm_pair_kernel<Q8_0, f16 operands> (CTA pairs, tcgen05.mma.cta_group::2)"
 SM_MAX_FALLBACK = 1965.0
 
@@ -129,32 +130,37 @@ class ClockSampler:
 
 
 def cpu_oracle_sample(fmt, batch, target_s=12.0):
-    """Times the oracle (dequantise + fp64 GEMM) on the first rows of each matrix of the step,
-    sized to roughly `target_s` seconds.  Returns (GB/s of weight bytes, description, threads)."""
-    import numpy as np
+    """Times the oracle on the first rows of each matrix of the step, sized to roughly
+    `target_s` seconds: the fused gate+up (dequantise + fp64 GEMMs + SiLU) on `rows` rows of
+    gate and up, and the down GEMM on `rows` rows of down with a synthetic bf16 h.  Returns
+    (GB/s of weight bytes, description, threads, seconds)."""
     import oracle
     from block_quantized_weight_qgemm_b200 import inputs
     threads = oracle.default_threads()
 
     def run(rows):
-        t_total, nbytes = 0.0, 0
-        for name, N, K, seed in matrices():
-            W = inputs.weights(rows, K, seed=seed).numpy()
-            codes, scales, ts = oracle.pack(fmt, W)
-            x = inputs.bf16_bits(inputs.activations(batch, K, seed=1))
-            t0 = time.perf_counter()
-            Wd = oracle.dequant(fmt, codes, scales, ts, rows, K)
-            oracle.gemm(x, Wd, nthreads=threads)
-            t_total += time.perf_counter() - t0
-            nbytes += weight_bytes(fmt, rows, K)
-        return t_total, nbytes
+        Wg = inputs.weights(rows, HIDDEN, seed=0).numpy()
+        Wu = inputs.weights(rows, HIDDEN, seed=2).numpy()
+        Wd = inputs.weights(rows, INTER, seed=3).numpy()
+        pg, pu, pd = oracle.pack(fmt, Wg), oracle.pack(fmt, Wu), oracle.pack(fmt, Wd)
+        x = inputs.bf16_bits(inputs.activations(batch, HIDDEN, seed=1))
+        h = inputs.bf16_bits(inputs.activations(batch, INTER, seed=4))
+        t0 = time.perf_counter()
+        Wgd = oracle.dequant(fmt, *pg, rows, HIDDEN)
+        Wud = oracle.dequant(fmt, *pu, rows, HIDDEN)
+        oracle.ffn_gate_up(x, Wgd, Wud, nthreads=threads)
+        Wdd = oracle.dequant(fmt, *pd, rows, INTER)
+        oracle.gemm(h, Wdd, nthreads=threads)
+        t = time.perf_counter() - t0
+        nbytes = 2 * weight_bytes(fmt, rows, HIDDEN) + weight_bytes(fmt, rows, INTER)
+        return t, nbytes
 
     t, nb = run(64)
     rows = int(max(64, min(HIDDEN, 64 * target_s / max(t, 1e-3))))
     rows = (rows // 32) * 32
     t, nb = run(rows)
-    desc = "first %d rows of each of gate/up/down (%.1f MB of packed weights), B=%d, dequant+fp64 GEMM" % (
-        rows, nb / 1e6, batch)
+    desc = ("first %d rows of each of gate, up (fused FFN) and down (%.1f MB of packed weights), "
+            "B=%d, dequant + fp64 GEMMs" % (rows, nb / 1e6, batch))
     return nb / t / 1e9, desc, threads, t
 
 
@@ -233,28 +239,36 @@ def main():
     qgemm.lib()
 
     fmt, B = args.fmt, args.batch
-    # weight rings, activations, outputs, workspaces
-    calls = []
+    # weight rings (gate, up, down), activations, h, y, workspaces
+    rings = {}
     for name, N, K, seed in matrices():
-        ring = []
+        rings[name] = []
         for i in range(RING):
             W = inputs.weights(N, K, seed=seed + 1000 * i).to(dev)
-            ring.append(qgemm.pack(fmt, W))
+            rings[name].append(qgemm.pack(fmt, W))
             del W
-        x = inputs.activations(B, K, seed=1 if name != "down" else 4).to(dev)
-        y = torch.empty(B, N, device=dev)
-        ws = torch.empty(max(qgemm.workspace_size(fmt, N, K, B), 16), dtype=torch.uint8, device=dev)
-        calls.append(dict(name=name, N=N, K=K, ring=ring, x=x, y=y, ws=ws))
+    x = inputs.activations(B, HIDDEN, seed=1).to(dev)
+    h = torch.empty(B, INTER, dtype=torch.bfloat16, device=dev)
+    y = torch.empty(B, HIDDEN, device=dev)
+    ws_ffn = torch.empty(max(qgemm.ffn_workspace_size(fmt, INTER, HIDDEN, B), 16), dtype=torch.uint8,
+                         device=dev)
+    ws_down = torch.empty(max(qgemm.workspace_size(fmt, HIDDEN, INTER, B), 16), dtype=torch.uint8,
+                          device=dev)
     torch.cuda.synchronize()
-    step_bytes = sum(weight_bytes(fmt, c["N"], c["K"]) for c in calls)
+    ffn_bytes = 2 * weight_bytes(fmt, INTER, HIDDEN)
+    down_bytes = weight_bytes(fmt, HIDDEN, INTER)
+    step_bytes = ffn_bytes + down_bytes
 
-    def step(i, events=None, stream=None):
-        for j, c in enumerate(calls):
-            if events is not None:
-                qgemm.profile_events(*events[j])
-            qgemm.run(c["x"], c["ring"][i % RING], y=c["y"], workspace=c["ws"], stream=stream)
-        if events is not None:
-            qgemm.profile_events(None, None)
+    def launch_ffn(i, xin, stream=None):
+        qgemm.ffn_gate_up(xin, rings["gate"][i % RING], rings["up"][i % RING], h=h,
+                          workspace=ws_ffn, stream=stream)
+
+    def launch_down(i, stream=None):
+        qgemm.run(h, rings["down"][i % RING], y=y, workspace=ws_down, stream=stream)
+
+    def step(i, stream=None):
+        launch_ffn(i, x, stream)
+        launch_down(i, stream)
 
     # one CUDA graph per weight copy of the ring: a step is the replay of graph[i % RING]
     gstream = torch.cuda.Stream(device=dev)
@@ -295,41 +309,52 @@ def main():
     clk = clocks.stop()
     ms = t0.elapsed_time(t1) / args.steps
 
-    # ---- the dominant kernel alone: events around each GEMM launch (stream launches) ----
-    kev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            for _ in calls] for _ in range(args.steps)]
-    for pairs in kev:  # torch creates the CUDA events lazily, on first record
-        for a, b in pairs:
-            a.record()
-            b.record()
+    # ---- the dominant kernel: for each of the two launches of a step, one CUDA graph of K
+    # back-to-back launches cycling the weight ring, timed between events; per-launch time =
+    # elapsed / K (each launch includes its x preparation, overlapped by the GEMM, and for
+    # the down projection the split-K reduce) ------------------------------------------
+    kgraphs = []
+    with torch.cuda.stream(gstream):
+        for fn in (lambda i: launch_ffn(i, x, gstream), lambda i: launch_down(i, gstream)):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=gstream):
+                for i in range(args.steps):
+                    fn(i)
+            kgraphs.append(g)
     torch.cuda.synchronize()
-    for i in range(args.steps):
-        step(i, kev[i])
+    for g in kgraphs:  # warm
+        g.replay()
     torch.cuda.synchronize()
-    kernel_ms = [[a.elapsed_time(b) for (a, b) in kev[i]] for i in range(args.steps)]
-    per_launch = []
-    for i in range(args.steps):
-        for j, c in enumerate(calls):
-            per_launch.append((weight_bytes(fmt, c["N"], c["K"]), kernel_ms[i][j]))
-    k_bytes = sum(b for b, _ in per_launch) / len(per_launch)
-    k_ms = sum(t for _, t in per_launch) / len(per_launch)
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in kgraphs]
+    with torch.cuda.stream(gstream):
+        for (ea, eb), g in zip(kev, kgraphs):
+            ea.record(gstream)
+            g.replay()
+            eb.record(gstream)
+    torch.cuda.synchronize()
+    launch_ms = [ea.elapsed_time(eb) / args.steps for ea, eb in kev]
+    # achieved = the launches' algorithmic bytes over their time (both launches are the pair
+    # kernel; the fused one reads two matrices)
+    k_bytes = (ffn_bytes + down_bytes) / 2
+    k_ms = sum(launch_ms) / 2
 
     ms_max = max_over_ranks(ms, dev, world)
     value = job_rate(step_bytes, ms_max, world)
 
     # ---- end-to-end through the public API with host buffers ---------------------------
-    hx = [c["x"].cpu().pin_memory() for c in calls]
-    hy = [torch.empty(c["y"].shape, dtype=c["y"].dtype).pin_memory() for c in calls]
-    dx = [torch.empty_like(c["x"]) for c in calls]
-    h2d = sum(t.numel() * t.element_size() for t in hx)
-    d2h = sum(t.numel() * t.element_size() for t in hy)
+    hx = x.cpu().pin_memory()
+    hy = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    dx = torch.empty_like(x)
+    h2d = hx.numel() * hx.element_size()
+    d2h = hy.numel() * hy.element_size()
     stream = torch.cuda.current_stream()
 
     def e2e_step(i):
-        for j, c in enumerate(calls):
-            dx[j].copy_(hx[j], non_blocking=True)
-            qgemm.run(dx[j], c["ring"][i % RING], y=c["y"], workspace=c["ws"])
-            hy[j].copy_(c["y"], non_blocking=True)
+        dx.copy_(hx, non_blocking=True)
+        launch_ffn(i, dx)
+        launch_down(i)
+        hy.copy_(y, non_blocking=True)
         stream.synchronize()
 
     for i in range(max(2, args.warmup)):
@@ -367,8 +392,10 @@ def main():
                    "weight_bytes_per_step": step_bytes,
                    "l2": "weights cycle through %d distinct copies per matrix (%.2f GB) > 126 MB L2"
                          % (RING, RING * step_bytes / 1e9),
-                   "timing": "step = CUDA-graph replay of the three qgemm_run calls; the kernel "
-                             "figure times each GEMM launch between events on its stream",
+                   "timing": "step = CUDA-graph replay of the two calls (fused gate+up, down); "
+                             "the kernel figure is, per call, one graph of K back-to-back calls "
+                             "between events / K (x preparation + GEMM [+ split-K reduce] per "
+                             "call: an upper bound on the GEMM kernel)",
                    "parallelism": "replicas" if world > 1 else "single GPU"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
@@ -377,7 +404,8 @@ def main():
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": sum(launches_per_call(fmt, c["N"], c["K"], B) for c in calls) * args.steps,
+        "gpu_launches": (launches_per_call(fmt, INTER, HIDDEN, B) + launches_per_call(fmt, HIDDEN, INTER, B))
+                        * args.steps,
         "clocks": clk,
         "device_status": status,
     }
