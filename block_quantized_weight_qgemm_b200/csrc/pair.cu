@@ -236,6 +236,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     const bool by_matrix = (p.NMAT == 2);
     if (rank == 0 && lane == 0 && (by_matrix || e < p.NACC)) {
       const uint32_t idesc = idesc_f16_pair(BF16OP, (uint32_t)p.NB);
+      const uint32_t xs16 = xslice >> 4;
       RingPos xc;  // x stage of the current group
       RingPos ap;  // A ring
       bool ok = true;
@@ -266,11 +267,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           const uint32_t d = tmem + (uint32_t)(acc_i * p.NB);
           const uint32_t a = tmem + a_col0 + (uint32_t)(ap.slot * kPairACols);
           const bool first = by_matrix ? (gi == 0) : (gi < p.NACC);  // accumulator's first group
-#pragma unroll 4
-          for (int ks = 0; ks < ksteps; ++ks) {
-            const uint32_t bx = xbase + (uint32_t)(ks >> 2) * xslice + (uint32_t)((ks & 3) * 32);
-            mma_f16_ts_pair(d, a + (uint32_t)(ks * 8), smem_desc_sw128(bx), idesc,
-                            (!first || ks > 0) ? 1u : 0u);
+          // The issuing thread, not the tensor pipe, bounds small-N MMA streams, so a full slot
+          // is one straight run of 16 MMAs whose operand addresses are the group's descriptor
+          // plus constants (descriptor address units are 16 bytes).
+          const uint64_t bd0 = smem_desc_sw128(xbase);
+          if (ksteps == 16) {
+#pragma unroll
+            for (int ks = 0; ks < 16; ++ks)
+              mma_f16_ts_pair(d, a + (uint32_t)(ks * 8),
+                              bd0 + (uint64_t)((ks >> 2) * xs16 + (ks & 3) * 2), idesc,
+                              (first && ks == 0) ? 0u : 1u);
+          } else {
+            for (int ks = 0; ks < ksteps; ++ks)
+              mma_f16_ts_pair(d, a + (uint32_t)(ks * 8),
+                              bd0 + (uint64_t)((ks >> 2) * xs16 + (ks & 3) * 2), idesc,
+                              (first && ks == 0) ? 0u : 1u);
           }
           mma_commit_pair(bar_a_empty + 8 * ap.slot);
           ap.next(AS);
