@@ -144,7 +144,7 @@ __global__ void __launch_bounds__(256) qgemm_splitk_reduce_kernel(const ReducePa
     } else {
       const float gv = g[e] * ts0, uv = u[e] * ts1;
       reinterpret_cast<__nv_bfloat16*>(p.out)[off + e] =
-          __float2bfloat16_rn(gv / (1.0f + expf(-gv)) * uv);
+          __float2bfloat16_rn(silu_mul(gv, uv));
     }
   }
 }
