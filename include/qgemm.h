@@ -176,17 +176,22 @@ int qgemm_run_noalloc(int fmt, const void* x_dev, int64_t B, int64_t K, const vo
                       const void* scales_dev, const float* tensor_scale_dev, int64_t N,
                       void* y_dev, int y_dtype, void* stream);
 
-/* Bytes of device workspace qgemm_ffn_gate_up needs for (fmt, N, K, M). */
+/* Bytes of device workspace qgemm_ffn_gate_up needs for (fmt, N, K, M).  Above M = 256 it
+ * holds the fp32 g and u of one chunk of rows (at most 2048 rows: 2 * rows * N * 4 bytes). */
 int qgemm_ffn_workspace_size(int fmt, int64_t N, int64_t K, int64_t M, size_t* bytes);
 
 /*
  * Fused gate+up projection with a SiLU(gate)*up epilogue (Atlas issue, "fused gate+up
  * with dual accumulators ... gate/up are never written to global"):
- *   g = x Wg^T, u = x Wu^T (fp32 accumulators, never stored);
+ *   g = x Wg^T, u = x Wu^T (fp32);
  *   h_dev[M][N] = bf16_RNE( g / (1 + exp(-g)) * u ).
  * Both matrices use the same format and shape [N][K]; x_dev is bf16 [M][K].
  * g_ts_dev / u_ts_dev: NVFP4 tensor scales (NULL for the other formats).
- * For M <= 256 row m of h depends only on x row m (as for qgemm_run).
+ * For M <= 256 one kernel keeps g and u in its accumulators and never stores them, and row m
+ * of h depends only on x row m (as for qgemm_run).  Above 256 rows, each chunk of rows runs
+ * as two GEMMs into fp32 g and u in the workspace and one SiLU pass (prefill widths, where
+ * the single kernel's narrower batch tiles would cost more than the round trip).
+ * Asynchronous on `stream`; errors as for qgemm_run.
  */
 int qgemm_ffn_gate_up(int fmt, const void* x_dev, int64_t M, int64_t K, const void* g_codes_dev,
                       const void* g_scales_dev, const float* g_ts_dev, const void* u_codes_dev,

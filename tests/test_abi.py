@@ -107,4 +107,16 @@ def test_split_rule_depends_only_on_shape(lib):
 
 def test_prefill_path_needs_no_workspace(lib):
     assert qgemm.workspace_size("nvfp4", 17408, 5120, 2048) == 0
-    assert qgemm.ffn_workspace_size("nvfp4", 17408, 5120, 2048) == 0
+
+
+def test_wide_fused_ffn_workspace_holds_g_and_u_of_one_chunk(lib):
+    # above 256 rows the fused gate+up runs, per chunk of rows, two plain GEMMs into fp32
+    # g and u and one SiLU pass; chunks of 2048 rows, balanced (multiples of 8 rows) only
+    # when a full-chunk split would leave a last chunk of 256 rows or fewer
+    N = 17408
+    assert qgemm.ffn_workspace_size("nvfp4", N, 5120, 2048) == 2 * 2048 * N * 4
+    assert qgemm.ffn_workspace_size("nvfp4", N, 5120, 2049) == 2 * 1032 * N * 4
+    assert qgemm.ffn_workspace_size("nvfp4", N, 5120, 7235) == 2 * 2048 * N * 4
+    assert qgemm.ffn_workspace_size("q8_0", N, 5120, 300) == 2 * 304 * N * 4
+    # at or below 256 rows the single fused kernel runs
+    assert qgemm.ffn_workspace_size("q8_0", N, 5120, 256) < 256 * N * 4
