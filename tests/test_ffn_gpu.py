@@ -73,3 +73,20 @@ def test_ffn_batch_invariance(pairs, fmt):
         assert np.array_equal(_h(x[:M], cg, cu), full[:M]), "width %d differs from width 256" % M
     for s0, M in [(3, 64), (100, 70)]:
         assert np.array_equal(_h(x[s0:s0 + M], cg, cu), full[s0:s0 + M]), (s0, M)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_ffn_wide_chunks_parity_and_row_independence(pairs, fmt):
+    # 4300 rows run as three balanced chunks (1440, 1440, 1420 rows) of two GEMMs and a SiLU
+    # pass each; above 256 rows a row of h still depends only on its own row of x, so a
+    # 300-row window across a chunk boundary (a single chunk when run alone) matches bitwise
+    cg, cu = pairs[fmt]
+    M = 4300
+    x = inputs.activations(M, cg.K, seed=26)
+    xb = inputs.bf16_bits(x)
+    g, u, _ = oracle.ffn_gate_up(xb, cg.Wd, cu.Wd)
+    h = _h(x, cg, cu)
+    bad, worst = h_bound_violations(h, g, u, xb, cg.Wd, cu.Wd)
+    assert bad == 0, "%d outputs outside the bound (worst ratio %.3g)" % (bad, worst)
+    s0 = 1300
+    assert np.array_equal(_h(x[s0:s0 + 300], cg, cu), h[s0:s0 + 300])
