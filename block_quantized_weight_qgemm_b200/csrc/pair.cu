@@ -7,9 +7,10 @@
 // Swap-AB on the 5th-generation tensor cores, two SMs per MMA:
 //   * A cluster of two CTAs shares one tcgen05.mma.cta_group::2 stream.  The MMA M operand
 //     is 256 weight rows: the even CTA's 128 rows in its tensor memory (TMEM), the odd CTA's
-//     128 rows at the same TMEM address of its own SM.  One M=256 instruction costs the
-//     tensor pipe about what an M=128 one does on a single SM, so the pair halves the
-//     instruction count per weight byte -- the limit of the one-SM form at small widths.
+//     128 rows at the same TMEM address of its own SM.  At small widths the issuing thread,
+//     not the tensor pipe, bounds the MMA stream (about 58 cycles per instruction), and one
+//     M=256 instruction costs it what an M=128 one does, so the pair halves the instruction
+//     count per weight byte.
 //   * The MMA N operand is NB batch rows of x: rows [0, NB/2) in the even CTA's shared
 //     memory, [NB/2, NB) in the odd CTA's, both loaded by TMA in the 128-byte swizzle.
 //     Each CTA's TMEM receives the fp32 accumulator of its own 128 rows x all NB columns.
@@ -22,8 +23,8 @@
 //   * K is split into S contiguous ranges, S fixed by (format, N, K).  Partials are summed
 //     in the fixed order s = 0..S-1 by the reduce kernel; nothing in the arithmetic depends
 //     on the batch width, so row b of y is bit-identical for every width up to 256.
-//   * Operand types as in the one-SM design: f16 (x rescaled per row by a power of two) for
-//     widths up to 256, bf16 straight from the caller above that.
+//   * Operand types: f16 (x rescaled per row by a power of two) for widths up to 256, bf16
+//     straight from the caller above that.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
