@@ -28,6 +28,8 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "dequant.cuh"
 #include "ptx.cuh"
@@ -518,15 +520,17 @@ template <int FMT, bool BF16OP>
 cudaError_t launch_pair_impl(const GemmParams& p, size_t smem_bytes, int units,
                              const CUtensorMap* maps, bool pdl, cudaStream_t stream) {
   auto kern = qgemm_pair_kernel<FMT, BF16OP>;
-  // raise the dynamic shared-memory limit once per instantiation (to the device maximum)
-  static int set_device = -1;
+  // raise the dynamic shared-memory limit (a per-device function attribute) once per device
+  // and instantiation; devices beyond 64 set it on every launch
+  static std::atomic<uint64_t> set_mask{0};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (set_device != dev) {
+  const uint64_t bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+  if (bit == 0 || !(set_mask.load(std::memory_order_acquire) & bit)) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
     if (e != cudaSuccess) return e;
-    set_device = dev;
+    set_mask.fetch_or(bit, std::memory_order_release);
   }
   if (smem_bytes > (size_t)kSmemLimit) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
