@@ -16,8 +16,8 @@ import threading
 
 import numpy as np
 
-Q8_0, NVFP4, MXFP4 = 0, 1, 2
-FORMATS = {"q8_0": Q8_0, "nvfp4": NVFP4, "mxfp4": MXFP4}
+Q8_0, NVFP4, MXFP4, FP8 = 0, 1, 2, 3
+FORMATS = {"q8_0": Q8_0, "nvfp4": NVFP4, "mxfp4": MXFP4, "fp8": FP8}
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "qgemm_oracle.c")
@@ -50,6 +50,8 @@ def _load():
             lib.orc_e2m1_encode.argtypes = [d]
             lib.orc_e4m3_encode_pos.restype = u
             lib.orc_e4m3_encode_pos.argtypes = [d]
+            lib.orc_e4m3_encode.restype = u
+            lib.orc_e4m3_encode.argtypes = [d]
             lib.orc_f16_encode_satfinite.restype = u
             lib.orc_f16_encode_satfinite.argtypes = [d]
             lib.orc_bf16_encode.restype = u
@@ -63,6 +65,7 @@ def _load():
             lib.orc_pack_q8_0.argtypes = [vp, i64, i64, vp, vp]
             lib.orc_pack_nvfp4.argtypes = [vp, i64, i64, vp, vp, vp]
             lib.orc_pack_mxfp4.argtypes = [vp, i64, i64, vp, vp]
+            lib.orc_pack_fp8.argtypes = [vp, i64, i64, vp, vp]
             lib.orc_dequant.argtypes = [ctypes.c_int, vp, vp, ctypes.c_float, i64, i64, vp]
             lib.orc_gemm.argtypes = [vp, i64, i64, vp, i64, vp, ctypes.c_int]
             lib.orc_ffn_gate_up.argtypes = [vp, i64, i64, vp, vp, i64, vp, vp, vp, ctypes.c_int]
@@ -116,6 +119,10 @@ def e4m3_encode_pos(v: float) -> int:
     return _load().orc_e4m3_encode_pos(v)
 
 
+def e4m3_encode(v: float) -> int:
+    return _load().orc_e4m3_encode(v)
+
+
 def f16_encode_satfinite(v: float) -> int:
     return _load().orc_f16_encode_satfinite(v)
 
@@ -131,7 +138,7 @@ def silu(g: float) -> float:
 # ---- layout -----------------------------------------------------------------------------
 
 def block_size(fmt) -> int:
-    return 16 if _fmt(fmt) == NVFP4 else 32
+    return 16 if _fmt(fmt) in (NVFP4, FP8) else 32
 
 
 def code_pitch(fmt, K: int) -> int:
@@ -145,7 +152,9 @@ def scale_pitch(fmt, K: int) -> int:
 # ---- array routines ---------------------------------------------------------------------
 
 def pack(fmt, W: np.ndarray):
-    """W: float32 [N, K].  Returns (codes uint8 [N, cpitch], scales uint8 [N, spitch], ts)."""
+    """W: float32 [N, K].  Returns (codes uint8 [N, cpitch], scales uint8 [N, spitch], ts).
+    FP8 has no block scales (spitch = 0); NVFP4 and FP8 return their fp32 tensor scale, the
+    other formats 1.0."""
     f = _fmt(fmt)
     W = np.ascontiguousarray(W, dtype=np.float32)
     N, K = W.shape
@@ -158,6 +167,9 @@ def pack(fmt, W: np.ndarray):
         tsv = 1.0
     elif f == NVFP4:
         lib.orc_pack_nvfp4(_ptr(W), N, K, _ptr(codes), _ptr(scales), _ptr(ts))
+        tsv = float(ts[0])
+    elif f == FP8:
+        lib.orc_pack_fp8(_ptr(W), N, K, _ptr(codes), _ptr(ts))
         tsv = float(ts[0])
     else:
         lib.orc_pack_mxfp4(_ptr(W), N, K, _ptr(codes), _ptr(scales))

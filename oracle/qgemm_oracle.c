@@ -7,12 +7,13 @@
  *
  * What it computes (the definition, in fp64, sequential k):
  *     y[b][n] = sum_k  x[b][k] * deq(W)[n][k]
- * with x given as bf16 bit patterns (decoded exactly) and W given in one of three
- * block-quantized encodings:
+ * with x given as bf16 bit patterns (decoded exactly) and W given in one of four
+ * quantized encodings:
  *   Q8_0  : int8 codes, one fp16 scale per 32 consecutive k        (w = q * d16)
  *   NVFP4 : E2M1 codes, one E4M3 scale per 16 consecutive k, plus
  *           one fp32 tensor scale                                   (w = e2m1 * e4m3 * ts)
  *   MXFP4 : E2M1 codes, one E8M0 scale per 32 consecutive k        (w = e2m1 * 2^(e-127))
+ *   FP8   : E4M3 codes, one fp32 tensor scale                       (w = e4m3 * ts)
  *
  * Sources (web pages on block-quantized GEMMs):
  *   - hipfire PR "chunk scalar Q8 batched GEMM above 64 rows": the batched Q8_0 GEMM
@@ -23,6 +24,8 @@
  *     FP64 host reference with exact weights, and the fused gate+up with a
  *     SiLU(gate)*up epilogue.
  *   - "Qwen3.8-27B MXFP4 (AMD Quark) for RDNA4" model card: the MXFP4 weight format.
+ *   - Atlas issue, kernel ranking and verify-tier sections: the FP8 (E4M3) weight layers of
+ *     the NVIDIA pack behind w8a16_gemm_n_m128 and w8a16_gemv_batch8.
  * Where the pages are silent (bit layouts, scale recipes, nibble order, rounding of
  * the packers) the readings are stated beside each function.
  *
@@ -38,7 +41,8 @@
  *   scales : row-major [N][spitch] bytes.  Q8_0: little-endian fp16 per 32-block,
  *            spitch = roundup(2*K/32,16).  NVFP4: one E4M3 byte per 16-block,
  *            spitch = roundup(K/16,16).  MXFP4: one E8M0 byte per 32-block,
- *            spitch = roundup(K/32,16).
+ *            spitch = roundup(K/32,16).  FP8: no block scales, spitch = 0.
+ *   FP8 codes: byte k = the E4M3 code of element k, cpitch = roundup(K,16).
  */
 #include <math.h>
 #include <pthread.h>
@@ -49,6 +53,7 @@
 #define ORC_Q8_0 0
 #define ORC_NVFP4 1
 #define ORC_MXFP4 2
+#define ORC_FP8 3
 
 /* ------------------------------------------------------------------------- */
 /* Element and scale decoders: each is the format's definition written out.  */
@@ -144,6 +149,13 @@ unsigned orc_e4m3_encode_pos(double a) {
     return best;
 }
 
+/* Signed E4M3 code of a finite value: the magnitude as orc_e4m3_encode_pos, the sign
+ * from v (a negative value whose magnitude rounds to zero keeps the sign bit, 0x80). */
+unsigned orc_e4m3_encode(double v) {
+    unsigned sign = (v < 0.0) ? 0x80u : 0u;
+    return sign | orc_e4m3_encode_pos(fabs(v));
+}
+
 /* IEEE binary16 nearest to v, ties to even, saturating to +-65504 (the Q8_0
  * scale is kept finite).  Works by exact power-of-two rescaling and the C
  * library's round-half-even (nearbyint in the default rounding mode). */
@@ -206,15 +218,17 @@ unsigned orc_bf16_encode(double v) {
 
 static int64_t roundup16(int64_t v) { return (v + 15) / 16 * 16; }
 
-int orc_block_size(int fmt) { return fmt == ORC_NVFP4 ? 16 : 32; }
+/* K granularity of each format: its scale block (FP8 has none; 16 keeps x rows aligned). */
+int orc_block_size(int fmt) { return (fmt == ORC_NVFP4 || fmt == ORC_FP8) ? 16 : 32; }
 
 int64_t orc_code_pitch(int fmt, int64_t K) {
-    return fmt == ORC_Q8_0 ? roundup16(K) : roundup16(K / 2);
+    return (fmt == ORC_Q8_0 || fmt == ORC_FP8) ? roundup16(K) : roundup16(K / 2);
 }
 
 int64_t orc_scale_pitch(int fmt, int64_t K) {
     if (fmt == ORC_Q8_0) return roundup16(2 * (K / 32));
     if (fmt == ORC_NVFP4) return roundup16(K / 16);
+    if (fmt == ORC_FP8) return 0;
     return roundup16(K / 32);
 }
 
@@ -226,7 +240,8 @@ static void put_nibble(uint8_t *row, int64_t k, unsigned code) {
 
 /* ORC_MUTATE plants one known mistake (for the tests that show the pins catch it; the
    library build never defines it): 1 nibble order, 2 dropped NVFP4 tensor scale,
-   3 dropped last term of each dot product, 4 Q8_0 scale bytes swapped. */
+   3 dropped last term of each dot product, 4 Q8_0 scale bytes swapped, 5 dropped FP8
+   tensor scale, 6 FP8 sign bit ignored. */
 #ifndef ORC_MUTATE
 #define ORC_MUTATE 0
 #endif
@@ -247,6 +262,9 @@ static unsigned get_nibble(const uint8_t *row, int64_t k) {
 /*         zero ts, or a scale that rounds to 0, gets scale 0 and codes 0.    */
 /*  MXFP4: e = clamp(floor(log2 amax_blk) - 2 + 127, 0, 254) (OCP MX v1.0);   */
 /*         code = E2M1_RNE_sat(w/2^(e-127)); amax 0 gives e = 0, codes 0.     */
+/*  FP8  : ts = fp32_RNE(amax(W)/448) (one scale per matrix: the pages' FP8   */
+/*         layers come from an NVIDIA pack, whose FP8 recipe scales per       */
+/*         tensor); code = E4M3_RNE_sat(w/ts); a zero ts gives codes 0.       */
 /* All quotients are formed once in fp64 from exact operands.                 */
 /* ------------------------------------------------------------------------- */
 
@@ -333,6 +351,21 @@ void orc_pack_mxfp4(const float *W, int64_t N, int64_t K, uint8_t *codes, uint8_
     }
 }
 
+/* Returns the fp32 tensor scale through *ts_out. */
+void orc_pack_fp8(const float *W, int64_t N, int64_t K, uint8_t *codes, float *ts_out) {
+    int64_t cp = orc_code_pitch(ORC_FP8, K);
+    double amax = 0.0;
+    float ts;
+    memset(codes, 0, (size_t)(N * cp));
+    for (int64_t i = 0; i < N * K; ++i) amax = fmax(amax, fabs((double)W[i]));
+    ts = (float)(amax / 448.0);
+    *ts_out = ts;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k)
+            codes[n * cp + k] =
+                (uint8_t)(ts != 0.0f ? orc_e4m3_encode((double)W[n * K + k] / (double)ts) : 0u);
+}
+
 /* ------------------------------------------------------------------------- */
 /* Dequantisation to fp64 (exact).                                            */
 /* ------------------------------------------------------------------------- */
@@ -352,6 +385,9 @@ void orc_dequant(int fmt, const uint8_t *codes, const uint8_t *scales, float ts,
             } else if (fmt == ORC_NVFP4) {
                 v = orc_e2m1(get_nibble(cr, k)) * orc_e4m3(sr[k / 16]) *
                     (ORC_MUTATE == 2 ? 1.0 : (double)ts);
+            } else if (fmt == ORC_FP8) {
+                v = orc_e4m3(ORC_MUTATE == 6 ? (cr[k] & 0x7Fu) : cr[k]) *
+                    (ORC_MUTATE == 5 ? 1.0 : (double)ts);
             } else {
                 v = orc_e2m1(get_nibble(cr, k)) * orc_e8m0(sr[k / 32]);
             }

@@ -152,6 +152,24 @@ def test_e4m3_encode_against_torch_and_ties():
     assert oracle.e4m3_encode_pos(1e30) == 0x7E
 
 
+def test_e4m3_signed_encode_against_torch_and_sign_rule():
+    # the FP8 weight encoder: torch's float -> float8_e4m3fn conversion (round to nearest even)
+    # on values of both signs within the finite range, and the sign rule for zero
+    rng = np.random.default_rng(3)
+    vals = (rng.standard_normal(4000).astype(np.float32)
+            * np.float32(2.0) ** rng.integers(-14, 9, 4000).astype(np.float32))
+    vals = vals[np.abs(vals) < 448.0]
+    ref = torch.from_numpy(vals).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    for v, r in zip(vals, ref):
+        if int(r) & 0x7F:   # a non-zero result: torch and the oracle agree on sign and magnitude
+            assert oracle.e4m3_encode(float(v)) == int(r), v
+        else:               # rounds to zero: the oracle keeps the sign bit of v
+            assert oracle.e4m3_encode(float(v)) == (0x80 if v < 0 else 0x00), v
+    assert oracle.e4m3_encode(-448.0) == 0xFE and oracle.e4m3_encode(-1e9) == 0xFE
+    assert oracle.e4m3_encode(-2.0 ** -10) == 0x80 and oracle.e4m3_encode(2.0 ** -10) == 0x00
+    assert oracle.e4m3_encode(-(2.0 ** -10 + 2.0 ** -20)) == 0x81  # above half the subnormal step
+
+
 def _e2m1_nearest_code(v: Fraction) -> int:
     """Brute force: nearest E2M1 magnitude, ties to the even code, saturate at 6."""
     a = abs(v)
@@ -277,6 +295,32 @@ def test_pitches_and_footprint(golden):
 # Dequantisation and GEMM
 # ------------------------------------------------------------------------------------------
 
+def test_fp8_pack_brute_force():
+    # per-tensor scale ts = fp32(amax/448); each code the E4M3 value nearest to w/ts in exact
+    # arithmetic (ties to the even code, saturating at 448), with the sign of w
+    N, K = 5, 96
+    W = _rows_with_specials(N, K, 14)
+    W[4, 5] = -np.abs(W).max() * 1.5      # the matrix maximum is negative
+    W[4, 6] = np.float32(1e-12)           # far below the smallest subnormal step
+    W[4, 7] = np.float32(-1e-12)
+    codes, scales, ts = oracle.pack("fp8", W)
+    assert scales.shape == (N, 0)
+    amax = float(np.abs(W.astype(np.float64)).max())
+    assert ts == float(np.float32(amax / 448.0))
+    vals = [Fraction(oracle.e4m3(b)) for b in range(0x7F)]   # the finite non-negative values
+    for n in range(N):
+        for k in range(K):
+            q = Fraction(float(W[n, k])) / Fraction(ts)
+            want = min(range(0x7F), key=lambda b: (abs(abs(q) - vals[b]), b & 1))
+            want |= 0x80 if q < 0 else 0
+            assert int(codes[n, k]) == want, (n, k)
+    assert int(codes[4, 5]) == 0xFE      # -amax -> -448 (saturated after the fp32 rounding of ts)
+    assert int(codes[4, 6]) == 0x00 and int(codes[4, 7]) == 0x80
+    # a zero matrix: ts = 0 and all codes 0
+    c0, _, t0 = oracle.pack("fp8", np.zeros((2, 32), dtype=np.float32))
+    assert t0 == 0.0 and not c0.any()
+
+
 def test_dequant_hand_built_rows():
     K = 32
     # Q8_0: codes -127, 1, 5 with scale 1.0 (0x3C00) and 0.5 (0x3800) in block 2
@@ -305,6 +349,12 @@ def test_dequant_hand_built_rows():
     scales[0, 0] = 128
     Wd = oracle.dequant("mxfp4", codes, scales, 1.0, 1, K)
     assert Wd[0, 0] == 12.0 and Wd[0, 1] == -1.0
+    # FP8: E4M3 0x38 = 1.0, 0xC0 = -2.0, 0x7E = 448, 0x01 = 2^-9, 0x80 = -0; ts = 0.25
+    codes = np.zeros((1, oracle.code_pitch("fp8", K)), dtype=np.uint8)
+    scales = np.zeros((1, 0), dtype=np.uint8)
+    codes[0, :5] = [0x38, 0xC0, 0x7E, 0x01, 0x80]
+    Wd = oracle.dequant("fp8", codes, scales, 0.25, 1, K)
+    assert list(Wd[0, :6]) == [0.25, -0.5, 112.0, 2.0 ** -11, 0.0, 0.0]
 
 
 def _fraction_gemm(x16, Wd):
@@ -315,7 +365,7 @@ def _fraction_gemm(x16, Wd):
     return [[sum(xf[b][k] * wf[n][k] for k in range(K)) for n in range(N)] for b in range(B)]
 
 
-@pytest.mark.parametrize("fmt", ["q8_0", "nvfp4", "mxfp4"])
+@pytest.mark.parametrize("fmt", ["q8_0", "nvfp4", "mxfp4", "fp8"])
 @pytest.mark.parametrize("K", [32, 64])
 def test_gemm_brute_force_rational(fmt, K):
     N, B = 4, 3
@@ -332,7 +382,7 @@ def test_gemm_brute_force_rational(fmt, K):
             assert abs(Fraction(float(y[b, n])) - exact[b][n]) <= Fraction(bound)
 
 
-@pytest.mark.parametrize("fmt", ["q8_0", "nvfp4", "mxfp4"])
+@pytest.mark.parametrize("fmt", ["q8_0", "nvfp4", "mxfp4", "fp8"])
 def test_gemm_one_hot_and_ones(fmt):
     N, K = 7, 96
     W = inputs.weights(N, K, seed=23).numpy()
@@ -451,6 +501,11 @@ def _hand_rows_hold(lib):
     scales[0, 0] = 0x38
     Wd = _dequant_with(lib, "nvfp4", codes, scales, 0.5, 1, K)
     ok &= bool(Wd[0, 0] == -3.0 and Wd[0, 1] == 3.0)
+    codes = np.zeros((1, oracle.code_pitch("fp8", K)), dtype=np.uint8)
+    scales = np.zeros((1, 16), dtype=np.uint8)
+    codes[0, :2] = [0x38, 0xC0]
+    Wd = _dequant_with(lib, "fp8", codes, scales, 0.25, 1, K)
+    ok &= bool(Wd[0, 0] == 0.25 and Wd[0, 1] == -0.5)
     return ok
 
 
@@ -473,3 +528,5 @@ def test_pins_catch_planted_mistakes(tmp_path):
     assert not _hand_rows_hold(_mutant(tmp_path, 2))        # NVFP4 tensor scale dropped
     assert not _gemm_matches_fractions(_mutant(tmp_path, 3))  # last term of each sum dropped
     assert not _hand_rows_hold(_mutant(tmp_path, 4))        # Q8_0 scale bytes swapped
+    assert not _hand_rows_hold(_mutant(tmp_path, 5))        # FP8 tensor scale dropped
+    assert not _hand_rows_hold(_mutant(tmp_path, 6))        # FP8 sign bit ignored
