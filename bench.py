@@ -1,24 +1,28 @@
 """Benchmark of the block-quantized-weight GEMM hot path on B200.
 
-Default workload (one "step"): the Q8_0 27B FFN at decode width B = 64 -- h = bf16(SiLU(x Wg^T)
+Headline workload (one "step"): the Q8_0 27B FFN at decode width B = 64 -- h = bf16(SiLU(x Wg^T)
 * (x Wu^T)) with qgemm_ffn_gate_up on the gate and up [17408, 5120] matrices, then
 y = h Wd^T (fp32) with qgemm_run on the down [5120, 17408] matrix.  Steps are timed as replays
 of a CUDA graph holding the two calls.  The metric is weight GB/s: packed weight bytes read
-per step / step time (the pages' weight-streaming bound for widths <= 64).  Weights cycle
-through a ring of distinct copies so that no step finds its weights in L2.
+per step / step time (the weight-streaming bound for widths <= 64).  Weights cycle through a
+ring of distinct copies so that no step finds its weights in L2.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+The same JSON line carries a `configs` record with every workload configuration of the
+method, each timed per call on the device: decode widths as weight GB/s against the measured
+copy bandwidth, prefill chunks (M >= 2048) as TFLOP/s against the measured burst dense bf16
+peak.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--no-configs]
 
 With N > 1 (torchrun, one process per GPU) every rank runs an independent replica of the
 same workload ("replicas only": the path has no exchange step); value = all ranks' bytes /
-max-over-ranks device time.  --impl reference times the CPU oracle on a bounded sample of
-the same workload (rank 0 only).  Prints one JSON line on rank 0.
+max-over-ranks device time.  --impl reference times the CPU oracle on a bounded sample of the
+same workload (rank 0 only), W warm-up and K timed steps.  Prints one JSON line on rank 0.
 """
 from __future__ import annotations
 
 import argparse
 import json
-import math
 import os
 import statistics
 import subprocess
@@ -37,7 +41,6 @@ METRIC = "qGEMM weight GB/s (B≤64) & TFLOP/s (prefill) as % of B200 roofline"
 WORKLOAD = ("Q8_0 27B FFN decode step, B=64: h = SiLU(x Wg^T)*(x Wu^T) with gate/up W[17408,5120] "
             "(qgemm_ffn_gate_up), then y = h Wd^T with down W[5120,17408] (qgemm_run)")
 KERNEL = "qgemm_pair_kernel<Q8_0, f16 operands> (CTA pairs, tcgen05.mma.cta_group::2)"
-SM_MAX_FALLBACK = 1965.0
 
 
 def parse():
@@ -48,27 +51,33 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--batch", type=int, default=BATCH)
     ap.add_argument("--fmt", default=FMT)
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-configuration record (headline step only)")
     return ap.parse_args()
 
 
 def peaks():
+    """(HBM GB/s, burst bf16 TFLOP/s, source) from the driver's measurement, else fallback."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
             d = json.load(f)
-        return float(d["hbm_gbs"]), "measured"
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
     except Exception:
-        return 6650.0, "fallback"
+        return 6650.0, 1590.0, "fallback"
 
 
 def matrices():
-    # (name, N, K, weight seed, activation width K, activation seed)
+    # (name, N, K, weight seed)
     return [("gate", INTER, HIDDEN, 0), ("up", INTER, HIDDEN, 2), ("down", HIDDEN, INTER, 3)]
 
 
 def weight_bytes(fmt, N, K):
+    """Algorithmic bytes of one packed matrix: codes + block scales (no padding)."""
     if fmt == "q8_0":
         return N * K + N * (K // 32) * 2
+    if fmt == "fp8":
+        return N * K
     if fmt == "nvfp4":
         return N * K // 2 + N * (K // 16)
     return N * K // 2 + N * (K // 32)
@@ -129,65 +138,75 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def cpu_oracle_sample(fmt, batch, target_s=12.0):
-    """Times the oracle on the first rows of each matrix of the step, sized to roughly
-    `target_s` seconds: the fused gate+up (dequantise + fp64 GEMMs + SiLU) on `rows` rows of
-    gate and up, and the down GEMM on `rows` rows of down with a synthetic bf16 h.  Returns
-    (GB/s of weight bytes, description, threads, seconds)."""
-    import oracle
-    from block_quantized_weight_qgemm_b200 import inputs
-    threads = oracle.default_threads()
+# ---- the oracle on the host cores (reference arm and cpu_baseline) -------------------------
 
-    def run(rows):
-        Wg = inputs.weights(rows, HIDDEN, seed=0).numpy()
-        Wu = inputs.weights(rows, HIDDEN, seed=2).numpy()
-        Wd = inputs.weights(rows, INTER, seed=3).numpy()
-        pg, pu, pd = oracle.pack(fmt, Wg), oracle.pack(fmt, Wu), oracle.pack(fmt, Wd)
-        x = inputs.bf16_bits(inputs.activations(batch, HIDDEN, seed=1))
-        h = inputs.bf16_bits(inputs.activations(batch, INTER, seed=4))
+class OracleSample:
+    """The oracle (as it stands) on the first `rows` rows of each matrix of the step: the fused
+    gate+up (dequantise + fp64 GEMMs + SiLU) on gate and up, and the down GEMM on a synthetic
+    bf16 h.  Packing happens once, outside the timed calls."""
+
+    def __init__(self, fmt, batch, rows):
+        import oracle
+        from block_quantized_weight_qgemm_b200 import inputs
+        self.oracle, self.fmt, self.rows = oracle, fmt, rows
+        self.threads = oracle.default_threads()
+        self.pg = oracle.pack(fmt, inputs.weights(rows, HIDDEN, seed=0).numpy())
+        self.pu = oracle.pack(fmt, inputs.weights(rows, HIDDEN, seed=2).numpy())
+        self.pd = oracle.pack(fmt, inputs.weights(rows, INTER, seed=3).numpy())
+        self.x = inputs.bf16_bits(inputs.activations(batch, HIDDEN, seed=1))
+        self.h = inputs.bf16_bits(inputs.activations(batch, INTER, seed=4))
+        self.nbytes = 2 * weight_bytes(fmt, rows, HIDDEN) + weight_bytes(fmt, rows, INTER)
+        self.batch = batch
+
+    def run(self) -> float:
+        o, f, r = self.oracle, self.fmt, self.rows
         t0 = time.perf_counter()
-        Wgd = oracle.dequant(fmt, *pg, rows, HIDDEN)
-        Wud = oracle.dequant(fmt, *pu, rows, HIDDEN)
-        oracle.ffn_gate_up(x, Wgd, Wud, nthreads=threads)
-        Wdd = oracle.dequant(fmt, *pd, rows, INTER)
-        oracle.gemm(h, Wdd, nthreads=threads)
-        t = time.perf_counter() - t0
-        nbytes = 2 * weight_bytes(fmt, rows, HIDDEN) + weight_bytes(fmt, rows, INTER)
-        return t, nbytes
+        Wgd = o.dequant(f, *self.pg, r, HIDDEN)
+        Wud = o.dequant(f, *self.pu, r, HIDDEN)
+        o.ffn_gate_up(self.x, Wgd, Wud, nthreads=self.threads)
+        Wdd = o.dequant(f, *self.pd, r, INTER)
+        o.gemm(self.h, Wdd, nthreads=self.threads)
+        return time.perf_counter() - t0
 
-    t, nb = run(64)
+    def describe(self):
+        return ("first %d rows of each of gate, up (fused FFN) and down (%.1f MB of packed "
+                "weights), B=%d, dequant + fp64 GEMMs" % (self.rows, self.nbytes / 1e6, self.batch))
+
+
+def oracle_sample(fmt, batch, target_s):
+    """An OracleSample sized to take about target_s seconds per run."""
+    probe = OracleSample(fmt, batch, 64)
+    t = probe.run()
     rows = int(max(64, min(HIDDEN, 64 * target_s / max(t, 1e-3))))
-    rows = (rows // 32) * 32
-    t, nb = run(rows)
-    desc = ("first %d rows of each of gate, up (fused FFN) and down (%.1f MB of packed weights), "
-            "B=%d, dequant + fp64 GEMMs" % (rows, nb / 1e6, batch))
-    return nb / t / 1e9, desc, threads, t
+    return OracleSample(fmt, batch, (rows // 32) * 32)
 
 
 def run_reference(args, rank, world):
+    """The reference arm: the CPU oracle, W warm-up and K timed steps of a bounded sample."""
     if rank != 0:
         return
-    gbs, desc, threads, t = cpu_oracle_sample(args.fmt, args.batch, target_s=6.0)
-    steps_t = []
-    # each step: one bounded sample of the workload through the oracle (as it stands)
+    sample = oracle_sample(args.fmt, args.batch, target_s=2.0)
     for _ in range(args.warmup):
-        pass
-    per_step_s = t
-    value = gbs
+        sample.run()
+    times = [sample.run() for _ in range(args.steps)]
+    per_step_s = sum(times) / len(times)
+    value = sample.nbytes / per_step_s / 1e9
+    desc = sample.describe()
     line = {
         "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_step_s * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "impl": "reference",
-        "config": {"workload": WORKLOAD, "fmt": args.fmt, "B": args.batch,
-                   "sample": desc},
-        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads,
+        "config": {"workload": WORKLOAD, "fmt": args.fmt, "B": args.batch, "sample": desc},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": sample.threads,
                          "kind": "oracle", "sample": desc},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
+
+# ---- device timing helpers ------------------------------------------------------------------
 
 def max_over_ranks(v: float, device, world: int) -> float:
     """The largest value of v over all ranks (every rank calls this, in the same order)."""
@@ -213,6 +232,177 @@ def launches_per_call(fmt, N, K, B):
     if B > 256:
         return 1
     return 2 + (1 if qgemm.split_k(fmt, N, K) > 1 else 0)
+
+
+def graph_us(fn, reps, stream):
+    """Device time per call of fn(i), i = 0..reps-1, captured in one CUDA graph on `stream`
+    and replayed between CUDA events on that stream (after one warm replay)."""
+    import torch
+    with torch.cuda.stream(stream):
+        for i in range(min(reps, 2)):
+            fn(i)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(reps):
+                fn(i)
+    torch.cuda.synchronize()
+    # replay() launches on the current stream: make it `stream`, where the events are recorded
+    with torch.cuda.stream(stream):
+        g.replay()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        g.replay()
+        b.record(stream)
+    torch.cuda.synchronize()
+    us = a.elapsed_time(b) * 1e3 / reps
+    del g
+    return us
+
+
+def clone_ring(pw, n):
+    """n packed copies at distinct addresses (the same bytes): a ring that defeats L2."""
+    from block_quantized_weight_qgemm_b200 import qgemm
+    out = [pw]
+    for _ in range(n - 1):
+        c = qgemm.PackedWeight(pw.fmt, pw.N, pw.K, pw.codes.device)
+        c.codes.copy_(pw.codes)
+        c.scales.copy_(pw.scales)
+        if pw.tensor_scale is not None:
+            c.tensor_scale.copy_(pw.tensor_scale)
+        out.append(c)
+    return out
+
+
+def run_configs(dev, stream, q8_rings, hbm_peak, tf_peak):
+    """Every workload configuration, timed per call on the device (kernel time: x preparation
+    + GEMM [+ split-K reduce] per call; graphs of back-to-back calls over a weight ring)."""
+    import torch
+    from block_quantized_weight_qgemm_b200 import inputs, qgemm
+
+    recs = []
+
+    def packed(fmt, N, K, seed):
+        W = inputs.weights(N, K, seed=seed).to(dev)
+        pw = qgemm.pack(fmt, W)
+        del W
+        return pw
+
+    def decode(name, fmt, ring, B, reps=40, note=None):
+        N, K = ring[0].N, ring[0].K
+        x = inputs.activations(B, K, seed=1).to(dev)
+        y = torch.empty(B, N, device=dev)
+        ws = torch.empty(max(qgemm.workspace_size(fmt, N, K, B), 16), dtype=torch.uint8, device=dev)
+        us = graph_us(lambda i: qgemm.run(x, ring[i % len(ring)], y=y, workspace=ws, stream=stream),
+                      reps, stream)
+        nb = weight_bytes(fmt, N, K)
+        gbs = nb / (us * 1e-6) / 1e9
+        r = {"config": name, "kind": "decode", "fmt": fmt, "N": N, "K": K, "B": B,
+             "us": round(us, 2), "weight_GBps": round(gbs, 1), "frac_hbm": round(gbs / hbm_peak, 4)}
+        if note:
+            r["note"] = note
+        recs.append(r)
+
+    def decode_ffn(name, fmt, gring, uring, B, reps=40):
+        N, K = gring[0].N, gring[0].K
+        x = inputs.activations(B, K, seed=1).to(dev)
+        h = torch.empty(B, N, dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(max(qgemm.ffn_workspace_size(fmt, N, K, B), 16), dtype=torch.uint8,
+                         device=dev)
+        us = graph_us(lambda i: qgemm.ffn_gate_up(x, gring[i % len(gring)], uring[i % len(uring)],
+                                                  h=h, workspace=ws, stream=stream), reps, stream)
+        nb = 2 * weight_bytes(fmt, N, K)
+        gbs = nb / (us * 1e-6) / 1e9
+        recs.append({"config": name, "kind": "decode", "fmt": fmt, "N": N, "K": K, "B": B,
+                     "op": "ffn_gate_up", "us": round(us, 2), "weight_GBps": round(gbs, 1),
+                     "frac_hbm": round(gbs / hbm_peak, 4)})
+
+    def prefill(name, fmt, pw, M, reps=4):
+        N, K = pw.N, pw.K
+        x = inputs.activations(M, K, seed=1).to(dev)
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(max(qgemm.workspace_size(fmt, N, K, M), 16), dtype=torch.uint8, device=dev)
+        us = graph_us(lambda i: qgemm.run(x, pw, y=y, workspace=ws, stream=stream), reps, stream)
+        tf = 2.0 * M * N * K / (us * 1e-6) / 1e12
+        recs.append({"config": name, "kind": "prefill", "fmt": fmt, "N": N, "K": K, "M": M,
+                     "us": round(us, 1), "TFLOPs": round(tf, 1), "frac_tensor": round(tf / tf_peak, 4)})
+        del x, y, ws
+
+    def prefill_ffn(name, fmt, pg, pu, pd, M, reps=3):
+        N, K = pg.N, pg.K
+        x = inputs.activations(M, K, seed=1).to(dev)
+        h = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        y = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+        wsf = torch.empty(max(qgemm.ffn_workspace_size(fmt, N, K, M), 16), dtype=torch.uint8,
+                          device=dev)
+        wsd = torch.empty(max(qgemm.workspace_size(fmt, K, N, M), 16), dtype=torch.uint8, device=dev)
+
+        def chain(i):
+            qgemm.ffn_gate_up(x, pg, pu, h=h, workspace=wsf, stream=stream)
+            qgemm.run(h, pd, y=y, workspace=wsd, stream=stream)
+
+        us = graph_us(chain, reps, stream)
+        us_ffn = graph_us(lambda i: qgemm.ffn_gate_up(x, pg, pu, h=h, workspace=wsf, stream=stream),
+                          reps, stream)
+        flop = 2.0 * M * (2 * N) * K + 2.0 * M * K * N
+        tf = flop / (us * 1e-6) / 1e12
+        tf_ffn = 2.0 * M * (2 * N) * K / (us_ffn * 1e-6) / 1e12
+        recs.append({"config": name, "kind": "prefill", "fmt": fmt, "N": N, "K": K, "M": M,
+                     "op": "ffn_gate_up + down", "us": round(us, 1), "TFLOPs": round(tf, 1),
+                     "frac_tensor": round(tf / tf_peak, 4), "ffn_gate_up_us": round(us_ffn, 1),
+                     "ffn_gate_up_TFLOPs": round(tf_ffn, 1),
+                     "down_us": round(us - us_ffn, 1)})
+        del x, h, y, wsf, wsd
+
+    # cfg 1: tiny Q8_0 [512, 1024] -- the whole matrix fits in L2; too small for a roofline
+    tiny = packed("q8_0", 512, 1024, 0)
+    for B in (1, 64, 65):
+        decode("q8_0 tiny [512,1024]", "q8_0", [tiny], B,
+               note="0.56 MB of weights: L2-resident, no roofline bar")
+    # cfg 2: Q8_0 at the 27B FFN shapes
+    gate, up, down = q8_rings["gate"], q8_rings["up"], q8_rings["down"]
+    for B in (1, 16, 64):
+        decode("q8_0 27B gate/up", "q8_0", gate, B)
+    decode("q8_0 27B gate/up", "q8_0", gate, 256)
+    decode("q8_0 27B down", "q8_0", down, 64)
+    for B in (1, 64):
+        decode_ffn("q8_0 27B fused gate+up", "q8_0", gate, up, B)
+    prefill("q8_0 27B gate/up prefill", "q8_0", gate[0], 2048)
+    # cfg 3: NVFP4 verify widths
+    nv_gate = packed("nvfp4", INTER, HIDDEN, 0)
+    ring = clone_ring(nv_gate, RING)
+    for B in (1, 4, 8, 16):
+        decode("nvfp4 27B gate/up verify", "nvfp4", ring, B)
+    del ring
+    # cfg 4: NVFP4 prefill FFN chunk (fused gate+up -> h -> down)
+    nv_up = packed("nvfp4", INTER, HIDDEN, 2)
+    nv_down = packed("nvfp4", HIDDEN, INTER, 3)
+    for M in (2048, 7235):
+        prefill_ffn("nvfp4 27B FFN prefill chunk", "nvfp4", nv_gate, nv_up, nv_down, M)
+    del nv_gate, nv_up, nv_down
+    torch.cuda.empty_cache()
+    # FP8 (E4M3, per-tensor scale) weights: the batch-8 verify GEMV widths and decode, the
+    # W8A16 prefill GEMM
+    fp8 = packed("fp8", INTER, HIDDEN, 0)
+    ring = clone_ring(fp8, RING)
+    for B in (1, 8, 16, 64):
+        decode("fp8 27B gate/up", "fp8", ring, B)
+    del ring
+    prefill("fp8 27B gate/up prefill", "fp8", fp8, 2048)
+    del fp8
+    torch.cuda.empty_cache()
+    # cfg 5: MXFP4 serving mix (B = 32 decode, M = 8192 prefill) on both shapes
+    for N, K, seed in ((INTER, HIDDEN, 0), (HIDDEN, INTER, 3)):
+        mx = packed("mxfp4", N, K, seed)
+        ring = clone_ring(mx, RING)
+        decode("mxfp4 27B serving mix", "mxfp4", ring, 32)
+        del ring
+        prefill("mxfp4 27B serving mix prefill", "mxfp4", mx, 8192, reps=3)
+        del mx
+        torch.cuda.empty_cache()
+    return recs
 
 
 def main():
@@ -242,11 +432,9 @@ def main():
     # weight rings (gate, up, down), activations, h, y, workspaces
     rings = {}
     for name, N, K, seed in matrices():
-        rings[name] = []
-        for i in range(RING):
-            W = inputs.weights(N, K, seed=seed + 1000 * i).to(dev)
-            rings[name].append(qgemm.pack(fmt, W))
-            del W
+        W = inputs.weights(N, K, seed=seed).to(dev)
+        rings[name] = clone_ring(qgemm.pack(fmt, W), RING)
+        del W
     x = inputs.activations(B, HIDDEN, seed=1).to(dev)
     h = torch.empty(B, INTER, dtype=torch.bfloat16, device=dev)
     y = torch.empty(B, HIDDEN, device=dev)
@@ -259,16 +447,16 @@ def main():
     down_bytes = weight_bytes(fmt, HIDDEN, INTER)
     step_bytes = ffn_bytes + down_bytes
 
-    def launch_ffn(i, xin, stream=None):
-        qgemm.ffn_gate_up(xin, rings["gate"][i % RING], rings["up"][i % RING], h=h,
+    def launch_ffn(i, xin, hout, stream=None):
+        qgemm.ffn_gate_up(xin, rings["gate"][i % RING], rings["up"][i % RING], h=hout,
                           workspace=ws_ffn, stream=stream)
 
-    def launch_down(i, stream=None):
-        qgemm.run(h, rings["down"][i % RING], y=y, workspace=ws_down, stream=stream)
+    def launch_down(i, hin, yout, stream=None):
+        qgemm.run(hin, rings["down"][i % RING], y=yout, workspace=ws_down, stream=stream)
 
     def step(i, stream=None):
-        launch_ffn(i, x, stream)
-        launch_down(i, stream)
+        launch_ffn(i, x, h, stream)
+        launch_down(i, h, y, stream)
 
     # one CUDA graph per weight copy of the ring: a step is the replay of graph[i % RING]
     gstream = torch.cuda.Stream(device=dev)
@@ -313,74 +501,88 @@ def main():
     # back-to-back launches cycling the weight ring, timed between events; per-launch time =
     # elapsed / K (each launch includes its x preparation, overlapped by the GEMM, and for
     # the down projection the split-K reduce) ------------------------------------------
-    kgraphs = []
-    with torch.cuda.stream(gstream):
-        for fn in (lambda i: launch_ffn(i, x, gstream), lambda i: launch_down(i, gstream)):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=gstream):
-                for i in range(args.steps):
-                    fn(i)
-            kgraphs.append(g)
-    torch.cuda.synchronize()
-    for g in kgraphs:  # warm
-        g.replay()
-    torch.cuda.synchronize()
-    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in kgraphs]
-    with torch.cuda.stream(gstream):
-        for (ea, eb), g in zip(kev, kgraphs):
-            ea.record(gstream)
-            g.replay()
-            eb.record(gstream)
-    torch.cuda.synchronize()
-    launch_ms = [ea.elapsed_time(eb) / args.steps for ea, eb in kev]
+    ffn_us = graph_us(lambda i: launch_ffn(i, x, h, gstream), args.steps, gstream)
+    down_us = graph_us(lambda i: launch_down(i, h, y, gstream), args.steps, gstream)
     # achieved = the launches' algorithmic bytes over their time (both launches are the pair
     # kernel; the fused one reads two matrices)
     k_bytes = (ffn_bytes + down_bytes) / 2
-    k_ms = sum(launch_ms) / 2
+    k_ms = (ffn_us + down_us) / 2 * 1e-3
 
     ms_max = max_over_ranks(ms, dev, world)
     value = job_rate(step_bytes, ms_max, world)
 
-    # ---- end-to-end through the public API with host buffers ---------------------------
-    hx = x.cpu().pin_memory()
-    hy = torch.empty(y.shape, dtype=y.dtype).pin_memory()
-    dx = torch.empty_like(x)
-    h2d = hx.numel() * hx.element_size()
-    d2h = hy.numel() * hy.element_size()
-    stream = torch.cuda.current_stream()
+    # ---- end to end through the public API with host buffers: every step copies its input
+    # from pinned host memory and its result back; a two-deep ring of device buffers lets the
+    # copies of neighbouring steps overlap the compute (copy stream and compute stream) -----
+    NSLOT = 2
+    hx = [x.cpu().pin_memory() for _ in range(NSLOT)]
+    hy = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for _ in range(NSLOT)]
+    dx = [torch.empty_like(x) for _ in range(NSLOT)]
+    dy = [torch.empty_like(y) for _ in range(NSLOT)]
+    h2d = hx[0].numel() * hx[0].element_size()
+    d2h = hy[0].numel() * hy[0].element_size()
+    comp = torch.cuda.current_stream()
+    copy_in = torch.cuda.Stream(device=dev)
+    copy_out = torch.cuda.Stream(device=dev)
+    in_done = [torch.cuda.Event() for _ in range(NSLOT)]
+    comp_done = [torch.cuda.Event() for _ in range(NSLOT)]
+    out_done = [torch.cuda.Event() for _ in range(NSLOT)]
+    used = [False] * NSLOT
 
     def e2e_step(i):
-        dx.copy_(hx, non_blocking=True)
-        launch_ffn(i, dx)
-        launch_down(i)
-        hy.copy_(y, non_blocking=True)
-        stream.synchronize()
+        s = i % NSLOT
+        with torch.cuda.stream(copy_in):
+            if used[s]:
+                copy_in.wait_event(comp_done[s])  # dx[s]'s previous step has consumed it
+            dx[s].copy_(hx[s], non_blocking=True)
+            in_done[s].record(copy_in)
+        comp.wait_event(in_done[s])
+        if used[s]:
+            comp.wait_event(out_done[s])  # dy[s]'s previous result has reached the host
+        launch_ffn(i, dx[s], h)
+        launch_down(i, h, dy[s])
+        comp_done[s].record(comp)
+        with torch.cuda.stream(copy_out):
+            copy_out.wait_event(comp_done[s])
+            hy[s].copy_(dy[s], non_blocking=True)
+            out_done[s].record(copy_out)
+        used[s] = True
 
     for i in range(max(2, args.warmup)):
         e2e_step(i)
+    torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record()
+    e0.record(comp)
     for i in range(args.steps):
         e2e_step(i)
-    e1.record()
+    for s in range(NSLOT):
+        comp.wait_event(out_done[s])
+    e1.record(comp)
     torch.cuda.synchronize()
     e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev, world)
     e2e_value = job_rate(step_bytes, e_ms, world)
 
     status = qgemm.device_status(reset=True)
 
+    hbm_peak, tf_peak, peak_kind = peaks()
+    configs, cfg_clk = None, None
+    if not args.no_configs:
+        cclk = ClockSampler(local)
+        cclk.start()
+        configs = run_configs(dev, gstream, rings, hbm_peak, tf_peak)
+        cfg_clk = cclk.stop()
+        status = status or qgemm.device_status(reset=True)
+
     cpu = None
     if rank == 0 and world == 1:
-        gbs, desc, threads, _ = cpu_oracle_sample(fmt, B)
-        cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
-               "sample": desc}
+        sample = oracle_sample(fmt, B, target_s=12.0)
+        t = sample.run()
+        cpu = {"value": round(sample.nbytes / t / 1e9, 4), "unit": "GB/s", "cores": sample.threads,
+               "kind": "oracle", "sample": sample.describe()}
 
-    peak, peak_kind = peaks()
     achieved = k_bytes / (k_ms * 1e-3) / 1e9
     traffic = _traffic_from_profiles()
     line = {
@@ -390,25 +592,37 @@ def main():
         "data": "synthetic (seeded N(0,0.02) weights, N(0,1) bf16 activations)",
         "config": {"workload": WORKLOAD, "fmt": fmt, "B": B, "accumulate": "f32",
                    "weight_bytes_per_step": step_bytes,
-                   "l2": "weights cycle through %d distinct copies per matrix (%.2f GB) > 126 MB L2"
-                         % (RING, RING * step_bytes / 1e9),
+                   "l2": "weights cycle through %d copies per matrix at distinct addresses "
+                         "(%.2f GB) > 126 MB L2" % (RING, RING * step_bytes / 1e9),
                    "timing": "step = CUDA-graph replay of the two calls (fused gate+up, down); "
                              "the kernel figure is, per call, one graph of K back-to-back calls "
                              "between events / K (x preparation + GEMM [+ split-K reduce] per "
                              "call: an upper bound on the GEMM kernel)",
                    "parallelism": "replicas" if world > 1 else "single GPU"},
-        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
-                     "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "kernel": KERNEL, "peak_source": peak_kind,
-                     "bytes_per_launch": int(k_bytes), "avg_launch_us": round(k_ms * 1e3, 3)},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
+                     "unit": "GB/s", "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
+                     "kernel": KERNEL, "peak_source": peak_kind + " (copy bandwidth, burst)",
+                     "bytes_per_launch": int(k_bytes), "avg_launch_us": round(k_ms * 1e3, 3),
+                     "ffn_gate_up_us": round(ffn_us, 2), "down_us": round(down_us, 2)},
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
+                "d2h_bytes_per_step": d2h,
+                "how": "qgemm_ffn_gate_up + qgemm_run per step with x copied in from pinned host "
+                       "memory and y copied back every step; copies on their own streams, two "
+                       "device buffer slots so neighbouring steps' copies overlap compute"},
         "gpu_launches": (launches_per_call(fmt, INTER, HIDDEN, B) + launches_per_call(fmt, HIDDEN, INTER, B))
                         * args.steps,
         "clocks": clk,
         "device_status": status,
     }
+    if configs is not None:
+        line["configs"] = {"peaks": {"hbm_GBps": hbm_peak, "bf16_TFLOPs_burst": tf_peak,
+                                     "source": peak_kind},
+                           "timing": "per call: one CUDA graph of back-to-back calls between "
+                                     "events (decode: 40 calls over a 4-copy weight ring; "
+                                     "prefill: 3-4 calls); frac_hbm = weight bytes / time / "
+                                     "copy bandwidth, frac_tensor = 2MNK / time / burst bf16 peak",
+                           "clocks": cfg_clk, "results": configs}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -96,27 +96,67 @@ bool make_map3(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_
 
 int64_t pad64(int64_t k) { return (k + 63) / 64 * 64; }
 
+// A weight matrix's buffers are present: codes; block scales unless the format has none
+// (FP8); the fp32 tensor scale for the formats that have one (NVFP4, FP8).
+bool weights_given(int fmt, const void* codes, const void* scales, const float* ts) {
+  return codes && (scales || scale_row_bytes(fmt) == 0) && (ts || !has_tensor_scale(fmt));
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int check_fmt_shape(int fmt, int64_t N, int64_t K) {
-  if (fmt != FMT_Q8_0 && fmt != FMT_NVFP4 && fmt != FMT_MXFP4) return QGEMM_ERR_FORMAT;
+  if (fmt != FMT_Q8_0 && fmt != FMT_NVFP4 && fmt != FMT_MXFP4 && fmt != FMT_FP8)
+    return QGEMM_ERR_FORMAT;
   if (N < 1 || K < 1 || N > 0x7FFFFFFF || K > 0x7FFFFFFF) return QGEMM_ERR_SHAPE;
   if (K % block_k(fmt) != 0) return QGEMM_ERR_K_BLOCK;
   return QGEMM_OK;
 }
 
+// Per-device facts looked up once: whether the device is an sm_100 part, and the device
+// addresses of the library's error word and no-alloc scratch there.  Devices beyond
+// kMaxDevices are looked up on every call.
+constexpr int kMaxDevices = 64;
+std::mutex g_dev_mu;
+int g_dev_cc[kMaxDevices] = {};          // 0 unknown, 1 sm_100, 2 other
+int* g_dev_err_ptr[kMaxDevices] = {};
+
+int current_device(int* dev) {
+  const cudaError_t e = cudaGetDevice(dev);
+  return e == cudaSuccess ? QGEMM_OK : cuda_fail(e, "cudaGetDevice");
+}
+
 int device_ok() {
-  static int ok = -1;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    int dev = 0, major = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
-      ok = 0;
-    else
-      ok = (major == 10) ? 1 : 0;
-  });
-  return ok;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < kMaxDevices) {
+    std::lock_guard<std::mutex> lock(g_dev_mu);
+    if (g_dev_cc[dev] != 0) return g_dev_cc[dev] == 1;
+  }
+  int major = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return 0;
+  const int v = (major == 10) ? 1 : 2;
+  if (dev >= 0 && dev < kMaxDevices) {
+    std::lock_guard<std::mutex> lock(g_dev_mu);
+    g_dev_cc[dev] = v;
+  }
+  return v == 1;
+}
+
+// Device address of the library's error word on the current device (nullptr on failure).
+int* error_word() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  if (dev >= 0 && dev < kMaxDevices) {
+    std::lock_guard<std::mutex> lock(g_dev_mu);
+    if (g_dev_err_ptr[dev]) return g_dev_err_ptr[dev];
+  }
+  int* w = device_error_word();
+  if (w && dev >= 0 && dev < kMaxDevices) {
+    std::lock_guard<std::mutex> lock(g_dev_mu);
+    g_dev_err_ptr[dev] = w;
+  }
+  return w;
 }
 
 // The K split of the CTA-pair kernel for widths 1..256: a function of (fmt, N, K) only.  A
@@ -198,7 +238,7 @@ bool make_plan_pair(int fmt, int64_t N, int64_t K, int64_t B, int nmat, Plan* pl
   p.tmem_cols = next_pow2_cols(p.R * p.NACC * p.NB + p.AS * kPairACols);
   if (p.tmem_cols > 512) return false;
   const size_t xstage = (size_t)(p.NB / 2) * 128 * (kPairAK / kSubK);
-  const size_t misc = 8 * (2 * 4 + 2 * kMaxWStages + 2 * 8 + 1) + 16 + 4 * kMaxNB + 64;
+  const size_t misc = 8 * (2 * 4 + 2 * kMaxWStages + 2 * 8 + 1) + 16 + 8 * kMaxNB + 64;
   const size_t budget = kSmemLimit - 1024 - misc;
   const size_t wstage = (size_t)pair_wstage_bytes(fmt);
   int XS = 4;
@@ -211,7 +251,8 @@ bool make_plan_pair(int fmt, int64_t N, int64_t K, int64_t B, int nmat, Plan* pl
   p.smem_w = (uint32_t)(XS * xstage);
   p.smem_bar = p.smem_w + (uint32_t)(WS * wstage);
   const size_t bar_bytes = 8 * (2 * XS + 2 * WS + 2 * p.AS + 1);
-  p.smem_bytes = 1024 + p.smem_bar + bar_bytes + 16 + 4 * p.NB + 64;
+  // control words, then per-column exponents and factors (int and float per batch column)
+  p.smem_bytes = 1024 + p.smem_bar + bar_bytes + 16 + 8 * p.NB + 64;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t o = off;
@@ -227,8 +268,80 @@ bool make_plan_pair(int fmt, int64_t N, int64_t K, int64_t B, int nmat, Plan* pl
   return true;
 }
 
+// Plans are pure functions of (fmt, N, K, B, nmat); each host thread keeps its last few.
+struct PlanKey {
+  int fmt, nmat;
+  int64_t N, K, B;
+  bool operator==(const PlanKey& o) const {
+    return fmt == o.fmt && nmat == o.nmat && N == o.N && K == o.K && B == o.B;
+  }
+};
+constexpr int kCacheEntries = 8;
+struct PlanCache {
+  PlanKey key[kCacheEntries];
+  Plan plan[kCacheEntries];
+  bool ok[kCacheEntries];
+  int used = 0, next = 0;
+};
+thread_local PlanCache g_plans;
+
 bool make_plan(int fmt, int64_t N, int64_t K, int64_t B, int nmat, Plan* pl) {
-  return make_plan_pair(fmt, N, K, B, nmat, pl);
+  const PlanKey k{fmt, nmat, N, K, B};
+  for (int i = 0; i < g_plans.used; ++i)
+    if (g_plans.key[i] == k) {
+      *pl = g_plans.plan[i];
+      return g_plans.ok[i];
+    }
+  const bool ok = make_plan_pair(fmt, N, K, B, nmat, pl);
+  const int i = g_plans.next;
+  g_plans.key[i] = k;
+  g_plans.plan[i] = *pl;
+  g_plans.ok[i] = ok;
+  g_plans.next = (i + 1) % kCacheEntries;
+  if (g_plans.used < kCacheEntries) ++g_plans.used;
+  return ok;
+}
+
+// The x tensor map of a call depends on the operand's address, type and geometry only; each
+// host thread keeps its last few encoded maps (a map holds no device state).
+struct MapKey {
+  int dev, dt, x3d;
+  const void* base;
+  int64_t rows, pitch, K;
+  uint32_t box_rows, box_slices;
+  bool operator==(const MapKey& o) const {
+    return dev == o.dev && dt == o.dt && x3d == o.x3d && base == o.base && rows == o.rows &&
+           pitch == o.pitch && K == o.K && box_rows == o.box_rows && box_slices == o.box_slices;
+  }
+};
+struct MapCache {
+  MapKey key[kCacheEntries];
+  CUtensorMap map[kCacheEntries];
+  int used = 0, next = 0;
+};
+thread_local MapCache g_maps;
+
+// x operand map: 3-D {64, rows, pitch/64} slices when the row pitch is a multiple of 64
+// elements, else 2-D {K, rows} with 64-element boxes.
+bool x_map(CUtensorMap* out, int dev, CUtensorMapDataType dt, const void* base, int64_t rows,
+           int64_t pitch, int64_t K, bool x3d, uint32_t box_rows, uint32_t box_slices) {
+  const MapKey k{dev, (int)dt, x3d ? 1 : 0, base, rows, pitch, K, box_rows, box_slices};
+  for (int i = 0; i < g_maps.used; ++i)
+    if (g_maps.key[i] == k) {
+      *out = g_maps.map[i];
+      return true;
+    }
+  const bool ok = x3d ? make_map3(out, dt, base, (uint64_t)rows, (uint64_t)pitch, box_rows,
+                                  box_slices)
+                      : make_map(out, dt, 2, base, (uint64_t)K, (uint64_t)rows,
+                                 (uint64_t)pitch * 2, kSubK, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!ok) return false;
+  const int i = g_maps.next;
+  g_maps.key[i] = k;
+  g_maps.map[i] = *out;
+  g_maps.next = (i + 1) % kCacheEntries;
+  if (g_maps.used < kCacheEntries) ++g_maps.used;
+  return true;
 }
 
 int run_impl(int fmt, const void* x, int64_t B, int64_t K, const void* const* codes,
@@ -238,7 +351,10 @@ int run_impl(int fmt, const void* x, int64_t B, int64_t K, const void* const* co
   if (!make_plan(fmt, N, K, B, nmat, &pl)) return QGEMM_ERR_SHAPE;
   if (pl.ws_total > 0 && (workspace == nullptr || ws_bytes < pl.ws_total)) return QGEMM_ERR_WORKSPACE;
   if (workspace && !aligned16(workspace)) return QGEMM_ERR_ALIGN;
-  int* dev_err = device_error_word();
+  int dev = 0;
+  int st = current_device(&dev);
+  if (st != QGEMM_OK) return st;
+  int* dev_err = error_word();
   if (!dev_err) return cuda_fail(cudaGetLastError(), "cudaGetSymbolAddress");
   uint8_t* wsb = static_cast<uint8_t*>(workspace);
 
@@ -292,11 +408,8 @@ int run_impl(int fmt, const void* x, int64_t B, int64_t K, const void* const* co
       pl.f16ops ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const int64_t xpitch = pl.f16ops ? pad64(K) : K;  // elements per row of the x operand
   p.x3d = (xpitch % 64 == 0) ? 1 : 0;
-  const bool mapped =
-      p.x3d ? make_map3(&xmap, xdt, xop, (uint64_t)B, (uint64_t)xpitch, (uint32_t)(pl.NB / 2),
-                        (uint32_t)(kPairAK / kSubK))
-            : make_map(&xmap, xdt, 2, xop, (uint64_t)K, (uint64_t)B, (uint64_t)xpitch * 2, kSubK,
-                       (uint32_t)(pl.NB / 2), CU_TENSOR_MAP_SWIZZLE_128B);
+  const bool mapped = x_map(&xmap, dev, xdt, xop, B, xpitch, K, p.x3d != 0,
+                            (uint32_t)(pl.NB / 2), (uint32_t)(kPairAK / kSubK));
   if (!mapped) {
     snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled failed");
     return QGEMM_ERR_CUDA;
@@ -314,8 +427,6 @@ int run_impl(int fmt, const void* x, int64_t B, int64_t K, const void* const* co
     rp.NMAT = nmat;
     rp.B = (int)B;
     rp.N = (int)N;
-    rp.ts[0] = p.ts[0];
-    rp.ts[1] = (nmat == 2) ? p.ts[1] : nullptr;
     rp.out = out;
     rp.out_bf16 = out_bf16;
     e = launch_reduce(rp, stream);
@@ -327,15 +438,14 @@ int run_impl(int fmt, const void* x, int64_t B, int64_t K, const void* const* co
 // Device address of g_noalloc_scratch on the current device, looked up once per device (the
 // lookup may load this library's device code on that device, so it must not happen inside a
 // stream capture).
-constexpr int kMaxNoAllocDevices = 64;
 std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kMaxNoAllocDevices] = {};
+void* g_noalloc_ptr[kMaxDevices] = {};
 
 int noalloc_scratch(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  if (dev < 0 || dev >= kMaxNoAllocDevices) return QGEMM_ERR_DEVICE;
+  if (dev < 0 || dev >= kMaxDevices) return QGEMM_ERR_DEVICE;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
   if (!g_noalloc_ptr[dev]) {
     void* p = nullptr;
@@ -386,7 +496,8 @@ int qgemm_repack_rowmajor(int fmt, int64_t N, int64_t K, const void* codes_rm, i
                           void* stream) {
   const int st = check_fmt_shape(fmt, N, K);
   if (st != QGEMM_OK) return st;
-  if (!codes_rm || !scales_rm || !codes || !scales) return QGEMM_ERR_NULL;
+  if (!codes_rm || !codes || (scale_row_bytes(fmt) > 0 && (!scales_rm || !scales)))
+    return QGEMM_ERR_NULL;
   if (code_pitch < rm_code_bytes_per_row(fmt, K) || scale_pitch < rm_scale_bytes_per_row(fmt, K))
     return QGEMM_ERR_SHAPE;
   if (!aligned16(codes) || !aligned16(scales)) return QGEMM_ERR_ALIGN;
@@ -410,9 +521,10 @@ int qgemm_pack(int fmt, const float* W, int64_t N, int64_t K, void* codes, void*
                float* tensor_scale, void* stream) {
   const int st = check_fmt_shape(fmt, N, K);
   if (st != QGEMM_OK) return st;
-  if (!W || !codes || !scales || (fmt == FMT_NVFP4 && !tensor_scale)) return QGEMM_ERR_NULL;
+  if (!W || !weights_given(fmt, codes, scales, tensor_scale)) return QGEMM_ERR_NULL;
   if (!aligned16(W) || !aligned16(codes) || !aligned16(scales)) return QGEMM_ERR_ALIGN;
-  if (fmt == FMT_NVFP4 && (reinterpret_cast<uintptr_t>(tensor_scale) & 3u)) return QGEMM_ERR_ALIGN;
+  if (has_tensor_scale(fmt) && (reinterpret_cast<uintptr_t>(tensor_scale) & 3u))
+    return QGEMM_ERR_ALIGN;
   if (!device_ok()) return QGEMM_ERR_DEVICE;
   cudaError_t e = launch_pack(fmt, W, N, K, codes, scales, tensor_scale,
                               static_cast<cudaStream_t>(stream));
@@ -498,7 +610,7 @@ int qgemm_run(int fmt, const void* x, int64_t B, int64_t K, const void* codes, c
   if (st != QGEMM_OK) return st;
   if (B < 1 || B > 0x7FFFFFFF) return QGEMM_ERR_SHAPE;
   if (y_dtype != QGEMM_Y_F32 && y_dtype != QGEMM_Y_BF16) return QGEMM_ERR_FORMAT;
-  if (!x || !codes || !scales || !y || (fmt == FMT_NVFP4 && !tensor_scale)) return QGEMM_ERR_NULL;
+  if (!x || !y || !weights_given(fmt, codes, scales, tensor_scale)) return QGEMM_ERR_NULL;
   if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || !aligned16(y))
     return QGEMM_ERR_ALIGN;
   if (!device_ok()) return QGEMM_ERR_DEVICE;
@@ -516,7 +628,7 @@ int qgemm_run_noalloc(int fmt, const void* x, int64_t B, int64_t K, const void* 
   if (st != QGEMM_OK) return st;
   if (B < 1 || B > 0x7FFFFFFF) return QGEMM_ERR_SHAPE;
   if (y_dtype != QGEMM_Y_F32 && y_dtype != QGEMM_Y_BF16) return QGEMM_ERR_FORMAT;
-  if (!x || !codes || !scales || !y || (fmt == FMT_NVFP4 && !tensor_scale)) return QGEMM_ERR_NULL;
+  if (!x || !y || !weights_given(fmt, codes, scales, tensor_scale)) return QGEMM_ERR_NULL;
   if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || !aligned16(y))
     return QGEMM_ERR_ALIGN;
   // the same plan qgemm_run would use; its workspace must fit the fixed scratch
@@ -541,8 +653,9 @@ int qgemm_ffn_gate_up(int fmt, const void* x, int64_t M, int64_t K, const void* 
   int st = check_fmt_shape(fmt, N, K);
   if (st != QGEMM_OK) return st;
   if (M < 1 || M > 0x7FFFFFFF) return QGEMM_ERR_SHAPE;
-  if (!x || !g_codes || !g_scales || !u_codes || !u_scales || !h) return QGEMM_ERR_NULL;
-  if (fmt == FMT_NVFP4 && (!g_ts || !u_ts)) return QGEMM_ERR_NULL;
+  if (!x || !h || !weights_given(fmt, g_codes, g_scales, g_ts) ||
+      !weights_given(fmt, u_codes, u_scales, u_ts))
+    return QGEMM_ERR_NULL;
   if (!aligned16(x) || !aligned16(g_codes) || !aligned16(g_scales) || !aligned16(u_codes) ||
       !aligned16(u_scales) || !aligned16(h))
     return QGEMM_ERR_ALIGN;
@@ -573,8 +686,6 @@ int qgemm_ffn_gate_up(int fmt, const void* x, int64_t M, int64_t K, const void* 
       rp.NMAT = 2;
       rp.B = (int)mc;
       rp.N = (int)N;
-      rp.ts[0] = nullptr;  // the GEMM epilogues applied the tensor scales
-      rp.ts[1] = nullptr;
       rp.out = static_cast<uint8_t*>(h) + (size_t)r0 * (size_t)N * 2;
       rp.out_bf16 = 1;
       const cudaError_t e = launch_reduce(rp, st);
@@ -592,7 +703,7 @@ int qgemm_ffn_gate_up(int fmt, const void* x, int64_t M, int64_t K, const void* 
 int qgemm_device_status(int reset) {
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
-  int* w = device_error_word();
+  int* w = error_word();
   if (!w) return cuda_fail(cudaGetLastError(), "cudaGetSymbolAddress");
   int v = 0;
   e = cudaMemcpy(&v, w, sizeof(int), cudaMemcpyDeviceToHost);

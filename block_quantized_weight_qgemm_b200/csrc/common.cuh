@@ -5,7 +5,7 @@
 
 namespace qg {
 
-enum Fmt : int { FMT_Q8_0 = 0, FMT_NVFP4 = 1, FMT_MXFP4 = 2 };
+enum Fmt : int { FMT_Q8_0 = 0, FMT_NVFP4 = 1, FMT_MXFP4 = 2, FMT_FP8 = 3 };
 
 // ---- tile geometry (tcgen05, swap-AB: weight rows are the MMA M dimension) -------------
 constexpr int kTileRows = 128;                    // weight rows per subtile (MMA M)
@@ -25,11 +25,22 @@ constexpr int kPairACols = kPairAK / 2;           // its TMEM columns
 constexpr int kMaxNB = 256;                       // MMA N limit
 constexpr int kSmemLimit = 227 * 1024;
 
+// one byte per element (Q8_0, FP8) or two (NVFP4, MXFP4)
+__host__ __device__ constexpr bool byte_codes(int fmt) { return fmt == FMT_Q8_0 || fmt == FMT_FP8; }
 // K covered by one weight stage (128 code bytes per row).
-__host__ __device__ constexpr int chunk_k(int fmt) { return fmt == FMT_Q8_0 ? 128 : 256; }
-__host__ __device__ constexpr int block_k(int fmt) { return fmt == FMT_NVFP4 ? 16 : 32; }
-// scale bytes per row per chunk: Q8_0 4 x fp16, NVFP4 16 x E4M3, MXFP4 8 x E8M0
-__host__ __device__ constexpr int scale_row_bytes(int fmt) { return fmt == FMT_NVFP4 ? 16 : 8; }
+__host__ __device__ constexpr int chunk_k(int fmt) { return byte_codes(fmt) ? 128 : 256; }
+// K granularity: the scale block (FP8 has none; 16 keeps every x row 32-byte aligned)
+__host__ __device__ constexpr int block_k(int fmt) {
+  return (fmt == FMT_NVFP4 || fmt == FMT_FP8) ? 16 : 32;
+}
+// scale bytes per row per chunk: Q8_0 4 x fp16, NVFP4 16 x E4M3, MXFP4 8 x E8M0, FP8 none
+__host__ __device__ constexpr int scale_row_bytes(int fmt) {
+  return fmt == FMT_NVFP4 ? 16 : fmt == FMT_FP8 ? 0 : 8;
+}
+// formats with an fp32 tensor scale applied in the epilogue
+__host__ __device__ constexpr bool has_tensor_scale(int fmt) {
+  return fmt == FMT_NVFP4 || fmt == FMT_FP8;
+}
 __host__ __device__ constexpr int64_t row_tiles(int64_t N) { return (N + kTileRows - 1) / kTileRows; }
 __host__ __device__ constexpr int64_t k_chunks(int fmt, int64_t K) {
   return (K + chunk_k(fmt) - 1) / chunk_k(fmt);
@@ -43,10 +54,10 @@ __host__ __device__ constexpr int pair_wstage_bytes(int fmt) {
 // scales [N][scale pitch], rows 16-byte aligned.
 __host__ __device__ constexpr int64_t roundup16(int64_t v) { return (v + 15) / 16 * 16; }
 __host__ __device__ constexpr int64_t rm_code_bytes_per_row(int fmt, int64_t K) {
-  return fmt == FMT_Q8_0 ? K : K / 2;
+  return byte_codes(fmt) ? K : K / 2;
 }
 __host__ __device__ constexpr int64_t rm_scale_bytes_per_row(int fmt, int64_t K) {
-  return fmt == FMT_Q8_0 ? 2 * (K / 32) : fmt == FMT_NVFP4 ? K / 16 : K / 32;
+  return fmt == FMT_Q8_0 ? 2 * (K / 32) : fmt == FMT_NVFP4 ? K / 16 : fmt == FMT_FP8 ? 0 : K / 32;
 }
 __host__ __device__ constexpr int64_t rm_code_pitch(int fmt, int64_t K) {
   return roundup16(rm_code_bytes_per_row(fmt, K));
@@ -90,20 +101,20 @@ struct GemmParams {
   int NACC;      // pair kernel: accumulators per subtile (1, or 2 for the f16 path)
   uint32_t smem_x, smem_w, smem_bar;  // byte offsets in the 1024-aligned dynamic smem
   const int* x_exp;          // f16 operands: x row b was scaled by 2^-x_exp[b]
-  const float* ts[2];        // NVFP4 tensor scales (device), else nullptr
+  const float* ts[2];        // NVFP4 / FP8 tensor scales (device), else nullptr
   const uint8_t* codes[2];   // tile-major packed codes of each matrix
   const uint8_t* scales[2];  // tile-major packed scales of each matrix
-  float* ws;                 // split-K partials [S][NMAT][B][N]
+  float* ws;                 // split-K partials [S][NMAT][B][N], fully scaled
   void* out;                 // y [B][N] (fp32 or bf16), or h [B][N] bf16 for NMAT == 2
   int out_bf16;
   int* dev_err;
 };
 
-// Fixed-order sum of the split-K partials and the output epilogue.
+// Fixed-order sum of the split-K partials and the output epilogue.  The partials carry every
+// scale already (the GEMM epilogue applies the tensor scale and the powers of two).
 struct ReduceParams {
   const float* ws;     // partials [S][NMAT][B][N]
   int S, NMAT, B, N;
-  const float* ts[2];  // NVFP4 tensor scales, else nullptr
   void* out;           // y [B][N] fp32 / bf16, or h [B][N] bf16 for NMAT == 2
   int out_bf16;
 };

@@ -151,6 +151,47 @@ struct Dequant<FMT_MXFP4, false> {
   }
 };
 
+// FP8 (E4M3) -> f16: the hardware E4M3x2 -> f16x2 conversion (every E4M3 value is exact in
+// f16); the tensor scale is applied in the epilogue.
+template <>
+struct Dequant<FMT_FP8, false> {
+  __device__ __forceinline__ static void run(const uint8_t* crow, int row, const uint8_t* /*srow*/,
+                                             int /*c*/, int e0, int /*ex*/, uint32_t (&v)[16]) {
+    const uint4 a = ld_sw128(crow, row, e0 >> 4);
+    const uint4 b = ld_sw128(crow, row, (e0 >> 4) + 1);
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[i] & 0xFFFFu), __NV_E4M3);
+      const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[i] >> 16), __NV_E4M3);
+      v[2 * i] = (uint32_t)lo.x | ((uint32_t)lo.y << 16);
+      v[2 * i + 1] = (uint32_t)hi.x | ((uint32_t)hi.y << 16);
+    }
+  }
+};
+
+// FP8 (E4M3) -> bf16 through f16 and fp32 (every E4M3 value is exact in each).
+template <>
+struct Dequant<FMT_FP8, true> {
+  __device__ __forceinline__ static void run(const uint8_t* crow, int row, const uint8_t* /*srow*/,
+                                             int /*c*/, int e0, int /*ex*/, uint32_t (&v)[16]) {
+    const uint4 a = ld_sw128(crow, row, e0 >> 4);
+    const uint4 b = ld_sw128(crow, row, (e0 >> 4) + 1);
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const __half2_raw r =
+            __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)((w[i] >> (16 * j)) & 0xFFFFu), __NV_E4M3);
+        __half2 h;
+        *reinterpret_cast<__half2_raw*>(&h) = r;
+        v[2 * i + j] = b2u(__float22bfloat162_rn(__half22float2(h)));
+      }
+    }
+  }
+};
+
 // E2M1 -> bf16 for 8 codes in one word (two prmt byte tables for the magnitude, prmt sign
 // replication for the sign bits), times a broadcast bf16 scale (exact).
 __device__ __forceinline__ void e2m1x8_bf16(uint32_t w, __nv_bfloat162 s, uint32_t* out) {
@@ -213,6 +254,19 @@ struct Dequant<FMT_MXFP4, true> {
 // ---------------------------------------------------------------------------------------
 // Epilogue helpers
 // ---------------------------------------------------------------------------------------
+// 2^e as a float, exact for -149 <= e <= 127 (subnormal below -126), 0 below -149.
+__device__ __forceinline__ float exp2_exact(int e) {
+  if (e >= -126) return __int_as_float((min(e, 127) + 127) << 23);
+  return e >= -149 ? __int_as_float(1 << (e + 149)) : 0.0f;
+}
+
+// Epilogue exponents within +-kFastExp take plain multiplies by exact powers of two.
+constexpr int kFastExp = 60;
+
+// v * 2^ex with a single rounding, for any ex (x rows of bf16 subnormals give ex down to
+// -147); kept out of line, off the epilogue's fast path.
+static __device__ __noinline__ float scale_pow2_exact(float v, int ex) { return ldexpf(v, ex); }
+
 __device__ __forceinline__ void store_y(const GemmParams& p, int b, int n, float v) {
   if (p.out_bf16)
     reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)b * p.N + n] = __float2bfloat16_rn(v);

@@ -16,10 +16,12 @@ namespace qg {
 __device__ int g_dev_err = 0;
 
 // ---------------------------------------------------------------------------------------
-// x preparation for the f16 path (Q8_0, widths <= 256): per row, e = floor(log2 amax) - 14,
+// x preparation for the f16 path (widths <= 256): per row, e = floor(log2 amax) - 14,
 // xh = f16(x * 2^-e) (exact for every bf16 value within 2^-38 of the row maximum), and the
 // row's exponent e, which the GEMM epilogue restores.  Rows of xh are padded with zeros to
-// a multiple of 64 elements.
+// a multiple of 64 elements.  e runs from -147 (a row of bf16 subnormals) to 113, so 2^-e
+// can exceed the largest fp32 power of two; it is applied as two exact factors, 2^n1 with
+// n1 = min(-e, 126) and 2^(-e - n1) (which is 1 unless the row's maximum is below 2^-112).
 // ---------------------------------------------------------------------------------------
 constexpr int kPrepThreads = 1024;  // one CTA per x row
 constexpr int kPrepRegs = 3;        // 16-byte words per thread held in registers (rows to 24576)
@@ -34,13 +36,15 @@ __device__ __forceinline__ float amax8(float m, const uint4& v) {
   return m;
 }
 
-__device__ __forceinline__ uint4 to_f16x8(const uint4& v, float sc) {
+// 8 bf16 values times 2^n1 * 2^n2 (both factors normal powers of two: each product is exact
+// unless it leaves the f16 range), rounded once to f16
+__device__ __forceinline__ uint4 to_f16x8(const uint4& v, float sc1, float sc2) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   uint32_t o[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const __half lo = __float2half_rn(__uint_as_float(w[i] << 16) * sc);
-    const __half hi = __float2half_rn(__uint_as_float(w[i] & 0xFFFF0000u) * sc);
+    const __half lo = __float2half_rn(__uint_as_float(w[i] << 16) * sc1 * sc2);
+    const __half hi = __float2half_rn(__uint_as_float(w[i] & 0xFFFF0000u) * sc1 * sc2);
     o[i] = (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
   }
   return make_uint4(o[0], o[1], o[2], o[3]);
@@ -85,15 +89,18 @@ __global__ void __launch_bounds__(kPrepThreads) qgemm_prep_x_kernel(const PrepPa
     (void)frexpf(amax, &ex);  // amax = f * 2^ex, f in [0.5, 1)
     e = (ex - 1) - 14;        // amax * 2^-e in [2^14, 2^15)
   }
-  const float sc = ldexpf(1.0f, -e);
+  const int n1 = min(-e, 126);
+  const float sc1 = __int_as_float((n1 + 127) << 23);      // 2^n1, n1 in [-113, 126]
+  const float sc2 = __int_as_float((-e - n1 + 127) << 23);  // 2^(-e-n1), exponent in [0, 21]
   uint16_t* xo = p.xh + (size_t)b * p.Kp;
 #pragma unroll
   for (int j = 0; j < kPrepRegs; ++j) {
     const int k = (threadIdx.x + j * kPrepThreads) * 8;
-    if (k < p.K) *reinterpret_cast<uint4*>(xo + k) = to_f16x8(v[j], sc);
+    if (k < p.K) *reinterpret_cast<uint4*>(xo + k) = to_f16x8(v[j], sc1, sc2);
   }
   for (int k = (threadIdx.x + kPrepRegs * kPrepThreads) * 8; k < p.K; k += kPrepThreads * 8)
-    *reinterpret_cast<uint4*>(xo + k) = to_f16x8(*reinterpret_cast<const uint4*>(xr + k), sc);
+    *reinterpret_cast<uint4*>(xo + k) =
+        to_f16x8(*reinterpret_cast<const uint4*>(xr + k), sc1, sc2);
   for (int k = p.K + threadIdx.x * 8; k < p.Kp; k += kPrepThreads * 8)
     *reinterpret_cast<uint4*>(xo + k) = make_uint4(0u, 0u, 0u, 0u);
   if (threadIdx.x == 0) p.x_exp[b] = e;
@@ -101,7 +108,8 @@ __global__ void __launch_bounds__(kPrepThreads) qgemm_prep_x_kernel(const PrepPa
 
 // ---------------------------------------------------------------------------------------
 // Split-K reduction: out = epilogue(sum_{s=0..S-1} partial_s), in that fixed order, one
-// 4-wide column group (b, n..n+3) per thread.
+// 4-wide column group (b, n..n+3) per thread.  The epilogue is the output conversion, or
+// SiLU(g) * u for the fused gate+up.
 // ---------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) qgemm_splitk_reduce_kernel(const ReduceParams p) {
   griddep_launch_dependents();  // the next call's preparation may launch and wait
@@ -132,19 +140,15 @@ __global__ void __launch_bounds__(256) qgemm_splitk_reduce_kernel(const ReducePa
       }
     }
   }
-  const float ts0 = p.ts[0] ? __ldg(p.ts[0]) : 1.0f;
-  const float ts1 = (p.NMAT == 2 && p.ts[1]) ? __ldg(p.ts[1]) : 1.0f;
+  // the partials already carry every scale (tensor scale, x and row exponents)
   for (int e = 0; e < lim; ++e) {
     if (p.NMAT == 1) {
-      const float v = g[e] * ts0;
       if (p.out_bf16)
-        reinterpret_cast<__nv_bfloat16*>(p.out)[off + e] = __float2bfloat16_rn(v);
+        reinterpret_cast<__nv_bfloat16*>(p.out)[off + e] = __float2bfloat16_rn(g[e]);
       else
-        reinterpret_cast<float*>(p.out)[off + e] = v;
+        reinterpret_cast<float*>(p.out)[off + e] = g[e];
     } else {
-      const float gv = g[e] * ts0, uv = u[e] * ts1;
-      reinterpret_cast<__nv_bfloat16*>(p.out)[off + e] =
-          __float2bfloat16_rn(silu_mul(gv, uv));
+      reinterpret_cast<__nv_bfloat16*>(p.out)[off + e] = __float2bfloat16_rn(silu_mul(g[e], u[e]));
     }
   }
 }

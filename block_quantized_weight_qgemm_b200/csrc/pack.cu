@@ -5,6 +5,7 @@
 //   NVFP4: ts = fp32_RNE(amax(W)/2688); s = E4M3_RNE_sat(amax_blk/(6 ts));
 //          code = E2M1_RNE_sat(w/(e4m3(s) ts)).
 //   MXFP4: e = clamp(floor(log2 amax_blk) - 2 + 127, 0, 254); code = E2M1_RNE_sat(w/2^(e-127)).
+//   FP8  : ts = fp32_RNE(amax(W)/448); code = E4M3_RNE_sat(w/ts), sign kept at zero.
 // Every quotient is formed once in fp64 from exact operands (the divisor products are exact
 // in fp64), then rounded once to the target format -- fp16 by the integer routine below,
 // E4M3 / E2M1 by NVIDIA's double -> fp8 / fp4 conversions -- so ties are decided on the
@@ -88,6 +89,10 @@ __device__ __forceinline__ float nvfp4_ts_from_amax(float amax) {
   return __double2float_rn((double)amax / (6.0 * 448.0));
 }
 
+__device__ __forceinline__ float fp8_ts_from_amax(float amax) {
+  return __double2float_rn((double)amax / 448.0);
+}
+
 // One thread per 16-element block.  amax_bits holds max|W| (written by amax_kernel).
 __global__ void pack_nvfp4_kernel(const float* __restrict__ W, int64_t N, int64_t K,
                                   uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
@@ -123,6 +128,34 @@ __global__ void pack_nvfp4_kernel(const float* __restrict__ W, int64_t N, int64_
 __global__ void nvfp4_finish_kernel(float* tensor_scale) {
   const unsigned int bits = *reinterpret_cast<unsigned int*>(tensor_scale);
   *tensor_scale = nvfp4_ts_from_amax(__uint_as_float(bits));
+}
+
+// One thread per 16 consecutive elements of a row.  amax_bits holds max|W|.
+__global__ void pack_fp8_kernel(const float* __restrict__ W, int64_t N, int64_t K,
+                                uint8_t* __restrict__ codes, const unsigned int* amax_bits) {
+  const int64_t nb = K / 16;
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= N * nb) return;
+  const int64_t n = idx / nb, kb = idx % nb;
+  const float ts = fp8_ts_from_amax(__uint_as_float(*amax_bits));
+  const float* w = W + n * K + kb * 16;
+  const int64_t C = k_chunks(FMT_FP8, K);
+  const int64_t k0 = kb * 16, c = k0 / 128;
+  const int b0 = (int)(k0 % 128);
+  for (int i = 0; i < 16; ++i) {
+    uint32_t code = 0;
+    if (ts != 0.f) {
+      const double v = (double)w[i] / (double)ts;
+      code = ((uint32_t)__nv_cvt_double_to_fp8(fabs(v), __NV_SATFINITE, __NV_E4M3) & 0x7Fu) |
+             (v < 0.0 ? 0x80u : 0u);
+    }
+    codes[code_offset(C, n, c, b0 + i)] = (uint8_t)code;
+  }
+}
+
+__global__ void fp8_finish_kernel(float* tensor_scale) {
+  const unsigned int bits = *reinterpret_cast<unsigned int*>(tensor_scale);
+  *tensor_scale = fp8_ts_from_amax(__uint_as_float(bits));
 }
 
 // One thread per 32-element block.
@@ -192,8 +225,10 @@ cudaError_t launch_pack(int fmt, const float* W, int64_t N, int64_t K, void* cod
   // padding rows and K past the last block are zero
   e = cudaMemsetAsync(codes, 0, (size_t)packed_code_bytes(fmt, N, K), stream);
   if (e != cudaSuccess) return e;
-  e = cudaMemsetAsync(scales, 0, (size_t)packed_scale_bytes(fmt, N, K), stream);
-  if (e != cudaSuccess) return e;
+  if (packed_scale_bytes(fmt, N, K) > 0) {
+    e = cudaMemsetAsync(scales, 0, (size_t)packed_scale_bytes(fmt, N, K), stream);
+    if (e != cudaSuccess) return e;
+  }
   const int threads = 256;
   if (fmt == FMT_Q8_0) {
     const int64_t blocks = (N * (K / 32) + threads - 1) / threads;
@@ -207,6 +242,14 @@ cudaError_t launch_pack(int fmt, const float* W, int64_t N, int64_t K, void* cod
     pack_nvfp4_kernel<<<(unsigned)blocks, threads, 0, stream>>>(
         W, N, K, (uint8_t*)codes, (uint8_t*)scales, reinterpret_cast<unsigned int*>(tensor_scale));
     nvfp4_finish_kernel<<<1, 1, 0, stream>>>(tensor_scale);
+  } else if (fmt == FMT_FP8) {
+    e = cudaMemsetAsync(tensor_scale, 0, sizeof(float), stream);
+    if (e != cudaSuccess) return e;
+    amax_kernel<<<1184, threads, 0, stream>>>(W, N * K, reinterpret_cast<unsigned int*>(tensor_scale));
+    const int64_t blocks = (N * (K / 16) + threads - 1) / threads;
+    pack_fp8_kernel<<<(unsigned)blocks, threads, 0, stream>>>(
+        W, N, K, (uint8_t*)codes, reinterpret_cast<unsigned int*>(tensor_scale));
+    fp8_finish_kernel<<<1, 1, 0, stream>>>(tensor_scale);
   } else {
     const int64_t blocks = (N * (K / 32) + threads - 1) / threads;
     pack_mxfp4_kernel<<<(unsigned)blocks, threads, 0, stream>>>(W, N, K, (uint8_t*)codes,

@@ -71,7 +71,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   const uint32_t bar_acc = bar_a_empty + 8 * AS;
   int* ctl = reinterpret_cast<int*>(bars + 2 * XS + 2 * WS + 2 * AS + 1);
   volatile int* abort_flag = ctl + 1;
-  float* col_fac = reinterpret_cast<float*>(ctl + 4);
+  // per batch column: the x row's power-of-two exponent, and 2^exponent as an exact float
+  int* col_exp = ctl + 4;
+  float* col_fac = reinterpret_cast<float*>(ctl + 4 + p.NB);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();  // 0: even CTA (issues the MMAs), 1: odd CTA
@@ -107,6 +109,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     mbar_init(bar_acc, 2);  // one final commit per issuer
     ctl[1] = 0;
     ctl[2] = 0;
+    ctl[3] = 0;  // set when a column's exponent leaves the epilogue's fast range
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -150,7 +153,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           const uint32_t sbytes = (uint32_t)n * (kTileRows * SB);
           mbar_arrive_expect_tx(fb, cbytes + sbytes);
           bulk_load(dst, p.codes[m] + blk * kWCodeBytes, cbytes, fb, pol_w);
-          bulk_load(dst + WSCALES, p.scales[m] + blk * (kTileRows * SB), sbytes, fb, pol_w);
+          if (SB > 0)
+            bulk_load(dst + WSCALES, p.scales[m] + blk * (kTileRows * SB), sbytes, fb, pol_w);
         } else {
           mbar_arrive(fb);  // a tile past the matrix: its rows are never stored
         }
@@ -394,12 +398,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 
     // the output may be read by a dependent grid only after it completes; let it launch
     griddep_launch_dependents();
-    // per-column factors 2^x_exp[b] (f16 path); x_exp comes from the preceding grid.  Loaded
+    // per-column exponents x_exp[b] (f16 path); x_exp comes from the preceding grid.  Loaded
     // before the accumulator wait so that their latency hides behind the last MMAs.
     griddep_wait();
     for (int i = threadIdx.x - kPairFirstDequantWarp * 32; i < p.NB; i += kPairDequantWarps * 32) {
       const int b = bt * p.NB + i;
-      col_fac[i] = (b < p.B) ? (p.x_exp ? ldexpf(1.0f, p.x_exp[b]) : 1.0f) : 0.0f;
+      const int ce = (b < p.B && p.x_exp) ? p.x_exp[b] : 0;
+      col_exp[i] = ce;
+      col_fac[i] = exp2_exact(ce);
+      if (ce < -kFastExp || ce > kFastExp) ctl[3] = 1;
     }
     asm volatile("bar.sync 1, %0;" ::"r"(kPairDequantWarps * 32) : "memory");
     if (ok) {
@@ -411,14 +418,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     const int cb0 = h * qcols;
     const size_t BN = (size_t)p.B * p.N;
     float ts[2] = {1.0f, 1.0f};
-    if (FMT == FMT_NVFP4) {
+    if (has_tensor_scale(FMT)) {
       ts[0] = __ldg(p.ts[0]);
       if (p.NMAT == 2) ts[1] = __ldg(p.ts[1]);
     }
-    float rowfac[4] = {1.0f, 1.0f, 1.0f, 1.0f};
-    if (FMT == FMT_MXFP4 && !BF16OP)
+    // per-row exponent restored by the epilogue: the MXFP4 f16 rebase (2^(E - Emax + 13) in
+    // the operand for a block scale 2^(E - 127))
+    constexpr bool kRowExp = (FMT == FMT_MXFP4 && !BF16OP);
+    int rowexp[4] = {0, 0, 0, 0};
+    if (kRowExp)
 #pragma unroll
-      for (int r = 0; r < 4; ++r) rowfac[r] = ldexpf(1.0f, emax[r] - 140);
+      for (int r = 0; r < 4; ++r) rowexp[r] = emax[r] - 140;
+    // Fast path: with every exponent within +-kFastExp, ((acc * ts) * 2^re) * 2^ce rounds once
+    // except at subnormal magnitudes far below the accuracy bound; otherwise (x rows near the
+    // ends of the bf16 range) each output is scaled by one exactly rounded ldexpf.
+    const bool cols_fast = (ctl[3] == 0);
     const bool two_acc = (p.NACC == 2 && ngroups > 1);
     if (ok) {
       // scale the accumulators; store finals (S == 1) or partials (S > 1)
@@ -426,8 +440,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         const int64_t t = 2 * ((int64_t)g * tpg + lt) + rank;
         const int64_t n64 = t * kTileRows + row;
         const int n = (int)n64;
-        const float rf_g = sel4(rowfac, lt * p.NMAT);
-        const float rf_u = sel4(rowfac, lt * p.NMAT + 1);
+        const int re_g = sel4(rowexp, lt * p.NMAT);
+        const int re_u = sel4(rowexp, lt * p.NMAT + 1);
+        const float rf_g = exp2_exact(re_g), rf_u = exp2_exact(re_u);
+        const bool fast_g = cols_fast && re_g >= -kFastExp && re_g <= kFastExp;
+        const bool fast_u = cols_fast && re_u >= -kFastExp && re_u <= kFastExp;
         for (int cb = cb0; cb < cb0 + qcols; cb += 16) {
           const int ngrp = min(16, cb0 + qcols - cb) >> 2;  // groups of 4 columns
           uint32_t va[4][4], vb[4][4];
@@ -472,18 +489,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
               const int col = cb + g4 * 4 + i;
               const int b = bt * p.NB + col;
               if (b >= p.B) break;
+              // tensor scale first, then the row's and the column's powers of two
               const float cf = col_fac[col];
-              const float ga = __uint_as_float(va[g4][i]) * cf * rf_g;
+              const float vg = __uint_as_float(va[g4][i]) * ts[0];
+              const float ga = fast_g ? (kRowExp ? vg * rf_g : vg) * cf
+                                      : scale_pow2_exact(vg, col_exp[col] + re_g);
               if (p.NMAT == 1) {
                 if (p.S > 1) p.ws[(size_t)s * BN + (size_t)b * p.N + n] = ga;
-                else store_y(p, b, n, ga * ts[0]);
+                else store_y(p, b, n, ga);
               } else {
-                const float ua = __uint_as_float(vb[g4][i]) * cf * rf_u;
+                const float vu = __uint_as_float(vb[g4][i]) * ts[1];
+                const float ua = fast_u ? (kRowExp ? vu * rf_u : vu) * cf
+                                        : scale_pow2_exact(vu, col_exp[col] + re_u);
                 if (p.S > 1) {
                   p.ws[(size_t)(2 * s) * BN + (size_t)b * p.N + n] = ga;
                   p.ws[(size_t)(2 * s + 1) * BN + (size_t)b * p.N + n] = ua;
                 } else {
-                  store_h(p, b, n, ga * ts[0], ua * ts[1]);
+                  store_h(p, b, n, ga, ua);
                 }
               }
             }
@@ -555,9 +577,12 @@ cudaError_t launch_pair(int fmt, bool bf16op, const GemmParams& p, size_t smem_b
     case FMT_NVFP4:
       return bf16op ? launch_pair_impl<FMT_NVFP4, true>(p, smem_bytes, units, maps, pdl, stream)
                     : launch_pair_impl<FMT_NVFP4, false>(p, smem_bytes, units, maps, pdl, stream);
-    default:
+    case FMT_MXFP4:
       return bf16op ? launch_pair_impl<FMT_MXFP4, true>(p, smem_bytes, units, maps, pdl, stream)
                     : launch_pair_impl<FMT_MXFP4, false>(p, smem_bytes, units, maps, pdl, stream);
+    default:
+      return bf16op ? launch_pair_impl<FMT_FP8, true>(p, smem_bytes, units, maps, pdl, stream)
+                    : launch_pair_impl<FMT_FP8, false>(p, smem_bytes, units, maps, pdl, stream);
   }
 }
 

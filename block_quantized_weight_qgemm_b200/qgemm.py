@@ -13,10 +13,11 @@ import threading
 
 import torch
 
-Q8_0, NVFP4, MXFP4 = 0, 1, 2
-FORMATS = {"q8_0": Q8_0, "nvfp4": NVFP4, "mxfp4": MXFP4}
+Q8_0, NVFP4, MXFP4, FP8 = 0, 1, 2, 3
+FORMATS = {"q8_0": Q8_0, "nvfp4": NVFP4, "mxfp4": MXFP4, "fp8": FP8}
 Y_F32, Y_BF16 = 0, 1
-BLOCK = {Q8_0: 32, NVFP4: 16, MXFP4: 32}
+BLOCK = {Q8_0: 32, NVFP4: 16, MXFP4: 32, FP8: 16}  # K granularity (FP8: no block scales)
+TENSOR_SCALE = (NVFP4, FP8)
 
 OK = 0
 STATUS = {
@@ -89,7 +90,8 @@ def _check(status: int, where: str):
 
 
 def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    """Device address of a tensor (None for a missing or empty one)."""
+    return None if (t is None or t.numel() == 0) else ctypes.c_void_p(t.data_ptr())
 
 
 def _stream(stream=None):
@@ -154,7 +156,8 @@ def profile_events(begin=None, end=None):
 # ---- packed weights ---------------------------------------------------------------------
 
 class PackedWeight:
-    """Device buffers of one packed [N, K] matrix (codes, scales, optional tensor scale)."""
+    """Device buffers of one packed [N, K] matrix (codes, block scales -- empty for FP8 --
+    and the fp32 tensor scale of NVFP4 and FP8)."""
 
     def __init__(self, fmt, N: int, K: int, device=None):
         self.fmt = _fmt(fmt)
@@ -164,13 +167,16 @@ class PackedWeight:
         self.codes = torch.empty(cb, dtype=torch.uint8, device=device)   # tile-major layout
         self.scales = torch.empty(sb, dtype=torch.uint8, device=device)
         self.tensor_scale = (torch.empty(1, dtype=torch.float32, device=device)
-                             if self.fmt == NVFP4 else None)
+                             if self.fmt in TENSOR_SCALE else None)
 
     @property
     def nbytes(self) -> int:
         """Algorithmic bytes a GEMM reads for this matrix (codes + scales, no row padding)."""
-        code = self.N * (self.K if self.fmt == Q8_0 else self.K // 2)
-        scale = self.N * (2 * self.K // 32 if self.fmt == Q8_0 else self.K // BLOCK[self.fmt])
+        code = self.N * (self.K if self.fmt in (Q8_0, FP8) else self.K // 2)
+        if self.fmt == FP8:
+            scale = 0
+        else:
+            scale = self.N * (2 * self.K // 32 if self.fmt == Q8_0 else self.K // BLOCK[self.fmt])
         return code + scale
 
 
@@ -189,8 +195,9 @@ def repack_rowmajor(fmt, codes_rm: torch.Tensor, scales_rm: torch.Tensor, N: int
     """qgemm_repack_rowmajor: row-major interchange layout [N, pitch] -> PackedWeight."""
     assert codes_rm.is_cuda and scales_rm.is_cuda and codes_rm.dim() == 2 and scales_rm.dim() == 2
     pw = out or PackedWeight(fmt, N, K, codes_rm.device)
+    spitch = scales_rm.stride(0) if scales_rm.numel() else 0
     _check(lib().qgemm_repack_rowmajor(pw.fmt, N, K, _ptr(codes_rm), codes_rm.stride(0),
-                                       _ptr(scales_rm), scales_rm.stride(0), _ptr(pw.codes),
+                                       _ptr(scales_rm), spitch, _ptr(pw.codes),
                                        _ptr(pw.scales), _stream(stream)), "qgemm_repack_rowmajor")
     return pw
 

@@ -18,23 +18,27 @@
  *                   the Atlas issue's exact-F16-dequant section).
  *   QGEMM_FMT_MXFP4 E2M1 codes; one E8M0 scale per 32 consecutive k (the MXFP4 model
  *                   card's format, OCP MX v1.0):  w = e2m1 * 2^(e-127).
+ *   QGEMM_FMT_FP8   E4M3 codes; no block scales; one fp32 tensor scale ts:  w = e4m3 * ts
+ *                   (the FP8 W8A16 layers of the Atlas issue's kernel ranking and verify-tier
+ *                   sections; ts applied in the epilogue).  K must be a multiple of 16.
  *
  * Packed layout (tile-major; what qgemm_pack writes and qgemm_run reads).  Rows are grouped
- * in tiles of 128 (T = ceil(N/128)), K in chunks of CK elements (CK = 128 for Q8_0, 256 for
- * NVFP4 and MXFP4; C = ceil(K/CK)).  Rows past N and elements past K are zero.
+ * in tiles of 128 (T = ceil(N/128)), K in chunks of CK elements (CK = 128 for Q8_0 and FP8,
+ * 256 for NVFP4 and MXFP4; C = ceil(K/CK)).  Rows past N and elements past K are zero.
  *   codes  [T][C][128 rows][128 bytes]: the row's CK elements of the chunk (Q8_0: one int8
- *          byte each; FP4: element 2j in the low nibble of byte j), with the row's 16-byte
- *          groups permuted: group g of row r is stored at position g ^ (r & 7).
- *          Size T*C*16384 bytes.
- *   scales [T][C][128 rows][SB bytes], SB = 8 (Q8_0: 4 little-endian fp16; MXFP4: 8 E8M0)
- *          or 16 (NVFP4: 16 E4M3), the row's block scales of the chunk in K order.
- *          Size T*C*128*SB bytes.
+ *          byte each; FP8: one E4M3 byte each; FP4: element 2j in the low nibble of byte j),
+ *          with the row's 16-byte groups permuted: group g of row r is stored at position
+ *          g ^ (r & 7).  Size T*C*16384 bytes.
+ *   scales [T][C][128 rows][SB bytes], SB = 8 (Q8_0: 4 little-endian fp16; MXFP4: 8 E8M0),
+ *          16 (NVFP4: 16 E4M3) or 0 (FP8), the row's block scales of the chunk in K order.
+ *          Size T*C*128*SB bytes (0 for FP8: scales_dev may then be NULL everywhere).
  * Each (tile, chunk) is one contiguous block of codes and one of scales, so the kernel
  * streams it with two 1-D bulk copies.
  *
  * Row-major interchange layout (input of qgemm_repack_rowmajor): codes [N][code pitch]
- * (Q8_0: K bytes; FP4: K/2 bytes, element 2j in the low nibble of byte j), scales
- * [N][scale pitch] (Q8_0: K/32 little-endian fp16; NVFP4: K/16 E4M3; MXFP4: K/32 E8M0);
+ * (Q8_0, FP8: K bytes; FP4: K/2 bytes, element 2j in the low nibble of byte j), scales
+ * [N][scale pitch] (Q8_0: K/32 little-endian fp16; NVFP4: K/16 E4M3; MXFP4: K/32 E8M0;
+ * FP8: none, pitch 0);
  * qgemm_row_pitches gives the smallest 16-byte-aligned pitches.
  *
  * Conventions for every entry point:
@@ -44,10 +48,12 @@
  *     abort or exit the process.  A status other than QGEMM_OK means nothing was
  *     launched (argument errors) or a launch failed (QGEMM_ERR_CUDA).
  *   - Device pointers must be 16-byte aligned (TMA); x, y and h must be contiguous.
- *   - The library keeps no device state between calls except a small cache of
- *     TMA descriptors and a device error word read by qgemm_device_status().
- *   - Calls that overlap on the device may share nothing writable: each needs its own
- *     workspace.
+ *   - Device state that outlives a call: the error word read by qgemm_device_status(), and
+ *     the fixed scratch of qgemm_run_noalloc (see there).  Host state: each calling thread
+ *     keeps its last few tile plans and encoded x tensor maps (TMA descriptors, keyed by
+ *     the operand's address and geometry; they hold no device memory).
+ *   - qgemm_run and qgemm_ffn_gate_up calls that may overlap on the device need their own
+ *     workspaces; qgemm_run_noalloc calls share one scratch and must not overlap.
  */
 #ifndef QGEMM_H
 #define QGEMM_H
@@ -63,6 +69,7 @@ extern "C" {
 #define QGEMM_FMT_Q8_0 0
 #define QGEMM_FMT_NVFP4 1
 #define QGEMM_FMT_MXFP4 2
+#define QGEMM_FMT_FP8 3
 
 /* Output element types of qgemm_run. */
 #define QGEMM_Y_F32 0
@@ -82,7 +89,8 @@ extern "C" {
 
 /*
  * Sizes of the tile-major packed buffers for an N x K weight matrix.  No device work.
- * Returns QGEMM_ERR_FORMAT / _SHAPE / _K_BLOCK / _NULL.
+ * Returns QGEMM_ERR_FORMAT / _SHAPE / _K_BLOCK / _NULL.  (No passage: a layout helper for
+ * this library's packed layout, described above.)
  */
 int qgemm_packed_size(int fmt, int64_t N, int64_t K, size_t* code_bytes, size_t* scale_bytes);
 
@@ -116,29 +124,36 @@ int qgemm_repack_rowmajor(int fmt, int64_t N, int64_t K, const void* codes_rm_de
  *          rounds to 0) gets scale 0 and codes 0.  Writes ts to *tensor_scale_dev.
  *   MXFP4: e = clamp(floor(log2 amax) - 2 + 127, 0, 254); code = E2M1_RNE_sat(w/2^(e-127));
  *          an all-zero block gets e = 0 and codes 0.
+ *   FP8  : ts = fp32_RNE(max|W|/448); code = E4M3_RNE_sat(w/ts); a zero matrix gets ts = 0
+ *          and codes 0.  Writes ts to *tensor_scale_dev.
  * Ties round to even.  A negative element whose magnitude rounds to 0 keeps its sign bit.
  * codes_dev / scales_dev: qgemm_packed_size() bytes (tile-major layout), 16-byte aligned.
- * tensor_scale_dev: one float (NVFP4 only; must be NULL or ignored otherwise).
+ * tensor_scale_dev: one float (NVFP4 and FP8; ignored otherwise).
  * Not performance critical (uses fp64 for exact tie decisions).
  */
 int qgemm_pack(int fmt, const float* W_dev, int64_t N, int64_t K, void* codes_dev,
                void* scales_dev, float* tensor_scale_dev, void* stream);
 
 /*
- * Bytes of device workspace qgemm_run needs for (fmt, N, K, B).  May be 0.
+ * Bytes of device workspace qgemm_run needs for (fmt, N, K, B).  May be 0.  (No passage: the
+ * workspace holds this design's f16 copy of x, its per-row exponents and the split-K
+ * partials of the fixed-order reduction.)
  */
 int qgemm_workspace_size(int fmt, int64_t N, int64_t K, int64_t B, size_t* bytes);
 
 /*
  * y_dev[B][N] = x_dev[B][K] (bf16) * dequant(W)^T, W given by codes_dev / scales_dev
- * (packed as above) and, for NVFP4, the fp32 tensor scale at *tensor_scale_dev.
+ * (packed as above) and, for NVFP4 and FP8, the fp32 tensor scale at *tensor_scale_dev.
  *   y_dtype    : QGEMM_Y_F32 (fp32) or QGEMM_Y_BF16 (bf16, round to nearest even).
  *   workspace  : qgemm_workspace_size() bytes of device memory (may be NULL if that
  *                size is 0).  Its contents need no initialisation.
  * Any B >= 1.  For B <= 256 the result row b depends only on x row b, W, and (N, K):
  * the split of K, the order of every sum and the arithmetic do not depend on B.
  * Accuracy: fp32 accumulation of exactly dequantized weights (Q8_0 products are rounded
- * once to the 16-bit operand type); see the project notes for the bound.
+ * once to the 16-bit operand type).  Up to 256 rows each x row is scaled by a power of two
+ * from its own maximum before the f16 conversion (exact for every element within 2^-38 of
+ * the row maximum, bf16 subnormals included); the epilogue restores it with the tensor scale
+ * applied first, so y is finite whenever the exact result is.
  */
 int qgemm_run(int fmt, const void* x_dev, int64_t B, int64_t K, const void* codes_dev,
               const void* scales_dev, const float* tensor_scale_dev, int64_t N, void* y_dev,
@@ -186,7 +201,7 @@ int qgemm_ffn_workspace_size(int fmt, int64_t N, int64_t K, int64_t M, size_t* b
  *   g = x Wg^T, u = x Wu^T (fp32);
  *   h_dev[M][N] = bf16_RNE( g / (1 + exp(-g)) * u ).
  * Both matrices use the same format and shape [N][K]; x_dev is bf16 [M][K].
- * g_ts_dev / u_ts_dev: NVFP4 tensor scales (NULL for the other formats).
+ * g_ts_dev / u_ts_dev: NVFP4 / FP8 tensor scales (NULL for the other formats).
  * For M <= 256 one kernel keeps g and u in its accumulators and never stores them, and row m
  * of h depends only on x row m (as for qgemm_run).  Above 256 rows, each chunk of rows runs
  * as two GEMMs into fp32 g and u in the workspace and one SiLU pass (prefill widths, where
@@ -219,7 +234,8 @@ int qgemm_device_status(int reset);
  */
 int qgemm_profile_events(void* begin_event, void* end_event);
 
-/* Static, human-readable text for a status code. */
+/* Static, human-readable text for a status code.  (No passage: error reporting; the pages'
+ * only error path is the batch > 64 rejection this library removes.) */
 const char* qgemm_status_str(int status);
 
 /* Text of the last CUDA error seen by this library in the calling thread ("" if none). */

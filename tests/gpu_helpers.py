@@ -21,11 +21,13 @@ def tile_packed(fmt, codes_rm: np.ndarray, scales_rm: np.ndarray, N: int, K: int
     """The tile-major layout of include/qgemm.h, built from the row-major packing with numpy
     (a byte permutation written from the header's description, independent of the library)."""
     f = oracle.FORMATS[fmt] if isinstance(fmt, str) else fmt
-    CK = 128 if f == oracle.Q8_0 else 256
-    SB = 16 if f == oracle.NVFP4 else 8
+    byte_codes = f in (oracle.Q8_0, oracle.FP8)
+    CK = 128 if byte_codes else 256
+    SB = {oracle.Q8_0: 8, oracle.NVFP4: 16, oracle.MXFP4: 8, oracle.FP8: 0}[f]
     T, C = -(-N // 128), -(-K // CK)
-    row_code = K if f == oracle.Q8_0 else K // 2
-    row_scale = {oracle.Q8_0: 2 * (K // 32), oracle.NVFP4: K // 16, oracle.MXFP4: K // 32}[f]
+    row_code = K if byte_codes else K // 2
+    row_scale = {oracle.Q8_0: 2 * (K // 32), oracle.NVFP4: K // 16, oracle.MXFP4: K // 32,
+                 oracle.FP8: 0}[f]
     cfull = np.zeros((T * 128, C * 128), dtype=np.uint8)
     cfull[:N, :row_code] = codes_rm[:, :row_code]
     grp = cfull.reshape(T, 128, C, 8, 16).transpose(0, 2, 1, 3, 4)  # [T][C][row][group][16]

@@ -44,20 +44,21 @@ def test_status_strings(lib):
     assert lib.qgemm_last_cuda_error().decode() == ""
 
 
-@pytest.mark.parametrize("fmt", ["q8_0", "nvfp4", "mxfp4"])
+@pytest.mark.parametrize("fmt", ["q8_0", "nvfp4", "mxfp4", "fp8"])
 @pytest.mark.parametrize("K", [32, 64, 96, 1024, 5120, 17408])
 def test_pitches_match_layout_spec(lib, fmt, K):
-    if fmt != "nvfp4" and K % 32:
+    if fmt in ("q8_0", "mxfp4") and K % 32:
         pytest.skip("K must be a multiple of 32")
     cp, sp = qgemm.row_pitches(fmt, K)
     assert (cp, sp) == (oracle.code_pitch(fmt, K), oracle.scale_pitch(fmt, K))
     T, C, CK, SB = qgemm.packed_geometry(fmt, 300, K)
-    assert T == 3 and CK == (128 if fmt == "q8_0" else 256) and C == -(-K // CK)
-    assert SB == (16 if fmt == "nvfp4" else 8)
+    byte_codes = fmt in ("q8_0", "fp8")
+    assert T == 3 and CK == (128 if byte_codes else 256) and C == -(-K // CK)
+    assert SB == {"q8_0": 8, "nvfp4": 16, "mxfp4": 8, "fp8": 0}[fmt]
     cb, sb = qgemm.packed_size(fmt, 300, K)
     assert (cb, sb) == (T * C * 128 * 128, T * C * 128 * SB)
     # the tiled layout holds every byte of the row-major packing (plus zero padding)
-    assert cb >= 300 * (K if fmt == "q8_0" else K // 2)
+    assert cb >= 300 * (K if byte_codes else K // 2)
 
 
 def test_argument_errors(lib):
@@ -79,6 +80,12 @@ def test_argument_errors(lib):
     assert lib.qgemm_run(0, 8, 4, 64, 16, 16, None, 8, 16, 0, None, 0, None) == 5    # misaligned
     assert lib.qgemm_run(0, 16, 0, 64, 16, 16, None, 8, 16, 0, None, 0, None) == 2   # B = 0
     assert lib.qgemm_pack(0, None, 4, 64, None, None, None, None) == 4
+    # FP8: no block scales (NULL accepted) but the tensor scale is required
+    assert lib.qgemm_run(3, 16, 4, 64, 16, None, None, 8, 16, 0, None, 0, None) == 4
+    assert lib.qgemm_packed_size(3, 4, 40, ctypes.byref(sz), ctypes.byref(sz)) == 3   # K % 16
+    assert lib.qgemm_packed_size(3, 4, 48, ctypes.byref(sz), ctypes.byref(sz)) == 0
+    assert sz.value == 0                                                              # no scales
+    assert lib.qgemm_packed_size(4, 4, 48, ctypes.byref(sz), ctypes.byref(sz)) == 1   # format
     assert lib.qgemm_ffn_gate_up(0, 16, 4, 64, 16, 16, None, None, 16, None, 8, 16, None, 0,
                                  None) == 4
 

@@ -14,7 +14,7 @@ from gpu_helpers import Case, bf16_bits_of, h_bound_violations
 
 pytestmark = pytest.mark.gpu
 
-FMTS = ["q8_0", "nvfp4", "mxfp4"]
+FMTS = ["q8_0", "nvfp4", "mxfp4", "fp8"]
 
 
 @pytest.fixture(scope="module", autouse=True)

@@ -5,6 +5,7 @@ batch invariance is checked bit for bit on the full outputs.
 Workloads (seeded, synthetic; weights ~N(0, 0.02), activations bf16 ~N(0, 1)):
   Q8_0 gate/up [17408, 5120] and down [5120, 17408], widths 1..256 and 257;
   NVFP4 verify widths B in {1, 4, 5, 8, 9, 16} on [17408, 5120];
+  FP8 (E4M3) verify and decode widths, the down shape and an M = 2048 chunk;
   NVFP4 prefill FFN chunk, M in {2048, 7235}: fused gate+up -> h -> down;
   MXFP4 serving mix: B = 32 decode and an M = 8192 prefill chunk on both shapes."""
 import numpy as np
@@ -115,6 +116,15 @@ def test_nvfp4_prefill_ffn_chain(nvfp4_ffn, M):
     bound = (TOL * np.sqrt((hg ** 2).sum(axis=1))[:, None]
              + np.sqrt(((hg - hr) ** 2).sum(axis=1))[:, None]) * wn
     assert np.all(np.abs(y[rows] - y_ref) <= bound)
+    # the down projection on the oracle's own h at the plain bar: the sampled rows of the
+    # GPU's h are replaced by h_ref, and the full M-row GEMM runs in the same launch
+    # configuration (rows are independent, so the others do not affect the sampled ones)
+    h_mix = h.clone()
+    h_mix[torch.from_numpy(rows).cuda()] = inputs.bits_to_bf16(h_ref).cuda()
+    y_mix = _np(qgemm.run(h_mix, cd.pw))
+    torch.cuda.synchronize()
+    err = norm_err(y_mix[rows], y_ref, h_ref, cd.Wd)
+    assert err <= TOL, "down projection on h_ref: normalised error %.3e" % err
 
 
 def test_mxfp4_serving_mix():
@@ -131,7 +141,32 @@ def test_mxfp4_serving_mix():
         del case
 
 
-@pytest.mark.parametrize("fmt", ["q8_0", "nvfp4"])
+def test_fp8_27b_widths_and_prefill():
+    """FP8 (E4M3, per-tensor scale) at the 27B shapes: the batch-8 verify widths and decode
+    widths on the gate/up shape, bitwise invariant; the down shape at B = 64; and an M = 2048
+    prefill chunk on sampled rows.  The device packer gives the oracle's bytes at full size."""
+    case = Case("fp8", INTER, HIDDEN, seed=inputs.W_SEED)
+    pw = qgemm.pack("fp8", torch.from_numpy(case.W).cuda())
+    torch.cuda.synchronize()
+    ct, _ = tile_packed("fp8", case.codes, case.scales, INTER, HIDDEN)
+    assert np.array_equal(pw.codes.cpu().numpy(), ct)
+    assert pw.tensor_scale.item() == case.ts
+    del pw
+    x = inputs.activations(64, HIDDEN, seed=inputs.X_SEED).cuda()
+    xb = inputs.bf16_bits(x.cpu())
+    full = _np(_run(case, x))
+    _check_rows(case, full, xb, list(range(64)))
+    for B in (1, 8, 9, 16):
+        assert np.array_equal(_np(_run(case, x[:B])), full[:B]), "width %d differs from 64" % B
+    xp = inputs.activations(2048, HIDDEN, seed=inputs.X_SEED + 100).cuda()
+    _check_rows(case, _np(_run(case, xp)), inputs.bf16_bits(xp.cpu()), inputs.sample_rows(2048))
+    del case
+    down = Case("fp8", HIDDEN, INTER, seed=inputs.W3_SEED)
+    xd = inputs.activations(64, INTER, seed=inputs.X_SEED + 1).cuda()
+    _check_rows(down, _np(_run(down, xd)), inputs.bf16_bits(xd.cpu()), [0, 31, 63])
+
+
+@pytest.mark.parametrize("fmt", ["q8_0", "nvfp4", "fp8"])
 def test_ffn_gate_up_decode_widths_27b(fmt):
     """The fused gate+up at the 27B gate/up shape and decode widths: every unit holds many
     A-slot groups, so both MMA issuers alternate through the A ring many times."""

@@ -16,7 +16,7 @@ from gpu_helpers import TOL, Case, gpu_run, norm_err, round_bf16, round_f16, til
 
 pytestmark = pytest.mark.gpu
 
-FMTS = ["q8_0", "nvfp4", "mxfp4"]
+FMTS = ["q8_0", "nvfp4", "mxfp4", "fp8"]
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -56,7 +56,7 @@ def test_pack_byte_exact(fmt, N, K):
         mism[:5].tolist(), gc[tuple(mism[0])], codes[tuple(mism[0])])
     mism = np.argwhere(gs != scales)
     assert mism.size == 0, "scales differ at %s" % mism[:5].tolist()
-    if fmt == "nvfp4":
+    if fmt in ("nvfp4", "fp8"):
         assert pw.tensor_scale.item() == ts
 
 
@@ -148,6 +148,37 @@ def test_run_special_rows():
         err = norm_err(y[b:b + 1], y_ref[b:b + 1], xb[b:b + 1], case.Wd)
         assert err <= TOL, (b, err)
     assert np.all(y[0] == 0.0)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_run_extreme_rows_f16_path(small_cases, fmt):
+    # rows at the ends of the bf16 range (widths <= 256 convert x to f16 after a per-row power
+    # of two): a maximum of 1e-36 (the row's scale 2^-e exceeds 2^127), bf16 subnormals only,
+    # the largest finite magnitude beside values near the smallest normal, and a zero row
+    case = small_cases[fmt]
+    K = case.K
+    x = inputs.activations(7, K, seed=15).float()
+    x[0] *= 1e-36 / x[0].abs().max()
+    sub = np.array([0x0001, 0x0003, 0x007F, 0x8005, 0x0040, 0x8001], dtype=np.uint16)
+    x[1] = inputs.bits_to_bf16(np.resize(sub, K)).float()
+    x[2, ::3] = 1e-38
+    x[2, 1::3] = -2e-38
+    x[2, 5] = 3.0e38
+    x[3] = 0.0
+    x[4, ::2] *= 2.0 ** -100
+    x[5, 17] = -3.0e38
+    x[5, 18] = 2.5e38
+    x = x.to(torch.bfloat16)
+    xb = x_bits(x)
+    y_ref = oracle.gemm(xb, case.Wd)
+    y = gpu_run(case, x)
+    assert np.isfinite(y).all()
+    for b in range(7):
+        err = norm_err(y[b:b + 1], y_ref[b:b + 1], xb[b:b + 1], case.Wd)
+        assert err <= TOL, (b, err)
+    assert np.all(y[3] == 0.0)
+    # bf16 output is still the fp32 result rounded once
+    assert np.array_equal(gpu_run(case, x, torch.bfloat16), round_bf16(y))
 
 
 # --------------------------------------------------------------------------------------
