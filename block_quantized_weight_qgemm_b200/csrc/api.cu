@@ -230,19 +230,22 @@ bool make_plan_pair(int fmt, int64_t N, int64_t K, int64_t B, int nmat, Plan* pl
   p.b_tiles = (int)((B + p.NB - 1) / p.NB);
   p.R = nmat;
   p.n_groups = (int)pairs;
-  p.AS = std::min(4, (512 - p.R * p.NACC * p.NB) / kPairACols);
-  // an issuer's consecutive A slots lie at most 2 apart in the ring (plain GEMM with two
-  // accumulators: alternate groups of one slot; fused: alternate slots), so AS >= 2 keeps a
+  // A ring: an even number of kPairSlotK slots (each stage half owns AS/2), at most 6, at least
+  // 4 -- an issuer's previous slot of the same half lies at most 2 stages back (two issuers
+  // alternate groups of one stage, or take alternate matrices), so AS/2 >= 2 keeps that
   // slot's previous use complete before its issuer waits for it
-  if (p.AS < 2 || (nmat == 1 && p.NACC == 2 && p.R != 1)) return false;
+  p.AS = std::min(6, (512 - p.R * p.NACC * p.NB) / kPairACols) & ~1;
+  if (p.AS < 4 || (nmat == 1 && p.NACC == 2 && p.R != 1)) return false;
   p.tmem_cols = next_pow2_cols(p.R * p.NACC * p.NB + p.AS * kPairACols);
   if (p.tmem_cols > 512) return false;
   const size_t xstage = (size_t)(p.NB / 2) * 128 * (kPairAK / kSubK);
-  const size_t misc = 8 * (2 * 4 + 2 * kMaxWStages + 2 * 8 + 1) + 16 + 8 * kMaxNB + 64;
+  const size_t misc = 8 * (2 * 4 + 2 * kMaxWStages + 2 * 6 + 1) + 16 + 8 * kMaxNB + 64;
   const size_t budget = kSmemLimit - 1024 - misc;
   const size_t wstage = (size_t)pair_wstage_bytes(fmt);
+  // x ring depth 4 or 2 (even): the two issuers take alternate groups, so an x stage's
+  // previous use then belongs to the same issuer, whose wait therefore never aliases a phase
   int XS = 4;
-  while (XS > 2 && XS * xstage + 4 * wstage > budget) --XS;
+  if (XS * xstage + 4 * wstage > budget) XS = 2;
   if (XS * xstage + 2 * wstage > budget) return false;
   const int WS = (int)std::min<size_t>(kMaxWStages, (budget - XS * xstage) / wstage);
   p.XS = XS;
@@ -344,11 +347,45 @@ bool x_map(CUtensorMap* out, int dev, CUtensorMapDataType dt, const void* base, 
   return true;
 }
 
+// Grouped experts: the rows of x are grouped by expert (device offsets), each expert's
+// weights come from device pointer tables.
+struct MoeArgs {
+  const int* off;
+  int E;
+  int64_t max_rows;
+  const void* const* codes[2];
+  const void* const* scales[2];
+  const float* const* ts[2];
+};
+
+// The tiling of a grouped call: the plain plan for max_rows rows (batch tile, rings, operand
+// type), with the K split fixed at 1 and a workspace for the f16 copy of all M rows.
+bool make_moe_plan(int fmt, int64_t N, int64_t K, int64_t M, int64_t max_rows, int nmat,
+                   Plan* pl) {
+  if (!make_plan(fmt, N, K, max_rows, nmat, pl)) return false;
+  pl->S = 1;
+  pl->b_tiles = (int)((max_rows + pl->NB - 1) / pl->NB);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += (bytes + 255) / 256 * 256;
+    return o;
+  };
+  pl->off_xh = pl->f16ops ? take((size_t)M * pad64(K) * 2) : 0;
+  pl->off_exp = pl->f16ops ? take((size_t)M * 4) : 0;
+  pl->off_ws = 0;
+  pl->ws_total = off;
+  return true;
+}
+
 int run_impl(int fmt, const void* x, int64_t B, int64_t K, const void* const* codes,
              const void* const* scales, const float* const* ts, int nmat, int64_t N, void* out,
-             int out_bf16, void* workspace, size_t ws_bytes, cudaStream_t stream) {
+             int out_bf16, void* workspace, size_t ws_bytes, cudaStream_t stream,
+             const MoeArgs* moe = nullptr) {
   Plan pl;
-  if (!make_plan(fmt, N, K, B, nmat, &pl)) return QGEMM_ERR_SHAPE;
+  if (moe ? !make_moe_plan(fmt, N, K, B, moe->max_rows, nmat, &pl)
+          : !make_plan(fmt, N, K, B, nmat, &pl))
+    return QGEMM_ERR_SHAPE;
   if (pl.ws_total > 0 && (workspace == nullptr || ws_bytes < pl.ws_total)) return QGEMM_ERR_WORKSPACE;
   if (workspace && !aligned16(workspace)) return QGEMM_ERR_ALIGN;
   int dev = 0;
@@ -383,6 +420,15 @@ int run_impl(int fmt, const void* x, int64_t B, int64_t K, const void* const* co
     p.codes[m] = static_cast<const uint8_t*>(codes[mm]);
     p.scales[m] = static_cast<const uint8_t*>(scales[mm]);
   }
+  if (moe) {
+    p.moe_off = moe->off;
+    for (int m = 0; m < 2; ++m) {
+      const int mm = (m < nmat) ? m : 0;
+      p.moe_codes[m] = reinterpret_cast<const uint8_t* const*>(moe->codes[mm]);
+      p.moe_scales[m] = reinterpret_cast<const uint8_t* const*>(moe->scales[mm]);
+      p.moe_ts[m] = moe->ts[mm];
+    }
+  }
   p.x_exp = pl.f16ops ? reinterpret_cast<const int*>(wsb + pl.off_exp) : nullptr;
   p.ws = (pl.S > 1) ? reinterpret_cast<float*>(wsb + pl.off_ws) : nullptr;
   p.out = out;
@@ -414,7 +460,9 @@ int run_impl(int fmt, const void* x, int64_t B, int64_t K, const void* const* co
     snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled failed");
     return QGEMM_ERR_CUDA;
   }
-  const int grid = pl.n_groups * pl.b_tiles * pl.S;
+  const int64_t grid64 = (int64_t)pl.n_groups * pl.b_tiles * (moe ? moe->E : pl.S);
+  if (grid64 > 0x3FFFFFFF) return QGEMM_ERR_SHAPE;
+  const int grid = (int)grid64;
   if (g_prof_begin) cudaEventRecord(g_prof_begin, stream);
   // with f16 operands the GEMM follows the x preparation as its programmatic dependent
   cudaError_t e = launch_pair(fmt, !pl.f16ops, p, pl.smem_bytes, grid, &xmap, pl.f16ops, stream);
@@ -713,7 +761,7 @@ int qgemm_device_status(int reset) {
     e = cudaMemcpy(w, &z, sizeof(int), cudaMemcpyHostToDevice);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy");
   }
-  return v ? QGEMM_ERR_DEVICE_TIMEOUT : QGEMM_OK;
+  return v == kErrArg ? QGEMM_ERR_DEVICE_ARG : v ? QGEMM_ERR_DEVICE_TIMEOUT : QGEMM_OK;
 }
 
 const char* qgemm_status_str(int status) {
@@ -728,11 +776,104 @@ const char* qgemm_status_str(int status) {
     case QGEMM_ERR_CUDA: return "a CUDA call or kernel launch failed";
     case QGEMM_ERR_DEVICE: return "the current device is not an sm_100 GPU";
     case QGEMM_ERR_DEVICE_TIMEOUT: return "a kernel wait hit its time limit";
+    case QGEMM_ERR_DEVICE_ARG: return "a kernel refused an argument read from device memory";
     default: return "unknown status";
   }
 }
 
 const char* qgemm_last_cuda_error(void) { return g_last_cuda_error; }
+
+namespace {
+int check_moe(int fmt, const void* x, int64_t M, int64_t K, int E, const int32_t* off,
+              int64_t max_rows, int64_t N) {
+  int st = check_fmt_shape(fmt, N, K);
+  if (st != QGEMM_OK) return st;
+  if (M < 1 || M > 0x7FFFFFFF || E < 1 || max_rows < 1 || max_rows > 0x7FFFFFFF)
+    return QGEMM_ERR_SHAPE;
+  if (!x || !off) return QGEMM_ERR_NULL;
+  if (!aligned16(x) || (reinterpret_cast<uintptr_t>(off) & 3u)) return QGEMM_ERR_ALIGN;
+  return QGEMM_OK;
+}
+// a weight pointer table: codes always, scales unless the format has none, tensor scales
+// for the formats that have one; each 8-byte aligned
+int check_tables(int fmt, const void* const* c, const void* const* sc, const float* const* ts) {
+  if (!c || (scale_row_bytes(fmt) > 0 && !sc) || (has_tensor_scale(fmt) && !ts))
+    return QGEMM_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(c) & 7u) || (reinterpret_cast<uintptr_t>(sc) & 7u) ||
+      (reinterpret_cast<uintptr_t>(ts) & 7u))
+    return QGEMM_ERR_ALIGN;
+  return QGEMM_OK;
+}
+}  // namespace
+
+int qgemm_moe_workspace_size(int fmt, int64_t N, int64_t K, int64_t M, int64_t max_rows,
+                             size_t* bytes) {
+  int st = check_fmt_shape(fmt, N, K);
+  if (st != QGEMM_OK) return st;
+  if (M < 1 || M > 0x7FFFFFFF || max_rows < 1 || max_rows > 0x7FFFFFFF) return QGEMM_ERR_SHAPE;
+  if (!bytes) return QGEMM_ERR_NULL;
+  Plan pl;
+  if (!make_moe_plan(fmt, N, K, M, max_rows, 2, &pl)) return QGEMM_ERR_SHAPE;
+  Plan p1;
+  if (!make_moe_plan(fmt, N, K, M, max_rows, 1, &p1)) return QGEMM_ERR_SHAPE;
+  *bytes = std::max(pl.ws_total, p1.ws_total);  // one size serves both grouped entry points
+  return QGEMM_OK;
+}
+
+int qgemm_moe_run(int fmt, const void* x, int64_t M, int64_t K, int E, const int32_t* off,
+                  int64_t max_rows, const void* const* codes_tab, const void* const* scales_tab,
+                  const float* const* ts_tab, int64_t N, void* y, int y_dtype, void* workspace,
+                  size_t workspace_bytes, void* stream) {
+  int st = check_moe(fmt, x, M, K, E, off, max_rows, N);
+  if (st != QGEMM_OK) return st;
+  if (y_dtype != QGEMM_Y_F32 && y_dtype != QGEMM_Y_BF16) return QGEMM_ERR_FORMAT;
+  if (!y) return QGEMM_ERR_NULL;
+  if (!aligned16(y)) return QGEMM_ERR_ALIGN;
+  st = check_tables(fmt, codes_tab, scales_tab, ts_tab);
+  if (st != QGEMM_OK) return st;
+  if (!device_ok()) return QGEMM_ERR_DEVICE;
+  MoeArgs ma{};
+  ma.off = off;
+  ma.E = E;
+  ma.max_rows = max_rows;
+  ma.codes[0] = ma.codes[1] = codes_tab;
+  ma.scales[0] = ma.scales[1] = scales_tab;
+  ma.ts[0] = ma.ts[1] = ts_tab;
+  const void* none[1] = {nullptr};
+  const float* nts[1] = {nullptr};
+  return run_impl(fmt, x, M, K, none, none, nts, 1, N, y, y_dtype == QGEMM_Y_BF16, workspace,
+                  workspace_bytes, static_cast<cudaStream_t>(stream), &ma);
+}
+
+int qgemm_moe_gate_up(int fmt, const void* x, int64_t M, int64_t K, int E, const int32_t* off,
+                      int64_t max_rows, const void* const* g_codes_tab,
+                      const void* const* g_scales_tab, const float* const* g_ts_tab,
+                      const void* const* u_codes_tab, const void* const* u_scales_tab,
+                      const float* const* u_ts_tab, int64_t N, void* h, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  int st = check_moe(fmt, x, M, K, E, off, max_rows, N);
+  if (st != QGEMM_OK) return st;
+  if (!h) return QGEMM_ERR_NULL;
+  if (!aligned16(h)) return QGEMM_ERR_ALIGN;
+  st = check_tables(fmt, g_codes_tab, g_scales_tab, g_ts_tab);
+  if (st == QGEMM_OK) st = check_tables(fmt, u_codes_tab, u_scales_tab, u_ts_tab);
+  if (st != QGEMM_OK) return st;
+  if (!device_ok()) return QGEMM_ERR_DEVICE;
+  MoeArgs ma{};
+  ma.off = off;
+  ma.E = E;
+  ma.max_rows = max_rows;
+  ma.codes[0] = g_codes_tab;
+  ma.codes[1] = u_codes_tab;
+  ma.scales[0] = g_scales_tab;
+  ma.scales[1] = u_scales_tab;
+  ma.ts[0] = g_ts_tab;
+  ma.ts[1] = u_ts_tab;
+  const void* none[2] = {nullptr, nullptr};
+  const float* nts[2] = {nullptr, nullptr};
+  return run_impl(fmt, x, M, K, none, none, nts, 2, N, h, 1, workspace, workspace_bytes,
+                  static_cast<cudaStream_t>(stream), &ma);
+}
 
 int qgemm_profile_events(void* begin_event, void* end_event) {
   g_prof_begin = static_cast<cudaEvent_t>(begin_event);

@@ -20,8 +20,9 @@ constexpr int kPairIssuer2Warp = kPairFirstDequantWarp + kPairDequantWarps;  // 
 constexpr int kPairXWarp = kPairIssuer2Warp + 1;  // x producer
 constexpr int kPairThreads = (kPairXWarp + 1) * 32;
 constexpr int kPairSMs = 74;                      // CTA pairs resident at once (148 SMs)
-constexpr int kPairAK = 256;                      // K per A slot of the pair kernel
-constexpr int kPairACols = kPairAK / 2;           // its TMEM columns
+constexpr int kPairAK = 256;                      // K per weight stage / x group of the pair kernel
+constexpr int kPairSlotK = 128;                   // K per A slot (one half of a stage)
+constexpr int kPairACols = kPairSlotK / 2;        // its TMEM columns (f16 pairs)
 constexpr int kMaxNB = 256;                       // MMA N limit
 constexpr int kSmemLimit = 227 * 1024;
 
@@ -95,7 +96,7 @@ struct GemmParams {
   int b_tiles;   // ceil(B / NB)
   int chunks;    // ceil(K / chunk_k)
   int XS, WS;    // x ring and weight ring depths
-  int AS;        // A ring depth (TMEM slots of kPairAK)
+  int AS;        // A ring depth (TMEM slots of kPairSlotK; even: each stage half owns AS/2)
   int tmem_cols; // allocated TMEM columns
   int x3d;       // pair kernel: x map is 3-D {64, B, K/64} (one TMA load per x stage)
   int NACC;      // pair kernel: accumulators per subtile (1, or 2 for the f16 path)
@@ -108,6 +109,14 @@ struct GemmParams {
   void* out;                 // y [B][N] (fp32 or bf16), or h [B][N] bf16 for NMAT == 2
   int out_bf16;
   int* dev_err;
+  // Grouped experts (routed mixture-of-experts): when moe_off is set, x's B rows are grouped
+  // by expert (rows moe_off[e] .. moe_off[e+1]-1 belong to expert e, offsets clamped to
+  // [0, B]); a work unit is (expert, row-tile pair group, batch tile) with S = 1, and expert
+  // e's weights come from the device pointer tables below instead of codes/scales/ts.
+  const int* moe_off;
+  const uint8_t* const* moe_codes[2];
+  const uint8_t* const* moe_scales[2];
+  const float* const* moe_ts[2];
 };
 
 // Fixed-order sum of the split-K partials and the output epilogue.  The partials carry every
@@ -140,5 +149,6 @@ struct PrepParams {
 
 // Device error codes written to the library's error word.
 constexpr int kErrTimeout = 1;
+constexpr int kErrArg = 2;  // an argument found in device memory is invalid (an expert table entry)
 
 }  // namespace qg

@@ -267,11 +267,12 @@ constexpr int kFastExp = 60;
 // -147); kept out of line, off the epilogue's fast path.
 static __device__ __noinline__ float scale_pow2_exact(float v, int ex) { return ldexpf(v, ex); }
 
-__device__ __forceinline__ void store_y(const GemmParams& p, int b, int n, float v) {
+// y[m][n] (m: row of x and y)
+__device__ __forceinline__ void store_y(const GemmParams& p, int m, int n, float v) {
   if (p.out_bf16)
-    reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)b * p.N + n] = __float2bfloat16_rn(v);
+    reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)m * p.N + n] = __float2bfloat16_rn(v);
   else
-    reinterpret_cast<float*>(p.out)[(size_t)b * p.N + n] = v;
+    reinterpret_cast<float*>(p.out)[(size_t)m * p.N + n] = v;
 }
 
 // SiLU(g) * u rounded to bf16.  The fast exponential's relative error (~2^-21) is far
@@ -280,8 +281,8 @@ __device__ __forceinline__ float silu_mul(float g, float u) {
   return g / (1.0f + __expf(-g)) * u;
 }
 
-__device__ __forceinline__ void store_h(const GemmParams& p, int b, int n, float g, float u) {
-  reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)b * p.N + n] = __float2bfloat16_rn(silu_mul(g, u));
+__device__ __forceinline__ void store_h(const GemmParams& p, int m, int n, float g, float u) {
+  reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)m * p.N + n] = __float2bfloat16_rn(silu_mul(g, u));
 }
 
 

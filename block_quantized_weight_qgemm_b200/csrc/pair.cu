@@ -66,6 +66,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   const uint32_t bar_x_empty = bar_x_full + 8 * XS;
   const uint32_t bar_w_full = bar_x_empty + 8 * XS;
   const uint32_t bar_w_empty = bar_w_full + 8 * WS;
+  // A ring: AS TMEM slots of kPairSlotK.  Stage s's half h goes to slot 2 (s % (AS/2)) + h, so
+  // each half owns the ring positions of its parity.
   const uint32_t bar_a_full = bar_w_empty + 8 * WS;
   const uint32_t bar_a_empty = bar_a_full + 8 * AS;
   const uint32_t bar_acc = bar_a_empty + 8 * AS;
@@ -77,11 +79,47 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();  // 0: even CTA (issues the MMAs), 1: odd CTA
+  // work unit: (row-tile pair group g, batch tile bt, K split s); for grouped experts,
+  // (expert, g, bt) over the expert's rows [rb, rb + nrows) of x
   int u = (int)(blockIdx.x >> 1);
-  const int g = u % p.n_groups;
-  u /= p.n_groups;
-  const int bt = u % p.b_tiles;
-  const int s = u / p.b_tiles;
+  int g, bt, s, rb = 0, nrows = p.B;
+  const uint8_t* wcodes[2] = {p.codes[0], p.codes[1]};
+  const uint8_t* wscales[2] = {p.scales[0], p.scales[1]};
+  const float* wts[2] = {p.ts[0], p.ts[1]};
+  if (p.moe_off) {
+    bt = u % p.b_tiles;
+    u /= p.b_tiles;
+    g = u % p.n_groups;
+    const int ex = u / p.n_groups;
+    s = 0;
+    const int lo = min(max(__ldg(p.moe_off + ex), 0), p.B);
+    const int hi = min(max(__ldg(p.moe_off + ex + 1), lo), p.B);
+    rb = lo;
+    nrows = hi - lo;
+    if (bt * p.NB >= nrows) return;  // no rows of this expert in the tile: both CTAs leave
+    bool bad = false;
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+      const int mm = (m < p.NMAT) ? m : 0;
+      wcodes[m] = p.moe_codes[mm][ex];
+      wscales[m] = p.moe_scales[mm] ? p.moe_scales[mm][ex] : nullptr;
+      wts[m] = p.moe_ts[mm] ? p.moe_ts[mm][ex] : nullptr;
+      // the bulk copies need 16-byte aligned, present buffers: refuse the expert otherwise
+      bad |= (wcodes[m] == nullptr) || ((reinterpret_cast<uintptr_t>(wcodes[m]) & 15u) != 0);
+      if (SB > 0) bad |= (wscales[m] == nullptr) || ((reinterpret_cast<uintptr_t>(wscales[m]) & 15u) != 0);
+      if (has_tensor_scale(FMT))
+        bad |= (wts[m] == nullptr) || ((reinterpret_cast<uintptr_t>(wts[m]) & 3u) != 0);
+    }
+    if (bad) {
+      if (threadIdx.x == 0) atomicExch(p.dev_err, kErrArg);
+      return;  // both CTAs read the same entries and leave together
+    }
+  } else {
+    g = u % p.n_groups;
+    u /= p.n_groups;
+    bt = u % p.b_tiles;
+    s = u / p.b_tiles;
+  }
   const int c0 = (int)((int64_t)s * p.chunks / p.S);
   const int c1 = (int)((int64_t)(s + 1) * p.chunks / p.S);
   const int tpg = p.R / p.NMAT;  // tile pairs per group
@@ -100,10 +138,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     }
     for (int i = 0; i < WS; ++i) {
       mbar_init(bar_w_full + 8 * i, 1);
-      mbar_init(bar_w_empty + 8 * i, kPairDequantWarps);
+      mbar_init(bar_w_empty + 8 * i, kPairDequantWarps);  // both halves' warps read the stage
     }
     for (int i = 0; i < AS; ++i) {
-      mbar_init(bar_a_full + 8 * i, 2 * kPairDequantWarps);  // both CTAs' dequant warps
+      mbar_init(bar_a_full + 8 * i, kPairDequantWarps);  // the half's 4 warps in each CTA
       mbar_init(bar_a_empty + 8 * i, 1);
     }
     mbar_init(bar_acc, 2);  // one final commit per issuer
@@ -152,9 +190,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           const uint32_t cbytes = (uint32_t)n * kWCodeBytes;
           const uint32_t sbytes = (uint32_t)n * (kTileRows * SB);
           mbar_arrive_expect_tx(fb, cbytes + sbytes);
-          bulk_load(dst, p.codes[m] + blk * kWCodeBytes, cbytes, fb, pol_w);
+          bulk_load(dst, wcodes[m] + blk * kWCodeBytes, cbytes, fb, pol_w);
           if (SB > 0)
-            bulk_load(dst + WSCALES, p.scales[m] + blk * (kTileRows * SB), sbytes, fb, pol_w);
+            bulk_load(dst + WSCALES, wscales[m] + blk * (kTileRows * SB), sbytes, fb, pol_w);
         } else {
           mbar_arrive(fb);  // a tile past the matrix: its rows are never stored
         }
@@ -200,7 +238,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         const int cg = c0 + x_issued * CPA;
         const uint32_t dst = sx + (uint32_t)xp.slot * xstage;
         const uint32_t cbar = xbar0 + 8u * (uint32_t)xp.slot;
-        const int row0 = bt * p.NB + (int)rank * half;
+        const int row0 = rb + bt * p.NB + (int)rank * half;
         if (p.x3d) {
           // one box of 4 slices (slices past K read zeros from the padded rows or the
           // out-of-range fill)
@@ -233,65 +271,77 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     //   * fused gate+up (NMAT = 2, NACC = 1): issuer e takes matrix e's subtiles (gate or up),
     //     one accumulator each;
     //   * NACC = 1 plain GEMM (widths > 256): issuer 0 alone.
-    // An issuer's consecutive slots are at most AS apart in the A ring (AS >= 2 for the
-    // first two; the planner checks), so a slot's previous use has always completed when
-    // its issuer waits for it.  Within each accumulator the K slices arrive in ascending
-    // order.  Per slot: wait for the A slot (a_full counts both CTAs' dequant warps), issue
-    // its K=16 MMAs, release it to both CTAs with a multicast commit; per group: wait for
-    // the pair's x stage first and release it after the issuer's last slot of the group.
+    // A-ring slots hold one half of a stage each (kPairSlotK of K); half h of stage s sits at
+    // slot 2 (s % (AS/2)) + h, so the two halves run as independent rings.  An issuer's
+    // previous slot of the same half lies at most AS/2 stages back (two issuers alternate
+    // groups of one stage, or take alternate matrices), so its wait on a slot's "full"
+    // barrier never aliases an older phase.  Within each accumulator the K slices arrive in
+    // ascending order.  Per slot: wait for it (a_full counts the half's warps of both CTAs),
+    // issue its K=16 MMAs, release it to both CTAs with a multicast commit; per group: wait
+    // for the pair's x stage first and release it after the issuer's last slot of the group.
     const int e = (warp == 1) ? 0 : 1;
     const bool by_matrix = (p.NMAT == 2);
     if (rank == 0 && lane == 0 && (by_matrix || e < p.NACC)) {
       const uint32_t idesc = idesc_f16_pair(BF16OP, (uint32_t)p.NB);
       const uint32_t xs16 = xslice >> 4;
       RingPos xc;  // x stage of the current group
-      RingPos ap;  // A ring
+      RingPos sp;  // stage position in the A ring (AS/2 per half)
+      const int HS = AS / 2;
       bool ok = true;
       for (int gi = 0; gi < ngroups && ok; ++gi) {
         if (!by_matrix && gi % p.NACC != e) {
           // another issuer's group: keep the ring positions in step
-          for (int i = 0; i < p.R; ++i) ap.next(AS);
+          for (int i = 0; i < p.R; ++i) sp.next(HS);
           xc.next(XS);
           continue;
         }
-        const int ksteps = min(CPA, c1 - (c0 + gi * CPA)) * (KW / 16);
+        const int kvalid = min(CPA, c1 - (c0 + gi * CPA)) * KW;  // K of the group with data
         if (!mbar_wait_spin(bar_x_full + 8 * xc.slot, xc.phase, false, abort_flag, p.dev_err,
                             kErrTimeout))
           break;
         const uint32_t xbase = sx + (uint32_t)xc.slot * xstage;
-        for (int i = 0; i < p.R; ++i) {
-          if (by_matrix && (i & 1) != e) {  // the other matrix's slot
-            ap.next(AS);
+        const uint64_t bd0 = smem_desc_sw128(xbase);
+        for (int i = 0; i < p.R && ok; ++i) {
+          if (by_matrix && (i & 1) != e) {  // the other matrix's stage
+            sp.next(HS);
             continue;
           }
-          if (!mbar_wait_spin(bar_a_full + 8 * ap.slot, ap.phase, false, abort_flag, p.dev_err,
-                              kErrTimeout)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
           const int acc_i = by_matrix ? i : i * p.NACC + e;
           const uint32_t d = tmem + (uint32_t)(acc_i * p.NB);
-          const uint32_t a = tmem + a_col0 + (uint32_t)(ap.slot * kPairACols);
           const bool first = by_matrix ? (gi == 0) : (gi < p.NACC);  // accumulator's first group
-          // The issuing thread, not the tensor pipe, bounds small-N MMA streams, so a full slot
-          // is one straight run of 16 MMAs whose operand addresses are the group's descriptor
-          // plus constants (descriptor address units are 16 bytes).
-          const uint64_t bd0 = smem_desc_sw128(xbase);
-          if (ksteps == 16) {
 #pragma unroll
-            for (int ks = 0; ks < 16; ++ks)
-              mma_f16_ts_pair(d, a + (uint32_t)(ks * 8),
-                              bd0 + (uint64_t)((ks >> 2) * xs16 + (ks & 3) * 2), idesc,
-                              (first && ks == 0) ? 0u : 1u);
-          } else {
-            for (int ks = 0; ks < ksteps; ++ks)
-              mma_f16_ts_pair(d, a + (uint32_t)(ks * 8),
-                              bd0 + (uint64_t)((ks >> 2) * xs16 + (ks & 3) * 2), idesc,
-                              (first && ks == 0) ? 0u : 1u);
+          for (int hh = 0; hh < kPairAK / kPairSlotK; ++hh) {
+            const int slot = 2 * sp.slot + hh;
+            if (!mbar_wait_spin(bar_a_full + 8 * slot, sp.phase, false, abort_flag, p.dev_err,
+                                kErrTimeout)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a = tmem + a_col0 + (uint32_t)(slot * kPairACols);
+            const int ksteps = max(0, min(kPairSlotK, kvalid - hh * kPairSlotK)) / 16;
+            // The issuing thread, not the tensor pipe, bounds small-N MMA streams, so a full
+            // slot is one straight run of 8 MMAs whose operand addresses are the group's
+            // descriptor plus constants (descriptor address units are 16 bytes).
+            if (ksteps == kPairSlotK / 16) {
+#pragma unroll
+              for (int ks = 0; ks < kPairSlotK / 16; ++ks) {
+                const int kk = hh * (kPairSlotK / 16) + ks;  // K=16 step within the group
+                mma_f16_ts_pair(d, a + (uint32_t)(ks * 8),
+                                bd0 + (uint64_t)((kk >> 2) * xs16 + (kk & 3) * 2), idesc,
+                                (first && kk == 0) ? 0u : 1u);
+              }
+            } else {
+              for (int ks = 0; ks < ksteps; ++ks) {
+                const int kk = hh * (kPairSlotK / 16) + ks;
+                mma_f16_ts_pair(d, a + (uint32_t)(ks * 8),
+                                bd0 + (uint64_t)((kk >> 2) * xs16 + (kk & 3) * 2), idesc,
+                                (first && kk == 0) ? 0u : 1u);
+              }
+            }
+            mma_commit_pair(bar_a_empty + 8 * slot);
           }
-          mma_commit_pair(bar_a_empty + 8 * ap.slot);
-          ap.next(AS);
+          sp.next(HS);
         }
         if (!ok) break;
         mma_commit_pair(bar_x_empty + 8 * xc.slot);
@@ -303,9 +353,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   } else {
     // ------------------------------------------------------------ dequant + epilogue
     // Warp w may touch TMEM lanes 32*(w%4)..+31 (its lane quarter q); the kWPQ warps of a
-    // quarter split each A slot into parts h of EPW elements.
+    // quarter take the halves of each weight stage (warp h half h), each into its own A slot,
+    // so the two halves advance independently within the weight ring.
     constexpr int kWPQ = kPairDequantWarps / 4;
-    constexpr int EPW = kPairAK / kWPQ;
+    static_assert(kWPQ * kPairSlotK == kPairAK, "one A slot per warp of a quarter per stage");
     const int dw = warp - kPairFirstDequantWarp;
     const int q = warp & 3;
     const int h = dw >> 2;
@@ -323,7 +374,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         const int64_t n = t * kTileRows + row;
         uint32_t mx = 0;
         if (n < p.N) {
-          const uint8_t* sb = p.scales[r % p.NMAT];
+          const uint8_t* sb = wscales[r % p.NMAT];
           for (int c = c0; c < c1; ++c) {
             const uint2 v = __ldg(reinterpret_cast<const uint2*>(sb + scale_offset(FMT, p.chunks, n, c)));
             mx = __vmaxu4(mx, __vmaxu4(v.x, v.y));
@@ -334,53 +385,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       }
     }
 
-    RingPos ap;  // A ring
-    int li = 0;  // A slots written so far
-    // this warp's EPW elements of each A slot: chunk ccw of the group, from element eo
-    const int ccw = (h * EPW) / KW;
-    const int eo = (h * EPW) % KW;
+    RingPos wp;  // weight stage
+    RingPos sp;  // this half's A-ring position (AS/2 per half)
+    const int HS = AS / 2;
+    const int ccw = (h * kPairSlotK) / KW;  // chunk of the stage holding this warp's half
+    const int eo = (h * kPairSlotK) % KW;   // its first element within the chunk
+    int ns = 0;                             // stages consumed
     bool ok = true;
     for (int gi = 0; gi < ngroups && ok; ++gi) {
       const int cg = c0 + gi * CPA;
       const int n = min(CPA, c1 - cg);
       for (int r = 0; r < p.R; ++r) {
-        if (li >= AS) {
-          // the pair MMAs of this slot's previous use have completed
-          ok = mbar_wait(bar_a_empty + 8 * ap.slot, ap.phase ^ 1u, abort_flag, p.dev_err,
+        const int slot = 2 * sp.slot + h;
+        if (ns >= HS) {
+          // the pair MMAs of this slot's previous use (this half's stage ns - AS/2) are done
+          ok = mbar_wait(bar_a_empty + 8 * slot, sp.phase ^ 1u, abort_flag, p.dev_err,
                          kErrTimeout);
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
         }
-        // weight stage li (one per A slot): this warp's chunk ccw of it, if the group has one
-        const int wslot = li % WS;
-        bool wdone = false;
+        ok = mbar_wait(bar_w_full + 8 * wp.slot, wp.phase, abort_flag, p.dev_err, kErrTimeout);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        const uint8_t* stage = smem + p.smem_w + wp.slot * WSTAGE;
+        tc_fence_after();
         if (ccw < n) {
-          ok = mbar_wait(bar_w_full + 8 * wslot, (uint32_t)(li / WS) & 1u, abort_flag, p.dev_err,
-                         kErrTimeout);
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) break;
-          const uint8_t* stage = smem + p.smem_w + wslot * WSTAGE;
+          // this warp's half of the stage: kPairSlotK elements of its 32 rows
           const uint8_t* crow = stage + ccw * kWCodeBytes + row * kWRowBytes;
           const uint8_t* srow = stage + WSCALES + ccw * (kTileRows * SB) + row * SB;
-          tc_fence_after();
-          uint32_t v[EPW / 2];
+          uint32_t v[kPairSlotK / 2];
           const int ex = sel4(emax, r);
 #pragma unroll
-          for (int i = 0; i < EPW / 32; ++i)
+          for (int i = 0; i < kPairSlotK / 32; ++i)
             Dequant<FMT, BF16OP>::run(crow, row, srow, cg + ccw, eo + 32 * i, ex,
                                       *reinterpret_cast<uint32_t(*)[16]>(&v[16 * i]));
           __syncwarp();
-          if (lane == 0) mbar_arrive(bar_w_empty + 8 * wslot);  // registers hold the data
-          wdone = true;
-          const uint32_t ta = tmem + lane_base + a_col0 + (uint32_t)(ap.slot * kPairACols + h * (EPW / 2));
+          if (lane == 0) mbar_arrive(bar_w_empty + 8 * wp.slot);  // registers hold the data
+          const uint32_t ta = tmem + lane_base + a_col0 + (uint32_t)(slot * kPairACols);
 #pragma unroll
-          for (int i = 0; i < EPW / 64; ++i)
+          for (int i = 0; i < kPairSlotK / 64; ++i)
             tmem_st32(ta + (uint32_t)(32 * i), *reinterpret_cast<const uint32_t(*)[32]>(&v[32 * i]));
           tmem_st_wait();
-        }
-        if (!wdone) {
+        } else {
           __syncwarp();
-          if (lane == 0) mbar_arrive(bar_w_empty + 8 * wslot);  // nothing of this stage to read
+          if (lane == 0) mbar_arrive(bar_w_empty + 8 * wp.slot);  // nothing of this stage to read
         }
         tc_fence_before();
         __syncwarp();
@@ -388,11 +436,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         // odd CTA's with a relaxed remote arrive (a cluster-scope release here would cost
         // about a thousand cycles per slot)
         if (lane == 0) {
-          if (rank == 0) mbar_arrive(bar_a_full + 8 * ap.slot);
-          else mbar_arrive_cluster_relaxed(afull0 + 8u * (uint32_t)ap.slot);
+          if (rank == 0) mbar_arrive(bar_a_full + 8 * slot);
+          else mbar_arrive_cluster_relaxed(afull0 + 8u * (uint32_t)slot);
         }
-        ap.next(AS);
-        ++li;
+        wp.next(WS);
+        sp.next(HS);
+        ++ns;
       }
     }
 
@@ -403,7 +452,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     griddep_wait();
     for (int i = threadIdx.x - kPairFirstDequantWarp * 32; i < p.NB; i += kPairDequantWarps * 32) {
       const int b = bt * p.NB + i;
-      const int ce = (b < p.B && p.x_exp) ? p.x_exp[b] : 0;
+      const int ce = (b < nrows && p.x_exp) ? p.x_exp[rb + b] : 0;
       col_exp[i] = ce;
       col_fac[i] = exp2_exact(ce);
       if (ce < -kFastExp || ce > kFastExp) ctl[3] = 1;
@@ -419,8 +468,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     const size_t BN = (size_t)p.B * p.N;
     float ts[2] = {1.0f, 1.0f};
     if (has_tensor_scale(FMT)) {
-      ts[0] = __ldg(p.ts[0]);
-      if (p.NMAT == 2) ts[1] = __ldg(p.ts[1]);
+      ts[0] = __ldg(wts[0]);
+      if (p.NMAT == 2) ts[1] = __ldg(wts[1]);
     }
     // per-row exponent restored by the epilogue: the MXFP4 f16 rebase (2^(E - Emax + 13) in
     // the operand for a block scale 2^(E - 127))
@@ -488,7 +537,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             for (int i = 0; i < 4; ++i) {
               const int col = cb + g4 * 4 + i;
               const int b = bt * p.NB + col;
-              if (b >= p.B) break;
+              if (b >= nrows) break;
               // tensor scale first, then the row's and the column's powers of two
               const float cf = col_fac[col];
               const float vg = __uint_as_float(va[g4][i]) * ts[0];
@@ -496,7 +545,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                                       : scale_pow2_exact(vg, col_exp[col] + re_g);
               if (p.NMAT == 1) {
                 if (p.S > 1) p.ws[(size_t)s * BN + (size_t)b * p.N + n] = ga;
-                else store_y(p, b, n, ga);
+                else store_y(p, rb + b, n, ga);
               } else {
                 const float vu = __uint_as_float(vb[g4][i]) * ts[1];
                 const float ua = fast_u ? (kRowExp ? vu * rf_u : vu) * cf
@@ -505,7 +554,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                   p.ws[(size_t)(2 * s) * BN + (size_t)b * p.N + n] = ga;
                   p.ws[(size_t)(2 * s + 1) * BN + (size_t)b * p.N + n] = ua;
                 } else {
-                  store_h(p, b, n, ga, ua);
+                  store_h(p, rb + b, n, ga, ua);
                 }
               }
             }

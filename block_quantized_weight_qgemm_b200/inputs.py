@@ -55,3 +55,19 @@ def one_hot(B: int, K: int, cols) -> torch.Tensor:
     for b, c in enumerate(cols):
         x[b, int(c)] = 1.0
     return x
+
+
+def routing(T: int, E: int, k: int, seed: int = ROW_SEED):
+    """Top-k routing of T tokens over E experts drawn at random (distinct experts per token).
+    Returns (token index of each routed row, expert of each row, offsets int32 [E+1]) with the
+    rows grouped by expert, tokens ascending within an expert."""
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    choice = torch.stack([torch.randperm(E, generator=g)[:k] for _ in range(T)])  # [T, k]
+    tok = torch.arange(T).repeat_interleave(k)
+    exp = choice.reshape(-1)
+    order = torch.argsort(exp * T + tok)
+    tok, exp = tok[order], exp[order]
+    counts = torch.bincount(exp, minlength=E)
+    off = torch.zeros(E + 1, dtype=torch.int32)
+    off[1:] = torch.cumsum(counts, 0).to(torch.int32)
+    return tok.numpy(), exp.numpy(), off.numpy()

@@ -23,7 +23,7 @@ OK = 0
 STATUS = {
     0: "QGEMM_OK", 1: "QGEMM_ERR_FORMAT", 2: "QGEMM_ERR_SHAPE", 3: "QGEMM_ERR_K_BLOCK",
     4: "QGEMM_ERR_NULL", 5: "QGEMM_ERR_ALIGN", 6: "QGEMM_ERR_WORKSPACE", 7: "QGEMM_ERR_CUDA",
-    8: "QGEMM_ERR_DEVICE", 9: "QGEMM_ERR_DEVICE_TIMEOUT",
+    8: "QGEMM_ERR_DEVICE", 9: "QGEMM_ERR_DEVICE_TIMEOUT", 10: "QGEMM_ERR_DEVICE_ARG",
 }
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libqgemm.so")
@@ -45,6 +45,11 @@ SIGNATURES = [
     ("qgemm_ffn_workspace_size", _I, [_I, _I64, _I64, _I64, ctypes.POINTER(_SZ)]),
     ("qgemm_ffn_gate_up", _I, [_I, _VP, _I64, _I64, _VP, _VP, _VP, _VP, _VP, _VP, _I64, _VP, _VP,
                                _SZ, _VP]),
+    ("qgemm_moe_workspace_size", _I, [_I, _I64, _I64, _I64, _I64, ctypes.POINTER(_SZ)]),
+    ("qgemm_moe_run", _I, [_I, _VP, _I64, _I64, _I, _VP, _I64, _VP, _VP, _VP, _I64, _VP, _I, _VP,
+                           _SZ, _VP]),
+    ("qgemm_moe_gate_up", _I, [_I, _VP, _I64, _I64, _I, _VP, _I64, _VP, _VP, _VP, _VP, _VP, _VP,
+                               _I64, _VP, _VP, _SZ, _VP]),
     ("qgemm_split_k", _I, [_I, _I64, _I64, ctypes.POINTER(_I)]),
     ("qgemm_device_status", _I, [_I]),
     ("qgemm_profile_events", _I, [_VP, _VP]),
@@ -235,4 +240,74 @@ def ffn_gate_up(x: torch.Tensor, wg: PackedWeight, wu: PackedWeight, h: torch.Te
                                    _ptr(wg.tensor_scale), _ptr(wu.codes), _ptr(wu.scales),
                                    _ptr(wu.tensor_scale), wg.N, _ptr(h), _ptr(workspace),
                                    workspace.numel(), _stream(stream)), "qgemm_ffn_gate_up")
+    return h
+
+
+# ---- routed mixture-of-experts --------------------------------------------------------
+
+def moe_workspace_size(fmt, N: int, K: int, M: int, max_rows: int) -> int:
+    b = _SZ()
+    _check(lib().qgemm_moe_workspace_size(_fmt(fmt), N, K, M, max_rows, ctypes.byref(b)),
+           "qgemm_moe_workspace_size")
+    return b.value
+
+
+class ExpertTable:
+    """Device pointer tables of a list of packed experts (one PackedWeight each, same format
+    and shape): codes, scales (absent for FP8) and tensor scales (NVFP4, FP8)."""
+
+    def __init__(self, experts):
+        assert experts and all(e.fmt == experts[0].fmt and e.N == experts[0].N and
+                               e.K == experts[0].K for e in experts)
+        self.fmt, self.N, self.K, self.E = experts[0].fmt, experts[0].N, experts[0].K, len(experts)
+        dev = experts[0].codes.device
+
+        def table(ts):
+            return torch.tensor([t.data_ptr() for t in ts], dtype=torch.int64, device=dev)
+        self.codes = table([e.codes for e in experts])
+        self.scales = table([e.scales for e in experts]) if experts[0].scales.numel() else None
+        self.ts = (table([e.tensor_scale for e in experts])
+                   if experts[0].tensor_scale is not None else None)
+        self.experts = experts  # keeps the buffers alive
+
+
+def _moe_common(x, offsets, tab):
+    assert x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous() and x.dim() == 2
+    assert offsets.is_cuda and offsets.dtype == torch.int32 and offsets.numel() == tab.E + 1
+    assert x.shape[1] == tab.K
+
+
+def moe_run(x: torch.Tensor, offsets: torch.Tensor, tab: ExpertTable, max_rows: int,
+            y: torch.Tensor | None = None, y_dtype=torch.float32, workspace=None, stream=None):
+    """qgemm_moe_run: rows of x grouped by expert (int32 offsets[E+1] on the device)."""
+    _moe_common(x, offsets, tab)
+    M, K = x.shape
+    if y is None:
+        y = torch.empty((M, tab.N), dtype=y_dtype, device=x.device)
+    ydt = Y_BF16 if y.dtype == torch.bfloat16 else Y_F32
+    if workspace is None:
+        nbytes = moe_workspace_size(tab.fmt, tab.N, K, M, max_rows)
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=x.device)
+    _check(lib().qgemm_moe_run(tab.fmt, _ptr(x), M, K, tab.E, _ptr(offsets), max_rows,
+                               _ptr(tab.codes), _ptr(tab.scales), _ptr(tab.ts), tab.N, _ptr(y), ydt,
+                               _ptr(workspace), workspace.numel(), _stream(stream)), "qgemm_moe_run")
+    return y
+
+
+def moe_gate_up(x: torch.Tensor, offsets: torch.Tensor, gate: ExpertTable, up: ExpertTable,
+                max_rows: int, h: torch.Tensor | None = None, workspace=None, stream=None):
+    """qgemm_moe_gate_up: h = bf16(SiLU(x Wg_e^T) * (x Wu_e^T)) per routed row."""
+    _moe_common(x, offsets, gate)
+    assert gate.fmt == up.fmt and gate.N == up.N and gate.K == up.K and gate.E == up.E
+    M, K = x.shape
+    if h is None:
+        h = torch.empty((M, gate.N), dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        nbytes = moe_workspace_size(gate.fmt, gate.N, K, M, max_rows)
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=x.device)
+    _check(lib().qgemm_moe_gate_up(gate.fmt, _ptr(x), M, K, gate.E, _ptr(offsets), max_rows,
+                                   _ptr(gate.codes), _ptr(gate.scales), _ptr(gate.ts),
+                                   _ptr(up.codes), _ptr(up.scales), _ptr(up.ts), gate.N, _ptr(h),
+                                   _ptr(workspace), workspace.numel(), _stream(stream)),
+           "qgemm_moe_gate_up")
     return h

@@ -86,6 +86,7 @@ extern "C" {
 #define QGEMM_ERR_CUDA 7           /* a CUDA call or kernel launch failed                */
 #define QGEMM_ERR_DEVICE 8         /* the current device is not an sm_100 part           */
 #define QGEMM_ERR_DEVICE_TIMEOUT 9 /* a kernel's bounded wait ran out (see device_status) */
+#define QGEMM_ERR_DEVICE_ARG 10    /* a kernel refused an argument read from device memory */
 
 /*
  * Sizes of the tile-major packed buffers for an N x K weight matrix.  No device work.
@@ -214,14 +215,56 @@ int qgemm_ffn_gate_up(int fmt, const void* x_dev, int64_t M, int64_t K, const vo
                       void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Routed mixture-of-experts variants (Atlas issue, "Per-32-K-step hot loop" table: the routed
+ * expert kernels moe_w4a16_fused_gate_up_t and its pointer-table twin; Strix Halo prefill
+ * journey: "a fused gate/up + SwiGLU for the MoE, and routed down-projections").  Every
+ * expert's matrices are packed separately (qgemm_pack) with the same format and shape; the
+ * kernel finds them through pointer tables, so they need not be contiguous.
+ *   x_dev        bf16 [M][K]: the routed rows grouped by expert -- rows offsets[e] ..
+ *                offsets[e+1]-1 belong to expert e (an expert may have none).
+ *   offsets_dev  int32 [E+1] in device memory, non-decreasing, offsets[0] = 0, offsets[E] = M
+ *                (values are clamped to [0, M], so no row outside x is read or written).
+ *   max_rows     an upper bound on any expert's row count (1 <= max_rows); it sizes the
+ *                launch, and rows of an expert past it are not computed.
+ *   *_codes_tab / *_scales_tab / *_ts_tab: device arrays of E device pointers to each
+ *                expert's packed codes, scales (NULL table allowed for FP8) and tensor scale
+ *                (NVFP4 and FP8; else NULL).  Each buffer 16-byte aligned (tensor scales 4);
+ *                an expert whose entry is NULL or misaligned is skipped and the device status
+ *                becomes QGEMM_ERR_DEVICE_ARG.
+ * Per expert the arithmetic is that of qgemm_run / qgemm_ffn_gate_up with the K split fixed
+ * at 1: for max_rows <= 256 a row's output depends only on that row, its expert's weights
+ * and (fmt, N, K) -- not on how many rows the expert or the call has.
+ * Workspace: qgemm_moe_workspace_size() bytes (the f16 copy of x and its row exponents).
+ */
+int qgemm_moe_workspace_size(int fmt, int64_t N, int64_t K, int64_t M, int64_t max_rows,
+                             size_t* bytes);
+
+/* y[m][n] = x[m] W_e^T for the rows m of expert e (the routed down projection). */
+int qgemm_moe_run(int fmt, const void* x_dev, int64_t M, int64_t K, int E,
+                  const int32_t* offsets_dev, int64_t max_rows, const void* const* codes_tab_dev,
+                  const void* const* scales_tab_dev, const float* const* ts_tab_dev, int64_t N,
+                  void* y_dev, int y_dtype, void* workspace, size_t workspace_bytes, void* stream);
+
+/* h[m][n] = bf16(SiLU(x[m] Wg_e^T) * (x[m] Wu_e^T)) for the rows m of expert e (the routed
+ * fused gate+up with the SiLU(gate)*up epilogue; g and u never leave the chip). */
+int qgemm_moe_gate_up(int fmt, const void* x_dev, int64_t M, int64_t K, int E,
+                      const int32_t* offsets_dev, int64_t max_rows,
+                      const void* const* g_codes_tab_dev, const void* const* g_scales_tab_dev,
+                      const float* const* g_ts_tab_dev, const void* const* u_codes_tab_dev,
+                      const void* const* u_scales_tab_dev, const float* const* u_ts_tab_dev,
+                      int64_t N, void* h_dev, void* workspace, size_t workspace_bytes,
+                      void* stream);
+
+/*
  * Number of K splits qgemm_run uses for 1 <= B <= 256 (a function of fmt, N, K only).
  */
 int qgemm_split_k(int fmt, int64_t N, int64_t K, int* splits);
 
 /*
  * Synchronizes the current device and reports whether any kernel of this library hit a
- * bounded-wait limit since the last reset (QGEMM_ERR_DEVICE_TIMEOUT), else QGEMM_OK or
- * QGEMM_ERR_CUDA.  reset != 0 clears the flag.
+ * bounded-wait limit (QGEMM_ERR_DEVICE_TIMEOUT) or refused an argument it read from device
+ * memory (QGEMM_ERR_DEVICE_ARG) since the last reset, else QGEMM_OK or QGEMM_ERR_CUDA.
+ * reset != 0 clears the flag.
  */
 int qgemm_device_status(int reset);
 

@@ -134,19 +134,30 @@ unsigned orc_e2m1_encode(double v) {
 }
 
 /* E4M3 byte nearest to a >= 0 among the 127 finite non-negative values, ties to
- * the even byte, saturating at 448 (0x7E).  Scan of the table. */
+ * the even byte, saturating at 448 (0x7E).  The values grow with the byte (0x00..0x7E), so
+ * a binary search finds the largest byte lo whose value is <= a; the answer is lo or lo + 1,
+ * whichever is nearer, the even one on a tie. */
+static double e4m3_pos_table[0x7F];
+static int e4m3_pos_table_ready = 0;
+
 unsigned orc_e4m3_encode_pos(double a) {
-    unsigned best = 0;
-    if (a >= 448.0) return 0x7Eu; /* saturate at the largest finite value */
-    double bestd = fabs(a - orc_e4m3(0));
-    for (unsigned c = 1; c < 0x7Fu; ++c) {
-        double d = fabs(a - orc_e4m3(c));
-        if (d < bestd || (d == bestd && (c & 1u) == 0u && (best & 1u) == 1u)) {
-            best = c;
-            bestd = d;
-        }
+    unsigned lo = 0, hi = 0x7Eu, mid;
+    double dlo, dhi;
+    if (!e4m3_pos_table_ready) {  /* the decoder's values, once (callers are single-threaded) */
+        for (unsigned c = 0; c < 0x7Fu; ++c) e4m3_pos_table[c] = orc_e4m3(c);
+        e4m3_pos_table_ready = 1;
     }
-    return best;
+    if (a >= 448.0) return 0x7Eu; /* saturate at the largest finite value */
+    while (lo < hi) {             /* invariant: value(lo) <= a (value(0) = 0) */
+        mid = (lo + hi + 1u) / 2u;
+        if (e4m3_pos_table[mid] <= a) lo = mid;
+        else hi = mid - 1u;
+    }
+    dlo = a - e4m3_pos_table[lo];
+    dhi = e4m3_pos_table[lo + 1u] - a;  /* lo < 0x7E here because a < 448 */
+    if (dlo < dhi) return lo;
+    if (dhi < dlo) return lo + 1u;
+    return (lo & 1u) ? lo + 1u : lo;
 }
 
 /* Signed E4M3 code of a finite value: the magnitude as orc_e4m3_encode_pos, the sign

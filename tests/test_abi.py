@@ -37,7 +37,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_status_strings(lib):
-    for code in range(10):
+    for code in range(11):
         s = lib.qgemm_status_str(code).decode()
         assert s and s != "unknown status"
     assert lib.qgemm_status_str(99).decode() == "unknown status"
@@ -88,6 +88,17 @@ def test_argument_errors(lib):
     assert lib.qgemm_packed_size(4, 4, 48, ctypes.byref(sz), ctypes.byref(sz)) == 1   # format
     assert lib.qgemm_ffn_gate_up(0, 16, 4, 64, 16, 16, None, None, 16, None, 8, 16, None, 0,
                                  None) == 4
+    # routed experts: argument checks before any device work
+    assert lib.qgemm_moe_run(0, 16, 4, 64, 2, None, 4, 16, 16, None, 8, 16, 0, None, 0,
+                             None) == 4                                             # offsets
+    assert lib.qgemm_moe_run(0, 16, 4, 64, 0, 16, 4, 16, 16, None, 8, 16, 0, None, 0,
+                             None) == 2                                             # E = 0
+    assert lib.qgemm_moe_run(1, 16, 4, 64, 2, 16, 4, 16, 16, None, 8, 16, 0, None, 0,
+                             None) == 4                                             # NVFP4 ts table
+    assert lib.qgemm_moe_run(0, 16, 4, 64, 2, 16, 4, 20, 16, None, 8, 16, 0, None, 0,
+                             None) == 5                                             # table alignment
+    assert lib.qgemm_moe_gate_up(3, 16, 4, 64, 2, 16, 4, 16, None, 16, 16, None, None, 8, 16,
+                                 None, 0, None) == 4                                # up ts table
 
 
 def test_no_width_limit_in_sizes(lib):
@@ -127,3 +138,11 @@ def test_wide_fused_ffn_workspace_holds_g_and_u_of_one_chunk(lib):
     assert qgemm.ffn_workspace_size("q8_0", N, 5120, 300) == 2 * 304 * N * 4
     # at or below 256 rows the single fused kernel runs
     assert qgemm.ffn_workspace_size("q8_0", N, 5120, 256) < 256 * N * 4
+
+
+def test_moe_workspace_holds_f16_rows(lib):
+    # routed experts: the f16 copy of all M rows (row pitch K rounded up to 64) and their
+    # exponents, 256-byte aligned pieces; none on the wide path
+    M, K = 480, 2048
+    assert qgemm.moe_workspace_size("nvfp4", 512, K, M, 25) == M * K * 2 + (M * 4 + 255) // 256 * 256
+    assert qgemm.moe_workspace_size("nvfp4", 512, K, M, 300) == 0
