@@ -66,6 +66,7 @@ def _load():
             lib.orc_pack_nvfp4.argtypes = [vp, i64, i64, vp, vp, vp]
             lib.orc_pack_mxfp4.argtypes = [vp, i64, i64, vp, vp]
             lib.orc_pack_fp8.argtypes = [vp, i64, i64, vp, vp]
+            lib.orc_split_x.argtypes = [vp, i64, i64, ctypes.c_int, ctypes.c_int, vp]
             lib.orc_dequant.argtypes = [ctypes.c_int, vp, vp, ctypes.c_float, i64, i64, vp]
             lib.orc_gemm.argtypes = [vp, i64, i64, vp, i64, vp, ctypes.c_int]
             lib.orc_ffn_gate_up.argtypes = [vp, i64, i64, vp, vp, i64, vp, vp, vp, ctypes.c_int]
@@ -197,6 +198,21 @@ def gemm(x16: np.ndarray, Wd: np.ndarray, nthreads: int | None = None) -> np.nda
     y = np.zeros((B, N), dtype=np.float64)
     _load().orc_gemm(_ptr(x16), B, K, _ptr(Wd), N, _ptr(y), nthreads or default_threads())
     return y
+
+
+def split_x(x16: np.ndarray, elem: str, terms: int) -> np.ndarray:
+    """x (bf16 bits [B, K]) peeled into `terms` E4M3 ("e4m3") or E2M1 ("e2m1") terms per
+    32-block, each with its own power-of-two scale; returns the sum of the terms (fp64)."""
+    x16 = np.ascontiguousarray(x16, dtype=np.uint16)
+    B, K = x16.shape
+    xs = np.zeros((B, K), dtype=np.float64)
+    _load().orc_split_x(_ptr(x16), B, K, 0 if elem == "e4m3" else 1, terms, _ptr(xs))
+    return xs
+
+
+def gemm_f64(xd: np.ndarray, Wd: np.ndarray) -> np.ndarray:
+    """y = xd Wd^T for an fp64 x (the split activations) -- numpy's fp64 matmul."""
+    return np.asarray(xd, dtype=np.float64) @ np.asarray(Wd, dtype=np.float64).T
 
 
 def ffn_gate_up(x16: np.ndarray, Wg: np.ndarray, Wu: np.ndarray, nthreads: int | None = None):

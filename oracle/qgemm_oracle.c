@@ -463,6 +463,52 @@ void orc_gemm(const uint16_t *x16, int64_t B, int64_t K, const double *Wd, int64
 }
 
 /* ------------------------------------------------------------------------- */
+/* Activation split for a block-scaled MMA (the "on-the-fly activation          */
+/* quantisation" of a kind::mxf8f6f4 / kind::mxf4 path).  Reading: each 32-block */
+/* of a row is peeled into `terms` low-precision terms, each with its own E8M0   */
+/* (power-of-two) scale from the remaining block maximum:                        */
+/*   r_0 = x;  e_j = floor(log2 max|r_j|) - top;  q_j = ENC(r_j / 2^e_j);        */
+/*   r_{j+1} = r_j - q_j 2^e_j                                                   */
+/* with top = 7 for E4M3 (the maximum lands in [128, 256), below 448) and top = 2 */
+/* for E2M1 (the maximum lands in [4, 8), saturating at 6, as the MXFP4 packer).  */
+/* xs receives sum_j q_j 2^e_j, the x the block-scaled MMA would multiply.       */
+/* elem: 0 = E4M3, 1 = E2M1.                                                     */
+/* ------------------------------------------------------------------------- */
+void orc_split_x(const uint16_t *x16, int64_t B, int64_t K, int elem, int terms, double *xs) {
+    const int top = elem == 0 ? 7 : 2;
+    for (int64_t b = 0; b < B; ++b) {
+        for (int64_t k0 = 0; k0 < K; k0 += 32) {
+            double r[32], acc[32];
+            const int64_t n = (K - k0 < 32) ? K - k0 : 32;
+            for (int64_t i = 0; i < n; ++i) {
+                r[i] = orc_bf16(x16[b * K + k0 + i]);
+                acc[i] = 0.0;
+            }
+            for (int j = 0; j < terms; ++j) {
+                double amax = 0.0, sc;
+                int ex;
+                for (int64_t i = 0; i < n; ++i) amax = fmax(amax, fabs(r[i]));
+                if (amax == 0.0) break;
+                (void)frexp(amax, &ex);           /* floor(log2 amax) = ex - 1 */
+                sc = ldexp(1.0, (ex - 1) - top);
+                for (int64_t i = 0; i < n; ++i) {
+                    double q;
+                    if (elem == 0) {
+                        unsigned c = orc_e4m3_encode(r[i] / sc);
+                        q = orc_e4m3(c);
+                    } else {
+                        q = orc_e2m1(orc_e2m1_encode(r[i] / sc));
+                    }
+                    acc[i] += q * sc;
+                    r[i] -= q * sc;
+                }
+            }
+            for (int64_t i = 0; i < n; ++i) xs[b * K + k0 + i] = acc[i];
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------- */
 /* Fused FFN (Atlas issue: fused gate+up with dual accumulators; the pages'    */
 /* prefill path writes the activated product as bf16 for the down GEMM).      */
 /*   g = x Wg^T, u = x Wu^T (fp64); SiLU(g) = g / (1 + exp(-g));               */

@@ -530,3 +530,50 @@ def test_pins_catch_planted_mistakes(tmp_path):
     assert not _hand_rows_hold(_mutant(tmp_path, 4))        # Q8_0 scale bytes swapped
     assert not _hand_rows_hold(_mutant(tmp_path, 5))        # FP8 tensor scale dropped
     assert not _hand_rows_hold(_mutant(tmp_path, 6))        # FP8 sign bit ignored
+
+
+# ------------------------------------------------------------------------------------------
+# Activation split for a block-scaled MMA (the decision input of the block-scaled path)
+# ------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("elem,top", [("e4m3", 7), ("e2m1", 2)])
+def test_activation_split_first_term_brute_force(elem, top):
+    # one term: each element is the code value nearest to x / 2^e (ties to the even code,
+    # saturating), e = floor(log2 max|block|) - top, computed here from the definitions
+    x16 = inputs.bf16_bits(inputs.activations(3, 96, seed=51))
+    xs = oracle.split_x(x16, elem, 1)
+    if elem == "e4m3":
+        vals = [Fraction(oracle.e4m3(b)) for b in range(0x7F)]
+    else:
+        vals = [Fraction(v) for v in E2M1_MAG]
+    for b in range(3):
+        for k0 in range(0, 96, 32):
+            blk = [Fraction(oracle.bf16(int(v))) for v in x16[b, k0:k0 + 32]]
+            amax = max(abs(v) for v in blk)
+            _, ex = math.frexp(float(amax))
+            sc = Fraction(2) ** ((ex - 1) - top)
+            for i, v in enumerate(blk):
+                a = abs(v) / sc
+                best = min(range(len(vals)), key=lambda c: (abs(a - vals[c]), c & 1))
+                want = vals[best] * sc * (1 if v >= 0 else -1)
+                assert Fraction(float(xs[b, k0 + i])) == want, (b, k0 + i)
+
+
+def test_activation_split_accuracy_for_the_block_scaled_path():
+    # the 1e-3 bar of the method, for x ~ N(0, 1) in bf16 and NVFP4 / MXFP4 weights, at the
+    # 27B FFN reduction lengths: one E4M3 term is not enough, two are exact for all but a
+    # handful of elements; three E2M1 terms keep a wide margin
+    for K in (5120, 17408):
+        x16 = inputs.bf16_bits(inputs.activations(4, K, seed=52))
+        xd = oracle.bf16_decode_array(x16)
+        for fmt in ("nvfp4", "mxfp4"):
+            W = inputs.weights(16, K, seed=53).numpy()
+            Wd = oracle.dequant(fmt, *oracle.pack(fmt, W), 16, K)
+            y = oracle.gemm(x16, Wd)
+            err = {}
+            for elem, t in (("e4m3", 1), ("e4m3", 2), ("e4m3", 3), ("e2m1", 3), ("e2m1", 4)):
+                xs = oracle.split_x(x16, elem, t)
+                err[(elem, t)] = oracle.normalised_error(oracle.gemm_f64(xs, Wd), y, x16, Wd)
+            assert err[("e4m3", 1)] > 1e-4
+            assert err[("e4m3", 2)] < 1e-8 and err[("e4m3", 3)] < 1e-10
+            assert err[("e2m1", 3)] < 2e-4 and err[("e2m1", 4)] < 2e-5
+            assert np.array_equal(oracle.split_x(x16, "e4m3", 3), xd)  # three terms: exact
