@@ -279,6 +279,7 @@ def clone_ring(pw, n):
 def run_configs(dev, stream, q8_rings, hbm_peak, tf_peak):
     """Every workload configuration, timed per call on the device (kernel time: x preparation
     + GEMM [+ split-K reduce] per call; graphs of back-to-back calls over a weight ring)."""
+    import numpy as np
     import torch
     from block_quantized_weight_qgemm_b200 import inputs, qgemm
 
@@ -392,6 +393,45 @@ def run_configs(dev, stream, q8_rings, hbm_peak, tf_peak):
     del ring
     prefill("fp8 27B gate/up prefill", "fp8", fp8, 2048)
     del fp8
+    torch.cuda.empty_cache()
+    # routed experts (Flash-Next-style MoE: 512 experts, top-10; expert shape hidden 2048 x
+    # expert FFN 512): fused gate+up then the routed down projection, NVFP4
+    E, H, F = 512, 2048, 512
+    gen = torch.Generator(device=dev).manual_seed(0)
+    mats = {}
+    for name, (n, k) in (("gate", (F, H)), ("up", (F, H)), ("down", (H, F))):
+        W = torch.randn(E, n, k, generator=gen, device=dev) * 0.02
+        mats[name] = qgemm.ExpertTable([qgemm.pack("nvfp4", W[e]) for e in range(E)])
+        del W
+    for T, reps in ((64, 20), (2048, 4)):
+        tok, _, off_np = inputs.routing(T, E, 10, seed=0)
+        M = len(tok)
+        x = inputs.activations(M, H, seed=1).to(dev)
+        off = torch.from_numpy(off_np).to(dev)
+        mr = int(np.diff(off_np).max())
+        h = torch.empty(M, F, dtype=torch.bfloat16, device=dev)
+        y = torch.empty(M, H, dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(max(qgemm.moe_workspace_size("nvfp4", F, H, M, mr),
+                             qgemm.moe_workspace_size("nvfp4", H, F, M, mr), 16),
+                         dtype=torch.uint8, device=dev)
+
+        def moe_step(i):
+            qgemm.moe_gate_up(x, off, mats["gate"], mats["up"], mr, h=h, workspace=ws, stream=stream)
+            qgemm.moe_run(h, off, mats["down"], mr, y=y, workspace=ws, stream=stream)
+
+        us = graph_us(moe_step, reps, stream)
+        active = int((np.diff(off_np) > 0).sum())
+        nb = active * (2 * weight_bytes("nvfp4", F, H) + weight_bytes("nvfp4", H, F))
+        flop = 2.0 * M * (2 * F) * H + 2.0 * M * H * F
+        r = {"config": "nvfp4 routed MoE (512 experts, top-10, 2048x512)", "kind": "decode" if T <= 64 else "prefill",
+             "fmt": "nvfp4", "tokens": T, "routed_rows": M, "active_experts": active,
+             "max_rows": mr, "us": round(us, 1), "weight_GBps": round(nb / (us * 1e-6) / 1e9, 1),
+             "frac_hbm": round(nb / (us * 1e-6) / 1e9 / hbm_peak, 4),
+             "TFLOPs": round(flop / (us * 1e-6) / 1e12, 1),
+             "frac_tensor": round(flop / (us * 1e-6) / 1e12 / tf_peak, 4)}
+        recs.append(r)
+        del x, h, y, ws
+    del mats
     torch.cuda.empty_cache()
     # cfg 5: MXFP4 serving mix (B = 32 decode, M = 8192 prefill) on both shapes
     for N, K, seed in ((INTER, HIDDEN, 0), (HIDDEN, INTER, 3)):

@@ -239,7 +239,7 @@ bool make_plan_pair(int fmt, int64_t N, int64_t K, int64_t B, int nmat, Plan* pl
   p.tmem_cols = next_pow2_cols(p.R * p.NACC * p.NB + p.AS * kPairACols);
   if (p.tmem_cols > 512) return false;
   const size_t xstage = (size_t)(p.NB / 2) * 128 * (kPairAK / kSubK);
-  const size_t misc = 8 * (2 * 4 + 2 * kMaxWStages + 2 * 6 + 1) + 16 + 8 * kMaxNB + 64;
+  const size_t misc = 8 * (2 * 4 + 2 * kMaxWStages + 2 * 6 + 4) + 16 + 8 * kMaxNB + 64;
   const size_t budget = kSmemLimit - 1024 - misc;
   const size_t wstage = (size_t)pair_wstage_bytes(fmt);
   // x ring depth 4 or 2 (even): the two issuers take alternate groups, so an x stage's
@@ -253,7 +253,8 @@ bool make_plan_pair(int fmt, int64_t N, int64_t K, int64_t B, int nmat, Plan* pl
   p.smem_x = 0;
   p.smem_w = (uint32_t)(XS * xstage);
   p.smem_bar = p.smem_w + (uint32_t)(WS * wstage);
-  const size_t bar_bytes = 8 * (2 * XS + 2 * WS + 2 * p.AS + 1);
+  // ring barriers, then the accumulator hand-over pair and the issuers' two drain barriers
+  const size_t bar_bytes = 8 * (2 * XS + 2 * WS + 2 * p.AS + 4);
   // control words, then per-column exponents and factors (int and float per batch column)
   p.smem_bytes = 1024 + p.smem_bar + bar_bytes + 16 + 8 * p.NB + 64;
   size_t off = 0;
@@ -463,6 +464,7 @@ int run_impl(int fmt, const void* x, int64_t B, int64_t K, const void* const* co
   const int64_t grid64 = (int64_t)pl.n_groups * pl.b_tiles * (moe ? moe->E : pl.S);
   if (grid64 > 0x3FFFFFFF) return QGEMM_ERR_SHAPE;
   const int grid = (int)grid64;
+  p.units = grid;
   if (g_prof_begin) cudaEventRecord(g_prof_begin, stream);
   // with f16 operands the GEMM follows the x preparation as its programmatic dependent
   cudaError_t e = launch_pair(fmt, !pl.f16ops, p, pl.smem_bytes, grid, &xmap, pl.f16ops, stream);

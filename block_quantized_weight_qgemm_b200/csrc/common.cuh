@@ -94,6 +94,7 @@ struct GemmParams {
   int S;         // K splits (fixed by fmt, N, K for B <= 256)
   int n_groups;  // ceil(row tiles / (R / NMAT))
   int b_tiles;   // ceil(B / NB)
+  int units;     // work units of the call; the persistent grid's CTA pairs share them out
   int chunks;    // ceil(K / chunk_k)
   int XS, WS;    // x ring and weight ring depths
   int AS;        // A ring depth (TMEM slots of kPairSlotK; even: each stage half owns AS/2)

@@ -184,6 +184,21 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
   return r;
 }
 
+// Named barrier `id` over `nthreads` threads (whole warps) that also reduces a predicate:
+// true for every thread when it was true for all of them.
+__device__ __forceinline__ bool bar_and(uint32_t id, uint32_t nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
+
 // Every thread of both CTAs: release this CTA's prior writes, acquire the peer's.
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile(
