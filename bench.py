@@ -672,17 +672,18 @@ def main():
 
 def _traffic_from_profiles():
     """DRAM bytes per launch of the timed kernel from the committed ncu summary, if it was
-    taken on the current kernel source (else null)."""
+    taken on the current source of that kernel (the files listed in the summary, hashed in
+    order); else null."""
     import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             d = json.load(f)
         h = hashlib.sha256()
-        for name in sorted(os.listdir(os.path.join(ROOT, "block_quantized_weight_qgemm_b200", "csrc"))):
-            with open(os.path.join(ROOT, "block_quantized_weight_qgemm_b200", "csrc", name), "rb") as f:
+        for rel in d["sources"]:
+            with open(os.path.join(ROOT, rel), "rb") as f:
                 h.update(f.read())
-        if d.get("csrc_sha256") != h.hexdigest():
+        if d.get("sources_sha256") != h.hexdigest():
             return None
         return d.get("dram_bytes_per_launch_scaled")
     except Exception:
