@@ -1,0 +1,638 @@
+// bs.cu -- the block-scaled tensor-core path for MXFP4 weights at prefill widths (sm_100a).
+//
+// y[m][n] = sum_k x[m][k] * dequant(W)[n][k] with W in MXFP4 (E2M1 codes, one E8M0 scale per
+// 32 elements; OCP Microscaling format as the Atlas issue's "Fix: F16 operands with an exact
+// dequant" section describes it) and x in bf16, on tcgen05.mma.kind::mxf4nvf4 with 32-element
+// E8M0 block scales on both operands, so that the packed weights reach the tensor cores as
+// they are, without a dequantisation pass.
+//
+// x is not an MMA type here.  The split kernel writes each row as the sum of three E2M1 terms
+// with their own E8M0 scale per 32 elements: per block, r_0 = x * 2^-x_exp (x_exp = the row's
+// floor(log2 max|x|), an exact power of two that the epilogue restores), e_j = floor(log2
+// max|r_j|) - 2, q_j = E2M1(r_j / 2^e_j) (round to nearest even, saturating at 6),
+// r_{j+1} = r_j - q_j 2^e_j.  Three terms leave a residual below 2^-6 of each block's maximum
+// before rounding; measured against the exact product the normalised error is below 1e-4 at
+// the 27B shapes.  A term whose scale would fall below 2^-127 (blocks more than 2^125 below
+// the row maximum) is dropped.
+//
+// Layout of the split x (device, written by qgemm_bs_split_x, read by the GEMM):
+//   codes : [Mt][C][3][128 rows][128 bytes]   Mt = ceil(M/128) token tiles, C = ceil(K/256)
+//           chunks; row r of a (tile, chunk, term) block holds elements 256c .. 256c+255 of
+//           token 128 t + r, two per byte (even element in the low nibble), its 16-byte
+//           groups stored at group ^ (r & 7) (the 128-byte swizzle of the MMA operand, as the
+//           tile-major weights).  Tokens past M and elements past K are zero.
+//   scales: [Mt][C][3][128 rows][8]   E8M0 per 32 elements (bias 127).
+//   x_exp : [Mt * 128] int32.
+//
+// GEMM: one CTA per SM (persistent).  A tile is 128 tokens (MMA M, the x terms as operand A)
+// x 256 weight rows (MMA N, two tile-major weight tiles as operand B) over all of K.  Per
+// 256-K chunk the producer brings the three x-term blocks and the two weight blocks with their
+// scales into one of two shared-memory stages (1-D bulk copies); four staging warps place the
+// stage's scale factors in tensor memory with tcgen05.st in the layout the block-scaled MMA
+// reads (per 64-K block: scale j of row r = r0 + 32 r1 at lane r0 of every lane quarter,
+// column r1, byte j); one thread issues 4 K-blocks x 3 terms of M128 N256 K64 MMAs into one
+// fp32 accumulator; four epilogue warps read it out, restore 2^x_exp and store y.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp4.h>
+
+#include <atomic>
+
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace qg {
+
+constexpr int kBsTerms = 3;
+constexpr int kBsM = 128;                     // tokens per tile
+constexpr int kBsN = 256;                     // weight rows per tile (two weight tiles)
+constexpr int kBsK = 256;                     // K per stage (one MXFP4 chunk)
+constexpr int kBsStages = 2;
+constexpr int kBsBlock = kBsM * 128;          // one 128-row x 128-byte code block: 16 KB
+constexpr int kBsSBlock = kBsM * 8;           // its scales: 1 KB
+constexpr int kBsACodes = kBsTerms * kBsBlock;
+constexpr int kBsBCodes = 2 * kBsBlock;
+constexpr int kBsAScales = kBsTerms * kBsSBlock;
+constexpr int kBsBScales = 2 * kBsSBlock;
+constexpr int kBsStage = kBsACodes + kBsBCodes + kBsAScales + kBsBScales;  // 85 KB
+static_assert(kBsStage % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
+// tensor memory: the accumulator in columns [0, 256), then per stage kBsSfCols columns of
+// scale factors: x term t, K-block kb at (t * 4 + kb) * 4 (4 columns: row groups r1 = 0..3),
+// the weights' K-block kb at 48 + kb * 8 (8 columns: r1 = 0..7)
+constexpr int kBsSfCols = kBsTerms * 4 * 4 + 4 * 8;  // 80
+constexpr int kBsTmemCols = 512;
+static_assert(kBsN + kBsStages * kBsSfCols <= kBsTmemCols, "TMEM budget");
+constexpr int kBsStageWarp0 = 2;  // warps 2..5 stage the scale factors
+constexpr int kBsEpiWarp0 = 6;    // warps 6..9 run the epilogue
+constexpr int kBsThreads = 10 * 32;
+constexpr int kBsSmem = 1024 + kBsStages * kBsStage + 256;
+
+struct BsSplitParams {
+  const uint16_t* x;  // bf16 [M][K]
+  int M, K, C, Mt;
+  uint8_t* codes;
+  uint8_t* scales;
+  int* x_exp;
+};
+
+struct BsParams {
+  int M, N, K, C, Mt, Nt, units;
+  const uint8_t* xcodes;
+  const uint8_t* xscales;
+  const int* x_exp;
+  const uint8_t* wcodes;   // tile-major MXFP4 codes
+  const uint8_t* wscales;  // tile-major MXFP4 scales
+  void* out;               // y [M][N] fp32 or bf16
+  int out_bf16;
+  int* dev_err;
+};
+
+// ---------------------------------------------------------------------------------------
+// Split: one CTA of 256 threads per token row of the padded tile range (rows past M write
+// zeros).  Phase 1: the row maximum and x_exp.  Phase 2: each 256-element chunk is one warp's,
+// lane l holding elements 8l .. 8l+7 of it, so four lanes share a 32-element block.
+// Every step is exact in fp32: bf16 values times powers of two, an E2M1 code times a power of
+// two, and r - q 2^e, whose significand fits 24 bits because |r - q 2^e| is at most half an
+// E2M1 step at |r|'s magnitude (or the saturation error, 2^(e+1), where |r| >= 2^(e+2)).
+// ---------------------------------------------------------------------------------------
+constexpr int kBsSplitThreads = 256;
+constexpr int kBsSplitRegs = 3;  // 8-element words per thread kept from phase 1 (rows to 6144)
+
+__device__ __forceinline__ float bs_pow2(int e) {  // 2^e for -149 <= e <= 127, exact
+  return e >= -126 ? __int_as_float((e + 127) << 23) : __int_as_float(1 << (e + 149));
+}
+__device__ __forceinline__ float bs_amax8(float m, const uint4& v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    m = fmaxf(m, fmaxf(fabsf(__uint_as_float(w[i] << 16)), fabsf(__uint_as_float(w[i] & 0xFFFF0000u))));
+  return m;
+}
+
+// The three terms of one lane's 8 elements (its quarter of a 32-element block), written to
+// the split layout.  All four lanes of the block take the same decisions (the block maximum
+// is reduced over them first).
+__device__ __forceinline__ void bs_split8(const BsSplitParams& p, const uint4& v, bool in, float f1,
+                                          float f2, int t, int r, int c, int lane) {
+  float rv[8];
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    rv[2 * i] = in ? (__uint_as_float(w[i] << 16) * f1) * f2 : 0.f;
+    rv[2 * i + 1] = in ? (__uint_as_float(w[i] & 0xFFFF0000u) * f1) * f2 : 0.f;
+  }
+  const int j = lane >> 2;  // 32-element block of the chunk
+  bool done = false;
+#pragma unroll
+  for (int term = 0; term < kBsTerms; ++term) {
+    float bmax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) bmax = fmaxf(bmax, fabsf(rv[i]));
+    bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 1));
+    bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 2));
+    int sb = 0;  // E8M0 byte
+    uint32_t packed = 0u;
+    if (!done && bmax > 0.f) {
+      int ex;
+      (void)frexpf(bmax, &ex);
+      const int e = (ex - 1) - 2;  // block maximum / 2^e in [4, 8)
+      if (e >= -127) {
+        sb = e + 127;
+        const float inv = bs_pow2(-e), sc = bs_pow2(e);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          // two codes (element 2i in the low nibble), rounded to nearest even and saturated
+          // at 6 by the hardware conversion, and their values back as f16 (exact)
+          const __nv_fp4x2_storage_t c2 = __nv_cvt_float2_to_fp4x2(
+              make_float2(rv[2 * i] * inv, rv[2 * i + 1] * inv), __NV_E2M1, cudaRoundNearest);
+          const __half2_raw h = __nv_cvt_fp4x2_to_halfraw2(c2, __NV_E2M1);
+          rv[2 * i] = fmaf(-__half2float(__half(__half_raw{h.x})), sc, rv[2 * i]);
+          rv[2 * i + 1] = fmaf(-__half2float(__half(__half_raw{h.y})), sc, rv[2 * i + 1]);
+          packed |= (uint32_t)c2 << (8 * i);
+        }
+      } else {
+        done = true;  // below the E8M0 range: this and the later terms are dropped
+      }
+    } else {
+      done = true;
+    }
+    const size_t bidx = ((size_t)t * p.C + c) * kBsTerms + term;
+    // the block's 16 bytes are group j of the row, stored at group j ^ (r & 7)
+    uint8_t* crow = p.codes + bidx * kBsBlock + (size_t)r * 128;
+    *reinterpret_cast<uint32_t*>(crow + (((j ^ (r & 7)) & 7) << 4) + (lane & 3) * 4) = packed;
+    if ((lane & 3) == 0) p.scales[bidx * kBsSBlock + (size_t)r * 8 + j] = (uint8_t)(done ? 0 : sb);
+  }
+}
+
+__global__ void __launch_bounds__(kBsSplitThreads) qgemm_bs_split_kernel(const BsSplitParams p) {
+  // x may come from the preceding grid.  Only once that grid has completed may the GEMM
+  // launch: it reads the weights before it waits for this grid, and the grid before may have
+  // written them.
+  griddep_wait();
+  griddep_launch_dependents();
+  const int m = blockIdx.x;
+  const bool live = m < p.M;
+  const uint16_t* xr = p.x + (size_t)(live ? m : 0) * p.K;
+  __shared__ float red[kBsSplitThreads / 32];
+  // Phase 1: the row maximum.  Thread i reads the 8-element words k = 8 (i + 256 n); the same
+  // thread converts them in phase 2 (word n is lane i % 32 of chunk 8 n + i / 32), so the first
+  // kBsSplitRegs words stay in registers.
+  const int Kp = p.C * kBsK;
+  uint4 v[kBsSplitRegs];
+  float amax = 0.f;
+#pragma unroll
+  for (int n = 0; n < kBsSplitRegs; ++n) {
+    const int k = (threadIdx.x + n * kBsSplitThreads) * 8;
+    v[n] = (live && k < p.K) ? *reinterpret_cast<const uint4*>(xr + k) : make_uint4(0u, 0u, 0u, 0u);
+    amax = bs_amax8(amax, v[n]);
+  }
+  if (live)
+    for (int k = (threadIdx.x + kBsSplitRegs * kBsSplitThreads) * 8; k < p.K; k += kBsSplitThreads * 8)
+      amax = bs_amax8(amax, *reinterpret_cast<const uint4*>(xr + k));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  amax = red[0];
+#pragma unroll
+  for (int i = 1; i < kBsSplitThreads / 32; ++i) amax = fmaxf(amax, red[i]);
+  int xe = 0;
+  if (amax > 0.f && amax <= 3.4e38f) {
+    int ex;
+    (void)frexpf(amax, &ex);
+    xe = ex - 1;  // row maximum * 2^-xe in [1, 2)
+  }
+  if (threadIdx.x == 0) p.x_exp[m] = live ? xe : 0;
+  // 2^-xe as two exact factors (xe runs from -133 to 127)
+  const int a1 = min(-xe, 126);
+  const float f1 = bs_pow2(a1), f2 = bs_pow2(-xe - a1);
+  const int t = m / kBsM, r = m % kBsM;
+  const int lane = threadIdx.x & 31;
+  // Phase 2: word n of this thread is lane `lane` of chunk c = 8 (i + 256 n) / 256
+#pragma unroll
+  for (int n = 0; n < kBsSplitRegs; ++n) {
+    const int k = (threadIdx.x + n * kBsSplitThreads) * 8;
+    if (k < Kp) bs_split8(p, v[n], live && k < p.K, f1, f2, t, r, k / kBsK, lane);
+  }
+  for (int k = (threadIdx.x + kBsSplitRegs * kBsSplitThreads) * 8; k < Kp; k += kBsSplitThreads * 8) {
+    const bool in = live && k < p.K;
+    const uint4 w = in ? *reinterpret_cast<const uint4*>(xr + k) : make_uint4(0u, 0u, 0u, 0u);
+    bs_split8(p, w, in, f1, f2, t, r, k / kBsK, lane);
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// GEMM
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ void bs_tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void bs_tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void bs_tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+// D (+)= A * B^T with 32-element E8M0 block scales: A, B K-major E2M1 in shared memory, the
+// scale factors in tensor memory at sfa / sfb.
+__device__ __forceinline__ void bs_mma(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t"
+      "}" ::"r"(d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+__device__ __forceinline__ void bs_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+// Each lane writes 16 consecutive 32-bit columns of its own TMEM lane.
+__device__ __forceinline__ void bs_tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+// Each lane reads 32 consecutive 32-bit columns of its own TMEM lane.
+__device__ __forceinline__ void bs_tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+      "%30, %31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+        "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]),
+        "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]),
+        "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr)
+      : "memory");
+}
+
+// Instruction descriptor, kind::mxf4nvf4: A and B E2M1 (K-major), E8M0 scales, M = 128,
+// N = 256, K = 64 per instruction, scale factor ids 0.
+constexpr uint32_t kBsIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(kBsN >> 3) << 17) | (1u << 23) |
+                              ((uint32_t)(kBsM >> 4) << 24);
+
+__device__ __forceinline__ float bs_scale_pow2(float v, int e) {
+  return (e >= -126 && e <= 127) ? v * __int_as_float((e + 127) << 23) : ldexpf(v, e);
+}
+
+__global__ void __launch_bounds__(kBsThreads, 1) qgemm_bs_kernel(const __grid_constant__ BsParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBsStages * kBsStage);
+  const uint32_t bar_full = smem_u32(bars);                  // [2] stage data landed
+  const uint32_t bar_empty = bar_full + 8 * kBsStages;       // [2] the stage's MMAs are done
+  const uint32_t bar_sf = bar_empty + 8 * kBsStages;         // [2] its scale factors are in TMEM
+  const uint32_t bar_acc = bar_sf + 8 * kBsStages;           // a tile's accumulator is complete
+  const uint32_t bar_acc_free = bar_acc + 8;                 // the epilogue has read it
+  const uint32_t bar_drain = bar_acc_free + 8;               // the issuer's MMAs are done
+  int* ctl = reinterpret_cast<int*>(bars + 3 * kBsStages + 3);
+  volatile int* abort_flag = ctl + 1;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < kBsStages; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, 1);
+      mbar_init(bar_sf + 8 * s, 4);
+    }
+    mbar_init(bar_acc, 1);
+    mbar_init(bar_acc_free, 4);
+    mbar_init(bar_drain, 1);
+    ctl[1] = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    bs_tmem_alloc(smem_u32(ctl), kBsTmemCols);
+    bs_tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = static_cast<uint32_t>(ctl[0]);
+  const int64_t n_row_tiles = row_tiles(p.N);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_last();
+      const uint64_t pol_x = policy_evict_last();
+      RingPos sp;
+      int issued = 0;
+      bool ok = true;
+      bool waited = false;
+      for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+        const int mt = u % p.Mt, nt = u / p.Mt;
+        for (int c = 0; c < p.C; ++c) {
+          if (issued >= kBsStages &&
+              !mbar_wait(bar_empty + 8 * sp.slot, sp.phase ^ 1u, abort_flag, p.dev_err, kErrTimeout)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = bar_full + 8 * sp.slot;
+          const uint32_t st = sbase + (uint32_t)(sp.slot * kBsStage);
+          uint32_t bytes = kBsACodes + kBsAScales;
+          for (int j = 0; j < 2; ++j)
+            if (2 * nt + j < n_row_tiles) bytes += kBsBlock + kBsSBlock;
+          mbar_arrive_expect_tx(fb, bytes);
+          for (int j = 0; j < 2; ++j) {
+            const int64_t t = 2 * (int64_t)nt + j;
+            if (t >= n_row_tiles) continue;
+            const int64_t blk = t * p.C + c;
+            bulk_load(st + kBsACodes + j * kBsBlock, p.wcodes + blk * kBsBlock, kBsBlock, fb, pol_w);
+            bulk_load(st + kBsACodes + kBsBCodes + kBsAScales + j * kBsSBlock,
+                      p.wscales + blk * kBsSBlock, kBsSBlock, fb, pol_w);
+          }
+          // the split x comes from the preceding grid
+          if (!waited) {
+            griddep_wait();
+            waited = true;
+          }
+          const int64_t xb = ((int64_t)mt * p.C + c) * kBsTerms;
+          bulk_load(st, p.xcodes + xb * kBsBlock, kBsACodes, fb, pol_x);
+          bulk_load(st + kBsACodes + kBsBCodes, p.xscales + xb * kBsSBlock, kBsAScales, fb, pol_x);
+          sp.next(kBsStages);
+          ++issued;
+        }
+      }
+      if (!ok) {
+        // let the copies in flight land before the CTA leaves
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 200000) __nanosleep(1000);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      RingPos sp;
+      bool ok = true;
+      int ti = 0;
+      for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x, ++ti) {
+        if (ti > 0) {
+          if (!mbar_wait_spin(bar_acc_free, (uint32_t)(ti - 1) & 1u, false, abort_flag, p.dev_err,
+                              kErrTimeout)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
+        for (int c = 0; c < p.C; ++c) {
+          if (!mbar_wait_spin(bar_full + 8 * sp.slot, sp.phase, false, abort_flag, p.dev_err, kErrTimeout) ||
+              !mbar_wait_spin(bar_sf + 8 * sp.slot, sp.phase, false, abort_flag, p.dev_err, kErrTimeout)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t st = sbase + (uint32_t)(sp.slot * kBsStage);
+          const uint64_t bdesc0 = smem_desc_sw128(st + kBsACodes);
+          const uint32_t sf0 = tmem + (uint32_t)(kBsN + sp.slot * kBsSfCols);
+#pragma unroll
+          for (int kb = 0; kb < kBsK / 64; ++kb) {
+#pragma unroll
+            for (int t = 0; t < kBsTerms; ++t) {
+              const uint64_t adesc = smem_desc_sw128(st + (uint32_t)(t * kBsBlock)) + (uint64_t)(kb * 2);
+              bs_mma(tmem, adesc, bdesc0 + (uint64_t)(kb * 2), kBsIdesc,
+                     sf0 + (uint32_t)((t * 4 + kb) * 4), sf0 + (uint32_t)(48 + kb * 8),
+                     (c | kb | t) != 0 ? 1u : 0u);
+            }
+          }
+          bs_commit(bar_empty + 8 * sp.slot);
+          sp.next(kBsStages);
+        }
+        if (!ok) break;
+        bs_commit(bar_acc);
+      }
+      bs_commit(bar_drain);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(bar_drain, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+      }
+    }
+    __syncwarp();
+  } else if (warp < kBsEpiWarp0) {
+    // ------------------------------------------------------------ scale-factor staging
+    // Every warp writes the same values into its own lane quarter (the MMA reads the scale
+    // factors of row r0 + 32 r1 from lane r0 of each quarter).
+    const int q = warp & 3;
+    const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+    RingPos sp;
+    int used = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+      for (int c = 0; c < p.C; ++c) {
+        if (used >= kBsStages) {
+          ok = mbar_wait(bar_empty + 8 * sp.slot, sp.phase ^ 1u, abort_flag, p.dev_err, kErrTimeout);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+        }
+        ok = mbar_wait(bar_full + 8 * sp.slot, sp.phase, abort_flag, p.dev_err, kErrTimeout);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        const uint8_t* st = smem + sp.slot * kBsStage;
+        const uint8_t* sa = st + kBsACodes + kBsBCodes;  // x-term scales [3][128][8]
+        const uint8_t* sb = sa + kBsAScales;              // weight scales [2][128][8]
+        uint32_t v[kBsSfCols];
+#pragma unroll
+        for (int t = 0; t < kBsTerms; ++t)
+#pragma unroll
+          for (int r1 = 0; r1 < 4; ++r1) {
+            const uint2 s8 = *reinterpret_cast<const uint2*>(sa + t * kBsSBlock + (r1 * 32 + lane) * 8);
+#pragma unroll
+            for (int kb = 0; kb < 4; ++kb) {
+              const uint32_t w = (kb < 2) ? s8.x : s8.y;
+              v[(t * 4 + kb) * 4 + r1] = (w >> ((kb & 1) * 16)) & 0xFFFFu;
+            }
+          }
+#pragma unroll
+        for (int r1 = 0; r1 < 8; ++r1) {
+          const uint2 s8 = *reinterpret_cast<const uint2*>(sb + (r1 >> 2) * kBsSBlock + ((r1 & 3) * 32 + lane) * 8);
+#pragma unroll
+          for (int kb = 0; kb < 4; ++kb) {
+            const uint32_t w = (kb < 2) ? s8.x : s8.y;
+            v[48 + kb * 8 + r1] = (w >> ((kb & 1) * 16)) & 0xFFFFu;
+          }
+        }
+        const uint32_t ta = tmem + lane_base + (uint32_t)(kBsN + sp.slot * kBsSfCols);
+#pragma unroll
+        for (int i = 0; i < kBsSfCols / 16; ++i)
+          bs_tmem_st16(ta + (uint32_t)(16 * i), *reinterpret_cast<const uint32_t(*)[16]>(&v[16 * i]));
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_sf + 8 * sp.slot);
+        sp.next(kBsStages);
+        ++used;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;
+    const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+    griddep_wait();  // x_exp comes from the split kernel
+    int ti = 0;
+    for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++ti) {
+      const int mt = u % p.Mt, nt = u / p.Mt;
+      const int m = mt * kBsM + q * 32 + lane;
+      const int xe = (m < p.M) ? p.x_exp[m] : 0;
+      bool ok = mbar_wait(bar_acc, (uint32_t)ti & 1u, abort_flag, p.dev_err, kErrTimeout);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll 1
+      for (int cb = 0; cb < kBsN; cb += 32) {
+        uint32_t v[32];
+        bs_tmem_ld32(tmem + lane_base + (uint32_t)cb, v);
+        tmem_ld_wait();
+        const int n0 = nt * kBsN + cb;
+        if (m < p.M && n0 < p.N) {
+          if (p.out_bf16) {
+            __nv_bfloat16* yr = reinterpret_cast<__nv_bfloat16*>(p.out) + (size_t)m * p.N + n0;
+            if (n0 + 32 <= p.N && (p.N % 8) == 0) {
+#pragma unroll
+              for (int i = 0; i < 32; i += 8) {
+                uint32_t w[4];
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                  const __nv_bfloat16 lo = __float2bfloat16_rn(bs_scale_pow2(__uint_as_float(v[i + 2 * h]), xe));
+                  const __nv_bfloat16 hi = __float2bfloat16_rn(bs_scale_pow2(__uint_as_float(v[i + 2 * h + 1]), xe));
+                  w[h] = (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
+                }
+                *reinterpret_cast<uint4*>(yr + i) = make_uint4(w[0], w[1], w[2], w[3]);
+              }
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if (n0 + i < p.N) yr[i] = __float2bfloat16_rn(bs_scale_pow2(__uint_as_float(v[i]), xe));
+            }
+          } else {
+            float* yr = reinterpret_cast<float*>(p.out) + (size_t)m * p.N + n0;
+            if (n0 + 32 <= p.N && (p.N % 4) == 0) {
+#pragma unroll
+              for (int i = 0; i < 32; i += 4)
+                *reinterpret_cast<float4*>(yr + i) =
+                    make_float4(bs_scale_pow2(__uint_as_float(v[i]), xe), bs_scale_pow2(__uint_as_float(v[i + 1]), xe),
+                                bs_scale_pow2(__uint_as_float(v[i + 2]), xe), bs_scale_pow2(__uint_as_float(v[i + 3]), xe));
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if (n0 + i < p.N) yr[i] = bs_scale_pow2(__uint_as_float(v[i]), xe);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_acc_free);
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    bs_tmem_dealloc(tmem, kBsTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Launchers
+// ---------------------------------------------------------------------------------------
+cudaError_t launch_bs_split(const uint16_t* x, int M, int K, uint8_t* codes, uint8_t* scales,
+                            int* x_exp, cudaStream_t stream) {
+  BsSplitParams p{};
+  p.x = x;
+  p.M = M;
+  p.K = K;
+  p.C = (K + kBsK - 1) / kBsK;
+  p.Mt = (M + kBsM - 1) / kBsM;
+  p.codes = codes;
+  p.scales = scales;
+  p.x_exp = x_exp;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(p.Mt * kBsM), 1, 1);
+  cfg.blockDim = dim3(kBsSplitThreads, 1, 1);
+  cfg.stream = stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, qgemm_bs_split_kernel, p);
+}
+
+// SMs of device `dev`, read once per device (devices beyond 64 read it on every launch).
+static int bs_sm_count(int dev) {
+  static std::atomic<int> cached[64];
+  int v = (dev >= 0 && dev < 64) ? cached[dev].load(std::memory_order_relaxed) : 0;
+  if (v > 0) return v;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v < 1) v = 148;
+  if (dev >= 0 && dev < 64) cached[dev].store(v, std::memory_order_relaxed);
+  return v;
+}
+
+cudaError_t launch_bs_gemm(int M, int N, int K, const uint8_t* xcodes, const uint8_t* xscales,
+                           const int* x_exp, const uint8_t* wcodes, const uint8_t* wscales,
+                           void* out, int out_bf16, int* dev_err, cudaStream_t stream) {
+  static std::atomic<uint64_t> set_mask{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+  if (bit == 0 || !(set_mask.load(std::memory_order_acquire) & bit)) {
+    e = cudaFuncSetAttribute(qgemm_bs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kBsSmem);
+    if (e != cudaSuccess) return e;
+    set_mask.fetch_or(bit, std::memory_order_release);
+  }
+  BsParams p{};
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.C = (K + kBsK - 1) / kBsK;
+  p.Mt = (M + kBsM - 1) / kBsM;
+  p.Nt = (N + kBsN - 1) / kBsN;
+  p.units = p.Mt * p.Nt;
+  p.xcodes = xcodes;
+  p.xscales = xscales;
+  p.x_exp = x_exp;
+  p.wcodes = wcodes;
+  p.wscales = wscales;
+  p.out = out;
+  p.out_bf16 = out_bf16;
+  p.dev_err = dev_err;
+  const int sms = bs_sm_count(dev);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)std::min(p.units, sms), 1, 1);
+  cfg.blockDim = dim3(kBsThreads, 1, 1);
+  cfg.dynamicSmemBytes = kBsSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, qgemm_bs_kernel, p);
+}
+
+// workspace of the block-scaled path: split codes, split scales, row exponents
+size_t bs_workspace_bytes(int64_t M, int64_t K, size_t* off_scales, size_t* off_exp) {
+  const int64_t C = (K + kBsK - 1) / kBsK, Mt = (M + kBsM - 1) / kBsM;
+  const size_t codes = (size_t)(Mt * C * kBsTerms) * kBsBlock;
+  const size_t scales = (size_t)(Mt * C * kBsTerms) * kBsSBlock;
+  if (off_scales) *off_scales = codes;
+  if (off_exp) *off_exp = codes + scales;
+  return codes + scales + (size_t)Mt * kBsM * 4;
+}
+
+}  // namespace qg

@@ -50,6 +50,11 @@ SIGNATURES = [
                            _SZ, _VP]),
     ("qgemm_moe_gate_up", _I, [_I, _VP, _I64, _I64, _I, _VP, _I64, _VP, _VP, _VP, _VP, _VP, _VP,
                                _I64, _VP, _VP, _SZ, _VP]),
+    ("qgemm_bs_split_size", _I, [_I64, _I64, ctypes.POINTER(_SZ), ctypes.POINTER(_SZ),
+                                 ctypes.POINTER(_SZ)]),
+    ("qgemm_bs_split_x", _I, [_VP, _I64, _I64, _VP, _VP, _VP, _VP]),
+    ("qgemm_bs_workspace_size", _I, [_I, _I64, _I64, _I64, ctypes.POINTER(_SZ)]),
+    ("qgemm_bs_run", _I, [_I, _VP, _I64, _I64, _VP, _VP, _VP, _I64, _VP, _I, _VP, _SZ, _VP]),
     ("qgemm_split_k", _I, [_I, _I64, _I64, ctypes.POINTER(_I)]),
     ("qgemm_device_status", _I, [_I]),
     ("qgemm_profile_events", _I, [_VP, _VP]),
@@ -222,6 +227,52 @@ def run(x: torch.Tensor, pw: PackedWeight, y: torch.Tensor | None = None, y_dtyp
     _check(lib().qgemm_run(pw.fmt, _ptr(x), B, K, _ptr(pw.codes), _ptr(pw.scales),
                            _ptr(pw.tensor_scale), pw.N, _ptr(y), ydt, _ptr(workspace),
                            workspace.numel(), _stream(stream)), "qgemm_run")
+    return y
+
+
+def bs_split_size(M: int, K: int) -> tuple[int, int, int]:
+    """qgemm_bs_split_size: (code bytes, scale bytes, exponent bytes) of the split of x."""
+    c, sc, e = _SZ(), _SZ(), _SZ()
+    _check(lib().qgemm_bs_split_size(M, K, ctypes.byref(c), ctypes.byref(sc), ctypes.byref(e)),
+           "qgemm_bs_split_size")
+    return c.value, sc.value, e.value
+
+
+def bs_split_x(x: torch.Tensor, stream=None):
+    """qgemm_bs_split_x: x bf16 [M, K] -> (codes u8, scales u8, x_exp int32) in the layout of
+    include/qgemm.h (three E2M1 terms per row with E8M0 scales per 32 elements)."""
+    assert x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous() and x.dim() == 2
+    M, K = x.shape
+    nc, ns, ne = bs_split_size(M, K)
+    codes = torch.empty(nc, dtype=torch.uint8, device=x.device)
+    scales = torch.empty(ns, dtype=torch.uint8, device=x.device)
+    x_exp = torch.empty(ne // 4, dtype=torch.int32, device=x.device)
+    _check(lib().qgemm_bs_split_x(_ptr(x), M, K, _ptr(codes), _ptr(scales), _ptr(x_exp),
+                                  _stream(stream)), "qgemm_bs_split_x")
+    return codes, scales, x_exp
+
+
+def bs_workspace_size(fmt: int, N: int, K: int, M: int) -> int:
+    n = _SZ()
+    _check(lib().qgemm_bs_workspace_size(fmt, N, K, M, ctypes.byref(n)), "qgemm_bs_workspace_size")
+    return n.value
+
+
+def bs_run(x: torch.Tensor, pw: PackedWeight, y: torch.Tensor | None = None, y_dtype=torch.float32,
+           workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """qgemm_bs_run: the block-scaled path (MXFP4 weights): x bf16 [M, K] -> y [M, N]."""
+    assert x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous() and x.dim() == 2
+    M, K = x.shape
+    assert K == pw.K
+    if y is None:
+        y = torch.empty((M, pw.N), dtype=y_dtype, device=x.device)
+    ydt = Y_BF16 if y.dtype == torch.bfloat16 else Y_F32
+    if workspace is None:
+        nbytes = bs_workspace_size(pw.fmt, pw.N, K, M)
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=x.device)
+    _check(lib().qgemm_bs_run(pw.fmt, _ptr(x), M, K, _ptr(pw.codes), _ptr(pw.scales),
+                              _ptr(pw.tensor_scale), pw.N, _ptr(y), ydt, _ptr(workspace),
+                              workspace.numel(), _stream(stream)), "qgemm_bs_run")
     return y
 
 

@@ -101,6 +101,27 @@ def test_argument_errors(lib):
                                  None, 0, None) == 4                                # up ts table
 
 
+def test_block_scaled_argument_errors(lib):
+    sz = ctypes.c_size_t()
+    # the block-scaled path takes MXFP4 weights only, and checks before any device work
+    for fmt in (0, 1, 3):
+        assert lib.qgemm_bs_workspace_size(fmt, 256, 256, 128, ctypes.byref(sz)) == 1
+        assert lib.qgemm_bs_run(fmt, 16, 4, 64, 16, 16, 16, 8, 16, 0, 16, 1 << 20, None) == 1
+    assert lib.qgemm_bs_workspace_size(2, 256, 48, 128, ctypes.byref(sz)) == 3      # K % 32
+    assert lib.qgemm_bs_workspace_size(2, 256, 256, 0, ctypes.byref(sz)) == 2       # M < 1
+    assert lib.qgemm_bs_run(2, None, 4, 64, 16, 16, None, 8, 16, 0, 16, 1 << 20, None) == 4
+    assert lib.qgemm_bs_run(2, 8, 4, 64, 16, 16, None, 8, 16, 0, 16, 1 << 20, None) == 5
+    assert lib.qgemm_bs_run(2, 16, 4, 64, 16, 16, None, 8, 16, 0, 16, 16, None) == 6  # workspace
+    assert lib.qgemm_bs_split_x(16, 4, 48, 16, 16, 16, None) == 3                    # K % 32
+    assert lib.qgemm_bs_split_x(16, 4, 64, None, 16, 16, None) == 4
+    c, s, e = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    assert lib.qgemm_bs_split_size(300, 320, ctypes.byref(c), ctypes.byref(s), ctypes.byref(e)) == 0
+    # 3 token tiles x 2 chunks x 3 terms of 128 x 128 code bytes and 128 x 8 scale bytes
+    assert (c.value, s.value, e.value) == (3 * 2 * 3 * 16384, 3 * 2 * 3 * 1024, 3 * 128 * 4)
+    assert lib.qgemm_bs_workspace_size(2, 256, 320, 300, ctypes.byref(sz)) == 0
+    assert sz.value == c.value + s.value + e.value
+
+
 def test_no_width_limit_in_sizes(lib):
     # every width has a workspace size; nothing is rejected above 64 (the pages' MAX_BATCH)
     for B in (1, 63, 64, 65, 70, 76, 255, 256, 257, 1000, 8192):

@@ -1,0 +1,136 @@
+"""GPU parity of the block-scaled MXFP4 path (qgemm_bs_split_x / qgemm_bs_run) against the CPU
+oracle, through the C ABI.
+
+Bars:
+  * the split of x is exact: the sum of the three E2M1 terms the GPU writes (decoded on the
+    host from the layout of include/qgemm.h) equals oracle.split_x bit for bit;
+  * the GEMM is the product of that split with the dequantised weights up to fp32
+    accumulation (normalised error 2e-5), and within the method's 1e-3 of the exact product
+    at K >= 1024 (the split's own residual is measured in the oracle pins);
+  * one-hot rows of x reproduce the dequantised weight columns exactly.
+Shapes span several tiles with ragged M, N and K tails, and the 27B prefill shapes on sampled
+rows."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_quantized_weight_qgemm_b200 import inputs
+from block_quantized_weight_qgemm_b200 import qgemm
+from gpu_helpers import TOL, Case, norm_err, x_bits
+
+pytestmark = pytest.mark.gpu
+
+SPLIT_TOL = 2e-5  # fp32 accumulation of exact E2M1 x E2M1 products (K u bounds it by 1.2e-4)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from block_quantized_weight_qgemm_b200 import build
+    build.build()
+    qgemm.lib()
+    qgemm.device_status(reset=True)
+    yield
+    assert qgemm.device_status(reset=True) == qgemm.OK
+
+
+def _decode_split(codes, scales, x_exp, M, K):
+    """Sum of the three terms per element, from the documented layout (numpy only)."""
+    C, Mt = -(-K // 256), -(-M // 128)
+    vals = np.array([oracle.e2m1(c) for c in range(16)])
+    cb = codes.reshape(Mt, C, 3, 128, 8, 16)
+    un = np.empty_like(cb)
+    for r in range(128):
+        for g in range(8):
+            un[:, :, :, r, g, :] = cb[:, :, :, r, g ^ (r & 7), :]
+    un = un.reshape(Mt, C, 3, 128, 128)
+    el = np.stack([un & 15, un >> 4], axis=-1).reshape(Mt, C, 3, 128, 256)
+    sc = scales.reshape(Mt, C, 3, 128, 8).astype(np.float64)
+    val = vals[el] * np.repeat(np.exp2(sc - 127.0), 32, axis=-1)
+    tot = val.sum(axis=2).transpose(0, 2, 1, 3).reshape(Mt * 128, C * 256)
+    return tot, tot[:M, :K] * np.exp2(x_exp[:M].astype(np.float64))[:, None]
+
+
+def _special_rows(x: torch.Tensor) -> torch.Tensor:
+    x = x.clone()
+    M, K = x.shape
+    x[0] = 0.0                                        # all-zero row
+    x[1] = x[1] * 1e-30                                # tiny row (x_exp near -100)
+    x[2, : K // 2] = x[2, : K // 2] * 1e20             # blocks 2^66 apart in one row
+    x[3, 32:64] = 0.0                                  # a zero block
+    x[4, ::7] = -x[4, ::7] * 3.0e4                     # mixed signs and magnitudes
+    if M > 5:
+        x[5, :] = 6.0                                  # exactly representable in one term
+    return x
+
+
+@pytest.mark.parametrize("M,K", [(1, 32), (130, 288), (257, 1024), (200, 5120)])
+def test_split_bit_exact(M, K):
+    x = _special_rows(inputs.activations(M, K, seed=20 + M)) if M > 5 else inputs.activations(M, K, seed=20)
+    codes, scales, x_exp = qgemm.bs_split_x(x.cuda())
+    torch.cuda.synchronize()
+    codes, scales, x_exp = codes.cpu().numpy(), scales.cpu().numpy(), x_exp.cpu().numpy()
+    full, xs_gpu = _decode_split(codes, scales, x_exp, M, K)
+    xs = oracle.split_x(x_bits(x), "e2m1", 3)
+    bad = np.argwhere(xs_gpu != xs)
+    assert bad.size == 0, "split differs at %s: gpu %r oracle %r" % (
+        bad[:4].tolist(), xs_gpu[tuple(bad[0])], xs[tuple(bad[0])])
+    # padding rows and columns hold zeros
+    assert not full[M:].any() and not full[:, K:].any()
+    assert (x_exp[M:] == 0).all()
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 256, 256), (300, 400, 320), (129, 1000, 1056),
+                                   (517, 300, 2048)])
+def test_gemm_is_the_split_product(M, N, K):
+    case = Case("mxfp4", N, K, seed=30 + N)
+    x = _special_rows(inputs.activations(M, K, seed=31 + M))
+    y = qgemm.bs_run(x.cuda(), case.pw)
+    torch.cuda.synchronize()
+    y = y.cpu().numpy().astype(np.float64)
+    xb = x_bits(x)
+    ys = oracle.gemm_f64(oracle.split_x(xb, "e2m1", 3), case.Wd)
+    assert norm_err(y, ys, xb, case.Wd) <= SPLIT_TOL
+    if K >= 1024:
+        assert norm_err(y, oracle.gemm(xb, case.Wd), xb, case.Wd) <= TOL
+
+
+def test_one_hot_rows_give_weight_columns():
+    M, N, K = 256, 512, 768
+    case = Case("mxfp4", N, K, seed=41)
+    ks = (np.arange(M) * 37 + 3) % K
+    x = torch.zeros(M, K, dtype=torch.bfloat16)
+    x[np.arange(M), ks] = 1.0
+    x[7, ks[7]] = -0.375  # exactly one E2M1 term: -1.5 * 2^-2
+    y = qgemm.bs_run(x.cuda(), case.pw).cpu().numpy().astype(np.float64)
+    exp = case.Wd[:, ks].T.copy()
+    exp[7] *= -0.375
+    assert np.array_equal(y, exp)
+
+
+def test_bf16_output_and_workspace_reuse():
+    M, N, K = 300, 640, 1024
+    case = Case("mxfp4", N, K, seed=43)
+    x = inputs.activations(M, K, seed=44).cuda()
+    ws = torch.empty(qgemm.bs_workspace_size(qgemm._fmt("mxfp4"), N, K, M), dtype=torch.uint8,
+                     device="cuda")
+    y32 = qgemm.bs_run(x, case.pw, workspace=ws)
+    y16 = qgemm.bs_run(x, case.pw, y_dtype=torch.bfloat16, workspace=ws)
+    y32b = qgemm.bs_run(x, case.pw, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y32, y32b)  # deterministic
+    assert torch.equal(y16, y32.to(torch.bfloat16))
+
+
+@pytest.mark.parametrize("N,K,M", [(17408, 5120, 2048), (5120, 17408, 2048)])
+def test_27b_prefill_sampled_rows(N, K, M):
+    case = Case("mxfp4", N, K, seed=inputs.W_SEED if N == 17408 else inputs.W3_SEED)
+    x = inputs.activations(M, K, seed=50)
+    y = qgemm.bs_run(x.cuda(), case.pw)
+    torch.cuda.synchronize()
+    rows = np.array([0, 1, 127, 128, 1000, M - 1])
+    y = y[rows].cpu().numpy().astype(np.float64)
+    xb = x_bits(x)[rows]
+    ys = oracle.gemm_f64(oracle.split_x(xb, "e2m1", 3), case.Wd)
+    assert norm_err(y, ys, xb, case.Wd) <= SPLIT_TOL
+    assert norm_err(y, oracle.gemm(xb, case.Wd), xb, case.Wd) <= TOL
