@@ -331,6 +331,24 @@ def run_configs(dev, stream, q8_rings, hbm_peak, tf_peak):
                      "us": round(us, 1), "TFLOPs": round(tf, 1), "frac_tensor": round(tf / tf_peak, 4)})
         del x, y, ws
 
+    def prefill_bs(name, pw, M, reps=3):
+        # the block-scaled path (MXFP4 weights on kind::mxf4nvf4, x split into three E2M1
+        # terms): split + GEMM per call
+        N, K = pw.N, pw.K
+        x = inputs.activations(M, K, seed=1).to(dev)
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(qgemm.bs_workspace_size(qgemm._fmt("mxfp4"), N, K, M), dtype=torch.uint8,
+                         device=dev)
+        us = graph_us(lambda i: qgemm.bs_run(x, pw, y=y, workspace=ws, stream=stream), reps, stream)
+        tf = 2.0 * M * N * K / (us * 1e-6) / 1e12
+        # the MMAs run 3 x 2MNK of FP4 work; their own peak is the bf16 peak x 4 (the nominal
+        # dense FP4 : bf16 ratio, 9 : 2.25 PFLOP/s)
+        recs.append({"config": name, "kind": "prefill", "fmt": "mxfp4", "path": "block-scaled",
+                     "N": N, "K": K, "M": M, "us": round(us, 1), "TFLOPs": round(tf, 1),
+                     "frac_tensor": round(tf / tf_peak, 4),
+                     "fp4_mma_frac": round(3.0 * tf / (4.0 * tf_peak), 4)})
+        del x, y, ws
+
     def prefill_ffn(name, fmt, pg, pu, pd, M, reps=3):
         N, K = pg.N, pg.K
         x = inputs.activations(M, K, seed=1).to(dev)
@@ -440,6 +458,7 @@ def run_configs(dev, stream, q8_rings, hbm_peak, tf_peak):
         decode("mxfp4 27B serving mix", "mxfp4", ring, 32)
         del ring
         prefill("mxfp4 27B serving mix prefill", "mxfp4", mx, 8192, reps=3)
+        prefill_bs("mxfp4 27B serving mix prefill, block-scaled path", mx, 8192)
         del mx
         torch.cuda.empty_cache()
     return recs
