@@ -51,12 +51,13 @@ __device__ __forceinline__ uint4 to_f16x8(const uint4& v, float sc1, float sc2) 
 }
 
 __global__ void __launch_bounds__(kPrepThreads) qgemm_prep_x_kernel(const PrepParams p) {
+  // The GEMM that follows may start its set-up and weight streaming now; it waits for this
+  // grid before it reads xh or x_exp.  Its weight reads are not ordered after the grid before
+  // this one: weights must come from a grid that has completed, or that does not let its
+  // dependents launch early (the library's packers do not).
+  griddep_launch_dependents();
   // x may come from the grid before this one, which may also still read xh and x_exp
   griddep_wait();
-  // The GEMM that follows may start its set-up and weight streaming now; it waits for this
-  // grid before it reads xh or x_exp.  Not earlier: it reads the weights before that wait,
-  // and the grid before this one may have written them.
-  griddep_launch_dependents();
   const int b = blockIdx.x;
   const uint16_t* xr = p.x + (size_t)b * p.K;
   __shared__ float red[kPrepThreads / 32];

@@ -54,6 +54,12 @@
  *     the operand's address and geometry; they hold no device memory).
  *   - qgemm_run and qgemm_ffn_gate_up calls that may overlap on the device need their own
  *     workspaces; qgemm_run_noalloc calls share one scratch and must not overlap.
+ *   - The GEMM kernels are programmatic dependents of the small x-preparation kernel
+ *     launched just before them and start streaming weights before they wait for it.  x
+ *     (and every buffer a call writes) is ordered after all earlier work on the stream; the
+ *     packed weights are read assuming the kernel that wrote them has completed, which holds
+ *     for every kernel that does not trigger its dependents' launch early (this library's
+ *     packers, and any kernel launched without programmatic dependent launch).
  */
 #ifndef QGEMM_H
 #define QGEMM_H
