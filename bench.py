@@ -306,6 +306,21 @@ def run_configs(dev, stream, q8_rings, hbm_peak, tf_peak):
             r["note"] = note
         recs.append(r)
 
+    def decode_bs(name, ring, B, reps=40):
+        # the block-scaled path at a decode width (MXFP4 weights as the MMA M operand)
+        N, K = ring[0].N, ring[0].K
+        x = inputs.activations(B, K, seed=1).to(dev)
+        y = torch.empty(B, N, device=dev)
+        ws = torch.empty(max(qgemm.bs_workspace_size(qgemm._fmt("mxfp4"), N, K, B), 16),
+                         dtype=torch.uint8, device=dev)
+        us = graph_us(lambda i: qgemm.bs_run(x, ring[i % len(ring)], y=y, workspace=ws, stream=stream),
+                      reps, stream)
+        gbs = weight_bytes("mxfp4", N, K) / (us * 1e-6) / 1e9
+        recs.append({"config": name, "kind": "decode", "fmt": "mxfp4", "path": "block-scaled",
+                     "N": N, "K": K, "B": B, "us": round(us, 2), "weight_GBps": round(gbs, 1),
+                     "frac_hbm": round(gbs / hbm_peak, 4)})
+        del x, y, ws
+
     def decode_ffn(name, fmt, gring, uring, B, reps=40):
         N, K = gring[0].N, gring[0].K
         x = inputs.activations(B, K, seed=1).to(dev)
@@ -456,6 +471,7 @@ def run_configs(dev, stream, q8_rings, hbm_peak, tf_peak):
         mx = packed("mxfp4", N, K, seed)
         ring = clone_ring(mx, RING)
         decode("mxfp4 27B serving mix", "mxfp4", ring, 32)
+        decode_bs("mxfp4 27B serving mix, block-scaled path", ring, 32)
         del ring
         prefill("mxfp4 27B serving mix prefill", "mxfp4", mx, 8192, reps=3)
         prefill_bs("mxfp4 27B serving mix prefill, block-scaled path", mx, 8192)

@@ -19,7 +19,11 @@ cudaError_t launch_bs_split(const uint16_t* x, int M, int K, uint8_t* codes, uin
 cudaError_t launch_bs_gemm(int M, int N, int K, const uint8_t* xcodes, const uint8_t* xscales,
                            const int* x_exp, const uint8_t* wcodes, const uint8_t* wscales,
                            void* out, int out_bf16, int* dev_err, cudaStream_t stream);
-size_t bs_workspace_bytes(int64_t M, int64_t K, size_t* off_scales, size_t* off_exp);
+size_t bs_workspace_bytes(int64_t M, int64_t N, int64_t K, size_t* off_scales, size_t* off_exp,
+                          size_t* off_part);
+cudaError_t launch_bs_dec(int M, int N, int K, const uint8_t* xcodes, const uint8_t* xscales,
+                          const int* x_exp, const uint8_t* wcodes, const uint8_t* wscales,
+                          float* part, void* out, int out_bf16, int* dev_err, cudaStream_t stream);
 cudaError_t launch_pair(int fmt, bool bf16op, const GemmParams& p, size_t smem_bytes, int units,
                         const CUtensorMap* maps, bool pdl, cudaStream_t stream);
 cudaError_t launch_pack(int fmt, const float* W, int64_t N, int64_t K, void* codes, void* scales,
@@ -891,11 +895,12 @@ int qgemm_bs_split_size(int64_t M, int64_t K, size_t* code_bytes, size_t* scale_
   if (M < 1 || K < 1 || M > 0x7FFFFFFF || K > 0x7FFFFFFF) return QGEMM_ERR_SHAPE;
   if (K % 32 != 0) return QGEMM_ERR_K_BLOCK;
   if (!code_bytes || !scale_bytes || !exp_bytes) return QGEMM_ERR_NULL;
-  size_t off_s = 0, off_e = 0;
-  const size_t total = bs_workspace_bytes(M, K, &off_s, &off_e);
+  size_t off_s = 0, off_e = 0, off_p = 0;
+  (void)bs_workspace_bytes(M, 0, K, &off_s, &off_e, &off_p);
+  const int64_t Mt = (M + 127) / 128;
   *code_bytes = off_s;
   *scale_bytes = off_e - off_s;
-  *exp_bytes = total - off_e;
+  *exp_bytes = (size_t)Mt * 128 * 4;
   return QGEMM_OK;
 }
 
@@ -919,7 +924,7 @@ int qgemm_bs_workspace_size(int fmt, int64_t N, int64_t K, int64_t M, size_t* by
   if (st != QGEMM_OK) return st;
   if (M < 1 || M > 0x7FFFFFFF) return QGEMM_ERR_SHAPE;
   if (!bytes) return QGEMM_ERR_NULL;
-  *bytes = bs_workspace_bytes(M, K, nullptr, nullptr);
+  *bytes = bs_workspace_bytes(M, N, K, nullptr, nullptr, nullptr);
   return QGEMM_OK;
 }
 
@@ -934,8 +939,8 @@ int qgemm_bs_run(int fmt, const void* x, int64_t M, int64_t K, const void* codes
   if (!x || !y || !weights_given(fmt, codes, scales, tensor_scale)) return QGEMM_ERR_NULL;
   if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || !aligned16(y))
     return QGEMM_ERR_ALIGN;
-  size_t off_s = 0, off_e = 0;
-  const size_t need = bs_workspace_bytes(M, K, &off_s, &off_e);
+  size_t off_s = 0, off_e = 0, off_p = 0;
+  const size_t need = bs_workspace_bytes(M, N, K, &off_s, &off_e, &off_p);
   if (!workspace || workspace_bytes < need) return QGEMM_ERR_WORKSPACE;
   if (!aligned16(workspace)) return QGEMM_ERR_ALIGN;
   if (!device_ok()) return QGEMM_ERR_DEVICE;
@@ -947,9 +952,15 @@ int qgemm_bs_run(int fmt, const void* x, int64_t M, int64_t K, const void* codes
                                   reinterpret_cast<int*>(wsb + off_e), s);
   if (e != cudaSuccess) return cuda_fail(e, "split kernel launch");
   if (g_prof_begin) cudaEventRecord(g_prof_begin, s);
-  e = launch_bs_gemm((int)M, (int)N, (int)K, wsb, wsb + off_s, reinterpret_cast<const int*>(wsb + off_e),
-                     static_cast<const uint8_t*>(codes), static_cast<const uint8_t*>(scales), y,
-                     y_dtype == QGEMM_Y_BF16, dev_err, s);
+  // up to 128 rows the weights are the MMA M operand (decode tiling), above that x is
+  if (M <= 128)
+    e = launch_bs_dec((int)M, (int)N, (int)K, wsb, wsb + off_s, reinterpret_cast<const int*>(wsb + off_e),
+                      static_cast<const uint8_t*>(codes), static_cast<const uint8_t*>(scales),
+                      reinterpret_cast<float*>(wsb + off_p), y, y_dtype == QGEMM_Y_BF16, dev_err, s);
+  else
+    e = launch_bs_gemm((int)M, (int)N, (int)K, wsb, wsb + off_s, reinterpret_cast<const int*>(wsb + off_e),
+                       static_cast<const uint8_t*>(codes), static_cast<const uint8_t*>(scales), y,
+                       y_dtype == QGEMM_Y_BF16, dev_err, s);
   if (e != cudaSuccess) return cuda_fail(e, "block-scaled gemm launch");
   if (g_prof_end) cudaEventRecord(g_prof_end, s);
   return QGEMM_OK;

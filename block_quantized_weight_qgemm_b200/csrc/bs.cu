@@ -36,6 +36,7 @@
 #include <cuda_fp16.h>
 #include <cuda_fp4.h>
 
+#include <algorithm>
 #include <atomic>
 
 #include "common.cuh"
@@ -272,6 +273,18 @@ __device__ __forceinline__ void bs_tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) 
         "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]),
         "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]),
         "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr)
+      : "memory");
+}
+
+// Each lane reads 16 consecutive 32-bit columns of its own TMEM lane.
+__device__ __forceinline__ void bs_tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15}, [%16];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+        "=r"(v[14]), "=r"(v[15])
       : "r"(taddr)
       : "memory");
 }
@@ -547,6 +560,273 @@ __global__ void __launch_bounds__(kBsThreads, 1) qgemm_bs_kernel(const __grid_co
 }
 
 // ---------------------------------------------------------------------------------------
+// Decode widths (M <= 128): the roles of the operands swap.  The weights are the MMA M
+// operand (one 128-row weight tile per unit, its scales SFA), the split x the N operand
+// (N = M rounded up to 16 rows of the first token tile, its scales SFB), and K is split
+// over S ranges so that the units fill the SMs; S > 1 writes fp32 partials that the split-K
+// reduce kernel sums in the order s = 0..S-1.  Per 256-K chunk: 4 K-blocks x 3 terms of
+// M128 N(M) K64 MMAs.  Stage: [weight codes 16 KB][3 x N x 128 term codes][weight scales
+// 1 KB][3 x N x 8 term scales], rounded up to 1 KB.  TMEM: the accumulator (N columns), then
+// per stage 64 columns of scale factors: the weights' K-block kb at 4 kb (4 row groups), term
+// j's K-block kb at 16 + 4 (4 j + kb).
+// ---------------------------------------------------------------------------------------
+constexpr int kBdMaxStages = 6;
+constexpr int kBdSfCols = 16 + kBsTerms * 16;  // 64
+
+struct BsDecParams {
+  int M, N, K, C, Nb, S, units, stages, stage_bytes;
+  const uint8_t* xcodes;
+  const uint8_t* xscales;
+  const int* x_exp;
+  const uint8_t* wcodes;
+  const uint8_t* wscales;
+  float* ws;  // S > 1: partials [S][M][N], fully scaled
+  void* out;
+  int out_bf16;
+  int* dev_err;
+};
+
+__global__ void __launch_bounds__(kBsThreads, 1) qgemm_bs_dec_kernel(const __grid_constant__ BsDecParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const uint32_t sbase = smem_u32(smem);
+  const int NST = p.stages;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + NST * p.stage_bytes);
+  const uint32_t bar_full = smem_u32(bars);
+  const uint32_t bar_empty = bar_full + 8 * NST;
+  const uint32_t bar_sf = bar_empty + 8 * NST;
+  const uint32_t bar_acc = bar_sf + 8 * NST;
+  const uint32_t bar_acc_free = bar_acc + 8;
+  const uint32_t bar_drain = bar_acc_free + 8;
+  int* ctl = reinterpret_cast<int*>(bars + 3 * NST + 3);
+  volatile int* abort_flag = ctl + 1;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int Nb = p.Nb;
+  const uint32_t xterm = (uint32_t)Nb * 128u;      // one term's codes in a stage
+  const uint32_t off_ws = kBsBlock + kBsTerms * xterm;            // weight scales
+  const uint32_t off_xs = off_ws + kBsSBlock;                     // term scales
+  const uint32_t idesc = (1u << 7) | (1u << 10) | ((uint32_t)(Nb >> 3) << 17) | (1u << 23) |
+                         ((uint32_t)(kBsM >> 4) << 24);
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, 1);
+      mbar_init(bar_sf + 8 * s, 4);
+    }
+    mbar_init(bar_acc, 1);
+    mbar_init(bar_acc_free, 4);
+    mbar_init(bar_drain, 1);
+    ctl[1] = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    bs_tmem_alloc(smem_u32(ctl), kBsTmemCols);
+    bs_tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = static_cast<uint32_t>(ctl[0]);
+  const int64_t n_row_tiles = row_tiles(p.N);
+  auto unit_range = [&](int u, int& t, int& s, int& c0, int& c1) {
+    t = u % (int)n_row_tiles;
+    s = u / (int)n_row_tiles;
+    c0 = (int)((int64_t)s * p.C / p.S);
+    c1 = (int)((int64_t)(s + 1) * p.C / p.S);
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_x = policy_evict_last();
+      RingPos sp;
+      int issued = 0;
+      bool ok = true, waited = false;
+      for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+        int t, s, c0, c1;
+        unit_range(u, t, s, c0, c1);
+        for (int c = c0; c < c1; ++c) {
+          if (issued >= NST &&
+              !mbar_wait(bar_empty + 8 * sp.slot, sp.phase ^ 1u, abort_flag, p.dev_err, kErrTimeout)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = bar_full + 8 * sp.slot;
+          const uint32_t st = sbase + (uint32_t)(sp.slot * p.stage_bytes);
+          mbar_arrive_expect_tx(fb, kBsBlock + kBsSBlock + kBsTerms * (xterm + (uint32_t)Nb * 8u));
+          const int64_t blk = (int64_t)t * p.C + c;
+          bulk_load(st, p.wcodes + blk * kBsBlock, kBsBlock, fb, pol_w);
+          bulk_load(st + off_ws, p.wscales + blk * kBsSBlock, kBsSBlock, fb, pol_w);
+          if (!waited) {
+            griddep_wait();  // the split x comes from the preceding grid
+            waited = true;
+          }
+          for (int j = 0; j < kBsTerms; ++j) {
+            const int64_t xb = (int64_t)c * kBsTerms + j;  // token tile 0
+            bulk_load(st + kBsBlock + (uint32_t)j * xterm, p.xcodes + xb * kBsBlock, xterm, fb, pol_x);
+            bulk_load(st + off_xs + (uint32_t)(j * Nb * 8), p.xscales + xb * kBsSBlock, (uint32_t)Nb * 8u, fb, pol_x);
+          }
+          sp.next(NST);
+          ++issued;
+        }
+      }
+      if (!ok) {
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 200000) __nanosleep(1000);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      RingPos sp;
+      bool ok = true;
+      int ti = 0;
+      for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x, ++ti) {
+        int t, s, c0, c1;
+        unit_range(u, t, s, c0, c1);
+        if (ti > 0) {
+          if (!mbar_wait_spin(bar_acc_free, (uint32_t)(ti - 1) & 1u, false, abort_flag, p.dev_err,
+                              kErrTimeout)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
+        for (int c = c0; c < c1; ++c) {
+          if (!mbar_wait_spin(bar_full + 8 * sp.slot, sp.phase, false, abort_flag, p.dev_err, kErrTimeout) ||
+              !mbar_wait_spin(bar_sf + 8 * sp.slot, sp.phase, false, abort_flag, p.dev_err, kErrTimeout)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t st = sbase + (uint32_t)(sp.slot * p.stage_bytes);
+          const uint64_t adesc0 = smem_desc_sw128(st);
+          const uint32_t sf0 = tmem + (uint32_t)(Nb + sp.slot * kBdSfCols);
+#pragma unroll
+          for (int kb = 0; kb < kBsK / 64; ++kb) {
+#pragma unroll
+            for (int j = 0; j < kBsTerms; ++j) {
+              const uint64_t bdesc = smem_desc_sw128(st + kBsBlock + (uint32_t)j * xterm) + (uint64_t)(kb * 2);
+              bs_mma(tmem, adesc0 + (uint64_t)(kb * 2), bdesc, idesc, sf0 + (uint32_t)(kb * 4),
+                     sf0 + (uint32_t)(16 + (j * 4 + kb) * 4), (c != c0 || kb || j) ? 1u : 0u);
+            }
+          }
+          bs_commit(bar_empty + 8 * sp.slot);
+          sp.next(NST);
+        }
+        if (!ok) break;
+        bs_commit(bar_acc);
+      }
+      bs_commit(bar_drain);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(bar_drain, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+      }
+    }
+    __syncwarp();
+  } else if (warp < kBsEpiWarp0) {
+    // ------------------------------------------------------------ scale-factor staging
+    const int q = warp & 3;
+    const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+    RingPos sp;
+    int used = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+      int t, s, c0, c1;
+      unit_range(u, t, s, c0, c1);
+      for (int c = c0; c < c1; ++c) {
+        if (used >= NST) {
+          ok = mbar_wait(bar_empty + 8 * sp.slot, sp.phase ^ 1u, abort_flag, p.dev_err, kErrTimeout);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+        }
+        ok = mbar_wait(bar_full + 8 * sp.slot, sp.phase, abort_flag, p.dev_err, kErrTimeout);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        const uint8_t* st = smem + sp.slot * p.stage_bytes;
+        uint32_t v[kBdSfCols];
+#pragma unroll
+        for (int r1 = 0; r1 < 4; ++r1) {
+          const uint2 s8 = *reinterpret_cast<const uint2*>(st + off_ws + (r1 * 32 + lane) * 8);
+#pragma unroll
+          for (int kb = 0; kb < 4; ++kb) v[kb * 4 + r1] = (((kb < 2) ? s8.x : s8.y) >> ((kb & 1) * 16)) & 0xFFFFu;
+        }
+#pragma unroll
+        for (int j = 0; j < kBsTerms; ++j)
+#pragma unroll
+          for (int r1 = 0; r1 < 4; ++r1) {
+            const int row = r1 * 32 + lane;
+            uint2 s8 = make_uint2(0u, 0u);
+            if (row < Nb) s8 = *reinterpret_cast<const uint2*>(st + off_xs + j * Nb * 8 + row * 8);
+#pragma unroll
+            for (int kb = 0; kb < 4; ++kb)
+              v[16 + (j * 4 + kb) * 4 + r1] = (((kb < 2) ? s8.x : s8.y) >> ((kb & 1) * 16)) & 0xFFFFu;
+          }
+        const uint32_t ta = tmem + lane_base + (uint32_t)(Nb + sp.slot * kBdSfCols);
+#pragma unroll
+        for (int i = 0; i < kBdSfCols / 16; ++i)
+          bs_tmem_st16(ta + (uint32_t)(16 * i), *reinterpret_cast<const uint32_t(*)[16]>(&v[16 * i]));
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_sf + 8 * sp.slot);
+        sp.next(NST);
+        ++used;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    // lane = weight row n of the tile; columns = tokens b (scaled by 2^x_exp[b])
+    const int q = warp & 3;
+    const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+    griddep_wait();  // x_exp comes from the split kernel
+    const size_t MN = (size_t)p.M * p.N;
+    int ti = 0;
+    for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++ti) {
+      int t, s, c0, c1;
+      unit_range(u, t, s, c0, c1);
+      const int64_t n64 = (int64_t)t * kBsM + q * 32 + lane;
+      bool ok = mbar_wait(bar_acc, (uint32_t)ti & 1u, abort_flag, p.dev_err, kErrTimeout);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll 1
+      for (int cb = 0; cb < Nb; cb += 16) {
+        uint32_t v[16];
+        bs_tmem_ld16(tmem + lane_base + (uint32_t)cb, v);
+        tmem_ld_wait();
+        if (n64 < p.N) {
+          const int n = (int)n64;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int b = cb + i;
+            if (b < p.M) {
+              const float val = bs_scale_pow2(__uint_as_float(v[i]), __ldg(p.x_exp + b));
+              if (p.S > 1) p.ws[(size_t)s * MN + (size_t)b * p.N + n] = val;
+              else if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)b * p.N + n] = __float2bfloat16_rn(val);
+              else reinterpret_cast<float*>(p.out)[(size_t)b * p.N + n] = val;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_acc_free);
+    }
+    griddep_launch_dependents();  // the split-K reduce may launch
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    bs_tmem_dealloc(tmem, kBsTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------------------
 // Launchers
 // ---------------------------------------------------------------------------------------
 cudaError_t launch_bs_split(const uint16_t* x, int M, int K, uint8_t* codes, uint8_t* scales,
@@ -625,14 +905,104 @@ cudaError_t launch_bs_gemm(int M, int N, int K, const uint8_t* xcodes, const uin
   return cudaLaunchKernelEx(&cfg, qgemm_bs_kernel, p);
 }
 
-// workspace of the block-scaled path: split codes, split scales, row exponents
-size_t bs_workspace_bytes(int64_t M, int64_t K, size_t* off_scales, size_t* off_exp) {
+// K split of the decode kernel: a function of (N, K) only (the unit count is weighed against
+// the 148 SMs of a B200), the smallest S of least cost (waves of units x (chunks per unit + a
+// fixed cost of ~3 chunks) + a small charge per split for the partials).
+constexpr int kBsSplitSMs = 148;
+int bs_dec_split(int64_t N, int64_t K, int sms) {
+  const int64_t T = row_tiles(N), C = (K + kBsK - 1) / kBsK;
+  int best = 1;
+  double best_cost = 0.0;
+  for (int64_t S = 1; S <= std::min<int64_t>(16, C); ++S) {
+    const int64_t waves = (T * S + sms - 1) / sms;
+    const double cost = double(waves * ((C + S - 1) / S + 3)) + 0.25 * double(S);
+    if (S == 1 || cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best = (int)S;
+    }
+  }
+  return best;
+}
+
+// Workspace of the block-scaled path: split codes, split scales, row exponents and, for
+// decode widths with a K split, the fp32 partials.
+size_t bs_workspace_bytes(int64_t M, int64_t N, int64_t K, size_t* off_scales, size_t* off_exp,
+                          size_t* off_part) {
   const int64_t C = (K + kBsK - 1) / kBsK, Mt = (M + kBsM - 1) / kBsM;
   const size_t codes = (size_t)(Mt * C * kBsTerms) * kBsBlock;
   const size_t scales = (size_t)(Mt * C * kBsTerms) * kBsSBlock;
   if (off_scales) *off_scales = codes;
   if (off_exp) *off_exp = codes + scales;
-  return codes + scales + (size_t)Mt * kBsM * 4;
+  size_t total = codes + scales + (size_t)Mt * kBsM * 4;
+  total = (total + 255) / 256 * 256;
+  if (off_part) *off_part = total;
+  if (M <= kBsM && N > 0) {
+    const int S = bs_dec_split(N, K, kBsSplitSMs);
+    if (S > 1) total += (size_t)S * (size_t)M * (size_t)N * 4;
+  }
+  return total;
+}
+
+cudaError_t launch_reduce(const ReduceParams& rp, cudaStream_t stream);
+
+// Decode widths: returns cudaSuccess after queuing the GEMM (and the reduce when S > 1).
+cudaError_t launch_bs_dec(int M, int N, int K, const uint8_t* xcodes, const uint8_t* xscales,
+                          const int* x_exp, const uint8_t* wcodes, const uint8_t* wscales,
+                          float* part, void* out, int out_bf16, int* dev_err, cudaStream_t stream) {
+  static std::atomic<uint64_t> set_mask{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+  if (bit == 0 || !(set_mask.load(std::memory_order_acquire) & bit)) {
+    e = cudaFuncSetAttribute(qgemm_bs_dec_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
+    if (e != cudaSuccess) return e;
+    set_mask.fetch_or(bit, std::memory_order_release);
+  }
+  BsDecParams p{};
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.C = (K + kBsK - 1) / kBsK;
+  p.Nb = (M + 15) / 16 * 16;
+  const int sms = bs_sm_count(dev);
+  p.S = bs_dec_split(N, K, kBsSplitSMs);
+  p.units = (int)row_tiles(N) * p.S;
+  p.stage_bytes = (kBsBlock + kBsTerms * p.Nb * 128 + kBsSBlock + kBsTerms * p.Nb * 8 + 1023) / 1024 * 1024;
+  p.stages = std::min({kBdMaxStages, (kSmemLimit - 1024 - 256) / p.stage_bytes,
+                       (kBsTmemCols - p.Nb) / kBdSfCols});
+  if (p.stages < 2) return cudaErrorInvalidValue;
+  p.xcodes = xcodes;
+  p.xscales = xscales;
+  p.x_exp = x_exp;
+  p.wcodes = wcodes;
+  p.wscales = wscales;
+  p.ws = part;
+  p.out = out;
+  p.out_bf16 = out_bf16;
+  p.dev_err = dev_err;
+  const size_t smem = 1024 + (size_t)p.stages * p.stage_bytes + 256;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)std::min(p.units, sms), 1, 1);
+  cfg.blockDim = dim3(kBsThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, qgemm_bs_dec_kernel, p);
+  if (e != cudaSuccess || p.S == 1) return e;
+  ReduceParams rp{};
+  rp.ws = part;
+  rp.S = p.S;
+  rp.NMAT = 1;
+  rp.B = M;
+  rp.N = N;
+  rp.out = out;
+  rp.out_bf16 = out_bf16;
+  return launch_reduce(rp, stream);
 }
 
 }  // namespace qg

@@ -8,8 +8,9 @@ Bars:
     accumulation (normalised error 2e-5), and within the method's 1e-3 of the exact product
     at K >= 1024 (the split's own residual is measured in the oracle pins);
   * one-hot rows of x reproduce the dequantised weight columns exactly.
-Shapes span several tiles with ragged M, N and K tails, and the 27B prefill shapes on sampled
-rows."""
+Shapes span several tiles with ragged M, N and K tails, both tilings (up to 128 rows the
+weights are the MMA M operand and K is split over the SMs; above, x is), and the 27B shapes at
+prefill and decode widths on sampled rows."""
 import numpy as np
 import pytest
 import torch
@@ -52,21 +53,23 @@ def _decode_split(codes, scales, x_exp, M, K):
 
 
 def _special_rows(x: torch.Tensor) -> torch.Tensor:
+    """Rows 0..5 (as far as x has them) replaced by edge cases; a one-row x keeps its row."""
     x = x.clone()
     M, K = x.shape
+    if M < 6:
+        return x
     x[0] = 0.0                                        # all-zero row
     x[1] = x[1] * 1e-30                                # tiny row (x_exp near -100)
     x[2, : K // 2] = x[2, : K // 2] * 1e20             # blocks 2^66 apart in one row
     x[3, 32:64] = 0.0                                  # a zero block
     x[4, ::7] = -x[4, ::7] * 3.0e4                     # mixed signs and magnitudes
-    if M > 5:
-        x[5, :] = 6.0                                  # exactly representable in one term
+    x[5, :] = 6.0                                      # exactly representable in one term
     return x
 
 
 @pytest.mark.parametrize("M,K", [(1, 32), (130, 288), (257, 1024), (200, 5120)])
 def test_split_bit_exact(M, K):
-    x = _special_rows(inputs.activations(M, K, seed=20 + M)) if M > 5 else inputs.activations(M, K, seed=20)
+    x = _special_rows(inputs.activations(M, K, seed=20 + M))
     codes, scales, x_exp = qgemm.bs_split_x(x.cuda())
     torch.cuda.synchronize()
     codes, scales, x_exp = codes.cpu().numpy(), scales.cpu().numpy(), x_exp.cpu().numpy()
@@ -80,8 +83,9 @@ def test_split_bit_exact(M, K):
     assert (x_exp[M:] == 0).all()
 
 
-@pytest.mark.parametrize("M,N,K", [(128, 256, 256), (300, 400, 320), (129, 1000, 1056),
-                                   (517, 300, 2048)])
+@pytest.mark.parametrize("M,N,K", [(1, 300, 512), (16, 256, 256), (33, 1000, 1056),
+                                   (128, 640, 4096), (128, 256, 256), (300, 400, 320),
+                                   (129, 1000, 1056), (517, 300, 2048)])
 def test_gemm_is_the_split_product(M, N, K):
     case = Case("mxfp4", N, K, seed=30 + N)
     x = _special_rows(inputs.activations(M, K, seed=31 + M))
@@ -108,8 +112,9 @@ def test_one_hot_rows_give_weight_columns():
     assert np.array_equal(y, exp)
 
 
-def test_bf16_output_and_workspace_reuse():
-    M, N, K = 300, 640, 1024
+@pytest.mark.parametrize("M", [300, 40])
+def test_bf16_output_and_workspace_reuse(M):
+    N, K = 640, 1024
     case = Case("mxfp4", N, K, seed=43)
     x = inputs.activations(M, K, seed=44).cuda()
     ws = torch.empty(qgemm.bs_workspace_size(qgemm._fmt("mxfp4"), N, K, M), dtype=torch.uint8,
@@ -122,13 +127,14 @@ def test_bf16_output_and_workspace_reuse():
     assert torch.equal(y16, y32.to(torch.bfloat16))
 
 
-@pytest.mark.parametrize("N,K,M", [(17408, 5120, 2048), (5120, 17408, 2048)])
+@pytest.mark.parametrize("N,K,M", [(17408, 5120, 2048), (5120, 17408, 2048), (17408, 5120, 32),
+                                   (5120, 17408, 32)])
 def test_27b_prefill_sampled_rows(N, K, M):
     case = Case("mxfp4", N, K, seed=inputs.W_SEED if N == 17408 else inputs.W3_SEED)
     x = inputs.activations(M, K, seed=50)
     y = qgemm.bs_run(x.cuda(), case.pw)
     torch.cuda.synchronize()
-    rows = np.array([0, 1, 127, 128, 1000, M - 1])
+    rows = np.array([0, 1, 127, 128, 1000, M - 1]) if M > 1000 else np.array([0, 1, 17, M - 1])
     y = y[rows].cpu().numpy().astype(np.float64)
     xb = x_bits(x)[rows]
     ys = oracle.gemm_f64(oracle.split_x(xb, "e2m1", 3), case.Wd)
