@@ -565,13 +565,18 @@ __global__ void __launch_bounds__(kBsThreads, 1) qgemm_bs_kernel(const __grid_co
 // (N = M rounded up to 16 rows of the first token tile, its scales SFB), and K is split
 // over S ranges so that the units fill the SMs; S > 1 writes fp32 partials that the split-K
 // reduce kernel sums in the order s = 0..S-1.  Per 256-K chunk: 4 K-blocks x 3 terms of
-// M128 N(M) K64 MMAs.  Stage: [weight codes 16 KB][3 x N x 128 term codes][weight scales
-// 1 KB][3 x N x 8 term scales], rounded up to 1 KB.  TMEM: the accumulator (N columns), then
-// per stage 64 columns of scale factors: the weights' K-block kb at 4 kb (4 row groups), term
-// j's K-block kb at 16 + 4 (4 j + kb).
+// M128 N(M) K64 MMAs.  At these widths the issuing thread bounds the MMA stream, so two
+// issuers take alternate chunks of a unit, each into its own accumulator; the epilogue adds
+// them in the order even + odd.  Stage: [weight codes 16 KB][3 x N x 128 term codes][weight
+// scales 1 KB][3 x N x 8 term scales], rounded up to 1 KB; an even number of stages, so that a
+// stage's previous use belongs to the same issuer.  TMEM: the two accumulators (N columns
+// each), then per stage 64 columns of scale factors: the weights' K-block kb at 4 kb (4 row
+// groups), term j's K-block kb at 16 + 4 (4 j + kb).
 // ---------------------------------------------------------------------------------------
 constexpr int kBdMaxStages = 6;
 constexpr int kBdSfCols = 16 + kBsTerms * 16;  // 64
+constexpr int kBdIssuer2Warp = 10;
+constexpr int kBdThreads = 11 * 32;
 
 struct BsDecParams {
   int M, N, K, C, Nb, S, units, stages, stage_bytes;
@@ -586,7 +591,7 @@ struct BsDecParams {
   int* dev_err;
 };
 
-__global__ void __launch_bounds__(kBsThreads, 1) qgemm_bs_dec_kernel(const __grid_constant__ BsDecParams p) {
+__global__ void __launch_bounds__(kBdThreads, 1) qgemm_bs_dec_kernel(const __grid_constant__ BsDecParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sbase = smem_u32(smem);
@@ -598,7 +603,7 @@ __global__ void __launch_bounds__(kBsThreads, 1) qgemm_bs_dec_kernel(const __gri
   const uint32_t bar_acc = bar_sf + 8 * NST;
   const uint32_t bar_acc_free = bar_acc + 8;
   const uint32_t bar_drain = bar_acc_free + 8;
-  int* ctl = reinterpret_cast<int*>(bars + 3 * NST + 3);
+  int* ctl = reinterpret_cast<int*>(bars + 3 * NST + 4);
   volatile int* abort_flag = ctl + 1;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int Nb = p.Nb;
@@ -613,9 +618,10 @@ __global__ void __launch_bounds__(kBsThreads, 1) qgemm_bs_dec_kernel(const __gri
       mbar_init(bar_empty + 8 * s, 1);
       mbar_init(bar_sf + 8 * s, 4);
     }
-    mbar_init(bar_acc, 1);
+    mbar_init(bar_acc, 2);  // one commit of each issuer per unit
     mbar_init(bar_acc_free, 4);
     mbar_init(bar_drain, 1);
+    mbar_init(bar_drain + 8, 1);
     ctl[1] = 0;
     fence_mbar_init();
   }
@@ -628,6 +634,7 @@ __global__ void __launch_bounds__(kBsThreads, 1) qgemm_bs_dec_kernel(const __gri
   tc_fence_after();
   const uint32_t tmem = static_cast<uint32_t>(ctl[0]);
   const int64_t n_row_tiles = row_tiles(p.N);
+  const uint32_t sf_col0 = (uint32_t)(2 * Nb);  // scale factors after the two accumulators
   auto unit_range = [&](int u, int& t, int& s, int& c0, int& c1) {
     t = u % (int)n_row_tiles;
     s = u / (int)n_row_tiles;
@@ -677,12 +684,15 @@ __global__ void __launch_bounds__(kBsThreads, 1) qgemm_bs_dec_kernel(const __gri
       }
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp == kBdIssuer2Warp) {
+    // ------------------------------------------------------------ MMA issuers
+    // issuer e takes the chunks c of each unit with (c - c0) % 2 == e into accumulator e
+    const int e = (warp == 1) ? 0 : 1;
     if (lane == 0) {
       RingPos sp;
       bool ok = true;
       int ti = 0;
+      const uint32_t d = tmem + (uint32_t)(e * Nb);
       for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x, ++ti) {
         int t, s, c0, c1;
         unit_range(u, t, s, c0, c1);
@@ -695,6 +705,10 @@ __global__ void __launch_bounds__(kBsThreads, 1) qgemm_bs_dec_kernel(const __gri
           tc_fence_after();
         }
         for (int c = c0; c < c1; ++c) {
+          if (((c - c0) & 1) != e) {  // the other issuer's chunk: keep the ring position
+            sp.next(NST);
+            continue;
+          }
           if (!mbar_wait_spin(bar_full + 8 * sp.slot, sp.phase, false, abort_flag, p.dev_err, kErrTimeout) ||
               !mbar_wait_spin(bar_sf + 8 * sp.slot, sp.phase, false, abort_flag, p.dev_err, kErrTimeout)) {
             ok = false;
@@ -703,25 +717,25 @@ __global__ void __launch_bounds__(kBsThreads, 1) qgemm_bs_dec_kernel(const __gri
           tc_fence_after();
           const uint32_t st = sbase + (uint32_t)(sp.slot * p.stage_bytes);
           const uint64_t adesc0 = smem_desc_sw128(st);
-          const uint32_t sf0 = tmem + (uint32_t)(Nb + sp.slot * kBdSfCols);
+          const uint32_t sf0 = tmem + sf_col0 + (uint32_t)(sp.slot * kBdSfCols);
 #pragma unroll
           for (int kb = 0; kb < kBsK / 64; ++kb) {
 #pragma unroll
             for (int j = 0; j < kBsTerms; ++j) {
               const uint64_t bdesc = smem_desc_sw128(st + kBsBlock + (uint32_t)j * xterm) + (uint64_t)(kb * 2);
-              bs_mma(tmem, adesc0 + (uint64_t)(kb * 2), bdesc, idesc, sf0 + (uint32_t)(kb * 4),
-                     sf0 + (uint32_t)(16 + (j * 4 + kb) * 4), (c != c0 || kb || j) ? 1u : 0u);
+              bs_mma(d, adesc0 + (uint64_t)(kb * 2), bdesc, idesc, sf0 + (uint32_t)(kb * 4),
+                     sf0 + (uint32_t)(16 + (j * 4 + kb) * 4), (c - c0 >= 2 || kb || j) ? 1u : 0u);
             }
           }
           bs_commit(bar_empty + 8 * sp.slot);
           sp.next(NST);
         }
         if (!ok) break;
-        bs_commit(bar_acc);
+        bs_commit(bar_acc);  // this issuer's part of the unit (nothing pending if it had none)
       }
-      bs_commit(bar_drain);
+      bs_commit(bar_drain + 8 * e);
       const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait(bar_drain, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+      while (!mbar_try_wait(bar_drain + 8 * e, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
       }
     }
     __syncwarp();
@@ -764,7 +778,7 @@ __global__ void __launch_bounds__(kBsThreads, 1) qgemm_bs_dec_kernel(const __gri
             for (int kb = 0; kb < 4; ++kb)
               v[16 + (j * 4 + kb) * 4 + r1] = (((kb < 2) ? s8.x : s8.y) >> ((kb & 1) * 16)) & 0xFFFFu;
           }
-        const uint32_t ta = tmem + lane_base + (uint32_t)(Nb + sp.slot * kBdSfCols);
+        const uint32_t ta = tmem + lane_base + sf_col0 + (uint32_t)(sp.slot * kBdSfCols);
 #pragma unroll
         for (int i = 0; i < kBdSfCols / 16; ++i)
           bs_tmem_st16(ta + (uint32_t)(16 * i), *reinterpret_cast<const uint32_t(*)[16]>(&v[16 * i]));
@@ -792,11 +806,19 @@ __global__ void __launch_bounds__(kBsThreads, 1) qgemm_bs_dec_kernel(const __gri
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
+      const bool two = (c1 - c0) >= 2;  // the odd chunks' accumulator holds data
 #pragma unroll 1
       for (int cb = 0; cb < Nb; cb += 16) {
         uint32_t v[16];
         bs_tmem_ld16(tmem + lane_base + (uint32_t)cb, v);
         tmem_ld_wait();
+        if (two) {
+          uint32_t w[16];
+          bs_tmem_ld16(tmem + lane_base + (uint32_t)(Nb + cb), w);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) + __uint_as_float(w[i]));
+        }
         if (n64 < p.N) {
           const int n = (int)n64;
 #pragma unroll
@@ -970,7 +992,7 @@ cudaError_t launch_bs_dec(int M, int N, int K, const uint8_t* xcodes, const uint
   p.units = (int)row_tiles(N) * p.S;
   p.stage_bytes = (kBsBlock + kBsTerms * p.Nb * 128 + kBsSBlock + kBsTerms * p.Nb * 8 + 1023) / 1024 * 1024;
   p.stages = std::min({kBdMaxStages, (kSmemLimit - 1024 - 256) / p.stage_bytes,
-                       (kBsTmemCols - p.Nb) / kBdSfCols});
+                       (kBsTmemCols - 2 * p.Nb) / kBdSfCols}) & ~1;  // even
   if (p.stages < 2) return cudaErrorInvalidValue;
   p.xcodes = xcodes;
   p.xscales = xscales;
@@ -984,7 +1006,7 @@ cudaError_t launch_bs_dec(int M, int N, int K, const uint8_t* xcodes, const uint
   const size_t smem = 1024 + (size_t)p.stages * p.stage_bytes + 256;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)std::min(p.units, sms), 1, 1);
-  cfg.blockDim = dim3(kBsThreads, 1, 1);
+  cfg.blockDim = dim3(kBdThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute at[1];
