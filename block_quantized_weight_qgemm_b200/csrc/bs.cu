@@ -46,21 +46,24 @@ namespace qg {
 
 constexpr int kBsTerms = 3;
 constexpr int kBsM = 128;                     // tokens per tile
-constexpr int kBsN = 256;                     // weight rows per tile (two weight tiles)
+constexpr int kBsWT = 2;                      // weight tiles (of 128 rows) per tile
+constexpr int kBsN = 128 * kBsWT;             // weight rows per tile (MMA N)
 constexpr int kBsK = 256;                     // K per stage (one MXFP4 chunk)
-constexpr int kBsStages = 2;
+// (one weight tile per tile with three stages measured faster only at M = 2048 of the
+// 5120 x 17408 shape and slower at M = 8192: x is then re-read for every 128 weight rows)
+constexpr int kBsStages = kBsWT == 1 ? 3 : 2;
 constexpr int kBsBlock = kBsM * 128;          // one 128-row x 128-byte code block: 16 KB
 constexpr int kBsSBlock = kBsM * 8;           // its scales: 1 KB
 constexpr int kBsACodes = kBsTerms * kBsBlock;
-constexpr int kBsBCodes = 2 * kBsBlock;
+constexpr int kBsBCodes = kBsWT * kBsBlock;
 constexpr int kBsAScales = kBsTerms * kBsSBlock;
-constexpr int kBsBScales = 2 * kBsSBlock;
-constexpr int kBsStage = kBsACodes + kBsBCodes + kBsAScales + kBsBScales;  // 85 KB
+constexpr int kBsBScales = kBsWT * kBsSBlock;
+constexpr int kBsStage = kBsACodes + kBsBCodes + kBsAScales + kBsBScales;  // 85 KB at kBsWT = 2
 static_assert(kBsStage % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
 // tensor memory: the accumulator in columns [0, 256), then per stage kBsSfCols columns of
 // scale factors: x term t, K-block kb at (t * 4 + kb) * 4 (4 columns: row groups r1 = 0..3),
 // the weights' K-block kb at 48 + kb * 8 (8 columns: r1 = 0..7)
-constexpr int kBsSfCols = kBsTerms * 4 * 4 + 4 * 8;  // 80
+constexpr int kBsSfCols = kBsTerms * 4 * 4 + 4 * 4 * kBsWT;
 constexpr int kBsTmemCols = 512;
 static_assert(kBsN + kBsStages * kBsSfCols <= kBsTmemCols, "TMEM budget");
 constexpr int kBsStageWarp0 = 2;  // warps 2..5 stage the scale factors
@@ -355,11 +358,11 @@ __global__ void __launch_bounds__(kBsThreads, 1) qgemm_bs_kernel(const __grid_co
           const uint32_t fb = bar_full + 8 * sp.slot;
           const uint32_t st = sbase + (uint32_t)(sp.slot * kBsStage);
           uint32_t bytes = kBsACodes + kBsAScales;
-          for (int j = 0; j < 2; ++j)
-            if (2 * nt + j < n_row_tiles) bytes += kBsBlock + kBsSBlock;
+          for (int j = 0; j < kBsWT; ++j)
+            if (kBsWT * nt + j < n_row_tiles) bytes += kBsBlock + kBsSBlock;
           mbar_arrive_expect_tx(fb, bytes);
-          for (int j = 0; j < 2; ++j) {
-            const int64_t t = 2 * (int64_t)nt + j;
+          for (int j = 0; j < kBsWT; ++j) {
+            const int64_t t = kBsWT * (int64_t)nt + j;
             if (t >= n_row_tiles) continue;
             const int64_t blk = t * p.C + c;
             bulk_load(st + kBsACodes + j * kBsBlock, p.wcodes + blk * kBsBlock, kBsBlock, fb, pol_w);
@@ -416,7 +419,7 @@ __global__ void __launch_bounds__(kBsThreads, 1) qgemm_bs_kernel(const __grid_co
             for (int t = 0; t < kBsTerms; ++t) {
               const uint64_t adesc = smem_desc_sw128(st + (uint32_t)(t * kBsBlock)) + (uint64_t)(kb * 2);
               bs_mma(tmem, adesc, bdesc0 + (uint64_t)(kb * 2), kBsIdesc,
-                     sf0 + (uint32_t)((t * 4 + kb) * 4), sf0 + (uint32_t)(48 + kb * 8),
+                     sf0 + (uint32_t)((t * 4 + kb) * 4), sf0 + (uint32_t)(48 + kb * 4 * kBsWT),
                      (c | kb | t) != 0 ? 1u : 0u);
             }
           }
@@ -454,7 +457,7 @@ __global__ void __launch_bounds__(kBsThreads, 1) qgemm_bs_kernel(const __grid_co
         tc_fence_after();
         const uint8_t* st = smem + sp.slot * kBsStage;
         const uint8_t* sa = st + kBsACodes + kBsBCodes;  // x-term scales [3][128][8]
-        const uint8_t* sb = sa + kBsAScales;              // weight scales [2][128][8]
+        const uint8_t* sb = sa + kBsAScales;              // weight scales [kBsWT][128][8]
         uint32_t v[kBsSfCols];
 #pragma unroll
         for (int t = 0; t < kBsTerms; ++t)
@@ -468,12 +471,12 @@ __global__ void __launch_bounds__(kBsThreads, 1) qgemm_bs_kernel(const __grid_co
             }
           }
 #pragma unroll
-        for (int r1 = 0; r1 < 8; ++r1) {
+        for (int r1 = 0; r1 < 4 * kBsWT; ++r1) {
           const uint2 s8 = *reinterpret_cast<const uint2*>(sb + (r1 >> 2) * kBsSBlock + ((r1 & 3) * 32 + lane) * 8);
 #pragma unroll
           for (int kb = 0; kb < 4; ++kb) {
             const uint32_t w = (kb < 2) ? s8.x : s8.y;
-            v[48 + kb * 8 + r1] = (w >> ((kb & 1) * 16)) & 0xFFFFu;
+            v[48 + kb * 4 * kBsWT + r1] = (w >> ((kb & 1) * 16)) & 0xFFFFu;
           }
         }
         const uint32_t ta = tmem + lane_base + (uint32_t)(kBsN + sp.slot * kBsSfCols);
