@@ -67,6 +67,8 @@ def _load():
             lib.orc_pack_mxfp4.argtypes = [vp, i64, i64, vp, vp]
             lib.orc_pack_fp8.argtypes = [vp, i64, i64, vp, vp]
             lib.orc_split_x.argtypes = [vp, i64, i64, ctypes.c_int, ctypes.c_int, vp]
+            lib.orc_split_x_bs.argtypes = [vp, i64, i64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                           ctypes.c_int, vp]
             lib.orc_dequant.argtypes = [ctypes.c_int, vp, vp, ctypes.c_float, i64, i64, vp]
             lib.orc_gemm.argtypes = [vp, i64, i64, vp, i64, vp, ctypes.c_int]
             lib.orc_ffn_gate_up.argtypes = [vp, i64, i64, vp, vp, i64, vp, vp, vp, ctypes.c_int]
@@ -207,6 +209,22 @@ def split_x(x16: np.ndarray, elem: str, terms: int) -> np.ndarray:
     B, K = x16.shape
     xs = np.zeros((B, K), dtype=np.float64)
     _load().orc_split_x(_ptr(x16), B, K, 0 if elem == "e4m3" else 1, terms, _ptr(xs))
+    return xs
+
+
+# block size, prescale shift and smallest scale exponent of the block-scaled path's split
+BS_SPLIT = {"mxfp4": (32, 0, -127), "nvfp4": (16, 10, -9)}
+
+
+def split_x_bs(x16: np.ndarray, fmt: str, terms: int = 3) -> np.ndarray:
+    """The activation split as the block-scaled path of weight format `fmt` applies it: per-row
+    power-of-two prescale, E2M1 terms with power-of-two block scales in the MMA scale type's
+    range (orc_split_x_bs); returns 2^xe * the sum of the terms (fp64)."""
+    x16 = np.ascontiguousarray(x16, dtype=np.uint16)
+    B, K = x16.shape
+    blk, xshift, emin = BS_SPLIT[fmt]
+    xs = np.zeros((B, K), dtype=np.float64)
+    _load().orc_split_x_bs(_ptr(x16), B, K, blk, xshift, emin, terms, _ptr(xs))
     return xs
 
 

@@ -509,6 +509,58 @@ void orc_split_x(const uint16_t *x16, int64_t B, int64_t K, int elem, int terms,
 }
 
 /* ------------------------------------------------------------------------- */
+/* The activation split of the block-scaled path as the product applies it     */
+/* (reading: the split above with a per-row power-of-two prescale and a bounded */
+/* range of power-of-two block scales, so that each term's scale is a value of  */
+/* the MMA's scale type):                                                       */
+/*   xe = floor(log2 max|x_row|) - xshift   (0 for an all-zero row)            */
+/*   r_0 = x 2^-xe;  per block of `block` elements and term j:                  */
+/*   e_j = floor(log2 max|r_j|) - 2; if e_j < emin the term and the later ones  */
+/*   are dropped; q_j = E2M1_RNE_sat(r_j / 2^e_j); r_{j+1} = r_j - q_j 2^e_j.   */
+/* xs receives 2^xe sum_j q_j 2^e_j.  MXFP4 (E8M0 per 32): block 32, xshift 0,  */
+/* emin -127.  NVFP4 (UE4M3 per 16, powers of two only): block 16, xshift 10,   */
+/* emin -9 (2^-9 is the smallest UE4M3 power of two; the prescale puts the row  */
+/* maximum in [2^10, 2^11), so e_j <= 8 and 2^8 is representable).             */
+/* ------------------------------------------------------------------------- */
+void orc_split_x_bs(const uint16_t *x16, int64_t B, int64_t K, int block, int xshift, int emin,
+                    int terms, double *xs) {
+    for (int64_t b = 0; b < B; ++b) {
+        double rmax = 0.0;
+        int xe = 0;
+        for (int64_t k = 0; k < K; ++k) rmax = fmax(rmax, fabs(orc_bf16(x16[b * K + k])));
+        if (rmax > 0.0) {
+            int ex;
+            (void)frexp(rmax, &ex);
+            xe = (ex - 1) - xshift;
+        }
+        for (int64_t k0 = 0; k0 < K; k0 += block) {
+            double r[64], acc[64];
+            const int64_t n = (K - k0 < block) ? K - k0 : block;
+            for (int64_t i = 0; i < n; ++i) {
+                r[i] = ldexp(orc_bf16(x16[b * K + k0 + i]), -xe);
+                acc[i] = 0.0;
+            }
+            for (int j = 0; j < terms; ++j) {
+                double amax = 0.0, sc;
+                int ex, e;
+                for (int64_t i = 0; i < n; ++i) amax = fmax(amax, fabs(r[i]));
+                if (amax == 0.0) break;
+                (void)frexp(amax, &ex);
+                e = (ex - 1) - 2;
+                if (e < emin) break;
+                sc = ldexp(1.0, e);
+                for (int64_t i = 0; i < n; ++i) {
+                    const double q = orc_e2m1(orc_e2m1_encode(r[i] / sc));
+                    acc[i] += q * sc;
+                    r[i] -= q * sc;
+                }
+            }
+            for (int64_t i = 0; i < n; ++i) xs[b * K + k0 + i] = ldexp(acc[i], xe);
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------- */
 /* Fused FFN (Atlas issue: fused gate+up with dual accumulators; the pages'    */
 /* prefill path writes the activated product as bf16 for the down GEMM).      */
 /*   g = x Wg^T, u = x Wu^T (fp64); SiLU(g) = g / (1 + exp(-g));               */

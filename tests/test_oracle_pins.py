@@ -577,3 +577,59 @@ def test_activation_split_accuracy_for_the_block_scaled_path():
             assert err[("e4m3", 2)] < 1e-8 and err[("e4m3", 3)] < 1e-10
             assert err[("e2m1", 3)] < 2e-4 and err[("e2m1", 4)] < 2e-5
             assert np.array_equal(oracle.split_x(x16, "e4m3", 3), xd)  # three terms: exact
+
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
+def test_block_scaled_split_first_term_brute_force(fmt):
+    # one term, from the definitions: xe = floor(log2 max|row|) - xshift, each block's
+    # e = floor(log2 max|x 2^-xe|) - 2, the nearest E2M1 value of x 2^-xe / 2^e (ties to the even
+    # code, saturating at 6), times 2^e 2^xe; blocks with e below the smallest scale are zero
+    blk, xshift, emin = oracle.BS_SPLIT[fmt]
+    x = inputs.activations(3, 96, seed=61)
+    x[1, 16:32] *= 2.0 ** -40  # a block far below its row maximum
+    x16 = inputs.bf16_bits(x)
+    xs = oracle.split_x_bs(x16, fmt, 1)
+    vals = [Fraction(v) for v in E2M1_MAG]
+    for b in range(3):
+        row = [Fraction(oracle.bf16(int(v))) for v in x16[b]]
+        _, ex = math.frexp(float(max(abs(v) for v in row)))
+        xe = (ex - 1) - xshift
+        for k0 in range(0, 96, blk):
+            r = [v / Fraction(2) ** xe for v in row[k0:k0 + blk]]
+            _, ex = math.frexp(float(max(abs(v) for v in r)))
+            e = (ex - 1) - 2
+            for i, v in enumerate(r):
+                if e < emin:
+                    want = Fraction(0)
+                else:
+                    a = abs(v) / Fraction(2) ** e
+                    best = min(range(len(vals)), key=lambda c: (abs(a - vals[c]), c & 1))
+                    want = vals[best] * Fraction(2) ** (e + xe) * (1 if v >= 0 else -1)
+                assert Fraction(float(xs[b, k0 + i])) == want, (fmt, b, k0 + i)
+    if fmt == "nvfp4":
+        assert not xs[1, 16:32].any()  # 2^-40 below the maximum: below the UE4M3 range
+
+
+def test_block_scaled_split_prescale_invariance_and_mxfp4_reduction():
+    # a power-of-two factor on a row scales its split by the same factor (the prescale absorbs
+    # it); with MXFP4's parameters and no dropped block the split is the plain per-block peel
+    x = inputs.activations(4, 640, seed=62)
+    x16 = inputs.bf16_bits(x)
+    for fmt in ("mxfp4", "nvfp4"):
+        base = oracle.split_x_bs(x16, fmt, 3)
+        for k in (-60, 7, 90):
+            xk = inputs.bf16_bits(x * 2.0 ** k)
+            assert np.array_equal(oracle.split_x_bs(xk, fmt, 3), np.ldexp(base, k)), (fmt, k)
+    assert np.array_equal(oracle.split_x_bs(x16, "mxfp4", 3), oracle.split_x(x16, "e2m1", 3))
+
+
+def test_block_scaled_split_accuracy():
+    # three E2M1 terms in either variant stay well inside the 1e-3 bar at the 27B lengths
+    for K in (5120, 17408):
+        x16 = inputs.bf16_bits(inputs.activations(4, K, seed=63))
+        for fmt in ("nvfp4", "mxfp4"):
+            W = inputs.weights(16, K, seed=64).numpy()
+            Wd = oracle.dequant(fmt, *oracle.pack(fmt, W), 16, K)
+            y = oracle.gemm(x16, Wd)
+            err = oracle.normalised_error(oracle.gemm_f64(oracle.split_x_bs(x16, fmt, 3), Wd), y, x16, Wd)
+            assert err < 2e-4, (K, fmt, err)
