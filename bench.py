@@ -306,17 +306,17 @@ def run_configs(dev, stream, q8_rings, hbm_peak, tf_peak):
             r["note"] = note
         recs.append(r)
 
-    def decode_bs(name, ring, B, reps=40):
-        # the block-scaled path at a decode width (MXFP4 weights as the MMA M operand)
+    def decode_bs(name, ring, B, fmt="mxfp4", reps=40):
+        # the block-scaled path at a decode width (the weights as the MMA M operand)
         N, K = ring[0].N, ring[0].K
         x = inputs.activations(B, K, seed=1).to(dev)
         y = torch.empty(B, N, device=dev)
-        ws = torch.empty(max(qgemm.bs_workspace_size(qgemm._fmt("mxfp4"), N, K, B), 16),
+        ws = torch.empty(max(qgemm.bs_workspace_size(qgemm._fmt(fmt), N, K, B), 16),
                          dtype=torch.uint8, device=dev)
         us = graph_us(lambda i: qgemm.bs_run(x, ring[i % len(ring)], y=y, workspace=ws, stream=stream),
                       reps, stream)
-        gbs = weight_bytes("mxfp4", N, K) / (us * 1e-6) / 1e9
-        recs.append({"config": name, "kind": "decode", "fmt": "mxfp4", "path": "block-scaled",
+        gbs = weight_bytes(fmt, N, K) / (us * 1e-6) / 1e9
+        recs.append({"config": name, "kind": "decode", "fmt": fmt, "path": "block-scaled",
                      "N": N, "K": K, "B": B, "us": round(us, 2), "weight_GBps": round(gbs, 1),
                      "frac_hbm": round(gbs / hbm_peak, 4)})
         del x, y, ws
@@ -346,19 +346,19 @@ def run_configs(dev, stream, q8_rings, hbm_peak, tf_peak):
                      "us": round(us, 1), "TFLOPs": round(tf, 1), "frac_tensor": round(tf / tf_peak, 4)})
         del x, y, ws
 
-    def prefill_bs(name, pw, M, reps=3):
-        # the block-scaled path (MXFP4 weights on kind::mxf4nvf4, x split into three E2M1
-        # terms): split + GEMM per call
+    def prefill_bs(name, pw, M, fmt="mxfp4", reps=3):
+        # the block-scaled path (MXFP4 / NVFP4 weights on kind::mxf4nvf4, x split into three
+        # E2M1 terms): split + GEMM per call
         N, K = pw.N, pw.K
         x = inputs.activations(M, K, seed=1).to(dev)
         y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-        ws = torch.empty(qgemm.bs_workspace_size(qgemm._fmt("mxfp4"), N, K, M), dtype=torch.uint8,
+        ws = torch.empty(qgemm.bs_workspace_size(qgemm._fmt(fmt), N, K, M), dtype=torch.uint8,
                          device=dev)
         us = graph_us(lambda i: qgemm.bs_run(x, pw, y=y, workspace=ws, stream=stream), reps, stream)
         tf = 2.0 * M * N * K / (us * 1e-6) / 1e12
         # the MMAs run 3 x 2MNK of FP4 work; their own peak is the bf16 peak x 4 (the nominal
         # dense FP4 : bf16 ratio, 9 : 2.25 PFLOP/s)
-        recs.append({"config": name, "kind": "prefill", "fmt": "mxfp4", "path": "block-scaled",
+        recs.append({"config": name, "kind": "prefill", "fmt": fmt, "path": "block-scaled",
                      "N": N, "K": K, "M": M, "us": round(us, 1), "TFLOPs": round(tf, 1),
                      "frac_tensor": round(tf / tf_peak, 4),
                      "fp4_mma_frac": round(3.0 * tf / (4.0 * tf_peak), 4)})
@@ -409,7 +409,11 @@ def run_configs(dev, stream, q8_rings, hbm_peak, tf_peak):
     ring = clone_ring(nv_gate, RING)
     for B in (1, 4, 8, 16):
         decode("nvfp4 27B gate/up verify", "nvfp4", ring, B)
+    for B in (1, 16):
+        decode_bs("nvfp4 27B gate/up verify, block-scaled path", ring, B, fmt="nvfp4")
     del ring
+    prefill("nvfp4 27B gate/up prefill", "nvfp4", nv_gate, 2048)
+    prefill_bs("nvfp4 27B gate/up prefill, block-scaled path", nv_gate, 2048, fmt="nvfp4")
     # cfg 4: NVFP4 prefill FFN chunk (fused gate+up -> h -> down)
     nv_up = packed("nvfp4", INTER, HIDDEN, 2)
     nv_down = packed("nvfp4", HIDDEN, INTER, 3)

@@ -14,16 +14,18 @@
 
 namespace qg {
 cudaError_t launch_prep(const PrepParams& pp, cudaStream_t stream);
-cudaError_t launch_bs_split(const uint16_t* x, int M, int K, uint8_t* codes, uint8_t* scales,
-                            int* x_exp, cudaStream_t stream);
-cudaError_t launch_bs_gemm(int M, int N, int K, const uint8_t* xcodes, const uint8_t* xscales,
-                           const int* x_exp, const uint8_t* wcodes, const uint8_t* wscales,
-                           void* out, int out_bf16, int* dev_err, cudaStream_t stream);
-size_t bs_workspace_bytes(int64_t M, int64_t N, int64_t K, size_t* off_scales, size_t* off_exp,
-                          size_t* off_part);
-cudaError_t launch_bs_dec(int M, int N, int K, const uint8_t* xcodes, const uint8_t* xscales,
-                          const int* x_exp, const uint8_t* wcodes, const uint8_t* wscales,
-                          float* part, void* out, int out_bf16, int* dev_err, cudaStream_t stream);
+cudaError_t launch_bs_split(bool nv, const uint16_t* x, int M, int K, uint8_t* codes,
+                            uint8_t* scales, int* x_exp, cudaStream_t stream);
+cudaError_t launch_bs_gemm(bool nv, int M, int N, int K, const uint8_t* xcodes,
+                           const uint8_t* xscales, const int* x_exp, const uint8_t* wcodes,
+                           const uint8_t* wscales, const float* ts, void* out, int out_bf16,
+                           int* dev_err, cudaStream_t stream);
+size_t bs_workspace_bytes(bool nv, int64_t M, int64_t N, int64_t K, size_t* off_scales,
+                          size_t* off_exp, size_t* off_part);
+cudaError_t launch_bs_dec(bool nv, int M, int N, int K, const uint8_t* xcodes,
+                          const uint8_t* xscales, const int* x_exp, const uint8_t* wcodes,
+                          const uint8_t* wscales, const float* ts, float* part, void* out,
+                          int out_bf16, int* dev_err, cudaStream_t stream);
 cudaError_t launch_pair(int fmt, bool bf16op, const GemmParams& p, size_t smem_bytes, int units,
                         const CUtensorMap* maps, bool pdl, cudaStream_t stream);
 cudaError_t launch_pack(int fmt, const float* W, int64_t N, int64_t K, void* codes, void* scales,
@@ -888,15 +890,20 @@ int qgemm_moe_gate_up(int fmt, const void* x, int64_t M, int64_t K, int E, const
 }
 
 // ---------------------------------------------------------------------------------------
-// Block-scaled path (MXFP4 weights, x split into three E2M1 terms)
+// Block-scaled path (MXFP4 / NVFP4 weights, x split into three E2M1 terms)
 // ---------------------------------------------------------------------------------------
-int qgemm_bs_split_size(int64_t M, int64_t K, size_t* code_bytes, size_t* scale_bytes,
+namespace {
+bool bs_fmt(int fmt) { return fmt == QGEMM_FMT_MXFP4 || fmt == QGEMM_FMT_NVFP4; }
+}  // namespace
+
+int qgemm_bs_split_size(int fmt, int64_t M, int64_t K, size_t* code_bytes, size_t* scale_bytes,
                         size_t* exp_bytes) {
+  if (!bs_fmt(fmt)) return QGEMM_ERR_FORMAT;
   if (M < 1 || K < 1 || M > 0x7FFFFFFF || K > 0x7FFFFFFF) return QGEMM_ERR_SHAPE;
   if (K % 32 != 0) return QGEMM_ERR_K_BLOCK;
   if (!code_bytes || !scale_bytes || !exp_bytes) return QGEMM_ERR_NULL;
   size_t off_s = 0, off_e = 0, off_p = 0;
-  (void)bs_workspace_bytes(M, 0, K, &off_s, &off_e, &off_p);
+  (void)bs_workspace_bytes(fmt == QGEMM_FMT_NVFP4, M, 0, K, &off_s, &off_e, &off_p);
   const int64_t Mt = (M + 127) / 128;
   *code_bytes = off_s;
   *scale_bytes = off_e - off_s;
@@ -904,34 +911,36 @@ int qgemm_bs_split_size(int64_t M, int64_t K, size_t* code_bytes, size_t* scale_
   return QGEMM_OK;
 }
 
-int qgemm_bs_split_x(const void* x, int64_t M, int64_t K, void* codes, void* scales,
+int qgemm_bs_split_x(int fmt, const void* x, int64_t M, int64_t K, void* codes, void* scales,
                      int32_t* x_exp, void* stream) {
+  if (!bs_fmt(fmt)) return QGEMM_ERR_FORMAT;
   if (M < 1 || K < 1 || M > 0x7FFFFFFF || K > 0x7FFFFFFF) return QGEMM_ERR_SHAPE;
   if (K % 32 != 0) return QGEMM_ERR_K_BLOCK;
   if (!x || !codes || !scales || !x_exp) return QGEMM_ERR_NULL;
   if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || !aligned16(x_exp))
     return QGEMM_ERR_ALIGN;
   if (!device_ok()) return QGEMM_ERR_DEVICE;
-  const cudaError_t e = launch_bs_split(static_cast<const uint16_t*>(x), (int)M, (int)K,
+  const cudaError_t e = launch_bs_split(fmt == QGEMM_FMT_NVFP4, static_cast<const uint16_t*>(x), (int)M, (int)K,
                                         static_cast<uint8_t*>(codes), static_cast<uint8_t*>(scales),
                                         reinterpret_cast<int*>(x_exp), static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? QGEMM_OK : cuda_fail(e, "split kernel launch");
 }
 
 int qgemm_bs_workspace_size(int fmt, int64_t N, int64_t K, int64_t M, size_t* bytes) {
-  if (fmt != QGEMM_FMT_MXFP4) return QGEMM_ERR_FORMAT;
+  if (!bs_fmt(fmt)) return QGEMM_ERR_FORMAT;
   int st = check_fmt_shape(fmt, N, K);
   if (st != QGEMM_OK) return st;
   if (M < 1 || M > 0x7FFFFFFF) return QGEMM_ERR_SHAPE;
   if (!bytes) return QGEMM_ERR_NULL;
-  *bytes = bs_workspace_bytes(M, N, K, nullptr, nullptr, nullptr);
+  *bytes = bs_workspace_bytes(fmt == QGEMM_FMT_NVFP4, M, N, K, nullptr, nullptr, nullptr);
   return QGEMM_OK;
 }
 
 int qgemm_bs_run(int fmt, const void* x, int64_t M, int64_t K, const void* codes,
                  const void* scales, const float* tensor_scale, int64_t N, void* y, int y_dtype,
                  void* workspace, size_t workspace_bytes, void* stream) {
-  if (fmt != QGEMM_FMT_MXFP4) return QGEMM_ERR_FORMAT;
+  if (!bs_fmt(fmt)) return QGEMM_ERR_FORMAT;
+  const bool nv = fmt == QGEMM_FMT_NVFP4;
   int st = check_fmt_shape(fmt, N, K);
   if (st != QGEMM_OK) return st;
   if (M < 1 || M > 0x7FFFFFFF) return QGEMM_ERR_SHAPE;
@@ -940,7 +949,7 @@ int qgemm_bs_run(int fmt, const void* x, int64_t M, int64_t K, const void* codes
   if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || !aligned16(y))
     return QGEMM_ERR_ALIGN;
   size_t off_s = 0, off_e = 0, off_p = 0;
-  const size_t need = bs_workspace_bytes(M, N, K, &off_s, &off_e, &off_p);
+  const size_t need = bs_workspace_bytes(nv, M, N, K, &off_s, &off_e, &off_p);
   if (!workspace || workspace_bytes < need) return QGEMM_ERR_WORKSPACE;
   if (!aligned16(workspace)) return QGEMM_ERR_ALIGN;
   if (!device_ok()) return QGEMM_ERR_DEVICE;
@@ -948,18 +957,19 @@ int qgemm_bs_run(int fmt, const void* x, int64_t M, int64_t K, const void* codes
   if (!dev_err) return cuda_fail(cudaGetLastError(), "cudaGetSymbolAddress");
   uint8_t* wsb = static_cast<uint8_t*>(workspace);
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = launch_bs_split(static_cast<const uint16_t*>(x), (int)M, (int)K, wsb, wsb + off_s,
+  cudaError_t e = launch_bs_split(nv, static_cast<const uint16_t*>(x), (int)M, (int)K, wsb, wsb + off_s,
                                   reinterpret_cast<int*>(wsb + off_e), s);
   if (e != cudaSuccess) return cuda_fail(e, "split kernel launch");
   if (g_prof_begin) cudaEventRecord(g_prof_begin, s);
   // up to 128 rows the weights are the MMA M operand (decode tiling), above that x is
+  const float* ts = nv ? tensor_scale : nullptr;
   if (M <= 128)
-    e = launch_bs_dec((int)M, (int)N, (int)K, wsb, wsb + off_s, reinterpret_cast<const int*>(wsb + off_e),
-                      static_cast<const uint8_t*>(codes), static_cast<const uint8_t*>(scales),
+    e = launch_bs_dec(nv, (int)M, (int)N, (int)K, wsb, wsb + off_s, reinterpret_cast<const int*>(wsb + off_e),
+                      static_cast<const uint8_t*>(codes), static_cast<const uint8_t*>(scales), ts,
                       reinterpret_cast<float*>(wsb + off_p), y, y_dtype == QGEMM_Y_BF16, dev_err, s);
   else
-    e = launch_bs_gemm((int)M, (int)N, (int)K, wsb, wsb + off_s, reinterpret_cast<const int*>(wsb + off_e),
-                       static_cast<const uint8_t*>(codes), static_cast<const uint8_t*>(scales), y,
+    e = launch_bs_gemm(nv, (int)M, (int)N, (int)K, wsb, wsb + off_s, reinterpret_cast<const int*>(wsb + off_e),
+                       static_cast<const uint8_t*>(codes), static_cast<const uint8_t*>(scales), ts, y,
                        y_dtype == QGEMM_Y_BF16, dev_err, s);
   if (e != cudaSuccess) return cuda_fail(e, "block-scaled gemm launch");
   if (g_prof_end) cudaEventRecord(g_prof_end, s);

@@ -53,13 +53,8 @@ constexpr int kBsK = 256;                     // K per stage (one MXFP4 chunk)
 // 5120 x 17408 shape and slower at M = 8192: x is then re-read for every 128 weight rows)
 constexpr int kBsStages = kBsWT == 1 ? 3 : 2;
 constexpr int kBsBlock = kBsM * 128;          // one 128-row x 128-byte code block: 16 KB
-constexpr int kBsSBlock = kBsM * 8;           // its scales: 1 KB
 constexpr int kBsACodes = kBsTerms * kBsBlock;
 constexpr int kBsBCodes = kBsWT * kBsBlock;
-constexpr int kBsAScales = kBsTerms * kBsSBlock;
-constexpr int kBsBScales = kBsWT * kBsSBlock;
-constexpr int kBsStage = kBsACodes + kBsBCodes + kBsAScales + kBsBScales;  // 85 KB at kBsWT = 2
-static_assert(kBsStage % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
 // tensor memory: the accumulator in columns [0, 256), then per stage kBsSfCols columns of
 // scale factors: x term t, K-block kb at (t * 4 + kb) * 4 (4 columns: row groups r1 = 0..3),
 // the weights' K-block kb at 48 + kb * 8 (8 columns: r1 = 0..7)
@@ -69,14 +64,47 @@ static_assert(kBsN + kBsStages * kBsSfCols <= kBsTmemCols, "TMEM budget");
 constexpr int kBsStageWarp0 = 2;  // warps 2..5 stage the scale factors
 constexpr int kBsEpiWarp0 = 6;    // warps 6..9 run the epilogue
 constexpr int kBsThreads = 10 * 32;
-constexpr int kBsSmem = 1024 + kBsStages * kBsStage + 256;
 
 struct BsSplitParams {
   const uint16_t* x;  // bf16 [M][K]
   int M, K, C, Mt;
+  int nv;             // 1: NVFP4 (16-element blocks, UE4M3 powers of two), 0: MXFP4 (32, E8M0)
   uint8_t* codes;
-  uint8_t* scales;
+  uint8_t* scales;    // [Mt][C][3][128][sbr], sbr = 16 (NVFP4) or 8 (MXFP4)
   int* x_exp;
+};
+
+// Parameters of the split per weight format: block size, prescale shift (the row maximum
+// lands in [2^xshift, 2^(xshift+1))), smallest block-scale exponent, scale bytes per row and
+// 256-K chunk.  MXFP4: E8M0 scales per 32 elements, whose range covers every bf16 row after a
+// prescale to [1, 2).  NVFP4: UE4M3 scales per 16, restricted to the powers of two it holds
+// exactly (2^-9 .. 2^8, so that every step stays exact); the prescale to [2^10, 2^11) keeps
+// every block scale <= 2^8 and gives blocks 2^17 of range below the row maximum.
+__host__ __device__ constexpr int bs_blk(bool nv) { return nv ? 16 : 32; }
+__host__ __device__ constexpr int bs_xshift(bool nv) { return nv ? 10 : 0; }
+__host__ __device__ constexpr int bs_emin(bool nv) { return nv ? -9 : -127; }
+__host__ __device__ constexpr int bs_sbr(bool nv) { return nv ? 16 : 8; }
+// The scale byte of 2^e: E8M0 e + 127; UE4M3 (bias 7, three mantissa bits) (e + 7) << 3 for a
+// normal value, 2^(e + 9) as the subnormal mantissa below 2^-6.
+__host__ __device__ constexpr int bs_scale_byte(bool nv, int e) {
+  return nv ? (e >= -6 ? (e + 7) << 3 : 1 << (e + 9)) : e + 127;
+}
+
+// Prefill-kernel stage layout per weight format: [x-term codes 48 KB][weight codes 32 KB]
+// [x-term scales 3 x 128 x sbr][weight scales 2 x 128 x sbr] (85 KB MXFP4, 90 KB NVFP4).
+template <bool NV>
+struct BsLay {
+  static constexpr int SB = kBsM * bs_sbr(NV);  // scales of one 128-row block
+  static constexpr int AScales = kBsTerms * SB;
+  static constexpr int BScales = kBsWT * SB;
+  static constexpr int Stage = kBsACodes + kBsBCodes + AScales + BScales;
+  static constexpr int Smem = 1024 + kBsStages * Stage + 256;
+  // instruction descriptor, kind::mxf4nvf4: A and B E2M1 (K-major), M = 128, N = kBsN,
+  // K = 64 per instruction, scale factor ids 0, scale type UE4M3 (NVFP4) or E8M0 (MXFP4)
+  static constexpr uint32_t Idesc = (1u << 7) | (1u << 10) | ((uint32_t)(kBsN >> 3) << 17) |
+                                    ((NV ? 0u : 1u) << 23) | ((uint32_t)(kBsM >> 4) << 24);
+  static_assert(Stage % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
+  static_assert(Smem <= 227 * 1024, "shared memory");
 };
 
 struct BsParams {
@@ -84,8 +112,9 @@ struct BsParams {
   const uint8_t* xcodes;
   const uint8_t* xscales;
   const int* x_exp;
-  const uint8_t* wcodes;   // tile-major MXFP4 codes
-  const uint8_t* wscales;  // tile-major MXFP4 scales
+  const uint8_t* wcodes;   // tile-major MXFP4 / NVFP4 codes
+  const uint8_t* wscales;  // tile-major scales
+  const float* ts;         // NVFP4 tensor scale (device), else nullptr
   void* out;               // y [M][N] fp32 or bf16
   int out_bf16;
   int* dev_err;
@@ -113,9 +142,9 @@ __device__ __forceinline__ float bs_amax8(float m, const uint4& v) {
   return m;
 }
 
-// The three terms of one lane's 8 elements (its quarter of a 32-element block), written to
-// the split layout.  All four lanes of the block take the same decisions (the block maximum
-// is reduced over them first).
+// The three terms of one lane's 8 elements (a quarter of a 32-element block or half of a
+// 16-element one), written to the split layout.  All lanes of the block take the same
+// decisions (the block maximum is reduced over them first).
 __device__ __forceinline__ void bs_split8(const BsSplitParams& p, const uint4& v, bool in, float f1,
                                           float f2, int t, int r, int c, int lane) {
   float rv[8];
@@ -125,7 +154,11 @@ __device__ __forceinline__ void bs_split8(const BsSplitParams& p, const uint4& v
     rv[2 * i] = in ? (__uint_as_float(w[i] << 16) * f1) * f2 : 0.f;
     rv[2 * i + 1] = in ? (__uint_as_float(w[i] & 0xFFFF0000u) * f1) * f2 : 0.f;
   }
-  const int j = lane >> 2;  // 32-element block of the chunk
+  const int g = lane >> 2;                  // 16-byte group (32 elements) of the chunk
+  const bool nv = p.nv != 0;
+  const int lpb = bs_blk(nv) / 8;           // lanes per block
+  const int j = lane / lpb;                 // block of the chunk
+  const int emin = bs_emin(nv);
   bool done = false;
 #pragma unroll
   for (int term = 0; term < kBsTerms; ++term) {
@@ -133,15 +166,16 @@ __device__ __forceinline__ void bs_split8(const BsSplitParams& p, const uint4& v
 #pragma unroll
     for (int i = 0; i < 8; ++i) bmax = fmaxf(bmax, fabsf(rv[i]));
     bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 1));
-    bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 2));
-    int sb = 0;  // E8M0 byte
+    const float b2 = __shfl_xor_sync(0xffffffffu, bmax, 2);
+    if (!nv) bmax = fmaxf(bmax, b2);
+    int sb = 0;  // scale byte
     uint32_t packed = 0u;
     if (!done && bmax > 0.f) {
       int ex;
       (void)frexpf(bmax, &ex);
       const int e = (ex - 1) - 2;  // block maximum / 2^e in [4, 8)
-      if (e >= -127) {
-        sb = e + 127;
+      if (e >= emin) {
+        sb = bs_scale_byte(nv, e);
         const float inv = bs_pow2(-e), sc = bs_pow2(e);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -155,16 +189,17 @@ __device__ __forceinline__ void bs_split8(const BsSplitParams& p, const uint4& v
           packed |= (uint32_t)c2 << (8 * i);
         }
       } else {
-        done = true;  // below the E8M0 range: this and the later terms are dropped
+        done = true;  // below the scale range: this and the later terms are dropped
       }
     } else {
       done = true;
     }
     const size_t bidx = ((size_t)t * p.C + c) * kBsTerms + term;
-    // the block's 16 bytes are group j of the row, stored at group j ^ (r & 7)
+    // 32 elements are 16 bytes: group g of the row, stored at group g ^ (r & 7)
     uint8_t* crow = p.codes + bidx * kBsBlock + (size_t)r * 128;
-    *reinterpret_cast<uint32_t*>(crow + (((j ^ (r & 7)) & 7) << 4) + (lane & 3) * 4) = packed;
-    if ((lane & 3) == 0) p.scales[bidx * kBsSBlock + (size_t)r * 8 + j] = (uint8_t)(done ? 0 : sb);
+    *reinterpret_cast<uint32_t*>(crow + (((g ^ (r & 7)) & 7) << 4) + (lane & 3) * 4) = packed;
+    const int sbr = bs_sbr(nv);
+    if (lane % lpb == 0) p.scales[bidx * (size_t)(kBsM * sbr) + (size_t)r * sbr + j] = (uint8_t)(done ? 0 : sb);
   }
 }
 
@@ -204,11 +239,11 @@ __global__ void __launch_bounds__(kBsSplitThreads) qgemm_bs_split_kernel(const B
   if (amax > 0.f && amax <= 3.4e38f) {
     int ex;
     (void)frexpf(amax, &ex);
-    xe = ex - 1;  // row maximum * 2^-xe in [1, 2)
+    xe = (ex - 1) - bs_xshift(p.nv != 0);  // row maximum * 2^-xe in [2^xshift, 2^(xshift+1))
   }
   if (threadIdx.x == 0) p.x_exp[m] = live ? xe : 0;
-  // 2^-xe as two exact factors (xe runs from -133 to 127)
-  const int a1 = min(-xe, 126);
+  // 2^-xe as two exact factors (xe runs from -143 to 127)
+  const int a1 = max(min(-xe, 126), -126);
   const float f1 = bs_pow2(a1), f2 = bs_pow2(-xe - a1);
   const int t = m / kBsM, r = m % kBsM;
   const int lane = threadIdx.x & 31;
@@ -240,17 +275,35 @@ __device__ __forceinline__ void bs_tmem_dealloc(uint32_t taddr, uint32_t ncols) 
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
                : "memory");
 }
-// D (+)= A * B^T with 32-element E8M0 block scales: A, B K-major E2M1 in shared memory, the
-// scale factors in tensor memory at sfa / sfb.
+// D (+)= A * B^T with block scales: A, B K-major E2M1 in shared memory, the scale factors in
+// tensor memory at sfa / sfb; 16-element UE4M3 blocks (NVFP4) or 32-element E8M0 (MXFP4).
+template <bool NV>
 __device__ __forceinline__ void bs_mma(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                        uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t"
-      "}" ::"r"(d),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
-      : "memory");
+  if (NV)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t"
+        "}" ::"r"(d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t"
+        "}" ::"r"(d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+}
+
+// The 4-byte scale word of one row for 64-K block kb: NVFP4 keeps 4 scales per 64 K (16 bytes
+// per row and chunk), MXFP4 2 (8 bytes; the upper bytes of the word are unused).
+template <bool NV>
+__device__ __forceinline__ uint32_t bs_sf_word(const uint8_t* row, int kb) {
+  if (NV) return reinterpret_cast<const uint32_t*>(row)[kb];
+  return (uint32_t)reinterpret_cast<const uint16_t*>(row)[kb];
 }
 __device__ __forceinline__ void bs_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
@@ -292,16 +345,18 @@ __device__ __forceinline__ void bs_tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) 
       : "memory");
 }
 
-// Instruction descriptor, kind::mxf4nvf4: A and B E2M1 (K-major), E8M0 scales, M = 128,
-// N = 256, K = 64 per instruction, scale factor ids 0.
-constexpr uint32_t kBsIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(kBsN >> 3) << 17) | (1u << 23) |
-                              ((uint32_t)(kBsM >> 4) << 24);
 
 __device__ __forceinline__ float bs_scale_pow2(float v, int e) {
   return (e >= -126 && e <= 127) ? v * __int_as_float((e + 127) << 23) : ldexpf(v, e);
 }
 
+template <bool NV>
 __global__ void __launch_bounds__(kBsThreads, 1) qgemm_bs_kernel(const __grid_constant__ BsParams p) {
+  using L = BsLay<NV>;
+  constexpr int kBsStage = L::Stage;
+  constexpr int kBsAScales = L::AScales;
+  constexpr int kBsSBlock = L::SB;
+  constexpr int kSbr = bs_sbr(NV);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sbase = smem_u32(smem);
@@ -418,7 +473,7 @@ __global__ void __launch_bounds__(kBsThreads, 1) qgemm_bs_kernel(const __grid_co
 #pragma unroll
             for (int t = 0; t < kBsTerms; ++t) {
               const uint64_t adesc = smem_desc_sw128(st + (uint32_t)(t * kBsBlock)) + (uint64_t)(kb * 2);
-              bs_mma(tmem, adesc, bdesc0 + (uint64_t)(kb * 2), kBsIdesc,
+              bs_mma<NV>(tmem, adesc, bdesc0 + (uint64_t)(kb * 2), L::Idesc,
                      sf0 + (uint32_t)((t * 4 + kb) * 4), sf0 + (uint32_t)(48 + kb * 4 * kBsWT),
                      (c | kb | t) != 0 ? 1u : 0u);
             }
@@ -457,27 +512,21 @@ __global__ void __launch_bounds__(kBsThreads, 1) qgemm_bs_kernel(const __grid_co
         tc_fence_after();
         const uint8_t* st = smem + sp.slot * kBsStage;
         const uint8_t* sa = st + kBsACodes + kBsBCodes;  // x-term scales [3][128][8]
-        const uint8_t* sb = sa + kBsAScales;              // weight scales [kBsWT][128][8]
+        const uint8_t* sb = sa + kBsAScales;              // weight scales [kBsWT][128][sbr]
         uint32_t v[kBsSfCols];
 #pragma unroll
         for (int t = 0; t < kBsTerms; ++t)
 #pragma unroll
           for (int r1 = 0; r1 < 4; ++r1) {
-            const uint2 s8 = *reinterpret_cast<const uint2*>(sa + t * kBsSBlock + (r1 * 32 + lane) * 8);
+            const uint8_t* row = sa + t * kBsSBlock + (r1 * 32 + lane) * kSbr;
 #pragma unroll
-            for (int kb = 0; kb < 4; ++kb) {
-              const uint32_t w = (kb < 2) ? s8.x : s8.y;
-              v[(t * 4 + kb) * 4 + r1] = (w >> ((kb & 1) * 16)) & 0xFFFFu;
-            }
+            for (int kb = 0; kb < 4; ++kb) v[(t * 4 + kb) * 4 + r1] = bs_sf_word<NV>(row, kb);
           }
 #pragma unroll
         for (int r1 = 0; r1 < 4 * kBsWT; ++r1) {
-          const uint2 s8 = *reinterpret_cast<const uint2*>(sb + (r1 >> 2) * kBsSBlock + ((r1 & 3) * 32 + lane) * 8);
+          const uint8_t* row = sb + (r1 >> 2) * kBsSBlock + ((r1 & 3) * 32 + lane) * kSbr;
 #pragma unroll
-          for (int kb = 0; kb < 4; ++kb) {
-            const uint32_t w = (kb < 2) ? s8.x : s8.y;
-            v[48 + kb * 4 * kBsWT + r1] = (w >> ((kb & 1) * 16)) & 0xFFFFu;
-          }
+          for (int kb = 0; kb < 4; ++kb) v[48 + kb * 4 * kBsWT + r1] = bs_sf_word<NV>(row, kb);
         }
         const uint32_t ta = tmem + lane_base + (uint32_t)(kBsN + sp.slot * kBsSfCols);
 #pragma unroll
@@ -501,6 +550,9 @@ __global__ void __launch_bounds__(kBsThreads, 1) qgemm_bs_kernel(const __grid_co
       const int mt = u % p.Mt, nt = u / p.Mt;
       const int m = mt * kBsM + q * 32 + lane;
       const int xe = (m < p.M) ? p.x_exp[m] : 0;
+      const float tsv = NV ? __ldg(p.ts) : 1.0f;  // NVFP4 tensor scale, applied before 2^xe
+      // y = (acc * ts) * 2^xe: the tensor scale (NVFP4) rounds once, the power of two is exact
+      auto yv = [&](uint32_t u) { return bs_scale_pow2(NV ? __uint_as_float(u) * tsv : __uint_as_float(u), xe); };
       bool ok = mbar_wait(bar_acc, (uint32_t)ti & 1u, abort_flag, p.dev_err, kErrTimeout);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
@@ -520,8 +572,8 @@ __global__ void __launch_bounds__(kBsThreads, 1) qgemm_bs_kernel(const __grid_co
                 uint32_t w[4];
 #pragma unroll
                 for (int h = 0; h < 4; ++h) {
-                  const __nv_bfloat16 lo = __float2bfloat16_rn(bs_scale_pow2(__uint_as_float(v[i + 2 * h]), xe));
-                  const __nv_bfloat16 hi = __float2bfloat16_rn(bs_scale_pow2(__uint_as_float(v[i + 2 * h + 1]), xe));
+                  const __nv_bfloat16 lo = __float2bfloat16_rn(yv(v[i + 2 * h]));
+                  const __nv_bfloat16 hi = __float2bfloat16_rn(yv(v[i + 2 * h + 1]));
                   w[h] = (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
                 }
                 *reinterpret_cast<uint4*>(yr + i) = make_uint4(w[0], w[1], w[2], w[3]);
@@ -529,7 +581,7 @@ __global__ void __launch_bounds__(kBsThreads, 1) qgemm_bs_kernel(const __grid_co
             } else {
 #pragma unroll
               for (int i = 0; i < 32; ++i)
-                if (n0 + i < p.N) yr[i] = __float2bfloat16_rn(bs_scale_pow2(__uint_as_float(v[i]), xe));
+                if (n0 + i < p.N) yr[i] = __float2bfloat16_rn(yv(v[i]));
             }
           } else {
             float* yr = reinterpret_cast<float*>(p.out) + (size_t)m * p.N + n0;
@@ -537,12 +589,12 @@ __global__ void __launch_bounds__(kBsThreads, 1) qgemm_bs_kernel(const __grid_co
 #pragma unroll
               for (int i = 0; i < 32; i += 4)
                 *reinterpret_cast<float4*>(yr + i) =
-                    make_float4(bs_scale_pow2(__uint_as_float(v[i]), xe), bs_scale_pow2(__uint_as_float(v[i + 1]), xe),
-                                bs_scale_pow2(__uint_as_float(v[i + 2]), xe), bs_scale_pow2(__uint_as_float(v[i + 3]), xe));
+                    make_float4(yv(v[i]), yv(v[i + 1]),
+                                yv(v[i + 2]), yv(v[i + 3]));
             } else {
 #pragma unroll
               for (int i = 0; i < 32; ++i)
-                if (n0 + i < p.N) yr[i] = bs_scale_pow2(__uint_as_float(v[i]), xe);
+                if (n0 + i < p.N) yr[i] = yv(v[i]);
             }
           }
         }
@@ -588,13 +640,17 @@ struct BsDecParams {
   const int* x_exp;
   const uint8_t* wcodes;
   const uint8_t* wscales;
+  const float* ts;  // NVFP4 tensor scale (device), else nullptr
   float* ws;  // S > 1: partials [S][M][N], fully scaled
   void* out;
   int out_bf16;
   int* dev_err;
 };
 
+template <bool NV>
 __global__ void __launch_bounds__(kBdThreads, 1) qgemm_bs_dec_kernel(const __grid_constant__ BsDecParams p) {
+  constexpr int kSbr = bs_sbr(NV);
+  constexpr int kSBlock = kBsM * kSbr;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sbase = smem_u32(smem);
@@ -612,8 +668,8 @@ __global__ void __launch_bounds__(kBdThreads, 1) qgemm_bs_dec_kernel(const __gri
   const int Nb = p.Nb;
   const uint32_t xterm = (uint32_t)Nb * 128u;      // one term's codes in a stage
   const uint32_t off_ws = kBsBlock + kBsTerms * xterm;            // weight scales
-  const uint32_t off_xs = off_ws + kBsSBlock;                     // term scales
-  const uint32_t idesc = (1u << 7) | (1u << 10) | ((uint32_t)(Nb >> 3) << 17) | (1u << 23) |
+  const uint32_t off_xs = off_ws + kSBlock;                       // term scales
+  const uint32_t idesc = (1u << 7) | (1u << 10) | ((uint32_t)(Nb >> 3) << 17) | ((NV ? 0u : 1u) << 23) |
                          ((uint32_t)(kBsM >> 4) << 24);
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < NST; ++s) {
@@ -664,10 +720,10 @@ __global__ void __launch_bounds__(kBdThreads, 1) qgemm_bs_dec_kernel(const __gri
           }
           const uint32_t fb = bar_full + 8 * sp.slot;
           const uint32_t st = sbase + (uint32_t)(sp.slot * p.stage_bytes);
-          mbar_arrive_expect_tx(fb, kBsBlock + kBsSBlock + kBsTerms * (xterm + (uint32_t)Nb * 8u));
+          mbar_arrive_expect_tx(fb, kBsBlock + kSBlock + kBsTerms * (xterm + (uint32_t)(Nb * kSbr)));
           const int64_t blk = (int64_t)t * p.C + c;
           bulk_load(st, p.wcodes + blk * kBsBlock, kBsBlock, fb, pol_w);
-          bulk_load(st + off_ws, p.wscales + blk * kBsSBlock, kBsSBlock, fb, pol_w);
+          bulk_load(st + off_ws, p.wscales + blk * kSBlock, kSBlock, fb, pol_w);
           if (!waited) {
             griddep_wait();  // the split x comes from the preceding grid
             waited = true;
@@ -675,7 +731,7 @@ __global__ void __launch_bounds__(kBdThreads, 1) qgemm_bs_dec_kernel(const __gri
           for (int j = 0; j < kBsTerms; ++j) {
             const int64_t xb = (int64_t)c * kBsTerms + j;  // token tile 0
             bulk_load(st + kBsBlock + (uint32_t)j * xterm, p.xcodes + xb * kBsBlock, xterm, fb, pol_x);
-            bulk_load(st + off_xs + (uint32_t)(j * Nb * 8), p.xscales + xb * kBsSBlock, (uint32_t)Nb * 8u, fb, pol_x);
+            bulk_load(st + off_xs + (uint32_t)(j * Nb * kSbr), p.xscales + xb * kSBlock, (uint32_t)(Nb * kSbr), fb, pol_x);
           }
           sp.next(NST);
           ++issued;
@@ -726,7 +782,7 @@ __global__ void __launch_bounds__(kBdThreads, 1) qgemm_bs_dec_kernel(const __gri
 #pragma unroll
             for (int j = 0; j < kBsTerms; ++j) {
               const uint64_t bdesc = smem_desc_sw128(st + kBsBlock + (uint32_t)j * xterm) + (uint64_t)(kb * 2);
-              bs_mma(d, adesc0 + (uint64_t)(kb * 2), bdesc, idesc, sf0 + (uint32_t)(kb * 4),
+              bs_mma<NV>(d, adesc0 + (uint64_t)(kb * 2), bdesc, idesc, sf0 + (uint32_t)(kb * 4),
                      sf0 + (uint32_t)(16 + (j * 4 + kb) * 4), (c - c0 >= 2 || kb || j) ? 1u : 0u);
             }
           }
@@ -766,20 +822,19 @@ __global__ void __launch_bounds__(kBdThreads, 1) qgemm_bs_dec_kernel(const __gri
         uint32_t v[kBdSfCols];
 #pragma unroll
         for (int r1 = 0; r1 < 4; ++r1) {
-          const uint2 s8 = *reinterpret_cast<const uint2*>(st + off_ws + (r1 * 32 + lane) * 8);
+          const uint8_t* row = st + off_ws + (r1 * 32 + lane) * kSbr;
 #pragma unroll
-          for (int kb = 0; kb < 4; ++kb) v[kb * 4 + r1] = (((kb < 2) ? s8.x : s8.y) >> ((kb & 1) * 16)) & 0xFFFFu;
+          for (int kb = 0; kb < 4; ++kb) v[kb * 4 + r1] = bs_sf_word<NV>(row, kb);
         }
 #pragma unroll
         for (int j = 0; j < kBsTerms; ++j)
 #pragma unroll
           for (int r1 = 0; r1 < 4; ++r1) {
-            const int row = r1 * 32 + lane;
-            uint2 s8 = make_uint2(0u, 0u);
-            if (row < Nb) s8 = *reinterpret_cast<const uint2*>(st + off_xs + j * Nb * 8 + row * 8);
+            const int rw = r1 * 32 + lane;
+            const uint8_t* row = st + off_xs + j * Nb * kSbr + rw * kSbr;
 #pragma unroll
             for (int kb = 0; kb < 4; ++kb)
-              v[16 + (j * 4 + kb) * 4 + r1] = (((kb < 2) ? s8.x : s8.y) >> ((kb & 1) * 16)) & 0xFFFFu;
+              v[16 + (j * 4 + kb) * 4 + r1] = rw < Nb ? bs_sf_word<NV>(row, kb) : 0u;
           }
         const uint32_t ta = tmem + lane_base + sf_col0 + (uint32_t)(sp.slot * kBdSfCols);
 #pragma unroll
@@ -800,6 +855,7 @@ __global__ void __launch_bounds__(kBdThreads, 1) qgemm_bs_dec_kernel(const __gri
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     griddep_wait();  // x_exp comes from the split kernel
     const size_t MN = (size_t)p.M * p.N;
+    const float tsv = NV ? __ldg(p.ts) : 1.0f;  // NVFP4 tensor scale, applied before 2^x_exp
     int ti = 0;
     for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++ti) {
       int t, s, c0, c1;
@@ -828,7 +884,8 @@ __global__ void __launch_bounds__(kBdThreads, 1) qgemm_bs_dec_kernel(const __gri
           for (int i = 0; i < 16; ++i) {
             const int b = cb + i;
             if (b < p.M) {
-              const float val = bs_scale_pow2(__uint_as_float(v[i]), __ldg(p.x_exp + b));
+              const float acc = NV ? __uint_as_float(v[i]) * tsv : __uint_as_float(v[i]);
+              const float val = bs_scale_pow2(acc, __ldg(p.x_exp + b));
               if (p.S > 1) p.ws[(size_t)s * MN + (size_t)b * p.N + n] = val;
               else if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)b * p.N + n] = __float2bfloat16_rn(val);
               else reinterpret_cast<float*>(p.out)[(size_t)b * p.N + n] = val;
@@ -854,14 +911,15 @@ __global__ void __launch_bounds__(kBdThreads, 1) qgemm_bs_dec_kernel(const __gri
 // ---------------------------------------------------------------------------------------
 // Launchers
 // ---------------------------------------------------------------------------------------
-cudaError_t launch_bs_split(const uint16_t* x, int M, int K, uint8_t* codes, uint8_t* scales,
-                            int* x_exp, cudaStream_t stream) {
+cudaError_t launch_bs_split(bool nv, const uint16_t* x, int M, int K, uint8_t* codes,
+                            uint8_t* scales, int* x_exp, cudaStream_t stream) {
   BsSplitParams p{};
   p.x = x;
   p.M = M;
   p.K = K;
   p.C = (K + kBsK - 1) / kBsK;
   p.Mt = (M + kBsM - 1) / kBsM;
+  p.nv = nv ? 1 : 0;
   p.codes = codes;
   p.scales = scales;
   p.x_exp = x_exp;
@@ -887,19 +945,36 @@ static int bs_sm_count(int dev) {
   return v;
 }
 
-cudaError_t launch_bs_gemm(int M, int N, int K, const uint8_t* xcodes, const uint8_t* xscales,
-                           const int* x_exp, const uint8_t* wcodes, const uint8_t* wscales,
-                           void* out, int out_bf16, int* dev_err, cudaStream_t stream) {
+// Raises a kernel's dynamic shared-memory limit once per device (devices beyond 64 on every
+// launch); one mask per kernel instantiation.
+static cudaError_t bs_smem_attr(const void* fn, std::atomic<uint64_t>& mask, int dev, int bytes) {
+  const uint64_t bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+  if (bit != 0 && (mask.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) mask.fetch_or(bit, std::memory_order_release);
+  return e;
+}
+
+static cudaError_t bs_launch_pdl(cudaLaunchConfig_t& cfg, cudaStream_t stream, cudaLaunchAttribute* at) {
+  cfg.stream = stream;
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaSuccess;
+}
+
+template <bool NV>
+static cudaError_t launch_bs_gemm_t(int M, int N, int K, const uint8_t* xcodes,
+                                    const uint8_t* xscales, const int* x_exp, const uint8_t* wcodes,
+                                    const uint8_t* wscales, const float* ts, void* out,
+                                    int out_bf16, int* dev_err, cudaStream_t stream) {
   static std::atomic<uint64_t> set_mask{0};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  const uint64_t bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
-  if (bit == 0 || !(set_mask.load(std::memory_order_acquire) & bit)) {
-    e = cudaFuncSetAttribute(qgemm_bs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kBsSmem);
-    if (e != cudaSuccess) return e;
-    set_mask.fetch_or(bit, std::memory_order_release);
-  }
+  e = bs_smem_attr((const void*)qgemm_bs_kernel<NV>, set_mask, dev, BsLay<NV>::Smem);
+  if (e != cudaSuccess) return e;
   BsParams p{};
   p.M = M;
   p.N = N;
@@ -913,21 +988,27 @@ cudaError_t launch_bs_gemm(int M, int N, int K, const uint8_t* xcodes, const uin
   p.x_exp = x_exp;
   p.wcodes = wcodes;
   p.wscales = wscales;
+  p.ts = ts;
   p.out = out;
   p.out_bf16 = out_bf16;
   p.dev_err = dev_err;
-  const int sms = bs_sm_count(dev);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)std::min(p.units, sms), 1, 1);
+  cfg.gridDim = dim3((unsigned)std::min(p.units, bs_sm_count(dev)), 1, 1);
   cfg.blockDim = dim3(kBsThreads, 1, 1);
-  cfg.dynamicSmemBytes = kBsSmem;
-  cfg.stream = stream;
+  cfg.dynamicSmemBytes = BsLay<NV>::Smem;
   cudaLaunchAttribute at[1];
-  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  at[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = at;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, qgemm_bs_kernel, p);
+  bs_launch_pdl(cfg, stream, at);
+  return cudaLaunchKernelEx(&cfg, qgemm_bs_kernel<NV>, p);
+}
+
+cudaError_t launch_bs_gemm(bool nv, int M, int N, int K, const uint8_t* xcodes,
+                           const uint8_t* xscales, const int* x_exp, const uint8_t* wcodes,
+                           const uint8_t* wscales, const float* ts, void* out, int out_bf16,
+                           int* dev_err, cudaStream_t stream) {
+  return nv ? launch_bs_gemm_t<true>(M, N, K, xcodes, xscales, x_exp, wcodes, wscales, ts, out,
+                                     out_bf16, dev_err, stream)
+            : launch_bs_gemm_t<false>(M, N, K, xcodes, xscales, x_exp, wcodes, wscales, ts, out,
+                                      out_bf16, dev_err, stream);
 }
 
 // K split of the decode kernel: a function of (N, K) only (the unit count is weighed against
@@ -951,11 +1032,11 @@ int bs_dec_split(int64_t N, int64_t K, int sms) {
 
 // Workspace of the block-scaled path: split codes, split scales, row exponents and, for
 // decode widths with a K split, the fp32 partials.
-size_t bs_workspace_bytes(int64_t M, int64_t N, int64_t K, size_t* off_scales, size_t* off_exp,
-                          size_t* off_part) {
+size_t bs_workspace_bytes(bool nv, int64_t M, int64_t N, int64_t K, size_t* off_scales,
+                          size_t* off_exp, size_t* off_part) {
   const int64_t C = (K + kBsK - 1) / kBsK, Mt = (M + kBsM - 1) / kBsM;
   const size_t codes = (size_t)(Mt * C * kBsTerms) * kBsBlock;
-  const size_t scales = (size_t)(Mt * C * kBsTerms) * kBsSBlock;
+  const size_t scales = (size_t)(Mt * C * kBsTerms) * (size_t)(kBsM * bs_sbr(nv));
   if (off_scales) *off_scales = codes;
   if (off_exp) *off_exp = codes + scales;
   size_t total = codes + scales + (size_t)Mt * kBsM * 4;
@@ -970,30 +1051,27 @@ size_t bs_workspace_bytes(int64_t M, int64_t N, int64_t K, size_t* off_scales, s
 
 cudaError_t launch_reduce(const ReduceParams& rp, cudaStream_t stream);
 
-// Decode widths: returns cudaSuccess after queuing the GEMM (and the reduce when S > 1).
-cudaError_t launch_bs_dec(int M, int N, int K, const uint8_t* xcodes, const uint8_t* xscales,
-                          const int* x_exp, const uint8_t* wcodes, const uint8_t* wscales,
-                          float* part, void* out, int out_bf16, int* dev_err, cudaStream_t stream) {
+template <bool NV>
+static cudaError_t launch_bs_dec_t(int M, int N, int K, const uint8_t* xcodes,
+                                   const uint8_t* xscales, const int* x_exp, const uint8_t* wcodes,
+                                   const uint8_t* wscales, const float* ts, float* part, void* out,
+                                   int out_bf16, int* dev_err, cudaStream_t stream) {
   static std::atomic<uint64_t> set_mask{0};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  const uint64_t bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
-  if (bit == 0 || !(set_mask.load(std::memory_order_acquire) & bit)) {
-    e = cudaFuncSetAttribute(qgemm_bs_dec_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
-    if (e != cudaSuccess) return e;
-    set_mask.fetch_or(bit, std::memory_order_release);
-  }
+  e = bs_smem_attr((const void*)qgemm_bs_dec_kernel<NV>, set_mask, dev, kSmemLimit);
+  if (e != cudaSuccess) return e;
+  constexpr int kSbr = bs_sbr(NV);
   BsDecParams p{};
   p.M = M;
   p.N = N;
   p.K = K;
   p.C = (K + kBsK - 1) / kBsK;
   p.Nb = (M + 15) / 16 * 16;
-  const int sms = bs_sm_count(dev);
   p.S = bs_dec_split(N, K, kBsSplitSMs);
   p.units = (int)row_tiles(N) * p.S;
-  p.stage_bytes = (kBsBlock + kBsTerms * p.Nb * 128 + kBsSBlock + kBsTerms * p.Nb * 8 + 1023) / 1024 * 1024;
+  p.stage_bytes = (kBsBlock + kBsTerms * p.Nb * 128 + kBsM * kSbr + kBsTerms * p.Nb * kSbr + 1023) / 1024 * 1024;
   p.stages = std::min({kBdMaxStages, (kSmemLimit - 1024 - 256) / p.stage_bytes,
                        (kBsTmemCols - 2 * p.Nb) / kBdSfCols}) & ~1;  // even
   if (p.stages < 2) return cudaErrorInvalidValue;
@@ -1002,22 +1080,18 @@ cudaError_t launch_bs_dec(int M, int N, int K, const uint8_t* xcodes, const uint
   p.x_exp = x_exp;
   p.wcodes = wcodes;
   p.wscales = wscales;
+  p.ts = ts;
   p.ws = part;
   p.out = out;
   p.out_bf16 = out_bf16;
   p.dev_err = dev_err;
-  const size_t smem = 1024 + (size_t)p.stages * p.stage_bytes + 256;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)std::min(p.units, sms), 1, 1);
+  cfg.gridDim = dim3((unsigned)std::min(p.units, bs_sm_count(dev)), 1, 1);
   cfg.blockDim = dim3(kBdThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
+  cfg.dynamicSmemBytes = 1024 + (size_t)p.stages * p.stage_bytes + 256;
   cudaLaunchAttribute at[1];
-  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  at[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = at;
-  cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, qgemm_bs_dec_kernel, p);
+  bs_launch_pdl(cfg, stream, at);
+  e = cudaLaunchKernelEx(&cfg, qgemm_bs_dec_kernel<NV>, p);
   if (e != cudaSuccess || p.S == 1) return e;
   ReduceParams rp{};
   rp.ws = part;
@@ -1028,6 +1102,17 @@ cudaError_t launch_bs_dec(int M, int N, int K, const uint8_t* xcodes, const uint
   rp.out = out;
   rp.out_bf16 = out_bf16;
   return launch_reduce(rp, stream);
+}
+
+// Decode widths: queues the GEMM (and the split-K reduce when S > 1).
+cudaError_t launch_bs_dec(bool nv, int M, int N, int K, const uint8_t* xcodes,
+                          const uint8_t* xscales, const int* x_exp, const uint8_t* wcodes,
+                          const uint8_t* wscales, const float* ts, float* part, void* out,
+                          int out_bf16, int* dev_err, cudaStream_t stream) {
+  return nv ? launch_bs_dec_t<true>(M, N, K, xcodes, xscales, x_exp, wcodes, wscales, ts, part,
+                                    out, out_bf16, dev_err, stream)
+            : launch_bs_dec_t<false>(M, N, K, xcodes, xscales, x_exp, wcodes, wscales, ts, part,
+                                     out, out_bf16, dev_err, stream);
 }
 
 }  // namespace qg

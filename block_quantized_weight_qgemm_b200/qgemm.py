@@ -50,9 +50,9 @@ SIGNATURES = [
                            _SZ, _VP]),
     ("qgemm_moe_gate_up", _I, [_I, _VP, _I64, _I64, _I, _VP, _I64, _VP, _VP, _VP, _VP, _VP, _VP,
                                _I64, _VP, _VP, _SZ, _VP]),
-    ("qgemm_bs_split_size", _I, [_I64, _I64, ctypes.POINTER(_SZ), ctypes.POINTER(_SZ),
+    ("qgemm_bs_split_size", _I, [_I, _I64, _I64, ctypes.POINTER(_SZ), ctypes.POINTER(_SZ),
                                  ctypes.POINTER(_SZ)]),
-    ("qgemm_bs_split_x", _I, [_VP, _I64, _I64, _VP, _VP, _VP, _VP]),
+    ("qgemm_bs_split_x", _I, [_I, _VP, _I64, _I64, _VP, _VP, _VP, _VP]),
     ("qgemm_bs_workspace_size", _I, [_I, _I64, _I64, _I64, ctypes.POINTER(_SZ)]),
     ("qgemm_bs_run", _I, [_I, _VP, _I64, _I64, _VP, _VP, _VP, _I64, _VP, _I, _VP, _SZ, _VP]),
     ("qgemm_split_k", _I, [_I, _I64, _I64, ctypes.POINTER(_I)]),
@@ -230,25 +230,26 @@ def run(x: torch.Tensor, pw: PackedWeight, y: torch.Tensor | None = None, y_dtyp
     return y
 
 
-def bs_split_size(M: int, K: int) -> tuple[int, int, int]:
-    """qgemm_bs_split_size: (code bytes, scale bytes, exponent bytes) of the split of x."""
+def bs_split_size(fmt, M: int, K: int) -> tuple[int, int, int]:
+    """qgemm_bs_split_size: (code bytes, scale bytes, exponent bytes) of the split of x for
+    weight format fmt (MXFP4 or NVFP4)."""
     c, sc, e = _SZ(), _SZ(), _SZ()
-    _check(lib().qgemm_bs_split_size(M, K, ctypes.byref(c), ctypes.byref(sc), ctypes.byref(e)),
-           "qgemm_bs_split_size")
+    _check(lib().qgemm_bs_split_size(_fmt(fmt), M, K, ctypes.byref(c), ctypes.byref(sc),
+                                     ctypes.byref(e)), "qgemm_bs_split_size")
     return c.value, sc.value, e.value
 
 
-def bs_split_x(x: torch.Tensor, stream=None):
+def bs_split_x(x: torch.Tensor, fmt="mxfp4", stream=None):
     """qgemm_bs_split_x: x bf16 [M, K] -> (codes u8, scales u8, x_exp int32) in the layout of
-    include/qgemm.h (three E2M1 terms per row with E8M0 scales per 32 elements)."""
+    include/qgemm.h (three E2M1 terms per row with the weight format's block scales)."""
     assert x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous() and x.dim() == 2
     M, K = x.shape
-    nc, ns, ne = bs_split_size(M, K)
+    nc, ns, ne = bs_split_size(fmt, M, K)
     codes = torch.empty(nc, dtype=torch.uint8, device=x.device)
     scales = torch.empty(ns, dtype=torch.uint8, device=x.device)
     x_exp = torch.empty(ne // 4, dtype=torch.int32, device=x.device)
-    _check(lib().qgemm_bs_split_x(_ptr(x), M, K, _ptr(codes), _ptr(scales), _ptr(x_exp),
-                                  _stream(stream)), "qgemm_bs_split_x")
+    _check(lib().qgemm_bs_split_x(_fmt(fmt), _ptr(x), M, K, _ptr(codes), _ptr(scales),
+                                  _ptr(x_exp), _stream(stream)), "qgemm_bs_split_x")
     return codes, scales, x_exp
 
 
@@ -260,7 +261,7 @@ def bs_workspace_size(fmt: int, N: int, K: int, M: int) -> int:
 
 def bs_run(x: torch.Tensor, pw: PackedWeight, y: torch.Tensor | None = None, y_dtype=torch.float32,
            workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """qgemm_bs_run: the block-scaled path (MXFP4 weights): x bf16 [M, K] -> y [M, N]."""
+    """qgemm_bs_run: the block-scaled path (MXFP4 or NVFP4 weights): x bf16 [M, K] -> y [M, N]."""
     assert x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous() and x.dim() == 2
     M, K = x.shape
     assert K == pw.K

@@ -262,38 +262,47 @@ int qgemm_moe_gate_up(int fmt, const void* x_dev, int64_t M, int64_t K, int E,
                       void* stream);
 
 /*
- * Block-scaled path for MXFP4 weights (tcgen05.mma.kind::mxf4nvf4 with 32-element E8M0
- * block scales on both operands; the packed weights feed the tensor cores without a
+ * Block-scaled path for MXFP4 and NVFP4 weights (tcgen05.mma.kind::mxf4nvf4 with block
+ * scales on both operands; the packed weights feed the tensor cores without a
  * dequantisation pass), with the activations quantised on the fly (Atlas issue, kernel-ranking
- * section: a block-scaled MMA path for prefill).  x is split per row into three E2M1 terms
- * with their own E8M0 scale per 32 elements,
- *   x_exp = floor(log2 max|x_row|),  r_0 = x * 2^-x_exp,
- *   e_j = floor(log2 max_block |r_j|) - 2,  q_j = E2M1_RNE_sat(r_j / 2^e_j),
- *   r_{j+1} = r_j - q_j 2^e_j   (j = 0, 1, 2),
- * and y = 2^x_exp * sum_j (q_j 2^e_j) W^T, accumulated in fp32.  A term whose e_j would be
- * below -127 is dropped (zero codes, scale byte 0).  The result differs from qgemm_run by the
- * split's residual (measured normalised error below 1e-4 at the 27B shapes); it is a separate
- * entry point, not a mode of qgemm_run.
+ * section: a block-scaled MMA path for prefill).  x is split per row into three E2M1 terms with
+ * a power-of-two scale per block, in the weight format's scale type:
+ *   MXFP4: 32-element blocks, E8M0 scales, xshift 0, emin -127;
+ *   NVFP4: 16-element blocks, UE4M3 scales (powers of two 2^-9 .. 2^8 only), xshift 10,
+ *          emin -9;
+ *   x_exp = floor(log2 max|x_row|) - xshift,  r_0 = x * 2^-x_exp,
+ *   e_j = floor(log2 max_block |r_j|) - 2  (a term with e_j < emin and the later ones are
+ *   dropped: zero codes, scale 0),  q_j = E2M1_RNE_sat(r_j / 2^e_j),  r_{j+1} = r_j - q_j 2^e_j
+ *   for j = 0, 1, 2,
+ * and y = 2^x_exp * (sum_j (q_j 2^e_j) W^T) [* tensor scale for NVFP4], accumulated in fp32.
+ * The result differs from qgemm_run by the split's residual (measured normalised error below
+ * 2e-4 at the 27B shapes); it is a separate entry point, not a mode of qgemm_run.  Up to 128
+ * rows the weights are the MMA M operand and K is split over the SMs by a rule of (N, K)
+ * alone (fp32 partials summed in a fixed order); above that x is.
  *
- * qgemm_bs_split_size / qgemm_bs_split_x: the split alone.  Layout (device, caller-owned,
- * 16-byte aligned), with Mt = ceil(M/128), C = ceil(K/256):
+ * qgemm_bs_split_size / qgemm_bs_split_x: the split alone, for fmt MXFP4 or NVFP4.  Layout
+ * (device, caller-owned, 16-byte aligned), with Mt = ceil(M/128), C = ceil(K/256),
+ * sbr = 8 (MXFP4) or 16 (NVFP4):
  *   codes  [Mt][C][3][128][128] bytes: row r of block (t, c, j) holds elements
  *          256c .. 256c+255 of row 128t + r of term j, two per byte (even element in the
  *          low nibble), its 16-byte groups stored at group ^ (r & 7).  Rows past M and
  *          elements past K are zero.
- *   scales [Mt][C][3][128][8] E8M0 bytes (bias 127), one per 32 elements.
+ *   scales [Mt][C][3][128][sbr] scale bytes (E8M0 bias 127; UE4M3 bias 7), one per block.
  *   x_exp  [Mt*128] int32 (0 for rows past M and all-zero rows).
- * K must be a multiple of 32.  Errors: QGEMM_ERR_SHAPE, _K_BLOCK, _NULL, _ALIGN, _DEVICE, _CUDA.
+ * K must be a multiple of 32.  Errors: QGEMM_ERR_FORMAT, _SHAPE, _K_BLOCK, _NULL, _ALIGN,
+ * _DEVICE, _CUDA.
  */
-int qgemm_bs_split_size(int64_t M, int64_t K, size_t* code_bytes, size_t* scale_bytes,
+int qgemm_bs_split_size(int fmt, int64_t M, int64_t K, size_t* code_bytes, size_t* scale_bytes,
                         size_t* exp_bytes);
-int qgemm_bs_split_x(const void* x_dev, int64_t M, int64_t K, void* codes_dev, void* scales_dev,
-                     int32_t* x_exp_dev, void* stream);
+int qgemm_bs_split_x(int fmt, const void* x_dev, int64_t M, int64_t K, void* codes_dev,
+                     void* scales_dev, int32_t* x_exp_dev, void* stream);
 
 /*
  * qgemm_bs_workspace_size / qgemm_bs_run: y[M][N] = x W^T on the block-scaled path.  fmt must
- * be QGEMM_FMT_MXFP4 (else QGEMM_ERR_FORMAT); the other arguments as for qgemm_run, with M
- * the number of x rows.  The workspace (qgemm_bs_workspace_size bytes) holds the split of x.
+ * be QGEMM_FMT_MXFP4 or QGEMM_FMT_NVFP4 (else QGEMM_ERR_FORMAT; NVFP4 needs its tensor scale);
+ * the other arguments as for qgemm_run, with M the number of x rows.  The workspace
+ * (qgemm_bs_workspace_size bytes) holds the split of x and, up to 128 rows, the K-split
+ * partials.
  */
 int qgemm_bs_workspace_size(int fmt, int64_t N, int64_t K, int64_t M, size_t* bytes);
 int qgemm_bs_run(int fmt, const void* x_dev, int64_t M, int64_t K, const void* codes_dev,

@@ -1,9 +1,9 @@
-"""GPU parity of the block-scaled MXFP4 path (qgemm_bs_split_x / qgemm_bs_run) against the CPU
-oracle, through the C ABI.
+"""GPU parity of the block-scaled path for MXFP4 and NVFP4 weights (qgemm_bs_split_x /
+qgemm_bs_run) against the CPU oracle, through the C ABI.
 
 Bars:
   * the split of x is exact: the sum of the three E2M1 terms the GPU writes (decoded on the
-    host from the layout of include/qgemm.h) equals oracle.split_x bit for bit;
+    host from the layout of include/qgemm.h) equals oracle.split_x_bs bit for bit;
   * the GEMM is the product of that split with the dequantised weights up to fp32
     accumulation (normalised error 2e-5), and within the method's 1e-3 of the exact product
     at K >= 1024 (the split's own residual is measured in the oracle pins);
@@ -35,10 +35,13 @@ def _lib():
     assert qgemm.device_status(reset=True) == qgemm.OK
 
 
-def _decode_split(codes, scales, x_exp, M, K):
+def _decode_split(fmt, codes, scales, x_exp, M, K):
     """Sum of the three terms per element, from the documented layout (numpy only)."""
     C, Mt = -(-K // 256), -(-M // 128)
+    blk, sbr = (16, 16) if fmt == "nvfp4" else (32, 8)
     vals = np.array([oracle.e2m1(c) for c in range(16)])
+    svals = (np.array([oracle.e4m3(b) if b < 0x7F else 0.0 for b in range(256)]) if fmt == "nvfp4"
+             else np.exp2(np.arange(256, dtype=np.float64) - 127.0))
     cb = codes.reshape(Mt, C, 3, 128, 8, 16)
     un = np.empty_like(cb)
     for r in range(128):
@@ -46,8 +49,8 @@ def _decode_split(codes, scales, x_exp, M, K):
             un[:, :, :, r, g, :] = cb[:, :, :, r, g ^ (r & 7), :]
     un = un.reshape(Mt, C, 3, 128, 128)
     el = np.stack([un & 15, un >> 4], axis=-1).reshape(Mt, C, 3, 128, 256)
-    sc = scales.reshape(Mt, C, 3, 128, 8).astype(np.float64)
-    val = vals[el] * np.repeat(np.exp2(sc - 127.0), 32, axis=-1)
+    sc = scales.reshape(Mt, C, 3, 128, sbr)
+    val = vals[el] * np.repeat(svals[sc], blk, axis=-1)
     tot = val.sum(axis=2).transpose(0, 2, 1, 3).reshape(Mt * 128, C * 256)
     return tot, tot[:M, :K] * np.exp2(x_exp[:M].astype(np.float64))[:, None]
 
@@ -67,14 +70,18 @@ def _special_rows(x: torch.Tensor) -> torch.Tensor:
     return x
 
 
+FMTS = ["mxfp4", "nvfp4"]
+
+
+@pytest.mark.parametrize("fmt", FMTS)
 @pytest.mark.parametrize("M,K", [(1, 32), (130, 288), (257, 1024), (200, 5120)])
-def test_split_bit_exact(M, K):
+def test_split_bit_exact(fmt, M, K):
     x = _special_rows(inputs.activations(M, K, seed=20 + M))
-    codes, scales, x_exp = qgemm.bs_split_x(x.cuda())
+    codes, scales, x_exp = qgemm.bs_split_x(x.cuda(), fmt)
     torch.cuda.synchronize()
     codes, scales, x_exp = codes.cpu().numpy(), scales.cpu().numpy(), x_exp.cpu().numpy()
-    full, xs_gpu = _decode_split(codes, scales, x_exp, M, K)
-    xs = oracle.split_x(x_bits(x), "e2m1", 3)
+    full, xs_gpu = _decode_split(fmt, codes, scales, x_exp, M, K)
+    xs = oracle.split_x_bs(x_bits(x), fmt, 3)
     bad = np.argwhere(xs_gpu != xs)
     assert bad.size == 0, "split differs at %s: gpu %r oracle %r" % (
         bad[:4].tolist(), xs_gpu[tuple(bad[0])], xs[tuple(bad[0])])
@@ -83,41 +90,46 @@ def test_split_bit_exact(M, K):
     assert (x_exp[M:] == 0).all()
 
 
+@pytest.mark.parametrize("fmt", FMTS)
 @pytest.mark.parametrize("M,N,K", [(1, 300, 512), (16, 256, 256), (33, 1000, 1056),
                                    (128, 640, 4096), (128, 256, 256), (300, 400, 320),
                                    (129, 1000, 1056), (517, 300, 2048)])
-def test_gemm_is_the_split_product(M, N, K):
-    case = Case("mxfp4", N, K, seed=30 + N)
+def test_gemm_is_the_split_product(fmt, M, N, K):
+    case = Case(fmt, N, K, seed=30 + N)
     x = _special_rows(inputs.activations(M, K, seed=31 + M))
     y = qgemm.bs_run(x.cuda(), case.pw)
     torch.cuda.synchronize()
     y = y.cpu().numpy().astype(np.float64)
     xb = x_bits(x)
-    ys = oracle.gemm_f64(oracle.split_x(xb, "e2m1", 3), case.Wd)
+    ys = oracle.gemm_f64(oracle.split_x_bs(xb, fmt, 3), case.Wd)
     assert norm_err(y, ys, xb, case.Wd) <= SPLIT_TOL
     if K >= 1024:
         assert norm_err(y, oracle.gemm(xb, case.Wd), xb, case.Wd) <= TOL
 
 
-def test_one_hot_rows_give_weight_columns():
-    M, N, K = 256, 512, 768
-    case = Case("mxfp4", N, K, seed=41)
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("M", [256, 64])
+def test_one_hot_rows_give_weight_columns(fmt, M):
+    N, K = 512, 768
+    case = Case(fmt, N, K, seed=41)
     ks = (np.arange(M) * 37 + 3) % K
     x = torch.zeros(M, K, dtype=torch.bfloat16)
     x[np.arange(M), ks] = 1.0
     x[7, ks[7]] = -0.375  # exactly one E2M1 term: -1.5 * 2^-2
-    y = qgemm.bs_run(x.cuda(), case.pw).cpu().numpy().astype(np.float64)
+    y = qgemm.bs_run(x.cuda(), case.pw).cpu().numpy()
     exp = case.Wd[:, ks].T.copy()
     exp[7] *= -0.375
-    assert np.array_equal(y, exp)
+    # one exact product per output (times the NVFP4 tensor scale, rounded once to fp32)
+    assert np.array_equal(y, exp.astype(np.float32))
 
 
+@pytest.mark.parametrize("fmt", FMTS)
 @pytest.mark.parametrize("M", [300, 40])
-def test_bf16_output_and_workspace_reuse(M):
+def test_bf16_output_and_workspace_reuse(fmt, M):
     N, K = 640, 1024
-    case = Case("mxfp4", N, K, seed=43)
+    case = Case(fmt, N, K, seed=43)
     x = inputs.activations(M, K, seed=44).cuda()
-    ws = torch.empty(qgemm.bs_workspace_size(qgemm._fmt("mxfp4"), N, K, M), dtype=torch.uint8,
+    ws = torch.empty(qgemm.bs_workspace_size(qgemm._fmt(fmt), N, K, M), dtype=torch.uint8,
                      device="cuda")
     y32 = qgemm.bs_run(x, case.pw, workspace=ws)
     y16 = qgemm.bs_run(x, case.pw, y_dtype=torch.bfloat16, workspace=ws)
@@ -127,16 +139,18 @@ def test_bf16_output_and_workspace_reuse(M):
     assert torch.equal(y16, y32.to(torch.bfloat16))
 
 
-@pytest.mark.parametrize("N,K,M", [(17408, 5120, 2048), (5120, 17408, 2048), (17408, 5120, 32),
-                                   (5120, 17408, 32)])
-def test_27b_prefill_sampled_rows(N, K, M):
-    case = Case("mxfp4", N, K, seed=inputs.W_SEED if N == 17408 else inputs.W3_SEED)
+@pytest.mark.parametrize("fmt,N,K,M", [("mxfp4", 17408, 5120, 2048), ("mxfp4", 5120, 17408, 2048),
+                                       ("mxfp4", 17408, 5120, 32), ("mxfp4", 5120, 17408, 32),
+                                       ("nvfp4", 17408, 5120, 2048), ("nvfp4", 17408, 5120, 16),
+                                       ("nvfp4", 5120, 17408, 16)])
+def test_27b_prefill_sampled_rows(fmt, N, K, M):
+    case = Case(fmt, N, K, seed=inputs.W_SEED if N == 17408 else inputs.W3_SEED)
     x = inputs.activations(M, K, seed=50)
     y = qgemm.bs_run(x.cuda(), case.pw)
     torch.cuda.synchronize()
-    rows = np.array([0, 1, 127, 128, 1000, M - 1]) if M > 1000 else np.array([0, 1, 17, M - 1])
-    y = y[rows].cpu().numpy().astype(np.float64)
+    rows = np.array([0, 1, 127, 128, 1000, M - 1]) if M > 1000 else np.array([0, 1, M // 2, M - 1])
+    y = y.cpu().numpy()[rows].astype(np.float64)  # rows picked on the host
     xb = x_bits(x)[rows]
-    ys = oracle.gemm_f64(oracle.split_x(xb, "e2m1", 3), case.Wd)
+    ys = oracle.gemm_f64(oracle.split_x_bs(xb, fmt, 3), case.Wd)
     assert norm_err(y, ys, xb, case.Wd) <= SPLIT_TOL
     assert norm_err(y, oracle.gemm(xb, case.Wd), xb, case.Wd) <= TOL
