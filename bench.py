@@ -364,6 +364,28 @@ def run_configs(dev, stream, q8_rings, hbm_peak, tf_peak):
                      "fp4_mma_frac": round(3.0 * tf / (4.0 * tf_peak), 4)})
         del x, y, ws
 
+    def prefill_ffn_bs(name, fmt, pg, pu, pd, M, reps=3):
+        # the FFN chunk on the block-scaled path: fused gate+up, then the down projection on h
+        N, K = pg.N, pg.K
+        x = inputs.activations(M, K, seed=1).to(dev)
+        h = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        y = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+        wsf = torch.empty(qgemm.bs_ffn_workspace_size(fmt, N, K, M), dtype=torch.uint8, device=dev)
+        wsd = torch.empty(qgemm.bs_workspace_size(qgemm._fmt(fmt), K, N, M), dtype=torch.uint8, device=dev)
+
+        def chain(i):
+            qgemm.bs_ffn_gate_up(x, pg, pu, h=h, workspace=wsf, stream=stream)
+            qgemm.bs_run(h, pd, y=y, workspace=wsd, stream=stream)
+
+        us = graph_us(chain, reps, stream)
+        flop = 2.0 * M * (2 * N) * K + 2.0 * M * K * N
+        tf = flop / (us * 1e-6) / 1e12
+        recs.append({"config": name, "kind": "prefill", "fmt": fmt, "path": "block-scaled",
+                     "N": N, "K": K, "M": M, "op": "bs_ffn_gate_up + bs_run down",
+                     "us": round(us, 1), "TFLOPs": round(tf, 1), "frac_tensor": round(tf / tf_peak, 4),
+                     "fp4_mma_frac": round(3.0 * tf / (4.0 * tf_peak), 4)})
+        del x, h, y, wsf, wsd
+
     def prefill_ffn(name, fmt, pg, pu, pd, M, reps=3):
         N, K = pg.N, pg.K
         x = inputs.activations(M, K, seed=1).to(dev)
@@ -419,6 +441,8 @@ def run_configs(dev, stream, q8_rings, hbm_peak, tf_peak):
     nv_down = packed("nvfp4", HIDDEN, INTER, 3)
     for M in (2048, 7235):
         prefill_ffn("nvfp4 27B FFN prefill chunk", "nvfp4", nv_gate, nv_up, nv_down, M)
+        prefill_ffn_bs("nvfp4 27B FFN prefill chunk, block-scaled path", "nvfp4", nv_gate, nv_up,
+                       nv_down, M)
     del nv_gate, nv_up, nv_down
     torch.cuda.empty_cache()
     # FP8 (E4M3, per-tensor scale) weights: the batch-8 verify GEMV widths and decode, the

@@ -976,6 +976,92 @@ int qgemm_bs_run(int fmt, const void* x, int64_t M, int64_t K, const void* codes
   return QGEMM_OK;
 }
 
+// Fused gate+up on the block-scaled path: per chunk of up to kBsFfnRows rows, one split of x
+// serves both GEMMs; g and u go to an fp32 workspace [2][rows][N] and the split-K reduce
+// kernel with S = 1 and both matrices writes h = bf16(SiLU(g) * u), the expression of the other
+// fused paths.
+namespace {
+constexpr int64_t kBsFfnRows = 2048;
+size_t bs_ffn_bytes(bool nv, int64_t N, int64_t K, int64_t M, size_t* off_gu) {
+  const int64_t mc = std::min<int64_t>(M, kBsFfnRows);
+  const size_t split = (bs_workspace_bytes(nv, mc, N, K, nullptr, nullptr, nullptr) + 255) / 256 * 256;
+  if (off_gu) *off_gu = split;
+  return split + (size_t)2 * (size_t)mc * (size_t)N * 4;
+}
+}  // namespace
+
+int qgemm_bs_ffn_workspace_size(int fmt, int64_t N, int64_t K, int64_t M, size_t* bytes) {
+  if (!bs_fmt(fmt)) return QGEMM_ERR_FORMAT;
+  int st = check_fmt_shape(fmt, N, K);
+  if (st != QGEMM_OK) return st;
+  if (M < 1 || M > 0x7FFFFFFF) return QGEMM_ERR_SHAPE;
+  if (!bytes) return QGEMM_ERR_NULL;
+  *bytes = bs_ffn_bytes(fmt == QGEMM_FMT_NVFP4, N, K, M, nullptr);
+  return QGEMM_OK;
+}
+
+int qgemm_bs_ffn_gate_up(int fmt, const void* x, int64_t M, int64_t K, const void* g_codes,
+                         const void* g_scales, const float* g_ts, const void* u_codes,
+                         const void* u_scales, const float* u_ts, int64_t N, void* h,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  if (!bs_fmt(fmt)) return QGEMM_ERR_FORMAT;
+  int st = check_fmt_shape(fmt, N, K);
+  if (st != QGEMM_OK) return st;
+  if (M < 1 || M > 0x7FFFFFFF) return QGEMM_ERR_SHAPE;
+  if (!x || !h || !weights_given(fmt, g_codes, g_scales, g_ts) ||
+      !weights_given(fmt, u_codes, u_scales, u_ts))
+    return QGEMM_ERR_NULL;
+  if (!aligned16(x) || !aligned16(h) || !aligned16(g_codes) || !aligned16(g_scales) ||
+      !aligned16(u_codes) || !aligned16(u_scales))
+    return QGEMM_ERR_ALIGN;
+  const bool nv = fmt == QGEMM_FMT_NVFP4;
+  size_t off_gu = 0;
+  const size_t need = bs_ffn_bytes(nv, N, K, M, &off_gu);
+  if (!workspace || workspace_bytes < need) return QGEMM_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return QGEMM_ERR_ALIGN;
+  if (!device_ok()) return QGEMM_ERR_DEVICE;
+  int* dev_err = error_word();
+  if (!dev_err) return cuda_fail(cudaGetLastError(), "cudaGetSymbolAddress");
+  uint8_t* wsb = static_cast<uint8_t*>(workspace);
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const float* gts = nv ? g_ts : nullptr;
+  const float* uts = nv ? u_ts : nullptr;
+  for (int64_t r0 = 0; r0 < M; r0 += kBsFfnRows) {
+    const int mc = (int)std::min<int64_t>(kBsFfnRows, M - r0);
+    size_t off_s = 0, off_e = 0, off_p = 0;
+    (void)bs_workspace_bytes(nv, mc, N, K, &off_s, &off_e, &off_p);
+    const uint16_t* xr = static_cast<const uint16_t*>(x) + (size_t)r0 * (size_t)K;
+    cudaError_t e = launch_bs_split(nv, xr, mc, (int)K, wsb, wsb + off_s,
+                                    reinterpret_cast<int*>(wsb + off_e), s);
+    if (e != cudaSuccess) return cuda_fail(e, "split kernel launch");
+    float* gbuf = reinterpret_cast<float*>(wsb + off_gu);
+    float* ubuf = gbuf + (size_t)mc * (size_t)N;
+    for (int m = 0; m < 2 && e == cudaSuccess; ++m) {
+      const uint8_t* wc = static_cast<const uint8_t*>(m ? u_codes : g_codes);
+      const uint8_t* wsc = static_cast<const uint8_t*>(m ? u_scales : g_scales);
+      float* out = m ? ubuf : gbuf;
+      if (mc <= 128)
+        e = launch_bs_dec(nv, mc, (int)N, (int)K, wsb, wsb + off_s, reinterpret_cast<const int*>(wsb + off_e),
+                          wc, wsc, m ? uts : gts, reinterpret_cast<float*>(wsb + off_p), out, 0, dev_err, s);
+      else
+        e = launch_bs_gemm(nv, mc, (int)N, (int)K, wsb, wsb + off_s, reinterpret_cast<const int*>(wsb + off_e),
+                           wc, wsc, m ? uts : gts, out, 0, dev_err, s);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "block-scaled gemm launch");
+    ReduceParams rp{};
+    rp.ws = gbuf;
+    rp.S = 1;
+    rp.NMAT = 2;
+    rp.B = mc;
+    rp.N = (int)N;
+    rp.out = static_cast<uint8_t*>(h) + (size_t)r0 * (size_t)N * 2;
+    rp.out_bf16 = 1;
+    e = launch_reduce(rp, s);
+    if (e != cudaSuccess) return cuda_fail(e, "SiLU pass launch");
+  }
+  return QGEMM_OK;
+}
+
 int qgemm_profile_events(void* begin_event, void* end_event) {
   g_prof_begin = static_cast<cudaEvent_t>(begin_event);
   g_prof_end = static_cast<cudaEvent_t>(end_event);

@@ -55,6 +55,9 @@ SIGNATURES = [
     ("qgemm_bs_split_x", _I, [_I, _VP, _I64, _I64, _VP, _VP, _VP, _VP]),
     ("qgemm_bs_workspace_size", _I, [_I, _I64, _I64, _I64, ctypes.POINTER(_SZ)]),
     ("qgemm_bs_run", _I, [_I, _VP, _I64, _I64, _VP, _VP, _VP, _I64, _VP, _I, _VP, _SZ, _VP]),
+    ("qgemm_bs_ffn_workspace_size", _I, [_I, _I64, _I64, _I64, ctypes.POINTER(_SZ)]),
+    ("qgemm_bs_ffn_gate_up", _I, [_I, _VP, _I64, _I64, _VP, _VP, _VP, _VP, _VP, _VP, _I64, _VP,
+                                  _VP, _SZ, _VP]),
     ("qgemm_split_k", _I, [_I, _I64, _I64, ctypes.POINTER(_I)]),
     ("qgemm_device_status", _I, [_I]),
     ("qgemm_profile_events", _I, [_VP, _VP]),
@@ -275,6 +278,31 @@ def bs_run(x: torch.Tensor, pw: PackedWeight, y: torch.Tensor | None = None, y_d
                               _ptr(pw.tensor_scale), pw.N, _ptr(y), ydt, _ptr(workspace),
                               workspace.numel(), _stream(stream)), "qgemm_bs_run")
     return y
+
+
+def bs_ffn_workspace_size(fmt, N: int, K: int, M: int) -> int:
+    n = _SZ()
+    _check(lib().qgemm_bs_ffn_workspace_size(_fmt(fmt), N, K, M, ctypes.byref(n)),
+           "qgemm_bs_ffn_workspace_size")
+    return n.value
+
+
+def bs_ffn_gate_up(x: torch.Tensor, wg: PackedWeight, wu: PackedWeight, h: torch.Tensor | None = None,
+                   workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """qgemm_bs_ffn_gate_up: h = bf16(SiLU(x Wg^T) * (x Wu^T)) on the block-scaled path."""
+    assert x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous()
+    M, K = x.shape
+    assert wg.fmt == wu.fmt and wg.N == wu.N and wg.K == wu.K == K
+    if h is None:
+        h = torch.empty((M, wg.N), dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(max(bs_ffn_workspace_size(wg.fmt, wg.N, K, M), 16),
+                                dtype=torch.uint8, device=x.device)
+    _check(lib().qgemm_bs_ffn_gate_up(wg.fmt, _ptr(x), M, K, _ptr(wg.codes), _ptr(wg.scales),
+                                      _ptr(wg.tensor_scale), _ptr(wu.codes), _ptr(wu.scales),
+                                      _ptr(wu.tensor_scale), wg.N, _ptr(h), _ptr(workspace),
+                                      workspace.numel(), _stream(stream)), "qgemm_bs_ffn_gate_up")
+    return h
 
 
 def ffn_gate_up(x: torch.Tensor, wg: PackedWeight, wu: PackedWeight, h: torch.Tensor | None = None,

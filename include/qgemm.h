@@ -310,6 +310,19 @@ int qgemm_bs_run(int fmt, const void* x_dev, int64_t M, int64_t K, const void* c
                  int y_dtype, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * qgemm_bs_ffn_workspace_size / qgemm_bs_ffn_gate_up: h = bf16(SiLU(x Wg^T) * (x Wu^T)) on the
+ * block-scaled path (fmt MXFP4 or NVFP4), the fused gate+up of the Atlas issue's kernel
+ * ranking.  Per chunk of up to 2048 rows one split of x serves both GEMMs; g and u go to an
+ * fp32 workspace and one pass writes h (the same SiLU(g) * u expression as
+ * qgemm_ffn_gate_up).  Arguments as for qgemm_ffn_gate_up.
+ */
+int qgemm_bs_ffn_workspace_size(int fmt, int64_t N, int64_t K, int64_t M, size_t* bytes);
+int qgemm_bs_ffn_gate_up(int fmt, const void* x_dev, int64_t M, int64_t K, const void* g_codes_dev,
+                         const void* g_scales_dev, const float* g_ts_dev, const void* u_codes_dev,
+                         const void* u_scales_dev, const float* u_ts_dev, int64_t N, void* h_dev,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Number of K splits qgemm_run uses for 1 <= B <= 256 (a function of fmt, N, K only).
  */
 int qgemm_split_k(int fmt, int64_t N, int64_t K, int* splits);

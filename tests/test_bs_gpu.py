@@ -154,3 +154,25 @@ def test_27b_prefill_sampled_rows(fmt, N, K, M):
     ys = oracle.gemm_f64(oracle.split_x_bs(xb, fmt, 3), case.Wd)
     assert norm_err(y, ys, xb, case.Wd) <= SPLIT_TOL
     assert norm_err(y, oracle.gemm(xb, case.Wd), xb, case.Wd) <= TOL
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("M", [40, 300, 2100])
+def test_fused_gate_up(fmt, M):
+    # h = bf16(SiLU(g) * u) with g, u the split's products: one bf16 ulp plus the split bar
+    # propagated to first order (the chunk of 2048 rows is crossed at M = 2100)
+    from gpu_helpers import bf16_bits_of, h_bound_violations
+    N, K = 640, 1024
+    cg, cu = Case(fmt, N, K, seed=71), Case(fmt, N, K, seed=72)
+    x = inputs.activations(M, K, seed=73)
+    x[0] = 0.0          # an all-zero row
+    x[1] = x[1] * 1e-4  # a small row (h in the linear part of SiLU)
+    h = qgemm.bs_ffn_gate_up(x.cuda(), cg.pw, cu.pw)
+    torch.cuda.synchronize()
+    xb = x_bits(x)
+    rows = np.arange(M) if M <= 300 else np.array([0, 1, 5, 1000, 2047, 2048, M - 1])
+    xs = oracle.split_x_bs(xb[rows], fmt, 3)
+    g = oracle.gemm_f64(xs, cg.Wd)
+    u = oracle.gemm_f64(xs, cu.Wd)
+    bad, worst = h_bound_violations(bf16_bits_of(h)[rows], g, u, xb[rows], cg.Wd, cu.Wd, tol=SPLIT_TOL)
+    assert bad == 0, "%d outputs outside the bound (worst ratio %.2f)" % (bad, worst)
