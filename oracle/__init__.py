@@ -68,7 +68,7 @@ def _load():
             lib.orc_pack_fp8.argtypes = [vp, i64, i64, vp, vp]
             lib.orc_split_x.argtypes = [vp, i64, i64, ctypes.c_int, ctypes.c_int, vp]
             lib.orc_split_x_bs.argtypes = [vp, i64, i64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                                           ctypes.c_int, vp]
+                                           ctypes.c_int, ctypes.c_int, vp]
             lib.orc_dequant.argtypes = [ctypes.c_int, vp, vp, ctypes.c_float, i64, i64, vp]
             lib.orc_gemm.argtypes = [vp, i64, i64, vp, i64, vp, ctypes.c_int]
             lib.orc_ffn_gate_up.argtypes = [vp, i64, i64, vp, vp, i64, vp, vp, vp, ctypes.c_int]
@@ -212,19 +212,22 @@ def split_x(x16: np.ndarray, elem: str, terms: int) -> np.ndarray:
     return xs
 
 
-# block size, prescale shift and smallest scale exponent of the block-scaled path's split
-BS_SPLIT = {"mxfp4": (32, 0, -127), "nvfp4": (16, 10, -9)}
+# block size, prescale shift, smallest scale exponent, term element (0 E4M3, 1 E2M1) and
+# number of terms of the block-scaled path's split, per weight format
+BS_SPLIT = {"mxfp4": (32, 0, -127, 1, 3), "nvfp4": (16, 10, -9, 1, 3), "fp8": (32, 0, -127, 0, 2)}
 
 
-def split_x_bs(x16: np.ndarray, fmt: str, terms: int = 3) -> np.ndarray:
+def split_x_bs(x16: np.ndarray, fmt: str, terms: int | None = None) -> np.ndarray:
     """The activation split as the block-scaled path of weight format `fmt` applies it: per-row
-    power-of-two prescale, E2M1 terms with power-of-two block scales in the MMA scale type's
-    range (orc_split_x_bs); returns 2^xe * the sum of the terms (fp64)."""
+    power-of-two prescale, E2M1 (FP4 weights) or E4M3 (FP8 weights) terms with power-of-two
+    block scales in the MMA scale type's range (orc_split_x_bs); returns 2^xe * the sum of the
+    terms (fp64).  terms defaults to the path's own (3 E2M1, 2 E4M3)."""
     x16 = np.ascontiguousarray(x16, dtype=np.uint16)
     B, K = x16.shape
-    blk, xshift, emin = BS_SPLIT[fmt]
+    blk, xshift, emin, elem, nterms = BS_SPLIT[fmt]
     xs = np.zeros((B, K), dtype=np.float64)
-    _load().orc_split_x_bs(_ptr(x16), B, K, blk, xshift, emin, terms, _ptr(xs))
+    _load().orc_split_x_bs(_ptr(x16), B, K, blk, xshift, emin, elem,
+                           nterms if terms is None else terms, _ptr(xs))
     return xs
 
 

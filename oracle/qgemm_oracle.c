@@ -515,15 +515,18 @@ void orc_split_x(const uint16_t *x16, int64_t B, int64_t K, int elem, int terms,
 /* the MMA's scale type):                                                       */
 /*   xe = floor(log2 max|x_row|) - xshift   (0 for an all-zero row)            */
 /*   r_0 = x 2^-xe;  per block of `block` elements and term j:                  */
-/*   e_j = floor(log2 max|r_j|) - 2; if e_j < emin the term and the later ones  */
-/*   are dropped; q_j = E2M1_RNE_sat(r_j / 2^e_j); r_{j+1} = r_j - q_j 2^e_j.   */
+/*   e_j = floor(log2 max|r_j|) - top; if e_j < emin the term and the later     */
+/*   ones are dropped; q_j = ENC(r_j / 2^e_j); r_{j+1} = r_j - q_j 2^e_j,        */
+/* with ENC = E2M1_RNE_sat, top = 2 (elem 1) or E4M3_RNE_sat, top = 7 (elem 0). */
 /* xs receives 2^xe sum_j q_j 2^e_j.  MXFP4 (E8M0 per 32): block 32, xshift 0,  */
-/* emin -127.  NVFP4 (UE4M3 per 16, powers of two only): block 16, xshift 10,   */
-/* emin -9 (2^-9 is the smallest UE4M3 power of two; the prescale puts the row  */
-/* maximum in [2^10, 2^11), so e_j <= 8 and 2^8 is representable).             */
+/* emin -127, E2M1.  NVFP4 (UE4M3 per 16, powers of two only): block 16,        */
+/* xshift 10, emin -9 (2^-9 is the smallest UE4M3 power of two; the prescale    */
+/* puts the row maximum in [2^10, 2^11), so e_j <= 8 and 2^8 is representable), */
+/* E2M1.  FP8 weights (E8M0 per 32): block 32, xshift 0, emin -127, E4M3.       */
 /* ------------------------------------------------------------------------- */
 void orc_split_x_bs(const uint16_t *x16, int64_t B, int64_t K, int block, int xshift, int emin,
-                    int terms, double *xs) {
+                    int elem, int terms, double *xs) {
+    const int top = elem == 0 ? 7 : 2;
     for (int64_t b = 0; b < B; ++b) {
         double rmax = 0.0;
         int xe = 0;
@@ -546,11 +549,12 @@ void orc_split_x_bs(const uint16_t *x16, int64_t B, int64_t K, int block, int xs
                 for (int64_t i = 0; i < n; ++i) amax = fmax(amax, fabs(r[i]));
                 if (amax == 0.0) break;
                 (void)frexp(amax, &ex);
-                e = (ex - 1) - 2;
+                e = (ex - 1) - top;
                 if (e < emin) break;
                 sc = ldexp(1.0, e);
                 for (int64_t i = 0; i < n; ++i) {
-                    const double q = orc_e2m1(orc_e2m1_encode(r[i] / sc));
+                    const double q = elem == 0 ? orc_e4m3(orc_e4m3_encode(r[i] / sc))
+                                               : orc_e2m1(orc_e2m1_encode(r[i] / sc));
                     acc[i] += q * sc;
                     r[i] -= q * sc;
                 }

@@ -579,17 +579,20 @@ def test_activation_split_accuracy_for_the_block_scaled_path():
             assert np.array_equal(oracle.split_x(x16, "e4m3", 3), xd)  # three terms: exact
 
 
-@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4", "fp8"])
 def test_block_scaled_split_first_term_brute_force(fmt):
     # one term, from the definitions: xe = floor(log2 max|row|) - xshift, each block's
-    # e = floor(log2 max|x 2^-xe|) - 2, the nearest E2M1 value of x 2^-xe / 2^e (ties to the even
-    # code, saturating at 6), times 2^e 2^xe; blocks with e below the smallest scale are zero
-    blk, xshift, emin = oracle.BS_SPLIT[fmt]
+    # e = floor(log2 max|x 2^-xe|) - top, the nearest code value of x 2^-xe / 2^e (E2M1, top 2,
+    # or E4M3, top 7; ties to the even code, saturating), times 2^e 2^xe; blocks with e below the
+    # smallest scale are zero
+    blk, xshift, emin, elem, _ = oracle.BS_SPLIT[fmt]
+    top = 7 if elem == 0 else 2
     x = inputs.activations(3, 96, seed=61)
     x[1, 16:32] *= 2.0 ** -40  # a block far below its row maximum
     x16 = inputs.bf16_bits(x)
     xs = oracle.split_x_bs(x16, fmt, 1)
-    vals = [Fraction(v) for v in E2M1_MAG]
+    vals = ([Fraction(oracle.e4m3(b)) for b in range(0x7F)] if elem == 0
+            else [Fraction(v) for v in E2M1_MAG])
     for b in range(3):
         row = [Fraction(oracle.bf16(int(v))) for v in x16[b]]
         _, ex = math.frexp(float(max(abs(v) for v in row)))
@@ -597,7 +600,7 @@ def test_block_scaled_split_first_term_brute_force(fmt):
         for k0 in range(0, 96, blk):
             r = [v / Fraction(2) ** xe for v in row[k0:k0 + blk]]
             _, ex = math.frexp(float(max(abs(v) for v in r)))
-            e = (ex - 1) - 2
+            e = (ex - 1) - top
             for i, v in enumerate(r):
                 if e < emin:
                     want = Fraction(0)
@@ -615,21 +618,23 @@ def test_block_scaled_split_prescale_invariance_and_mxfp4_reduction():
     # it); with MXFP4's parameters and no dropped block the split is the plain per-block peel
     x = inputs.activations(4, 640, seed=62)
     x16 = inputs.bf16_bits(x)
-    for fmt in ("mxfp4", "nvfp4"):
-        base = oracle.split_x_bs(x16, fmt, 3)
+    for fmt in ("mxfp4", "nvfp4", "fp8"):
+        base = oracle.split_x_bs(x16, fmt)
         for k in (-60, 7, 90):
             xk = inputs.bf16_bits(x * 2.0 ** k)
-            assert np.array_equal(oracle.split_x_bs(xk, fmt, 3), np.ldexp(base, k)), (fmt, k)
+            assert np.array_equal(oracle.split_x_bs(xk, fmt), np.ldexp(base, k)), (fmt, k)
     assert np.array_equal(oracle.split_x_bs(x16, "mxfp4", 3), oracle.split_x(x16, "e2m1", 3))
+    assert np.array_equal(oracle.split_x_bs(x16, "fp8", 2), oracle.split_x(x16, "e4m3", 2))
 
 
 def test_block_scaled_split_accuracy():
-    # three E2M1 terms in either variant stay well inside the 1e-3 bar at the 27B lengths
+    # three E2M1 terms (FP4 weights) and two E4M3 terms (FP8 weights) stay well inside the
+    # 1e-3 bar at the 27B lengths
     for K in (5120, 17408):
         x16 = inputs.bf16_bits(inputs.activations(4, K, seed=63))
-        for fmt in ("nvfp4", "mxfp4"):
+        for fmt in ("nvfp4", "mxfp4", "fp8"):
             W = inputs.weights(16, K, seed=64).numpy()
             Wd = oracle.dequant(fmt, *oracle.pack(fmt, W), 16, K)
             y = oracle.gemm(x16, Wd)
-            err = oracle.normalised_error(oracle.gemm_f64(oracle.split_x_bs(x16, fmt, 3), Wd), y, x16, Wd)
-            assert err < 2e-4, (K, fmt, err)
+            err = oracle.normalised_error(oracle.gemm_f64(oracle.split_x_bs(x16, fmt), Wd), y, x16, Wd)
+            assert err < (1e-8 if fmt == "fp8" else 2e-4), (K, fmt, err)
