@@ -14,15 +14,15 @@
 
 namespace qg {
 cudaError_t launch_prep(const PrepParams& pp, cudaStream_t stream);
-cudaError_t launch_bs_split(bool nv, const uint16_t* x, int M, int K, uint8_t* codes,
+cudaError_t launch_bs_split(int f, const uint16_t* x, int M, int K, uint8_t* codes,
                             uint8_t* scales, int* x_exp, cudaStream_t stream);
-cudaError_t launch_bs_gemm(bool nv, int M, int N, int K, const uint8_t* xcodes,
+cudaError_t launch_bs_gemm(int f, int M, int N, int K, const uint8_t* xcodes,
                            const uint8_t* xscales, const int* x_exp, const uint8_t* wcodes,
                            const uint8_t* wscales, const float* ts, void* out, int out_bf16,
                            int* dev_err, cudaStream_t stream);
-size_t bs_workspace_bytes(bool nv, int64_t M, int64_t N, int64_t K, size_t* off_scales,
+size_t bs_workspace_bytes(int f, int64_t M, int64_t N, int64_t K, size_t* off_scales,
                           size_t* off_exp, size_t* off_part);
-cudaError_t launch_bs_dec(bool nv, int M, int N, int K, const uint8_t* xcodes,
+cudaError_t launch_bs_dec(int f, int M, int N, int K, const uint8_t* xcodes,
                           const uint8_t* xscales, const int* x_exp, const uint8_t* wcodes,
                           const uint8_t* wscales, const float* ts, float* part, void* out,
                           int out_bf16, int* dev_err, cudaStream_t stream);
@@ -890,10 +890,17 @@ int qgemm_moe_gate_up(int fmt, const void* x, int64_t M, int64_t K, int E, const
 }
 
 // ---------------------------------------------------------------------------------------
-// Block-scaled path (MXFP4 / NVFP4 weights, x split into three E2M1 terms)
+// Block-scaled path (MXFP4 / NVFP4 weights with x split into three E2M1 terms, FP8 weights
+// with x split into two E4M3 terms)
 // ---------------------------------------------------------------------------------------
 namespace {
-bool bs_fmt(int fmt) { return fmt == QGEMM_FMT_MXFP4 || fmt == QGEMM_FMT_NVFP4; }
+bool bs_fmt(int fmt) {
+  return fmt == QGEMM_FMT_MXFP4 || fmt == QGEMM_FMT_NVFP4 || fmt == QGEMM_FMT_FP8;
+}
+// the kernels' format id: 0 MXFP4, 1 NVFP4, 2 FP8
+int bs_id(int fmt) { return fmt == QGEMM_FMT_NVFP4 ? 1 : fmt == QGEMM_FMT_FP8 ? 2 : 0; }
+// the per-tensor scale the epilogue applies (NVFP4, FP8), else none
+const float* bs_ts(int fmt, const float* ts) { return fmt == QGEMM_FMT_MXFP4 ? nullptr : ts; }
 }  // namespace
 
 int qgemm_bs_split_size(int fmt, int64_t M, int64_t K, size_t* code_bytes, size_t* scale_bytes,
@@ -903,7 +910,7 @@ int qgemm_bs_split_size(int fmt, int64_t M, int64_t K, size_t* code_bytes, size_
   if (K % 32 != 0) return QGEMM_ERR_K_BLOCK;
   if (!code_bytes || !scale_bytes || !exp_bytes) return QGEMM_ERR_NULL;
   size_t off_s = 0, off_e = 0, off_p = 0;
-  (void)bs_workspace_bytes(fmt == QGEMM_FMT_NVFP4, M, 0, K, &off_s, &off_e, &off_p);
+  (void)bs_workspace_bytes(bs_id(fmt), M, 0, K, &off_s, &off_e, &off_p);
   const int64_t Mt = (M + 127) / 128;
   *code_bytes = off_s;
   *scale_bytes = off_e - off_s;
@@ -920,7 +927,7 @@ int qgemm_bs_split_x(int fmt, const void* x, int64_t M, int64_t K, void* codes, 
   if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || !aligned16(x_exp))
     return QGEMM_ERR_ALIGN;
   if (!device_ok()) return QGEMM_ERR_DEVICE;
-  const cudaError_t e = launch_bs_split(fmt == QGEMM_FMT_NVFP4, static_cast<const uint16_t*>(x), (int)M, (int)K,
+  const cudaError_t e = launch_bs_split(bs_id(fmt), static_cast<const uint16_t*>(x), (int)M, (int)K,
                                         static_cast<uint8_t*>(codes), static_cast<uint8_t*>(scales),
                                         reinterpret_cast<int*>(x_exp), static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? QGEMM_OK : cuda_fail(e, "split kernel launch");
@@ -932,7 +939,7 @@ int qgemm_bs_workspace_size(int fmt, int64_t N, int64_t K, int64_t M, size_t* by
   if (st != QGEMM_OK) return st;
   if (M < 1 || M > 0x7FFFFFFF) return QGEMM_ERR_SHAPE;
   if (!bytes) return QGEMM_ERR_NULL;
-  *bytes = bs_workspace_bytes(fmt == QGEMM_FMT_NVFP4, M, N, K, nullptr, nullptr, nullptr);
+  *bytes = bs_workspace_bytes(bs_id(fmt), M, N, K, nullptr, nullptr, nullptr);
   return QGEMM_OK;
 }
 
@@ -940,7 +947,7 @@ int qgemm_bs_run(int fmt, const void* x, int64_t M, int64_t K, const void* codes
                  const void* scales, const float* tensor_scale, int64_t N, void* y, int y_dtype,
                  void* workspace, size_t workspace_bytes, void* stream) {
   if (!bs_fmt(fmt)) return QGEMM_ERR_FORMAT;
-  const bool nv = fmt == QGEMM_FMT_NVFP4;
+  const int f = bs_id(fmt);
   int st = check_fmt_shape(fmt, N, K);
   if (st != QGEMM_OK) return st;
   if (M < 1 || M > 0x7FFFFFFF) return QGEMM_ERR_SHAPE;
@@ -949,7 +956,7 @@ int qgemm_bs_run(int fmt, const void* x, int64_t M, int64_t K, const void* codes
   if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || !aligned16(y))
     return QGEMM_ERR_ALIGN;
   size_t off_s = 0, off_e = 0, off_p = 0;
-  const size_t need = bs_workspace_bytes(nv, M, N, K, &off_s, &off_e, &off_p);
+  const size_t need = bs_workspace_bytes(f, M, N, K, &off_s, &off_e, &off_p);
   if (!workspace || workspace_bytes < need) return QGEMM_ERR_WORKSPACE;
   if (!aligned16(workspace)) return QGEMM_ERR_ALIGN;
   if (!device_ok()) return QGEMM_ERR_DEVICE;
@@ -957,18 +964,18 @@ int qgemm_bs_run(int fmt, const void* x, int64_t M, int64_t K, const void* codes
   if (!dev_err) return cuda_fail(cudaGetLastError(), "cudaGetSymbolAddress");
   uint8_t* wsb = static_cast<uint8_t*>(workspace);
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = launch_bs_split(nv, static_cast<const uint16_t*>(x), (int)M, (int)K, wsb, wsb + off_s,
+  cudaError_t e = launch_bs_split(f, static_cast<const uint16_t*>(x), (int)M, (int)K, wsb, wsb + off_s,
                                   reinterpret_cast<int*>(wsb + off_e), s);
   if (e != cudaSuccess) return cuda_fail(e, "split kernel launch");
   if (g_prof_begin) cudaEventRecord(g_prof_begin, s);
   // up to 128 rows the weights are the MMA M operand (decode tiling), above that x is
-  const float* ts = nv ? tensor_scale : nullptr;
+  const float* ts = bs_ts(fmt, tensor_scale);
   if (M <= 128)
-    e = launch_bs_dec(nv, (int)M, (int)N, (int)K, wsb, wsb + off_s, reinterpret_cast<const int*>(wsb + off_e),
+    e = launch_bs_dec(f, (int)M, (int)N, (int)K, wsb, wsb + off_s, reinterpret_cast<const int*>(wsb + off_e),
                       static_cast<const uint8_t*>(codes), static_cast<const uint8_t*>(scales), ts,
                       reinterpret_cast<float*>(wsb + off_p), y, y_dtype == QGEMM_Y_BF16, dev_err, s);
   else
-    e = launch_bs_gemm(nv, (int)M, (int)N, (int)K, wsb, wsb + off_s, reinterpret_cast<const int*>(wsb + off_e),
+    e = launch_bs_gemm(f, (int)M, (int)N, (int)K, wsb, wsb + off_s, reinterpret_cast<const int*>(wsb + off_e),
                        static_cast<const uint8_t*>(codes), static_cast<const uint8_t*>(scales), ts, y,
                        y_dtype == QGEMM_Y_BF16, dev_err, s);
   if (e != cudaSuccess) return cuda_fail(e, "block-scaled gemm launch");
@@ -982,9 +989,9 @@ int qgemm_bs_run(int fmt, const void* x, int64_t M, int64_t K, const void* codes
 // fused paths.
 namespace {
 constexpr int64_t kBsFfnRows = 2048;
-size_t bs_ffn_bytes(bool nv, int64_t N, int64_t K, int64_t M, size_t* off_gu) {
+size_t bs_ffn_bytes(int f, int64_t N, int64_t K, int64_t M, size_t* off_gu) {
   const int64_t mc = std::min<int64_t>(M, kBsFfnRows);
-  const size_t split = (bs_workspace_bytes(nv, mc, N, K, nullptr, nullptr, nullptr) + 255) / 256 * 256;
+  const size_t split = (bs_workspace_bytes(f, mc, N, K, nullptr, nullptr, nullptr) + 255) / 256 * 256;
   if (off_gu) *off_gu = split;
   return split + (size_t)2 * (size_t)mc * (size_t)N * 4;
 }
@@ -996,7 +1003,7 @@ int qgemm_bs_ffn_workspace_size(int fmt, int64_t N, int64_t K, int64_t M, size_t
   if (st != QGEMM_OK) return st;
   if (M < 1 || M > 0x7FFFFFFF) return QGEMM_ERR_SHAPE;
   if (!bytes) return QGEMM_ERR_NULL;
-  *bytes = bs_ffn_bytes(fmt == QGEMM_FMT_NVFP4, N, K, M, nullptr);
+  *bytes = bs_ffn_bytes(bs_id(fmt), N, K, M, nullptr);
   return QGEMM_OK;
 }
 
@@ -1014,9 +1021,9 @@ int qgemm_bs_ffn_gate_up(int fmt, const void* x, int64_t M, int64_t K, const voi
   if (!aligned16(x) || !aligned16(h) || !aligned16(g_codes) || !aligned16(g_scales) ||
       !aligned16(u_codes) || !aligned16(u_scales))
     return QGEMM_ERR_ALIGN;
-  const bool nv = fmt == QGEMM_FMT_NVFP4;
+  const int f = bs_id(fmt);
   size_t off_gu = 0;
-  const size_t need = bs_ffn_bytes(nv, N, K, M, &off_gu);
+  const size_t need = bs_ffn_bytes(f, N, K, M, &off_gu);
   if (!workspace || workspace_bytes < need) return QGEMM_ERR_WORKSPACE;
   if (!aligned16(workspace)) return QGEMM_ERR_ALIGN;
   if (!device_ok()) return QGEMM_ERR_DEVICE;
@@ -1024,14 +1031,14 @@ int qgemm_bs_ffn_gate_up(int fmt, const void* x, int64_t M, int64_t K, const voi
   if (!dev_err) return cuda_fail(cudaGetLastError(), "cudaGetSymbolAddress");
   uint8_t* wsb = static_cast<uint8_t*>(workspace);
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const float* gts = nv ? g_ts : nullptr;
-  const float* uts = nv ? u_ts : nullptr;
+  const float* gts = bs_ts(fmt, g_ts);
+  const float* uts = bs_ts(fmt, u_ts);
   for (int64_t r0 = 0; r0 < M; r0 += kBsFfnRows) {
     const int mc = (int)std::min<int64_t>(kBsFfnRows, M - r0);
     size_t off_s = 0, off_e = 0, off_p = 0;
-    (void)bs_workspace_bytes(nv, mc, N, K, &off_s, &off_e, &off_p);
+    (void)bs_workspace_bytes(f, mc, N, K, &off_s, &off_e, &off_p);
     const uint16_t* xr = static_cast<const uint16_t*>(x) + (size_t)r0 * (size_t)K;
-    cudaError_t e = launch_bs_split(nv, xr, mc, (int)K, wsb, wsb + off_s,
+    cudaError_t e = launch_bs_split(f, xr, mc, (int)K, wsb, wsb + off_s,
                                     reinterpret_cast<int*>(wsb + off_e), s);
     if (e != cudaSuccess) return cuda_fail(e, "split kernel launch");
     float* gbuf = reinterpret_cast<float*>(wsb + off_gu);
@@ -1041,10 +1048,10 @@ int qgemm_bs_ffn_gate_up(int fmt, const void* x, int64_t M, int64_t K, const voi
       const uint8_t* wsc = static_cast<const uint8_t*>(m ? u_scales : g_scales);
       float* out = m ? ubuf : gbuf;
       if (mc <= 128)
-        e = launch_bs_dec(nv, mc, (int)N, (int)K, wsb, wsb + off_s, reinterpret_cast<const int*>(wsb + off_e),
+        e = launch_bs_dec(f, mc, (int)N, (int)K, wsb, wsb + off_s, reinterpret_cast<const int*>(wsb + off_e),
                           wc, wsc, m ? uts : gts, reinterpret_cast<float*>(wsb + off_p), out, 0, dev_err, s);
       else
-        e = launch_bs_gemm(nv, mc, (int)N, (int)K, wsb, wsb + off_s, reinterpret_cast<const int*>(wsb + off_e),
+        e = launch_bs_gemm(f, mc, (int)N, (int)K, wsb, wsb + off_s, reinterpret_cast<const int*>(wsb + off_e),
                            wc, wsc, m ? uts : gts, out, 0, dev_err, s);
     }
     if (e != cudaSuccess) return cuda_fail(e, "block-scaled gemm launch");

@@ -35,6 +35,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp4.h>
+#include <cuda_fp8.h>
 
 #include <algorithm>
 #include <atomic>
@@ -44,67 +45,89 @@
 
 namespace qg {
 
-constexpr int kBsTerms = 3;
+constexpr int kBsMaxTerms = 3;
 constexpr int kBsM = 128;                     // tokens per tile
 constexpr int kBsWT = 2;                      // weight tiles (of 128 rows) per tile
 constexpr int kBsN = 128 * kBsWT;             // weight rows per tile (MMA N)
-constexpr int kBsK = 256;                     // K per stage (one MXFP4 chunk)
 // (one weight tile per tile with three stages measured faster only at M = 2048 of the
-// 5120 x 17408 shape and slower at M = 8192: x is then re-read for every 128 weight rows)
-constexpr int kBsStages = kBsWT == 1 ? 3 : 2;
+// 5120 x 17408 MXFP4 shape and slower at M = 8192: x is then re-read for every 128 weight rows)
 constexpr int kBsBlock = kBsM * 128;          // one 128-row x 128-byte code block: 16 KB
-constexpr int kBsACodes = kBsTerms * kBsBlock;
 constexpr int kBsBCodes = kBsWT * kBsBlock;
-// tensor memory: the accumulator in columns [0, 256), then per stage kBsSfCols columns of
-// scale factors: x term t, K-block kb at (t * 4 + kb) * 4 (4 columns: row groups r1 = 0..3),
-// the weights' K-block kb at 48 + kb * 8 (8 columns: r1 = 0..7)
-constexpr int kBsSfCols = kBsTerms * 4 * 4 + 4 * 4 * kBsWT;
+constexpr int kBsKB = 4;                      // MMA K-blocks per chunk (32 bytes of codes each)
 constexpr int kBsTmemCols = 512;
-static_assert(kBsN + kBsStages * kBsSfCols <= kBsTmemCols, "TMEM budget");
 constexpr int kBsStageWarp0 = 2;  // warps 2..5 stage the scale factors
 constexpr int kBsEpiWarp0 = 6;    // warps 6..9 run the epilogue
 constexpr int kBsThreads = 10 * 32;
 
+// Weight formats of the path: 0 MXFP4, 1 NVFP4 (both kind::mxf4nvf4, E2M1 operands),
+// 2 FP8 E4M3 with a per-tensor scale (kind::mxf8f6f4, E4M3 operands).
+constexpr int kBsMx = 0, kBsNv = 1, kBsF8 = 2;
+
 struct BsSplitParams {
   const uint16_t* x;  // bf16 [M][K]
   int M, K, C, Mt;
-  int nv;             // 1: NVFP4 (16-element blocks, UE4M3 powers of two), 0: MXFP4 (32, E8M0)
-  uint8_t* codes;
-  uint8_t* scales;    // [Mt][C][3][128][sbr], sbr = 16 (NVFP4) or 8 (MXFP4)
+  int f;              // weight format (kBsMx, kBsNv, kBsF8)
+  uint8_t* codes;     // [Mt][C][terms][128][128]
+  uint8_t* scales;    // [Mt][C][terms][128][sbr]
   int* x_exp;
 };
 
-// Parameters of the split per weight format: block size, prescale shift (the row maximum
-// lands in [2^xshift, 2^(xshift+1))), smallest block-scale exponent, scale bytes per row and
-// 256-K chunk.  MXFP4: E8M0 scales per 32 elements, whose range covers every bf16 row after a
-// prescale to [1, 2).  NVFP4: UE4M3 scales per 16, restricted to the powers of two it holds
-// exactly (2^-9 .. 2^8, so that every step stays exact); the prescale to [2^10, 2^11) keeps
-// every block scale <= 2^8 and gives blocks 2^17 of range below the row maximum.
-__host__ __device__ constexpr int bs_blk(bool nv) { return nv ? 16 : 32; }
-__host__ __device__ constexpr int bs_xshift(bool nv) { return nv ? 10 : 0; }
-__host__ __device__ constexpr int bs_emin(bool nv) { return nv ? -9 : -127; }
-__host__ __device__ constexpr int bs_sbr(bool nv) { return nv ? 16 : 8; }
+// Parameters of the split per weight format: terms, K per chunk (one weight chunk of the
+// tile-major layout), block size, prescale shift (the row maximum lands in
+// [2^xshift, 2^(xshift+1))), smallest block-scale exponent, top (the block maximum / 2^e lands
+// in [2^top, 2^(top+1))), x-term and weight scale bytes per row and chunk.  MXFP4: three E2M1
+// terms, E8M0 scales per 32 elements, whose range covers every bf16 row after a prescale to
+// [1, 2).  NVFP4: three E2M1 terms, UE4M3 scales per 16, restricted to the powers of two it
+// holds exactly (2^-9 .. 2^8, so that every step stays exact); the prescale to [2^10, 2^11)
+// keeps every block scale <= 2^8 and gives blocks 2^17 of range below the row maximum.  FP8:
+// two E4M3 terms with E8M0 scales per 32 (the weights carry only a per-tensor scale; their
+// block scales are 1).
+__host__ __device__ constexpr int bs_terms(int f) { return f == kBsF8 ? 2 : 3; }
+__host__ __device__ constexpr int bs_chunk(int f) { return f == kBsF8 ? 128 : 256; }
+__host__ __device__ constexpr int bs_blk(int f) { return f == kBsNv ? 16 : 32; }
+__host__ __device__ constexpr int bs_xshift(int f) { return f == kBsNv ? 10 : 0; }
+__host__ __device__ constexpr int bs_emin(int f) { return f == kBsNv ? -9 : -127; }
+__host__ __device__ constexpr int bs_top(int f) { return f == kBsF8 ? 7 : 2; }
+__host__ __device__ constexpr int bs_sbr(int f) { return f == kBsNv ? 16 : (f == kBsF8 ? 4 : 8); }
+__host__ __device__ constexpr int bs_wsbr(int f) { return f == kBsNv ? 16 : (f == kBsF8 ? 0 : 8); }
 // The scale byte of 2^e: E8M0 e + 127; UE4M3 (bias 7, three mantissa bits) (e + 7) << 3 for a
 // normal value, 2^(e + 9) as the subnormal mantissa below 2^-6.
-__host__ __device__ constexpr int bs_scale_byte(bool nv, int e) {
-  return nv ? (e >= -6 ? (e + 7) << 3 : 1 << (e + 9)) : e + 127;
+__host__ __device__ constexpr int bs_scale_byte(int f, int e) {
+  return f == kBsNv ? (e >= -6 ? (e + 7) << 3 : 1 << (e + 9)) : e + 127;
 }
 
-// Prefill-kernel stage layout per weight format: [x-term codes 48 KB][weight codes 32 KB]
-// [x-term scales 3 x 128 x sbr][weight scales 2 x 128 x sbr] (85 KB MXFP4, 90 KB NVFP4).
-template <bool NV>
+// Instruction descriptor of the block-scaled MMA with M = 128 and N = n, both operands
+// K-major, scale factor ids 0.  kind::mxf4nvf4: A and B E2M1 (format 1), K = 64 per
+// instruction, scale type UE4M3 (NVFP4) or E8M0 (MXFP4).  kind::mxf8f6f4: A and B E4M3
+// (format 0), K = 32 per instruction, scale type E8M0.
+__host__ __device__ constexpr uint32_t bs_idesc(int f, int n) {
+  return (f == kBsF8 ? 0u : ((1u << 7) | (1u << 10))) | ((uint32_t)(n >> 3) << 17) |
+         ((f == kBsNv ? 0u : 1u) << 23) | ((uint32_t)(kBsM >> 4) << 24);
+}
+
+// Prefill-kernel stage layout per weight format: [x-term codes terms x 16 KB][weight codes
+// 32 KB][x-term scales terms x 128 x sbr][weight scales 2 x 128 x wsbr] (85 KB MXFP4, 90 KB
+// NVFP4, 65 KB FP8).  Tensor memory: the accumulator in columns [0, 256), then per stage SfCols
+// columns of scale factors: x term t, K-block kb at (t * 4 + kb) * 4 (4 columns: row groups
+// r1 = 0..3), the weights' K-block kb at ASf + kb * 8 (8 columns: r1 = 0..7).
+template <int F>
 struct BsLay {
-  static constexpr int SB = kBsM * bs_sbr(NV);  // scales of one 128-row block
-  static constexpr int AScales = kBsTerms * SB;
-  static constexpr int BScales = kBsWT * SB;
-  static constexpr int Stage = kBsACodes + kBsBCodes + AScales + BScales;
-  static constexpr int Smem = 1024 + kBsStages * Stage + 256;
-  // instruction descriptor, kind::mxf4nvf4: A and B E2M1 (K-major), M = 128, N = kBsN,
-  // K = 64 per instruction, scale factor ids 0, scale type UE4M3 (NVFP4) or E8M0 (MXFP4)
-  static constexpr uint32_t Idesc = (1u << 7) | (1u << 10) | ((uint32_t)(kBsN >> 3) << 17) |
-                                    ((NV ? 0u : 1u) << 23) | ((uint32_t)(kBsM >> 4) << 24);
+  static constexpr int Terms = bs_terms(F);
+  static constexpr int ACodes = Terms * kBsBlock;
+  static constexpr int SB = kBsM * bs_sbr(F);    // x-term scales of one 128-row block
+  static constexpr int WSB = kBsM * bs_wsbr(F);  // weight scales of one 128-row block
+  static constexpr int AScales = Terms * SB;
+  static constexpr int BScales = kBsWT * WSB;
+  static constexpr int Stage = ACodes + kBsBCodes + AScales + BScales;
+  static constexpr int Stages = F == kBsF8 ? 3 : 2;  // FP8 chunks hold half the K
+  static constexpr int ASf = Terms * kBsKB * 4;
+  static constexpr int SfCols = ASf + kBsKB * 4 * kBsWT;
+  static constexpr int Smem = 1024 + Stages * Stage + 256;
+  static constexpr uint32_t Idesc = bs_idesc(F, kBsN);
   static_assert(Stage % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
   static_assert(Smem <= 227 * 1024, "shared memory");
+  static_assert(kBsN + Stages * SfCols <= kBsTmemCols, "TMEM budget");
+  static_assert(SfCols % 16 == 0, "scale factors are stored 16 columns at a time");
 };
 
 struct BsParams {
@@ -114,7 +137,7 @@ struct BsParams {
   const int* x_exp;
   const uint8_t* wcodes;   // tile-major MXFP4 / NVFP4 codes
   const uint8_t* wscales;  // tile-major scales
-  const float* ts;         // NVFP4 tensor scale (device), else nullptr
+  const float* ts;         // NVFP4 / FP8 tensor scale (device), else nullptr
   void* out;               // y [M][N] fp32 or bf16
   int out_bf16;
   int* dev_err;
@@ -122,11 +145,12 @@ struct BsParams {
 
 // ---------------------------------------------------------------------------------------
 // Split: one CTA of 256 threads per token row of the padded tile range (rows past M write
-// zeros).  Phase 1: the row maximum and x_exp.  Phase 2: each 256-element chunk is one warp's,
-// lane l holding elements 8l .. 8l+7 of it, so four lanes share a 32-element block.
-// Every step is exact in fp32: bf16 values times powers of two, an E2M1 code times a power of
-// two, and r - q 2^e, whose significand fits 24 bits because |r - q 2^e| is at most half an
-// E2M1 step at |r|'s magnitude (or the saturation error, 2^(e+1), where |r| >= 2^(e+2)).
+// zeros).  Phase 1: the row maximum and x_exp.  Phase 2: each 256-element span is one warp's,
+// lane l holding elements 8l .. 8l+7 of it (one E2M1 chunk, or two E4M3 chunks of 128), so
+// four lanes share a 32-element block (two a 16-element one).
+// Every step is exact in fp32: bf16 values times powers of two, a code times a power of two,
+// and r - q 2^e, whose significand fits 24 bits because |r - q 2^e| is at most half a code
+// step at |r|'s magnitude (or, for E2M1, the saturation error 2^(e+1) where |r| >= 2^(e+2)).
 // ---------------------------------------------------------------------------------------
 constexpr int kBsSplitThreads = 256;
 constexpr int kBsSplitRegs = 3;  // 8-element words per thread kept from phase 1 (rows to 6144)
@@ -142,11 +166,33 @@ __device__ __forceinline__ float bs_amax8(float m, const uint4& v) {
   return m;
 }
 
-// The three terms of one lane's 8 elements (a quarter of a 32-element block or half of a
-// 16-element one), written to the split layout.  All lanes of the block take the same
-// decisions (the block maximum is reduced over them first).
-__device__ __forceinline__ void bs_split8(const BsSplitParams& p, const uint4& v, bool in, float f1,
-                                          float f2, int t, int r, int c, int lane) {
+// Two elements as one code pair (element 2i first: the low nibble or byte), rounded to
+// nearest even and saturated by the hardware conversion, and their values back (exact in f16).
+template <int F>
+__device__ __forceinline__ uint32_t bs_enc2(float a, float b, float& qa, float& qb) {
+  if (F == kBsF8) {
+    const __nv_fp8x2_storage_t c2 = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(c2, __NV_E4M3);
+    qa = __half2float(__half(__half_raw{h.x}));
+    qb = __half2float(__half(__half_raw{h.y}));
+    return (uint32_t)c2;
+  }
+  const __nv_fp4x2_storage_t c2 = __nv_cvt_float2_to_fp4x2(make_float2(a, b), __NV_E2M1, cudaRoundNearest);
+  const __half2_raw h = __nv_cvt_fp4x2_to_halfraw2(c2, __NV_E2M1);
+  qa = __half2float(__half(__half_raw{h.x}));
+  qb = __half2float(__half(__half_raw{h.y}));
+  return (uint32_t)c2;
+}
+
+// The terms of one lane's 8 elements (a quarter of a 32-element block or half of a 16-element
+// one), written to the split layout when `store` (lanes past the padded K only take part in
+// the block reductions).  All lanes of the block take the same decisions (the block maximum is
+// reduced over them first).
+template <int F>
+__device__ __forceinline__ void bs_split8(const BsSplitParams& p, const uint4& v, bool in, bool store,
+                                          float f1, float f2, int t, int r, int k, int lane) {
+  constexpr int kTerms = bs_terms(F), kChunk = bs_chunk(F), kBlk = bs_blk(F), kSbr = bs_sbr(F);
+  constexpr int kLpb = kBlk / 8;  // lanes per block
   float rv[8];
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -154,39 +200,38 @@ __device__ __forceinline__ void bs_split8(const BsSplitParams& p, const uint4& v
     rv[2 * i] = in ? (__uint_as_float(w[i] << 16) * f1) * f2 : 0.f;
     rv[2 * i + 1] = in ? (__uint_as_float(w[i] & 0xFFFF0000u) * f1) * f2 : 0.f;
   }
-  const int g = lane >> 2;                  // 16-byte group (32 elements) of the chunk
-  const bool nv = p.nv != 0;
-  const int lpb = bs_blk(nv) / 8;           // lanes per block
-  const int j = lane / lpb;                 // block of the chunk
-  const int emin = bs_emin(nv);
+  const int c = k / kChunk, o = k % kChunk;  // chunk, element offset in it
+  const int j = o / kBlk;                    // block of the chunk
+  // byte offset of the 8 elements' codes in the row: 16-byte group ob / 16, stored at group
+  // (ob / 16) ^ (r & 7)
+  const int ob = F == kBsF8 ? o : o / 2;
+  const int pos = ((((ob >> 4) ^ r) & 7) << 4) + (ob & 15);
   bool done = false;
 #pragma unroll
-  for (int term = 0; term < kBsTerms; ++term) {
+  for (int term = 0; term < kTerms; ++term) {
     float bmax = 0.f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) bmax = fmaxf(bmax, fabsf(rv[i]));
     bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 1));
     const float b2 = __shfl_xor_sync(0xffffffffu, bmax, 2);
-    if (!nv) bmax = fmaxf(bmax, b2);
+    if (kLpb == 4) bmax = fmaxf(bmax, b2);
     int sb = 0;  // scale byte
-    uint32_t packed = 0u;
+    uint32_t packed[2] = {0u, 0u};
     if (!done && bmax > 0.f) {
       int ex;
       (void)frexpf(bmax, &ex);
-      const int e = (ex - 1) - 2;  // block maximum / 2^e in [4, 8)
-      if (e >= emin) {
-        sb = bs_scale_byte(nv, e);
+      const int e = (ex - 1) - bs_top(F);  // block maximum / 2^e in [2^top, 2^(top+1))
+      if (e >= bs_emin(F)) {
+        sb = bs_scale_byte(F, e);
         const float inv = bs_pow2(-e), sc = bs_pow2(e);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          // two codes (element 2i in the low nibble), rounded to nearest even and saturated
-          // at 6 by the hardware conversion, and their values back as f16 (exact)
-          const __nv_fp4x2_storage_t c2 = __nv_cvt_float2_to_fp4x2(
-              make_float2(rv[2 * i] * inv, rv[2 * i + 1] * inv), __NV_E2M1, cudaRoundNearest);
-          const __half2_raw h = __nv_cvt_fp4x2_to_halfraw2(c2, __NV_E2M1);
-          rv[2 * i] = fmaf(-__half2float(__half(__half_raw{h.x})), sc, rv[2 * i]);
-          rv[2 * i + 1] = fmaf(-__half2float(__half(__half_raw{h.y})), sc, rv[2 * i + 1]);
-          packed |= (uint32_t)c2 << (8 * i);
+          float qa, qb;
+          const uint32_t c2 = bs_enc2<F>(rv[2 * i] * inv, rv[2 * i + 1] * inv, qa, qb);
+          rv[2 * i] = fmaf(-qa, sc, rv[2 * i]);
+          rv[2 * i + 1] = fmaf(-qb, sc, rv[2 * i + 1]);
+          if (F == kBsF8) packed[i >> 1] |= c2 << (16 * (i & 1));
+          else packed[0] |= c2 << (8 * i);
         }
       } else {
         done = true;  // below the scale range: this and the later terms are dropped
@@ -194,15 +239,17 @@ __device__ __forceinline__ void bs_split8(const BsSplitParams& p, const uint4& v
     } else {
       done = true;
     }
-    const size_t bidx = ((size_t)t * p.C + c) * kBsTerms + term;
-    // 32 elements are 16 bytes: group g of the row, stored at group g ^ (r & 7)
-    uint8_t* crow = p.codes + bidx * kBsBlock + (size_t)r * 128;
-    *reinterpret_cast<uint32_t*>(crow + (((g ^ (r & 7)) & 7) << 4) + (lane & 3) * 4) = packed;
-    const int sbr = bs_sbr(nv);
-    if (lane % lpb == 0) p.scales[bidx * (size_t)(kBsM * sbr) + (size_t)r * sbr + j] = (uint8_t)(done ? 0 : sb);
+    if (store) {
+      const size_t bidx = ((size_t)t * p.C + c) * kTerms + term;
+      uint8_t* crow = p.codes + bidx * kBsBlock + (size_t)r * 128;
+      if (F == kBsF8) *reinterpret_cast<uint2*>(crow + pos) = make_uint2(packed[0], packed[1]);
+      else *reinterpret_cast<uint32_t*>(crow + pos) = packed[0];
+      if (lane % kLpb == 0) p.scales[bidx * (size_t)(kBsM * kSbr) + (size_t)r * kSbr + j] = (uint8_t)(done ? 0 : sb);
+    }
   }
 }
 
+template <int F>
 __global__ void __launch_bounds__(kBsSplitThreads) qgemm_bs_split_kernel(const BsSplitParams p) {
   // x may come from the preceding grid.  Only once that grid has completed may the GEMM
   // launch: it reads the weights before it waits for this grid, and the grid before may have
@@ -214,9 +261,9 @@ __global__ void __launch_bounds__(kBsSplitThreads) qgemm_bs_split_kernel(const B
   const uint16_t* xr = p.x + (size_t)(live ? m : 0) * p.K;
   __shared__ float red[kBsSplitThreads / 32];
   // Phase 1: the row maximum.  Thread i reads the 8-element words k = 8 (i + 256 n); the same
-  // thread converts them in phase 2 (word n is lane i % 32 of chunk 8 n + i / 32), so the first
-  // kBsSplitRegs words stay in registers.
-  const int Kp = p.C * kBsK;
+  // thread converts them in phase 2 (word n is lane i % 32 of the warp span starting at
+  // 256 (8 n + i / 32)), so the first kBsSplitRegs words stay in registers.
+  const int Kp = p.C * bs_chunk(F);
   uint4 v[kBsSplitRegs];
   float amax = 0.f;
 #pragma unroll
@@ -239,7 +286,7 @@ __global__ void __launch_bounds__(kBsSplitThreads) qgemm_bs_split_kernel(const B
   if (amax > 0.f && amax <= 3.4e38f) {
     int ex;
     (void)frexpf(amax, &ex);
-    xe = (ex - 1) - bs_xshift(p.nv != 0);  // row maximum * 2^-xe in [2^xshift, 2^(xshift+1))
+    xe = (ex - 1) - bs_xshift(F);  // row maximum * 2^-xe in [2^xshift, 2^(xshift+1))
   }
   if (threadIdx.x == 0) p.x_exp[m] = live ? xe : 0;
   // 2^-xe as two exact factors (xe runs from -143 to 127)
@@ -247,16 +294,17 @@ __global__ void __launch_bounds__(kBsSplitThreads) qgemm_bs_split_kernel(const B
   const float f1 = bs_pow2(a1), f2 = bs_pow2(-xe - a1);
   const int t = m / kBsM, r = m % kBsM;
   const int lane = threadIdx.x & 31;
-  // Phase 2: word n of this thread is lane `lane` of chunk c = 8 (i + 256 n) / 256
+  // Phase 2, over the warp spans that start inside the padded K (warp-uniform conditions:
+  // every lane of a span takes part in its block reductions)
 #pragma unroll
   for (int n = 0; n < kBsSplitRegs; ++n) {
     const int k = (threadIdx.x + n * kBsSplitThreads) * 8;
-    if (k < Kp) bs_split8(p, v[n], live && k < p.K, f1, f2, t, r, k / kBsK, lane);
+    if (k - 8 * lane < Kp) bs_split8<F>(p, v[n], live && k < p.K, k < Kp, f1, f2, t, r, k, lane);
   }
-  for (int k = (threadIdx.x + kBsSplitRegs * kBsSplitThreads) * 8; k < Kp; k += kBsSplitThreads * 8) {
+  for (int k = (threadIdx.x + kBsSplitRegs * kBsSplitThreads) * 8; k - 8 * lane < Kp; k += kBsSplitThreads * 8) {
     const bool in = live && k < p.K;
     const uint4 w = in ? *reinterpret_cast<const uint4*>(xr + k) : make_uint4(0u, 0u, 0u, 0u);
-    bs_split8(p, w, in, f1, f2, t, r, k / kBsK, lane);
+    bs_split8<F>(p, w, in, k < Kp, f1, f2, t, r, k, lane);
   }
 }
 
@@ -275,12 +323,21 @@ __device__ __forceinline__ void bs_tmem_dealloc(uint32_t taddr, uint32_t ncols) 
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
                : "memory");
 }
-// D (+)= A * B^T with block scales: A, B K-major E2M1 in shared memory, the scale factors in
-// tensor memory at sfa / sfb; 16-element UE4M3 blocks (NVFP4) or 32-element E8M0 (MXFP4).
-template <bool NV>
+// D (+)= A * B^T with block scales: A, B K-major in shared memory, the scale factors in
+// tensor memory at sfa / sfb.  E2M1 with 16-element UE4M3 blocks (NVFP4) or 32-element E8M0
+// (MXFP4); E4M3 with 32-element E8M0 blocks (FP8).
+template <int F>
 __device__ __forceinline__ void bs_mma(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                        uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
-  if (NV)
+  if (F == kBsF8)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t"
+        "}" ::"r"(d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+  else if (F == kBsNv)
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
@@ -298,13 +355,17 @@ __device__ __forceinline__ void bs_mma(uint32_t d, uint64_t adesc, uint64_t bdes
         : "memory");
 }
 
-// The 4-byte scale word of one row for 64-K block kb: NVFP4 keeps 4 scales per 64 K (16 bytes
-// per row and chunk), MXFP4 2 (8 bytes; the upper bytes of the word are unused).
-template <bool NV>
+// The 4-byte scale word of one row for MMA K-block kb: NVFP4 keeps 4 scales per 64 K (16 bytes
+// per row and chunk), MXFP4 2 (8 bytes), FP8 x terms 1 per 32 K (4 bytes); the upper bytes of
+// the word are unused.
+template <int F>
 __device__ __forceinline__ uint32_t bs_sf_word(const uint8_t* row, int kb) {
-  if (NV) return reinterpret_cast<const uint32_t*>(row)[kb];
+  if (F == kBsNv) return reinterpret_cast<const uint32_t*>(row)[kb];
+  if (F == kBsF8) return (uint32_t)row[kb];
   return (uint32_t)reinterpret_cast<const uint16_t*>(row)[kb];
 }
+// The FP8 weights' block scales: 2^0 in E8M0 (their tensor scale is applied in the epilogue)
+constexpr uint32_t kBsUnitSf = 0x7F7F7F7Fu;
 __device__ __forceinline__ void bs_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                : "memory");
@@ -350,13 +411,20 @@ __device__ __forceinline__ float bs_scale_pow2(float v, int e) {
   return (e >= -126 && e <= 127) ? v * __int_as_float((e + 127) << 23) : ldexpf(v, e);
 }
 
-template <bool NV>
+template <int F>
 __global__ void __launch_bounds__(kBsThreads, 1) qgemm_bs_kernel(const __grid_constant__ BsParams p) {
-  using L = BsLay<NV>;
+  using L = BsLay<F>;
+  constexpr int kTerms = L::Terms;
+  constexpr int kBsStages = L::Stages;
   constexpr int kBsStage = L::Stage;
+  constexpr int kBsACodes = L::ACodes;
   constexpr int kBsAScales = L::AScales;
   constexpr int kBsSBlock = L::SB;
-  constexpr int kSbr = bs_sbr(NV);
+  constexpr int kBsWSBlock = L::WSB;
+  constexpr int kBsSfCols = L::SfCols;
+  constexpr int kSbr = bs_sbr(F);
+  constexpr int kWSbr = bs_wsbr(F);
+  constexpr bool kTs = F != kBsMx;  // a per-tensor scale (NVFP4, FP8)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sbase = smem_u32(smem);
@@ -414,22 +482,23 @@ __global__ void __launch_bounds__(kBsThreads, 1) qgemm_bs_kernel(const __grid_co
           const uint32_t st = sbase + (uint32_t)(sp.slot * kBsStage);
           uint32_t bytes = kBsACodes + kBsAScales;
           for (int j = 0; j < kBsWT; ++j)
-            if (kBsWT * nt + j < n_row_tiles) bytes += kBsBlock + kBsSBlock;
+            if (kBsWT * nt + j < n_row_tiles) bytes += kBsBlock + kBsWSBlock;
           mbar_arrive_expect_tx(fb, bytes);
           for (int j = 0; j < kBsWT; ++j) {
             const int64_t t = kBsWT * (int64_t)nt + j;
             if (t >= n_row_tiles) continue;
             const int64_t blk = t * p.C + c;
             bulk_load(st + kBsACodes + j * kBsBlock, p.wcodes + blk * kBsBlock, kBsBlock, fb, pol_w);
-            bulk_load(st + kBsACodes + kBsBCodes + kBsAScales + j * kBsSBlock,
-                      p.wscales + blk * kBsSBlock, kBsSBlock, fb, pol_w);
+            if (kBsWSBlock > 0)
+              bulk_load(st + kBsACodes + kBsBCodes + kBsAScales + j * kBsWSBlock,
+                        p.wscales + blk * kBsWSBlock, kBsWSBlock, fb, pol_w);
           }
           // the split x comes from the preceding grid
           if (!waited) {
             griddep_wait();
             waited = true;
           }
-          const int64_t xb = ((int64_t)mt * p.C + c) * kBsTerms;
+          const int64_t xb = ((int64_t)mt * p.C + c) * kTerms;
           bulk_load(st, p.xcodes + xb * kBsBlock, kBsACodes, fb, pol_x);
           bulk_load(st + kBsACodes + kBsBCodes, p.xscales + xb * kBsSBlock, kBsAScales, fb, pol_x);
           sp.next(kBsStages);
@@ -469,13 +538,13 @@ __global__ void __launch_bounds__(kBsThreads, 1) qgemm_bs_kernel(const __grid_co
           const uint64_t bdesc0 = smem_desc_sw128(st + kBsACodes);
           const uint32_t sf0 = tmem + (uint32_t)(kBsN + sp.slot * kBsSfCols);
 #pragma unroll
-          for (int kb = 0; kb < kBsK / 64; ++kb) {
+          for (int kb = 0; kb < kBsKB; ++kb) {
 #pragma unroll
-            for (int t = 0; t < kBsTerms; ++t) {
+            for (int t = 0; t < kTerms; ++t) {
               const uint64_t adesc = smem_desc_sw128(st + (uint32_t)(t * kBsBlock)) + (uint64_t)(kb * 2);
-              bs_mma<NV>(tmem, adesc, bdesc0 + (uint64_t)(kb * 2), L::Idesc,
-                     sf0 + (uint32_t)((t * 4 + kb) * 4), sf0 + (uint32_t)(48 + kb * 4 * kBsWT),
-                     (c | kb | t) != 0 ? 1u : 0u);
+              bs_mma<F>(tmem, adesc, bdesc0 + (uint64_t)(kb * 2), L::Idesc,
+                        sf0 + (uint32_t)((t * 4 + kb) * 4), sf0 + (uint32_t)(L::ASf + kb * 4 * kBsWT),
+                        (c | kb | t) != 0 ? 1u : 0u);
             }
           }
           bs_commit(bar_empty + 8 * sp.slot);
@@ -511,22 +580,23 @@ __global__ void __launch_bounds__(kBsThreads, 1) qgemm_bs_kernel(const __grid_co
         if (!ok) break;
         tc_fence_after();
         const uint8_t* st = smem + sp.slot * kBsStage;
-        const uint8_t* sa = st + kBsACodes + kBsBCodes;  // x-term scales [3][128][8]
-        const uint8_t* sb = sa + kBsAScales;              // weight scales [kBsWT][128][sbr]
+        const uint8_t* sa = st + kBsACodes + kBsBCodes;  // x-term scales [terms][128][sbr]
+        const uint8_t* sb = sa + kBsAScales;              // weight scales [kBsWT][128][wsbr]
         uint32_t v[kBsSfCols];
 #pragma unroll
-        for (int t = 0; t < kBsTerms; ++t)
+        for (int t = 0; t < kTerms; ++t)
 #pragma unroll
           for (int r1 = 0; r1 < 4; ++r1) {
             const uint8_t* row = sa + t * kBsSBlock + (r1 * 32 + lane) * kSbr;
 #pragma unroll
-            for (int kb = 0; kb < 4; ++kb) v[(t * 4 + kb) * 4 + r1] = bs_sf_word<NV>(row, kb);
+            for (int kb = 0; kb < kBsKB; ++kb) v[(t * 4 + kb) * 4 + r1] = bs_sf_word<F>(row, kb);
           }
 #pragma unroll
         for (int r1 = 0; r1 < 4 * kBsWT; ++r1) {
-          const uint8_t* row = sb + (r1 >> 2) * kBsSBlock + ((r1 & 3) * 32 + lane) * kSbr;
+          const uint8_t* row = sb + (r1 >> 2) * kBsWSBlock + ((r1 & 3) * 32 + lane) * kWSbr;
 #pragma unroll
-          for (int kb = 0; kb < 4; ++kb) v[48 + kb * 4 * kBsWT + r1] = bs_sf_word<NV>(row, kb);
+          for (int kb = 0; kb < kBsKB; ++kb)
+            v[L::ASf + kb * 4 * kBsWT + r1] = kWSbr == 0 ? kBsUnitSf : bs_sf_word<F>(row, kb);
         }
         const uint32_t ta = tmem + lane_base + (uint32_t)(kBsN + sp.slot * kBsSfCols);
 #pragma unroll
@@ -550,9 +620,9 @@ __global__ void __launch_bounds__(kBsThreads, 1) qgemm_bs_kernel(const __grid_co
       const int mt = u % p.Mt, nt = u / p.Mt;
       const int m = mt * kBsM + q * 32 + lane;
       const int xe = (m < p.M) ? p.x_exp[m] : 0;
-      const float tsv = NV ? __ldg(p.ts) : 1.0f;  // NVFP4 tensor scale, applied before 2^xe
-      // y = (acc * ts) * 2^xe: the tensor scale (NVFP4) rounds once, the power of two is exact
-      auto yv = [&](uint32_t u) { return bs_scale_pow2(NV ? __uint_as_float(u) * tsv : __uint_as_float(u), xe); };
+      const float tsv = kTs ? __ldg(p.ts) : 1.0f;  // tensor scale, applied before 2^xe
+      // y = (acc * ts) * 2^xe: the tensor scale rounds once, the power of two is exact
+      auto yv = [&](uint32_t u) { return bs_scale_pow2(kTs ? __uint_as_float(u) * tsv : __uint_as_float(u), xe); };
       bool ok = mbar_wait(bar_acc, (uint32_t)ti & 1u, abort_flag, p.dev_err, kErrTimeout);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
@@ -619,17 +689,17 @@ __global__ void __launch_bounds__(kBsThreads, 1) qgemm_bs_kernel(const __grid_co
 // operand (one 128-row weight tile per unit, its scales SFA), the split x the N operand
 // (N = M rounded up to 16 rows of the first token tile, its scales SFB), and K is split
 // over S ranges so that the units fill the SMs; S > 1 writes fp32 partials that the split-K
-// reduce kernel sums in the order s = 0..S-1.  Per 256-K chunk: 4 K-blocks x 3 terms of
-// M128 N(M) K64 MMAs.  At these widths the issuing thread bounds the MMA stream, so two
-// issuers take alternate chunks of a unit, each into its own accumulator; the epilogue adds
-// them in the order even + odd.  Stage: [weight codes 16 KB][3 x N x 128 term codes][weight
-// scales 1 KB][3 x N x 8 term scales], rounded up to 1 KB; an even number of stages, so that a
-// stage's previous use belongs to the same issuer.  TMEM: the two accumulators (N columns
-// each), then per stage 64 columns of scale factors: the weights' K-block kb at 4 kb (4 row
-// groups), term j's K-block kb at 16 + 4 (4 j + kb).
+// reduce kernel sums in the order s = 0..S-1.  Per chunk: 4 K-blocks x terms MMAs of
+// M128 N(M) (K64 E2M1 or K32 E4M3).  At these widths the issuing thread bounds the MMA stream,
+// so two issuers take alternate chunks of a unit, each into its own accumulator; the epilogue
+// adds them in the order even + odd.  Stage: [weight codes 16 KB][terms x N x 128 term codes]
+// [weight scales 128 x wsbr][terms x N x sbr term scales], rounded up to 1 KB; an even number
+// of stages, so that a stage's previous use belongs to the same issuer.  TMEM: the two
+// accumulators (N columns each), then per stage 16 + 16 terms columns of scale factors: the
+// weights' K-block kb at 4 kb (4 row groups), term j's K-block kb at 16 + 4 (4 j + kb).
 // ---------------------------------------------------------------------------------------
-constexpr int kBdMaxStages = 6;
-constexpr int kBdSfCols = 16 + kBsTerms * 16;  // 64
+__host__ __device__ constexpr int bd_sf_cols(int f) { return 16 + bs_terms(f) * 16; }
+__host__ __device__ constexpr int bd_max_stages(int f) { return f == kBsF8 ? 8 : 6; }
 constexpr int kBdIssuer2Warp = 10;
 constexpr int kBdThreads = 11 * 32;
 
@@ -640,17 +710,21 @@ struct BsDecParams {
   const int* x_exp;
   const uint8_t* wcodes;
   const uint8_t* wscales;
-  const float* ts;  // NVFP4 tensor scale (device), else nullptr
+  const float* ts;  // NVFP4 / FP8 tensor scale (device), else nullptr
   float* ws;  // S > 1: partials [S][M][N], fully scaled
   void* out;
   int out_bf16;
   int* dev_err;
 };
 
-template <bool NV>
+template <int F>
 __global__ void __launch_bounds__(kBdThreads, 1) qgemm_bs_dec_kernel(const __grid_constant__ BsDecParams p) {
-  constexpr int kSbr = bs_sbr(NV);
-  constexpr int kSBlock = kBsM * kSbr;
+  constexpr int kTerms = bs_terms(F);
+  constexpr int kSbr = bs_sbr(F), kWSbr = bs_wsbr(F);
+  constexpr int kSBlock = kBsM * kSbr;    // one 128-row block of term scales in the split
+  constexpr int kWSBlock = kBsM * kWSbr;  // one 128-row block of weight scales
+  constexpr int kBdSfCols = bd_sf_cols(F);
+  constexpr bool kTs = F != kBsMx;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sbase = smem_u32(smem);
@@ -667,10 +741,9 @@ __global__ void __launch_bounds__(kBdThreads, 1) qgemm_bs_dec_kernel(const __gri
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int Nb = p.Nb;
   const uint32_t xterm = (uint32_t)Nb * 128u;      // one term's codes in a stage
-  const uint32_t off_ws = kBsBlock + kBsTerms * xterm;            // weight scales
-  const uint32_t off_xs = off_ws + kSBlock;                       // term scales
-  const uint32_t idesc = (1u << 7) | (1u << 10) | ((uint32_t)(Nb >> 3) << 17) | ((NV ? 0u : 1u) << 23) |
-                         ((uint32_t)(kBsM >> 4) << 24);
+  const uint32_t off_ws = kBsBlock + kTerms * xterm;  // weight scales
+  const uint32_t off_xs = off_ws + kWSBlock;           // term scales
+  const uint32_t idesc = bs_idesc(F, Nb);
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < NST; ++s) {
       mbar_init(bar_full + 8 * s, 1);
@@ -720,16 +793,16 @@ __global__ void __launch_bounds__(kBdThreads, 1) qgemm_bs_dec_kernel(const __gri
           }
           const uint32_t fb = bar_full + 8 * sp.slot;
           const uint32_t st = sbase + (uint32_t)(sp.slot * p.stage_bytes);
-          mbar_arrive_expect_tx(fb, kBsBlock + kSBlock + kBsTerms * (xterm + (uint32_t)(Nb * kSbr)));
+          mbar_arrive_expect_tx(fb, kBsBlock + kWSBlock + kTerms * (xterm + (uint32_t)(Nb * kSbr)));
           const int64_t blk = (int64_t)t * p.C + c;
           bulk_load(st, p.wcodes + blk * kBsBlock, kBsBlock, fb, pol_w);
-          bulk_load(st + off_ws, p.wscales + blk * kSBlock, kSBlock, fb, pol_w);
+          if (kWSBlock > 0) bulk_load(st + off_ws, p.wscales + blk * kWSBlock, kWSBlock, fb, pol_w);
           if (!waited) {
             griddep_wait();  // the split x comes from the preceding grid
             waited = true;
           }
-          for (int j = 0; j < kBsTerms; ++j) {
-            const int64_t xb = (int64_t)c * kBsTerms + j;  // token tile 0
+          for (int j = 0; j < kTerms; ++j) {
+            const int64_t xb = (int64_t)c * kTerms + j;  // token tile 0
             bulk_load(st + kBsBlock + (uint32_t)j * xterm, p.xcodes + xb * kBsBlock, xterm, fb, pol_x);
             bulk_load(st + off_xs + (uint32_t)(j * Nb * kSbr), p.xscales + xb * kSBlock, (uint32_t)(Nb * kSbr), fb, pol_x);
           }
@@ -778,11 +851,11 @@ __global__ void __launch_bounds__(kBdThreads, 1) qgemm_bs_dec_kernel(const __gri
           const uint64_t adesc0 = smem_desc_sw128(st);
           const uint32_t sf0 = tmem + sf_col0 + (uint32_t)(sp.slot * kBdSfCols);
 #pragma unroll
-          for (int kb = 0; kb < kBsK / 64; ++kb) {
+          for (int kb = 0; kb < kBsKB; ++kb) {
 #pragma unroll
-            for (int j = 0; j < kBsTerms; ++j) {
+            for (int j = 0; j < kTerms; ++j) {
               const uint64_t bdesc = smem_desc_sw128(st + kBsBlock + (uint32_t)j * xterm) + (uint64_t)(kb * 2);
-              bs_mma<NV>(d, adesc0 + (uint64_t)(kb * 2), bdesc, idesc, sf0 + (uint32_t)(kb * 4),
+              bs_mma<F>(d, adesc0 + (uint64_t)(kb * 2), bdesc, idesc, sf0 + (uint32_t)(kb * 4),
                      sf0 + (uint32_t)(16 + (j * 4 + kb) * 4), (c - c0 >= 2 || kb || j) ? 1u : 0u);
             }
           }
@@ -822,19 +895,19 @@ __global__ void __launch_bounds__(kBdThreads, 1) qgemm_bs_dec_kernel(const __gri
         uint32_t v[kBdSfCols];
 #pragma unroll
         for (int r1 = 0; r1 < 4; ++r1) {
-          const uint8_t* row = st + off_ws + (r1 * 32 + lane) * kSbr;
+          const uint8_t* row = st + off_ws + (r1 * 32 + lane) * kWSbr;
 #pragma unroll
-          for (int kb = 0; kb < 4; ++kb) v[kb * 4 + r1] = bs_sf_word<NV>(row, kb);
+          for (int kb = 0; kb < kBsKB; ++kb) v[kb * 4 + r1] = kWSbr == 0 ? kBsUnitSf : bs_sf_word<F>(row, kb);
         }
 #pragma unroll
-        for (int j = 0; j < kBsTerms; ++j)
+        for (int j = 0; j < kTerms; ++j)
 #pragma unroll
           for (int r1 = 0; r1 < 4; ++r1) {
             const int rw = r1 * 32 + lane;
             const uint8_t* row = st + off_xs + j * Nb * kSbr + rw * kSbr;
 #pragma unroll
-            for (int kb = 0; kb < 4; ++kb)
-              v[16 + (j * 4 + kb) * 4 + r1] = rw < Nb ? bs_sf_word<NV>(row, kb) : 0u;
+            for (int kb = 0; kb < kBsKB; ++kb)
+              v[16 + (j * 4 + kb) * 4 + r1] = rw < Nb ? bs_sf_word<F>(row, kb) : 0u;
           }
         const uint32_t ta = tmem + lane_base + sf_col0 + (uint32_t)(sp.slot * kBdSfCols);
 #pragma unroll
@@ -855,7 +928,7 @@ __global__ void __launch_bounds__(kBdThreads, 1) qgemm_bs_dec_kernel(const __gri
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     griddep_wait();  // x_exp comes from the split kernel
     const size_t MN = (size_t)p.M * p.N;
-    const float tsv = NV ? __ldg(p.ts) : 1.0f;  // NVFP4 tensor scale, applied before 2^x_exp
+    const float tsv = kTs ? __ldg(p.ts) : 1.0f;  // tensor scale, applied before 2^x_exp
     int ti = 0;
     for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++ti) {
       int t, s, c0, c1;
@@ -884,7 +957,7 @@ __global__ void __launch_bounds__(kBdThreads, 1) qgemm_bs_dec_kernel(const __gri
           for (int i = 0; i < 16; ++i) {
             const int b = cb + i;
             if (b < p.M) {
-              const float acc = NV ? __uint_as_float(v[i]) * tsv : __uint_as_float(v[i]);
+              const float acc = kTs ? __uint_as_float(v[i]) * tsv : __uint_as_float(v[i]);
               const float val = bs_scale_pow2(acc, __ldg(p.x_exp + b));
               if (p.S > 1) p.ws[(size_t)s * MN + (size_t)b * p.N + n] = val;
               else if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)b * p.N + n] = __float2bfloat16_rn(val);
@@ -911,15 +984,16 @@ __global__ void __launch_bounds__(kBdThreads, 1) qgemm_bs_dec_kernel(const __gri
 // ---------------------------------------------------------------------------------------
 // Launchers
 // ---------------------------------------------------------------------------------------
-cudaError_t launch_bs_split(bool nv, const uint16_t* x, int M, int K, uint8_t* codes,
+cudaError_t launch_bs_split(int f, const uint16_t* x, int M, int K, uint8_t* codes,
                             uint8_t* scales, int* x_exp, cudaStream_t stream) {
+  if (f < kBsMx || f > kBsF8) return cudaErrorInvalidValue;
   BsSplitParams p{};
   p.x = x;
   p.M = M;
   p.K = K;
-  p.C = (K + kBsK - 1) / kBsK;
+  p.C = (K + bs_chunk(f) - 1) / bs_chunk(f);
   p.Mt = (M + kBsM - 1) / kBsM;
-  p.nv = nv ? 1 : 0;
+  p.f = f;
   p.codes = codes;
   p.scales = scales;
   p.x_exp = x_exp;
@@ -932,7 +1006,9 @@ cudaError_t launch_bs_split(bool nv, const uint16_t* x, int M, int K, uint8_t* c
   at[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, qgemm_bs_split_kernel, p);
+  return f == kBsF8   ? cudaLaunchKernelEx(&cfg, qgemm_bs_split_kernel<kBsF8>, p)
+         : f == kBsNv ? cudaLaunchKernelEx(&cfg, qgemm_bs_split_kernel<kBsNv>, p)
+                      : cudaLaunchKernelEx(&cfg, qgemm_bs_split_kernel<kBsMx>, p);
 }
 
 // SMs of device `dev`, read once per device (devices beyond 64 read it on every launch).
@@ -964,7 +1040,7 @@ static cudaError_t bs_launch_pdl(cudaLaunchConfig_t& cfg, cudaStream_t stream, c
   return cudaSuccess;
 }
 
-template <bool NV>
+template <int F>
 static cudaError_t launch_bs_gemm_t(int M, int N, int K, const uint8_t* xcodes,
                                     const uint8_t* xscales, const int* x_exp, const uint8_t* wcodes,
                                     const uint8_t* wscales, const float* ts, void* out,
@@ -973,13 +1049,13 @@ static cudaError_t launch_bs_gemm_t(int M, int N, int K, const uint8_t* xcodes,
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  e = bs_smem_attr((const void*)qgemm_bs_kernel<NV>, set_mask, dev, BsLay<NV>::Smem);
+  e = bs_smem_attr((const void*)qgemm_bs_kernel<F>, set_mask, dev, BsLay<F>::Smem);
   if (e != cudaSuccess) return e;
   BsParams p{};
   p.M = M;
   p.N = N;
   p.K = K;
-  p.C = (K + kBsK - 1) / kBsK;
+  p.C = (K + bs_chunk(F) - 1) / bs_chunk(F);
   p.Mt = (M + kBsM - 1) / kBsM;
   p.Nt = (N + kBsN - 1) / kBsN;
   p.units = p.Mt * p.Nt;
@@ -995,33 +1071,43 @@ static cudaError_t launch_bs_gemm_t(int M, int N, int K, const uint8_t* xcodes,
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)std::min(p.units, bs_sm_count(dev)), 1, 1);
   cfg.blockDim = dim3(kBsThreads, 1, 1);
-  cfg.dynamicSmemBytes = BsLay<NV>::Smem;
+  cfg.dynamicSmemBytes = BsLay<F>::Smem;
   cudaLaunchAttribute at[1];
   bs_launch_pdl(cfg, stream, at);
-  return cudaLaunchKernelEx(&cfg, qgemm_bs_kernel<NV>, p);
+  return cudaLaunchKernelEx(&cfg, qgemm_bs_kernel<F>, p);
 }
 
-cudaError_t launch_bs_gemm(bool nv, int M, int N, int K, const uint8_t* xcodes,
+cudaError_t launch_bs_gemm(int f, int M, int N, int K, const uint8_t* xcodes,
                            const uint8_t* xscales, const int* x_exp, const uint8_t* wcodes,
                            const uint8_t* wscales, const float* ts, void* out, int out_bf16,
                            int* dev_err, cudaStream_t stream) {
-  return nv ? launch_bs_gemm_t<true>(M, N, K, xcodes, xscales, x_exp, wcodes, wscales, ts, out,
-                                     out_bf16, dev_err, stream)
-            : launch_bs_gemm_t<false>(M, N, K, xcodes, xscales, x_exp, wcodes, wscales, ts, out,
-                                      out_bf16, dev_err, stream);
+  switch (f) {
+    case kBsMx:
+      return launch_bs_gemm_t<kBsMx>(M, N, K, xcodes, xscales, x_exp, wcodes, wscales, ts, out,
+                                     out_bf16, dev_err, stream);
+    case kBsNv:
+      return launch_bs_gemm_t<kBsNv>(M, N, K, xcodes, xscales, x_exp, wcodes, wscales, ts, out,
+                                     out_bf16, dev_err, stream);
+    case kBsF8:
+      return launch_bs_gemm_t<kBsF8>(M, N, K, xcodes, xscales, x_exp, wcodes, wscales, ts, out,
+                                     out_bf16, dev_err, stream);
+    default:
+      return cudaErrorInvalidValue;
+  }
 }
 
-// K split of the decode kernel: a function of (N, K) only (the unit count is weighed against
-// the 148 SMs of a B200), the smallest S of least cost (waves of units x (chunks per unit + a
-// fixed cost of ~3 chunks) + a small charge per split for the partials).
+// K split of the decode kernel: a function of (format, N, K) only (the unit count is weighed
+// against the 148 SMs of a B200), the smallest S of least cost (waves of units x (K per unit +
+// a fixed cost of ~768 K) + a small charge per split for the partials), in units of 256 K.
 constexpr int kBsSplitSMs = 148;
-int bs_dec_split(int64_t N, int64_t K, int sms) {
-  const int64_t T = row_tiles(N), C = (K + kBsK - 1) / kBsK;
+int bs_dec_split(int f, int64_t N, int64_t K, int sms) {
+  const int64_t T = row_tiles(N), C = (K + bs_chunk(f) - 1) / bs_chunk(f);
+  const double ck = double(bs_chunk(f)) / 256.0;
   int best = 1;
   double best_cost = 0.0;
   for (int64_t S = 1; S <= std::min<int64_t>(16, C); ++S) {
     const int64_t waves = (T * S + sms - 1) / sms;
-    const double cost = double(waves * ((C + S - 1) / S + 3)) + 0.25 * double(S);
+    const double cost = double(waves) * (double((C + S - 1) / S) * ck + 3.0) + 0.25 * double(S);
     if (S == 1 || cost < best_cost - 1e-9) {
       best_cost = cost;
       best = (int)S;
@@ -1032,18 +1118,18 @@ int bs_dec_split(int64_t N, int64_t K, int sms) {
 
 // Workspace of the block-scaled path: split codes, split scales, row exponents and, for
 // decode widths with a K split, the fp32 partials.
-size_t bs_workspace_bytes(bool nv, int64_t M, int64_t N, int64_t K, size_t* off_scales,
+size_t bs_workspace_bytes(int f, int64_t M, int64_t N, int64_t K, size_t* off_scales,
                           size_t* off_exp, size_t* off_part) {
-  const int64_t C = (K + kBsK - 1) / kBsK, Mt = (M + kBsM - 1) / kBsM;
-  const size_t codes = (size_t)(Mt * C * kBsTerms) * kBsBlock;
-  const size_t scales = (size_t)(Mt * C * kBsTerms) * (size_t)(kBsM * bs_sbr(nv));
+  const int64_t C = (K + bs_chunk(f) - 1) / bs_chunk(f), Mt = (M + kBsM - 1) / kBsM;
+  const size_t codes = (size_t)(Mt * C * bs_terms(f)) * kBsBlock;
+  const size_t scales = (size_t)(Mt * C * bs_terms(f)) * (size_t)(kBsM * bs_sbr(f));
   if (off_scales) *off_scales = codes;
   if (off_exp) *off_exp = codes + scales;
   size_t total = codes + scales + (size_t)Mt * kBsM * 4;
   total = (total + 255) / 256 * 256;
   if (off_part) *off_part = total;
   if (M <= kBsM && N > 0) {
-    const int S = bs_dec_split(N, K, kBsSplitSMs);
+    const int S = bs_dec_split(f, N, K, kBsSplitSMs);
     if (S > 1) total += (size_t)S * (size_t)M * (size_t)N * 4;
   }
   return total;
@@ -1051,7 +1137,7 @@ size_t bs_workspace_bytes(bool nv, int64_t M, int64_t N, int64_t K, size_t* off_
 
 cudaError_t launch_reduce(const ReduceParams& rp, cudaStream_t stream);
 
-template <bool NV>
+template <int F>
 static cudaError_t launch_bs_dec_t(int M, int N, int K, const uint8_t* xcodes,
                                    const uint8_t* xscales, const int* x_exp, const uint8_t* wcodes,
                                    const uint8_t* wscales, const float* ts, float* part, void* out,
@@ -1060,20 +1146,21 @@ static cudaError_t launch_bs_dec_t(int M, int N, int K, const uint8_t* xcodes,
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  e = bs_smem_attr((const void*)qgemm_bs_dec_kernel<NV>, set_mask, dev, kSmemLimit);
+  e = bs_smem_attr((const void*)qgemm_bs_dec_kernel<F>, set_mask, dev, kSmemLimit);
   if (e != cudaSuccess) return e;
-  constexpr int kSbr = bs_sbr(NV);
+  constexpr int kTerms = bs_terms(F);
   BsDecParams p{};
   p.M = M;
   p.N = N;
   p.K = K;
-  p.C = (K + kBsK - 1) / kBsK;
+  p.C = (K + bs_chunk(F) - 1) / bs_chunk(F);
   p.Nb = (M + 15) / 16 * 16;
-  p.S = bs_dec_split(N, K, kBsSplitSMs);
+  p.S = bs_dec_split(F, N, K, kBsSplitSMs);
   p.units = (int)row_tiles(N) * p.S;
-  p.stage_bytes = (kBsBlock + kBsTerms * p.Nb * 128 + kBsM * kSbr + kBsTerms * p.Nb * kSbr + 1023) / 1024 * 1024;
-  p.stages = std::min({kBdMaxStages, (kSmemLimit - 1024 - 256) / p.stage_bytes,
-                       (kBsTmemCols - 2 * p.Nb) / kBdSfCols}) & ~1;  // even
+  p.stage_bytes = (kBsBlock + kTerms * p.Nb * 128 + kBsM * bs_wsbr(F) + kTerms * p.Nb * bs_sbr(F) + 1023) /
+                  1024 * 1024;
+  p.stages = std::min({bd_max_stages(F), (kSmemLimit - 1024 - 256) / p.stage_bytes,
+                       (kBsTmemCols - 2 * p.Nb) / bd_sf_cols(F)}) & ~1;  // even
   if (p.stages < 2) return cudaErrorInvalidValue;
   p.xcodes = xcodes;
   p.xscales = xscales;
@@ -1091,7 +1178,7 @@ static cudaError_t launch_bs_dec_t(int M, int N, int K, const uint8_t* xcodes,
   cfg.dynamicSmemBytes = 1024 + (size_t)p.stages * p.stage_bytes + 256;
   cudaLaunchAttribute at[1];
   bs_launch_pdl(cfg, stream, at);
-  e = cudaLaunchKernelEx(&cfg, qgemm_bs_dec_kernel<NV>, p);
+  e = cudaLaunchKernelEx(&cfg, qgemm_bs_dec_kernel<F>, p);
   if (e != cudaSuccess || p.S == 1) return e;
   ReduceParams rp{};
   rp.ws = part;
@@ -1105,14 +1192,23 @@ static cudaError_t launch_bs_dec_t(int M, int N, int K, const uint8_t* xcodes,
 }
 
 // Decode widths: queues the GEMM (and the split-K reduce when S > 1).
-cudaError_t launch_bs_dec(bool nv, int M, int N, int K, const uint8_t* xcodes,
+cudaError_t launch_bs_dec(int f, int M, int N, int K, const uint8_t* xcodes,
                           const uint8_t* xscales, const int* x_exp, const uint8_t* wcodes,
                           const uint8_t* wscales, const float* ts, float* part, void* out,
                           int out_bf16, int* dev_err, cudaStream_t stream) {
-  return nv ? launch_bs_dec_t<true>(M, N, K, xcodes, xscales, x_exp, wcodes, wscales, ts, part,
-                                    out, out_bf16, dev_err, stream)
-            : launch_bs_dec_t<false>(M, N, K, xcodes, xscales, x_exp, wcodes, wscales, ts, part,
-                                     out, out_bf16, dev_err, stream);
+  switch (f) {
+    case kBsMx:
+      return launch_bs_dec_t<kBsMx>(M, N, K, xcodes, xscales, x_exp, wcodes, wscales, ts, part,
+                                    out, out_bf16, dev_err, stream);
+    case kBsNv:
+      return launch_bs_dec_t<kBsNv>(M, N, K, xcodes, xscales, x_exp, wcodes, wscales, ts, part,
+                                    out, out_bf16, dev_err, stream);
+    case kBsF8:
+      return launch_bs_dec_t<kBsF8>(M, N, K, xcodes, xscales, x_exp, wcodes, wscales, ts, part,
+                                    out, out_bf16, dev_err, stream);
+    default:
+      return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace qg

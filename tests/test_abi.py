@@ -103,8 +103,8 @@ def test_argument_errors(lib):
 
 def test_block_scaled_argument_errors(lib):
     sz = ctypes.c_size_t()
-    # the block-scaled path takes MXFP4 and NVFP4 weights, and checks before any device work
-    for fmt in (0, 3):
+    # the block-scaled path takes MXFP4, NVFP4 and FP8 weights, and checks before any device work
+    for fmt in (0, 7):
         assert lib.qgemm_bs_workspace_size(fmt, 256, 256, 128, ctypes.byref(sz)) == 1
         assert lib.qgemm_bs_run(fmt, 16, 4, 64, 16, 16, 16, 8, 16, 0, 16, 1 << 20, None) == 1
     assert lib.qgemm_bs_workspace_size(2, 256, 48, 128, ctypes.byref(sz)) == 3      # K % 32
@@ -113,15 +113,18 @@ def test_block_scaled_argument_errors(lib):
     assert lib.qgemm_bs_run(2, 8, 4, 64, 16, 16, None, 8, 16, 0, 16, 1 << 20, None) == 5
     assert lib.qgemm_bs_run(2, 16, 4, 64, 16, 16, None, 8, 16, 0, 16, 16, None) == 6  # workspace
     assert lib.qgemm_bs_run(1, 16, 4, 64, 16, 16, None, 8, 16, 0, 16, 1 << 20, None) == 4  # NVFP4 ts
+    assert lib.qgemm_bs_run(3, 16, 4, 64, 16, None, None, 8, 16, 0, 16, 1 << 20, None) == 4  # FP8 ts
     assert lib.qgemm_bs_split_x(2, 16, 4, 48, 16, 16, 16, None) == 3                 # K % 32
     assert lib.qgemm_bs_split_x(2, 16, 4, 64, None, 16, 16, None) == 4
     assert lib.qgemm_bs_split_x(0, 16, 4, 64, 16, 16, 16, None) == 1                 # format
     c, s, e = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
-    for fmt, sbr in ((2, 8), (1, 16)):
+    for fmt, chunks, terms, sbr in ((2, 2, 3, 8), (1, 2, 3, 16), (3, 3, 2, 4)):
         assert lib.qgemm_bs_split_size(fmt, 300, 320, ctypes.byref(c), ctypes.byref(s),
                                        ctypes.byref(e)) == 0
-        # 3 token tiles x 2 chunks x 3 terms of 128 x 128 code bytes and 128 x sbr scale bytes
-        assert (c.value, s.value, e.value) == (3 * 2 * 3 * 16384, 3 * 2 * 3 * 128 * sbr, 3 * 128 * 4)
+        # 3 token tiles x chunks (of 256 K, 128 for FP8) x terms of 128 x 128 code bytes and
+        # 128 x sbr scale bytes
+        n = 3 * chunks * terms
+        assert (c.value, s.value, e.value) == (n * 16384, n * 128 * sbr, 3 * 128 * 4)
         assert lib.qgemm_bs_workspace_size(fmt, 256, 320, 300, ctypes.byref(sz)) == 0
         assert sz.value == c.value + s.value + e.value
 

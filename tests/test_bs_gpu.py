@@ -1,9 +1,10 @@
-"""GPU parity of the block-scaled path for MXFP4 and NVFP4 weights (qgemm_bs_split_x /
+"""GPU parity of the block-scaled path for MXFP4, NVFP4 and FP8 weights (qgemm_bs_split_x /
 qgemm_bs_run) against the CPU oracle, through the C ABI.
 
 Bars:
-  * the split of x is exact: the sum of the three E2M1 terms the GPU writes (decoded on the
-    host from the layout of include/qgemm.h) equals oracle.split_x_bs bit for bit;
+  * the split of x is exact: the sum of the terms the GPU writes (three E2M1 terms for FP4
+    weights, two E4M3 terms for FP8; decoded on the host from the layout of include/qgemm.h)
+    equals oracle.split_x_bs bit for bit;
   * the GEMM is the product of that split with the dequantised weights up to fp32
     accumulation (normalised error 2e-5), and within the method's 1e-3 of the exact product
     at K >= 1024 (the split's own residual is measured in the oracle pins);
@@ -35,23 +36,31 @@ def _lib():
     assert qgemm.device_status(reset=True) == qgemm.OK
 
 
+# per weight format: terms, K per chunk, block, scale bytes per row and chunk
+SPLIT_GEOM = {"mxfp4": (3, 256, 32, 8), "nvfp4": (3, 256, 16, 16), "fp8": (2, 128, 32, 4)}
+
+
 def _decode_split(fmt, codes, scales, x_exp, M, K):
-    """Sum of the three terms per element, from the documented layout (numpy only)."""
-    C, Mt = -(-K // 256), -(-M // 128)
-    blk, sbr = (16, 16) if fmt == "nvfp4" else (32, 8)
-    vals = np.array([oracle.e2m1(c) for c in range(16)])
+    """Sum of the terms per element, from the documented layout (numpy only)."""
+    terms, ck, blk, sbr = SPLIT_GEOM[fmt]
+    C, Mt = -(-K // ck), -(-M // 128)
     svals = (np.array([oracle.e4m3(b) if b < 0x7F else 0.0 for b in range(256)]) if fmt == "nvfp4"
              else np.exp2(np.arange(256, dtype=np.float64) - 127.0))
-    cb = codes.reshape(Mt, C, 3, 128, 8, 16)
+    cb = codes.reshape(Mt, C, terms, 128, 8, 16)
     un = np.empty_like(cb)
     for r in range(128):
         for g in range(8):
             un[:, :, :, r, g, :] = cb[:, :, :, r, g ^ (r & 7), :]
-    un = un.reshape(Mt, C, 3, 128, 128)
-    el = np.stack([un & 15, un >> 4], axis=-1).reshape(Mt, C, 3, 128, 256)
-    sc = scales.reshape(Mt, C, 3, 128, sbr)
+    un = un.reshape(Mt, C, terms, 128, 128)
+    if fmt == "fp8":  # one E4M3 code per byte
+        vals = np.array([oracle.e4m3(b) for b in range(256)])
+        el = un
+    else:             # two E2M1 codes per byte, the even element in the low nibble
+        vals = np.array([oracle.e2m1(c) for c in range(16)])
+        el = np.stack([un & 15, un >> 4], axis=-1).reshape(Mt, C, terms, 128, 256)
+    sc = scales.reshape(Mt, C, terms, 128, sbr)
     val = vals[el] * np.repeat(svals[sc], blk, axis=-1)
-    tot = val.sum(axis=2).transpose(0, 2, 1, 3).reshape(Mt * 128, C * 256)
+    tot = val.sum(axis=2).transpose(0, 2, 1, 3).reshape(Mt * 128, C * ck)
     return tot, tot[:M, :K] * np.exp2(x_exp[:M].astype(np.float64))[:, None]
 
 
@@ -70,7 +79,7 @@ def _special_rows(x: torch.Tensor) -> torch.Tensor:
     return x
 
 
-FMTS = ["mxfp4", "nvfp4"]
+FMTS = ["mxfp4", "nvfp4", "fp8"]
 
 
 @pytest.mark.parametrize("fmt", FMTS)
@@ -81,7 +90,7 @@ def test_split_bit_exact(fmt, M, K):
     torch.cuda.synchronize()
     codes, scales, x_exp = codes.cpu().numpy(), scales.cpu().numpy(), x_exp.cpu().numpy()
     full, xs_gpu = _decode_split(fmt, codes, scales, x_exp, M, K)
-    xs = oracle.split_x_bs(x_bits(x), fmt, 3)
+    xs = oracle.split_x_bs(x_bits(x), fmt)
     bad = np.argwhere(xs_gpu != xs)
     assert bad.size == 0, "split differs at %s: gpu %r oracle %r" % (
         bad[:4].tolist(), xs_gpu[tuple(bad[0])], xs[tuple(bad[0])])
@@ -101,7 +110,7 @@ def test_gemm_is_the_split_product(fmt, M, N, K):
     torch.cuda.synchronize()
     y = y.cpu().numpy().astype(np.float64)
     xb = x_bits(x)
-    ys = oracle.gemm_f64(oracle.split_x_bs(xb, fmt, 3), case.Wd)
+    ys = oracle.gemm_f64(oracle.split_x_bs(xb, fmt), case.Wd)
     assert norm_err(y, ys, xb, case.Wd) <= SPLIT_TOL
     if K >= 1024:
         assert norm_err(y, oracle.gemm(xb, case.Wd), xb, case.Wd) <= TOL
@@ -115,11 +124,11 @@ def test_one_hot_rows_give_weight_columns(fmt, M):
     ks = (np.arange(M) * 37 + 3) % K
     x = torch.zeros(M, K, dtype=torch.bfloat16)
     x[np.arange(M), ks] = 1.0
-    x[7, ks[7]] = -0.375  # exactly one E2M1 term: -1.5 * 2^-2
+    x[7, ks[7]] = -0.375  # exactly one term: -1.5 * 2^-2
     y = qgemm.bs_run(x.cuda(), case.pw).cpu().numpy()
     exp = case.Wd[:, ks].T.copy()
     exp[7] *= -0.375
-    # one exact product per output (times the NVFP4 tensor scale, rounded once to fp32)
+    # one exact product per output (times the NVFP4 / FP8 tensor scale, rounded once to fp32)
     assert np.array_equal(y, exp.astype(np.float32))
 
 
@@ -142,7 +151,8 @@ def test_bf16_output_and_workspace_reuse(fmt, M):
 @pytest.mark.parametrize("fmt,N,K,M", [("mxfp4", 17408, 5120, 2048), ("mxfp4", 5120, 17408, 2048),
                                        ("mxfp4", 17408, 5120, 32), ("mxfp4", 5120, 17408, 32),
                                        ("nvfp4", 17408, 5120, 2048), ("nvfp4", 17408, 5120, 16),
-                                       ("nvfp4", 5120, 17408, 16)])
+                                       ("nvfp4", 5120, 17408, 16), ("fp8", 17408, 5120, 2048),
+                                       ("fp8", 5120, 17408, 2048), ("fp8", 17408, 5120, 32)])
 def test_27b_prefill_sampled_rows(fmt, N, K, M):
     case = Case(fmt, N, K, seed=inputs.W_SEED if N == 17408 else inputs.W3_SEED)
     x = inputs.activations(M, K, seed=50)
@@ -151,7 +161,7 @@ def test_27b_prefill_sampled_rows(fmt, N, K, M):
     rows = np.array([0, 1, 127, 128, 1000, M - 1]) if M > 1000 else np.array([0, 1, M // 2, M - 1])
     y = y.cpu().numpy()[rows].astype(np.float64)  # rows picked on the host
     xb = x_bits(x)[rows]
-    ys = oracle.gemm_f64(oracle.split_x_bs(xb, fmt, 3), case.Wd)
+    ys = oracle.gemm_f64(oracle.split_x_bs(xb, fmt), case.Wd)
     assert norm_err(y, ys, xb, case.Wd) <= SPLIT_TOL
     assert norm_err(y, oracle.gemm(xb, case.Wd), xb, case.Wd) <= TOL
 
@@ -171,7 +181,7 @@ def test_fused_gate_up(fmt, M):
     torch.cuda.synchronize()
     xb = x_bits(x)
     rows = np.arange(M) if M <= 300 else np.array([0, 1, 5, 1000, 2047, 2048, M - 1])
-    xs = oracle.split_x_bs(xb[rows], fmt, 3)
+    xs = oracle.split_x_bs(xb[rows], fmt)
     g = oracle.gemm_f64(xs, cg.Wd)
     u = oracle.gemm_f64(xs, cu.Wd)
     bad, worst = h_bound_violations(bf16_bits_of(h)[rows], g, u, xb[rows], cg.Wd, cu.Wd, tol=SPLIT_TOL)
