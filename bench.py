@@ -346,9 +346,17 @@ def run_configs(dev, stream, q8_rings, hbm_peak, tf_peak):
                      "us": round(us, 1), "TFLOPs": round(tf, 1), "frac_tensor": round(tf / tf_peak, 4)})
         del x, y, ws
 
+    def mma_frac(fmt, tf):
+        # the block-scaled MMAs run terms x 2MNK of FP4 (three terms) or FP8 (two) work; their
+        # own peak is the bf16 peak x 4 or x 2 (the nominal dense FP4 : FP8 : bf16 ratio,
+        # 9 : 4.5 : 2.25 PFLOP/s)
+        terms, rate = (2.0, 2.0) if fmt == "fp8" else (3.0, 4.0)
+        return round(terms * tf / (rate * tf_peak), 4)
+
     def prefill_bs(name, pw, M, fmt="mxfp4", reps=3):
-        # the block-scaled path (MXFP4 / NVFP4 weights on kind::mxf4nvf4, x split into three
-        # E2M1 terms): split + GEMM per call
+        # the block-scaled path (MXFP4 / NVFP4 weights on kind::mxf4nvf4 with x split into
+        # three E2M1 terms, FP8 weights on kind::mxf8f6f4 with two E4M3 terms): split + GEMM
+        # per call
         N, K = pw.N, pw.K
         x = inputs.activations(M, K, seed=1).to(dev)
         y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
@@ -356,12 +364,9 @@ def run_configs(dev, stream, q8_rings, hbm_peak, tf_peak):
                          device=dev)
         us = graph_us(lambda i: qgemm.bs_run(x, pw, y=y, workspace=ws, stream=stream), reps, stream)
         tf = 2.0 * M * N * K / (us * 1e-6) / 1e12
-        # the MMAs run 3 x 2MNK of FP4 work; their own peak is the bf16 peak x 4 (the nominal
-        # dense FP4 : bf16 ratio, 9 : 2.25 PFLOP/s)
         recs.append({"config": name, "kind": "prefill", "fmt": fmt, "path": "block-scaled",
                      "N": N, "K": K, "M": M, "us": round(us, 1), "TFLOPs": round(tf, 1),
-                     "frac_tensor": round(tf / tf_peak, 4),
-                     "fp4_mma_frac": round(3.0 * tf / (4.0 * tf_peak), 4)})
+                     "frac_tensor": round(tf / tf_peak, 4), "mma_frac": mma_frac(fmt, tf)})
         del x, y, ws
 
     def prefill_ffn_bs(name, fmt, pg, pu, pd, M, reps=3):
@@ -383,7 +388,7 @@ def run_configs(dev, stream, q8_rings, hbm_peak, tf_peak):
         recs.append({"config": name, "kind": "prefill", "fmt": fmt, "path": "block-scaled",
                      "N": N, "K": K, "M": M, "op": "bs_ffn_gate_up + bs_run down",
                      "us": round(us, 1), "TFLOPs": round(tf, 1), "frac_tensor": round(tf / tf_peak, 4),
-                     "fp4_mma_frac": round(3.0 * tf / (4.0 * tf_peak), 4)})
+                     "mma_frac": mma_frac(fmt, tf)})
         del x, h, y, wsf, wsd
 
     def prefill_ffn(name, fmt, pg, pu, pd, M, reps=3):
@@ -453,6 +458,7 @@ def run_configs(dev, stream, q8_rings, hbm_peak, tf_peak):
         decode("fp8 27B gate/up", "fp8", ring, B)
     del ring
     prefill("fp8 27B gate/up prefill", "fp8", fp8, 2048)
+    prefill_bs("fp8 27B gate/up prefill, block-scaled path", fp8, 2048, fmt="fp8")
     del fp8
     torch.cuda.empty_cache()
     # routed experts (Flash-Next-style MoE: 512 experts, top-10; expert shape hidden 2048 x

@@ -1,37 +1,41 @@
-// bs.cu -- the block-scaled tensor-core path for MXFP4 weights at prefill widths (sm_100a).
+// bs.cu -- the block-scaled tensor-core path (sm_100a).
 //
 // y[m][n] = sum_k x[m][k] * dequant(W)[n][k] with W in MXFP4 (E2M1 codes, one E8M0 scale per
 // 32 elements; OCP Microscaling format as the Atlas issue's "Fix: F16 operands with an exact
-// dequant" section describes it) and x in bf16, on tcgen05.mma.kind::mxf4nvf4 with 32-element
-// E8M0 block scales on both operands, so that the packed weights reach the tensor cores as
-// they are, without a dequantisation pass.
+// dequant" section describes it), NVFP4 (E2M1, one UE4M3 scale per 16, a tensor scale) or FP8
+// (E4M3 with a tensor scale), and x in bf16, on tcgen05.mma.kind::mxf4nvf4 (FP4) or
+// kind::mxf8f6f4 (FP8) with block scales on both operands, so that the packed weights reach
+// the tensor cores as they are, without a dequantisation pass.
 //
-// x is not an MMA type here.  The split kernel writes each row as the sum of three E2M1 terms
-// with their own E8M0 scale per 32 elements: per block, r_0 = x * 2^-x_exp (x_exp = the row's
-// floor(log2 max|x|), an exact power of two that the epilogue restores), e_j = floor(log2
-// max|r_j|) - 2, q_j = E2M1(r_j / 2^e_j) (round to nearest even, saturating at 6),
-// r_{j+1} = r_j - q_j 2^e_j.  Three terms leave a residual below 2^-6 of each block's maximum
-// before rounding; measured against the exact product the normalised error is below 1e-4 at
-// the 27B shapes.  A term whose scale would fall below 2^-127 (blocks more than 2^125 below
-// the row maximum) is dropped.
+// x is not an MMA type here.  The split kernel writes each row as the sum of terms in the
+// weights' element kind with their own power-of-two scale per block: per block, r_0 = x *
+// 2^-x_exp (x_exp = the row's floor(log2 max|x|) less a per-format shift, an exact power of
+// two that the epilogue restores), e_j = floor(log2 max|r_j|) - top, q_j = CODE(r_j / 2^e_j)
+// (round to nearest even, saturating), r_{j+1} = r_j - q_j 2^e_j.  Three E2M1 terms (top 2)
+// leave a residual below 2^-6 of each block's maximum before rounding; two E4M3 terms (top 7)
+// one below 2^-8.  Measured against the exact product the normalised error is below 1e-4 at
+// the 27B shapes.  A term whose scale would fall below the scale type's range is dropped.
 //
-// Layout of the split x (device, written by qgemm_bs_split_x, read by the GEMM):
-//   codes : [Mt][C][3][128 rows][128 bytes]   Mt = ceil(M/128) token tiles, C = ceil(K/256)
-//           chunks; row r of a (tile, chunk, term) block holds elements 256c .. 256c+255 of
-//           token 128 t + r, two per byte (even element in the low nibble), its 16-byte
-//           groups stored at group ^ (r & 7) (the 128-byte swizzle of the MMA operand, as the
-//           tile-major weights).  Tokens past M and elements past K are zero.
-//   scales: [Mt][C][3][128 rows][8]   E8M0 per 32 elements (bias 127).
+// Layout of the split x (device, written by qgemm_bs_split_x, read by the GEMM), with CK = 256
+// (FP4) or 128 (FP8) elements per chunk and T = 3 (FP4) or 2 (FP8) terms:
+//   codes : [Mt][C][T][128 rows][128 bytes]   Mt = ceil(M/128) token tiles, C = ceil(K/CK)
+//           chunks; row r of a (tile, chunk, term) block holds elements CK c .. CK c + CK-1 of
+//           token 128 t + r (E2M1: two per byte, even element in the low nibble; E4M3: one per
+//           byte), its 16-byte groups stored at group ^ (r & 7) (the 128-byte swizzle of the
+//           MMA operand, as the tile-major weights).  Tokens past M and elements past K are 0.
+//   scales: [Mt][C][T][128 rows][sbr]   one scale byte per block (sbr 8 MXFP4, 16 NVFP4, 4 FP8).
 //   x_exp : [Mt * 128] int32.
 //
-// GEMM: one CTA per SM (persistent).  A tile is 128 tokens (MMA M, the x terms as operand A)
-// x 256 weight rows (MMA N, two tile-major weight tiles as operand B) over all of K.  Per
-// 256-K chunk the producer brings the three x-term blocks and the two weight blocks with their
-// scales into one of two shared-memory stages (1-D bulk copies); four staging warps place the
-// stage's scale factors in tensor memory with tcgen05.st in the layout the block-scaled MMA
-// reads (per 64-K block: scale j of row r = r0 + 32 r1 at lane r0 of every lane quarter,
-// column r1, byte j); one thread issues 4 K-blocks x 3 terms of M128 N256 K64 MMAs into one
-// fp32 accumulator; four epilogue warps read it out, restore 2^x_exp and store y.
+// Prefill GEMM (more than 128 rows): one CTA per SM (persistent).  A tile is 128 tokens (MMA M,
+// the x terms as operand A) x 256 weight rows (MMA N, two tile-major weight tiles as operand B)
+// over all of K.  Per chunk the producer brings the x-term blocks and the two weight blocks
+// with their scales into one of the shared-memory stages (1-D bulk copies); four staging warps
+// place the stage's scale factors in tensor memory with tcgen05.st in the layout the
+// block-scaled MMA reads (per MMA K-block: scale j of row r = r0 + 32 r1 at lane r0 of every
+// lane quarter, column r1, byte j); one thread issues 4 K-blocks x T terms of M128 N256 MMAs
+// into one fp32 accumulator; four epilogue warps read it out, restore 2^x_exp (and the tensor
+// scale) and store y.  Decode widths use the second kernel below, with the operands' roles
+// swapped.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp4.h>

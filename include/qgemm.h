@@ -262,32 +262,35 @@ int qgemm_moe_gate_up(int fmt, const void* x_dev, int64_t M, int64_t K, int E,
                       void* stream);
 
 /*
- * Block-scaled path for MXFP4 and NVFP4 weights (tcgen05.mma.kind::mxf4nvf4 with block
- * scales on both operands; the packed weights feed the tensor cores without a
- * dequantisation pass), with the activations quantised on the fly (Atlas issue, kernel-ranking
- * section: a block-scaled MMA path for prefill).  x is split per row into three E2M1 terms with
- * a power-of-two scale per block, in the weight format's scale type:
- *   MXFP4: 32-element blocks, E8M0 scales, xshift 0, emin -127;
- *   NVFP4: 16-element blocks, UE4M3 scales (powers of two 2^-9 .. 2^8 only), xshift 10,
- *          emin -9;
+ * Block-scaled path for MXFP4, NVFP4 and FP8 weights (tcgen05.mma.kind::mxf4nvf4, or
+ * kind::mxf8f6f4 for FP8, with block scales on both operands; the packed weights feed the
+ * tensor cores without a dequantisation pass), with the activations quantised on the fly
+ * (Atlas issue, kernel-ranking section: a block-scaled MMA path for prefill).  x is split per
+ * row into terms with a power-of-two scale per block, in the MMA's scale type:
+ *   MXFP4: three E2M1 terms, 32-element blocks, E8M0 scales, xshift 0, emin -127, top 2;
+ *   NVFP4: three E2M1 terms, 16-element blocks, UE4M3 scales (powers of two 2^-9 .. 2^8
+ *          only), xshift 10, emin -9, top 2;
+ *   FP8:   two E4M3 terms, 32-element blocks, E8M0 scales, xshift 0, emin -127, top 7 (the
+ *          weights' block scales are 1);
  *   x_exp = floor(log2 max|x_row|) - xshift,  r_0 = x * 2^-x_exp,
- *   e_j = floor(log2 max_block |r_j|) - 2  (a term with e_j < emin and the later ones are
- *   dropped: zero codes, scale 0),  q_j = E2M1_RNE_sat(r_j / 2^e_j),  r_{j+1} = r_j - q_j 2^e_j
- *   for j = 0, 1, 2,
- * and y = 2^x_exp * (sum_j (q_j 2^e_j) W^T) [* tensor scale for NVFP4], accumulated in fp32.
+ *   e_j = floor(log2 max_block |r_j|) - top  (a term with e_j < emin and the later ones are
+ *   dropped: zero codes, scale 0),  q_j = CODE_RNE_sat(r_j / 2^e_j),  r_{j+1} = r_j - q_j 2^e_j,
+ * and y = 2^x_exp * (sum_j (q_j 2^e_j) W^T) [* tensor scale for NVFP4 and FP8], accumulated in
+ * fp32.
  * The result differs from qgemm_run by the split's residual (measured normalised error below
  * 2e-4 at the 27B shapes); it is a separate entry point, not a mode of qgemm_run.  Up to 128
  * rows the weights are the MMA M operand and K is split over the SMs by a rule of (N, K)
  * alone (fp32 partials summed in a fixed order); above that x is.
  *
- * qgemm_bs_split_size / qgemm_bs_split_x: the split alone, for fmt MXFP4 or NVFP4.  Layout
- * (device, caller-owned, 16-byte aligned), with Mt = ceil(M/128), C = ceil(K/256),
- * sbr = 8 (MXFP4) or 16 (NVFP4):
- *   codes  [Mt][C][3][128][128] bytes: row r of block (t, c, j) holds elements
- *          256c .. 256c+255 of row 128t + r of term j, two per byte (even element in the
- *          low nibble), its 16-byte groups stored at group ^ (r & 7).  Rows past M and
- *          elements past K are zero.
- *   scales [Mt][C][3][128][sbr] scale bytes (E8M0 bias 127; UE4M3 bias 7), one per block.
+ * qgemm_bs_split_size / qgemm_bs_split_x: the split alone, for fmt MXFP4, NVFP4 or FP8.
+ * Layout (device, caller-owned, 16-byte aligned), with Mt = ceil(M/128), CK = 256 (FP4) or
+ * 128 (FP8) elements per chunk, C = ceil(K/CK), T = 3 (FP4) or 2 (FP8) terms, sbr = 8 (MXFP4),
+ * 16 (NVFP4) or 4 (FP8):
+ *   codes  [Mt][C][T][128][128] bytes: row r of block (t, c, j) holds elements
+ *          CK c .. CK c + CK-1 of row 128t + r of term j (E2M1: two per byte, even element in
+ *          the low nibble; E4M3: one per byte), its 16-byte groups stored at group ^ (r & 7).
+ *          Rows past M and elements past K are zero.
+ *   scales [Mt][C][T][128][sbr] scale bytes (E8M0 bias 127; UE4M3 bias 7), one per block.
  *   x_exp  [Mt*128] int32 (0 for rows past M and all-zero rows).
  * K must be a multiple of 32.  Errors: QGEMM_ERR_FORMAT, _SHAPE, _K_BLOCK, _NULL, _ALIGN,
  * _DEVICE, _CUDA.
@@ -299,7 +302,8 @@ int qgemm_bs_split_x(int fmt, const void* x_dev, int64_t M, int64_t K, void* cod
 
 /*
  * qgemm_bs_workspace_size / qgemm_bs_run: y[M][N] = x W^T on the block-scaled path.  fmt must
- * be QGEMM_FMT_MXFP4 or QGEMM_FMT_NVFP4 (else QGEMM_ERR_FORMAT; NVFP4 needs its tensor scale);
+ * be QGEMM_FMT_MXFP4, QGEMM_FMT_NVFP4 or QGEMM_FMT_FP8 (else QGEMM_ERR_FORMAT; NVFP4 and FP8
+ * need their tensor scale);
  * the other arguments as for qgemm_run, with M the number of x rows.  The workspace
  * (qgemm_bs_workspace_size bytes) holds the split of x and, up to 128 rows, the K-split
  * partials.
@@ -311,7 +315,7 @@ int qgemm_bs_run(int fmt, const void* x_dev, int64_t M, int64_t K, const void* c
 
 /*
  * qgemm_bs_ffn_workspace_size / qgemm_bs_ffn_gate_up: h = bf16(SiLU(x Wg^T) * (x Wu^T)) on the
- * block-scaled path (fmt MXFP4 or NVFP4), the fused gate+up of the Atlas issue's kernel
+ * block-scaled path (fmt MXFP4, NVFP4 or FP8), the fused gate+up of the Atlas issue's kernel
  * ranking.  Per chunk of up to 2048 rows one split of x serves both GEMMs; g and u go to an
  * fp32 workspace and one pass writes h (the same SiLU(g) * u expression as
  * qgemm_ffn_gate_up).  Arguments as for qgemm_ffn_gate_up.
