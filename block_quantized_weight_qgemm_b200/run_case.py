@@ -5,7 +5,7 @@
 Weights: seeded N(0, 0.02), packed on the device with qgemm_pack; x: seeded N(0, 1) bf16.
 Without a flag each repetition is one qgemm_run of W[N, K]; with --ffn it is one
 qgemm_ffn_gate_up of a gate and an up matrix, both [N, K] (B is then the width M); with --bs
-it is one qgemm_bs_run (the block-scaled path, MXFP4 only)."""
+it is one qgemm_bs_run (the block-scaled path: MXFP4, NVFP4 or FP8)."""
 import sys
 
 import torch
