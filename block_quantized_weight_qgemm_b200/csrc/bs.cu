@@ -43,13 +43,13 @@
 
 #include <algorithm>
 #include <atomic>
+#include <type_traits>
 
 #include "common.cuh"
 #include "ptx.cuh"
 
 namespace qg {
 
-constexpr int kBsMaxTerms = 3;
 constexpr int kBsM = 128;                     // tokens per tile
 constexpr int kBsWT = 2;                      // weight tiles (of 128 rows) per tile
 constexpr int kBsN = 128 * kBsWT;             // weight rows per tile (MMA N)
@@ -59,7 +59,6 @@ constexpr int kBsBlock = kBsM * 128;          // one 128-row x 128-byte code blo
 constexpr int kBsBCodes = kBsWT * kBsBlock;
 constexpr int kBsKB = 4;                      // MMA K-blocks per chunk (32 bytes of codes each)
 constexpr int kBsTmemCols = 512;
-constexpr int kBsStageWarp0 = 2;  // warps 2..5 stage the scale factors
 constexpr int kBsEpiWarp0 = 6;    // warps 6..9 run the epilogue
 constexpr int kBsThreads = 10 * 32;
 
@@ -162,6 +161,12 @@ constexpr int kBsSplitRegs = 3;  // 8-element words per thread kept from phase 1
 __device__ __forceinline__ float bs_pow2(int e) {  // 2^e for -149 <= e <= 127, exact
   return e >= -126 ? __int_as_float((e + 127) << 23) : __int_as_float(1 << (e + 149));
 }
+// floor(log2 v) for a finite v > 0, from the bits (normal: biased exponent - 127; subnormal:
+// the leading mantissa bit's position - 149)
+__device__ __forceinline__ int bs_flog2(float v) {
+  const uint32_t b = __float_as_uint(v);
+  return (b >> 23) != 0u ? (int)(b >> 23) - 127 : -118 - __clz((int)b);
+}
 __device__ __forceinline__ float bs_amax8(float m, const uint4& v) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -191,8 +196,9 @@ __device__ __forceinline__ uint32_t bs_enc2(float a, float b, float& qa, float& 
 // The terms of one lane's 8 elements (a quarter of a 32-element block or half of a 16-element
 // one), written to the split layout when `store` (lanes past the padded K only take part in
 // the block reductions).  All lanes of the block take the same decisions (the block maximum is
-// reduced over them first).
-template <int F>
+// reduced over them first).  The prescale 2^-x_exp is f1 (TWO: f1 * f2, for exponents past
+// the normal range).
+template <int F, bool TWO>
 __device__ __forceinline__ void bs_split8(const BsSplitParams& p, const uint4& v, bool in, bool store,
                                           float f1, float f2, int t, int r, int k, int lane) {
   constexpr int kTerms = bs_terms(F), kChunk = bs_chunk(F), kBlk = bs_blk(F), kSbr = bs_sbr(F);
@@ -201,8 +207,9 @@ __device__ __forceinline__ void bs_split8(const BsSplitParams& p, const uint4& v
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    rv[2 * i] = in ? (__uint_as_float(w[i] << 16) * f1) * f2 : 0.f;
-    rv[2 * i + 1] = in ? (__uint_as_float(w[i] & 0xFFFF0000u) * f1) * f2 : 0.f;
+    const float lo = __uint_as_float(w[i] << 16) * f1, hi = __uint_as_float(w[i] & 0xFFFF0000u) * f1;
+    rv[2 * i] = in ? (TWO ? lo * f2 : lo) : 0.f;
+    rv[2 * i + 1] = in ? (TWO ? hi * f2 : hi) : 0.f;
   }
   const int c = k / kChunk, o = k % kChunk;  // chunk, element offset in it
   const int j = o / kBlk;                    // block of the chunk
@@ -222,18 +229,20 @@ __device__ __forceinline__ void bs_split8(const BsSplitParams& p, const uint4& v
     int sb = 0;  // scale byte
     uint32_t packed[2] = {0u, 0u};
     if (!done && bmax > 0.f) {
-      int ex;
-      (void)frexpf(bmax, &ex);
-      const int e = (ex - 1) - bs_top(F);  // block maximum / 2^e in [2^top, 2^(top+1))
+      const int e = bs_flog2(bmax) - bs_top(F);  // block maximum / 2^e in [2^top, 2^(top+1))
       if (e >= bs_emin(F)) {
         sb = bs_scale_byte(F, e);
-        const float inv = bs_pow2(-e), sc = bs_pow2(e);
+        // 2^-e is a normal float: e runs from emin >= -127 to at most 8 (the largest prescaled
+        // block maximum is below 2^11)
+        const float inv = __int_as_float((127 - e) << 23), sc = bs_pow2(e);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           float qa, qb;
           const uint32_t c2 = bs_enc2<F>(rv[2 * i] * inv, rv[2 * i + 1] * inv, qa, qb);
-          rv[2 * i] = fmaf(-qa, sc, rv[2 * i]);
-          rv[2 * i + 1] = fmaf(-qb, sc, rv[2 * i + 1]);
+          if (term + 1 < kTerms) {  // the last term's residual is not needed
+            rv[2 * i] = fmaf(-qa, sc, rv[2 * i]);
+            rv[2 * i + 1] = fmaf(-qb, sc, rv[2 * i + 1]);
+          }
           if (F == kBsF8) packed[i >> 1] |= c2 << (16 * (i & 1));
           else packed[0] |= c2 << (8 * i);
         }
@@ -287,11 +296,8 @@ __global__ void __launch_bounds__(kBsSplitThreads) qgemm_bs_split_kernel(const B
 #pragma unroll
   for (int i = 1; i < kBsSplitThreads / 32; ++i) amax = fmaxf(amax, red[i]);
   int xe = 0;
-  if (amax > 0.f && amax <= 3.4e38f) {
-    int ex;
-    (void)frexpf(amax, &ex);
-    xe = (ex - 1) - bs_xshift(F);  // row maximum * 2^-xe in [2^xshift, 2^(xshift+1))
-  }
+  if (amax > 0.f && amax <= 3.4e38f)
+    xe = bs_flog2(amax) - bs_xshift(F);  // row maximum * 2^-xe in [2^xshift, 2^(xshift+1))
   if (threadIdx.x == 0) p.x_exp[m] = live ? xe : 0;
   // 2^-xe as two exact factors (xe runs from -143 to 127)
   const int a1 = max(min(-xe, 126), -126);
@@ -300,16 +306,21 @@ __global__ void __launch_bounds__(kBsSplitThreads) qgemm_bs_split_kernel(const B
   const int lane = threadIdx.x & 31;
   // Phase 2, over the warp spans that start inside the padded K (warp-uniform conditions:
   // every lane of a span takes part in its block reductions)
+  auto phase2 = [&](auto two) {
+    constexpr bool kTwo = decltype(two)::value;
 #pragma unroll
-  for (int n = 0; n < kBsSplitRegs; ++n) {
-    const int k = (threadIdx.x + n * kBsSplitThreads) * 8;
-    if (k - 8 * lane < Kp) bs_split8<F>(p, v[n], live && k < p.K, k < Kp, f1, f2, t, r, k, lane);
-  }
-  for (int k = (threadIdx.x + kBsSplitRegs * kBsSplitThreads) * 8; k - 8 * lane < Kp; k += kBsSplitThreads * 8) {
-    const bool in = live && k < p.K;
-    const uint4 w = in ? *reinterpret_cast<const uint4*>(xr + k) : make_uint4(0u, 0u, 0u, 0u);
-    bs_split8<F>(p, w, in, k < Kp, f1, f2, t, r, k, lane);
-  }
+    for (int n = 0; n < kBsSplitRegs; ++n) {
+      const int k = (threadIdx.x + n * kBsSplitThreads) * 8;
+      if (k - 8 * lane < Kp) bs_split8<F, kTwo>(p, v[n], live && k < p.K, k < Kp, f1, f2, t, r, k, lane);
+    }
+    for (int k = (threadIdx.x + kBsSplitRegs * kBsSplitThreads) * 8; k - 8 * lane < Kp; k += kBsSplitThreads * 8) {
+      const bool in = live && k < p.K;
+      const uint4 w = in ? *reinterpret_cast<const uint4*>(xr + k) : make_uint4(0u, 0u, 0u, 0u);
+      bs_split8<F, kTwo>(p, w, in, k < Kp, f1, f2, t, r, k, lane);
+    }
+  };
+  if (f2 == 1.0f) phase2(std::false_type{});  // the row's 2^-xe is one normal float (uniform)
+  else phase2(std::true_type{});
 }
 
 // ---------------------------------------------------------------------------------------

@@ -86,6 +86,8 @@ FMTS = ["mxfp4", "nvfp4", "fp8"]
 @pytest.mark.parametrize("M,K", [(1, 32), (130, 288), (257, 1024), (200, 5120)])
 def test_split_bit_exact(fmt, M, K):
     x = _special_rows(inputs.activations(M, K, seed=20 + M))
+    if M >= 7:
+        x[6] = x[6] * 2.0 ** -128  # bf16 subnormals: 2^-x_exp is past the normal range
     codes, scales, x_exp = qgemm.bs_split_x(x.cuda(), fmt)
     torch.cuda.synchronize()
     codes, scales, x_exp = codes.cpu().numpy(), scales.cpu().numpy(), x_exp.cpu().numpy()
