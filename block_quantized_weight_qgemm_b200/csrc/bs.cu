@@ -636,17 +636,23 @@ __global__ void __launch_bounds__(kBsThreads, 1) qgemm_bs_kernel(const __grid_co
       const int m = mt * kBsM + q * 32 + lane;
       const int xe = (m < p.M) ? p.x_exp[m] : 0;
       const float tsv = kTs ? __ldg(p.ts) : 1.0f;  // tensor scale, applied before 2^xe
-      // y = (acc * ts) * 2^xe: the tensor scale rounds once, the power of two is exact
-      auto yv = [&](uint32_t u) { return bs_scale_pow2(kTs ? __uint_as_float(u) * tsv : __uint_as_float(u), xe); };
+      // y = (acc * ts) * 2^xe: the tensor scale rounds once, the power of two is exact.  When
+      // every row of the warp has a normal 2^xe (the common case) it is one multiply by a
+      // factor taken once per unit; otherwise the warp takes bs_scale_pow2 per element.
+      const bool fast = xe >= -126 && xe <= 127;
+      const float sc = __int_as_float(((fast ? xe : 0) + 127) << 23);
+      const bool all_fast = __all_sync(0xffffffffu, fast);
       bool ok = mbar_wait(bar_acc, (uint32_t)ti & 1u, abort_flag, p.dev_err, kErrTimeout);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-#pragma unroll 1
-      for (int cb = 0; cb < kBsN; cb += 32) {
-        uint32_t v[32];
-        bs_tmem_ld32(tmem + lane_base + (uint32_t)cb, v);
-        tmem_ld_wait();
+      // one 32-column block: scale and store (FAST: the one-multiply scale)
+      auto store_block = [&](const uint32_t (&v)[32], int cb, auto fastc) {
+        constexpr bool FAST = decltype(fastc)::value;
+        auto yv = [&](uint32_t w) {
+          const float a = kTs ? __uint_as_float(w) * tsv : __uint_as_float(w);
+          return FAST ? a * sc : bs_scale_pow2(a, xe);
+        };
         const int n0 = nt * kBsN + cb;
         if (m < p.M && n0 < p.N) {
           if (p.out_bf16) {
@@ -683,6 +689,14 @@ __global__ void __launch_bounds__(kBsThreads, 1) qgemm_bs_kernel(const __grid_co
             }
           }
         }
+      };
+#pragma unroll 1
+      for (int cb = 0; cb < kBsN; cb += 32) {
+        uint32_t v[32];
+        bs_tmem_ld32(tmem + lane_base + (uint32_t)cb, v);
+        tmem_ld_wait();
+        if (all_fast) store_block(v, cb, std::true_type{});
+        else store_block(v, cb, std::false_type{});
       }
       tc_fence_before();
       __syncwarp();
