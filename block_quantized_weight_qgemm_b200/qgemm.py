@@ -235,7 +235,7 @@ def run(x: torch.Tensor, pw: PackedWeight, y: torch.Tensor | None = None, y_dtyp
 
 def bs_split_size(fmt, M: int, K: int) -> tuple[int, int, int]:
     """qgemm_bs_split_size: (code bytes, scale bytes, exponent bytes) of the split of x for
-    weight format fmt (MXFP4 or NVFP4)."""
+    weight format fmt (MXFP4, NVFP4 or FP8)."""
     c, sc, e = _SZ(), _SZ(), _SZ()
     _check(lib().qgemm_bs_split_size(_fmt(fmt), M, K, ctypes.byref(c), ctypes.byref(sc),
                                      ctypes.byref(e)), "qgemm_bs_split_size")
@@ -244,7 +244,8 @@ def bs_split_size(fmt, M: int, K: int) -> tuple[int, int, int]:
 
 def bs_split_x(x: torch.Tensor, fmt="mxfp4", stream=None):
     """qgemm_bs_split_x: x bf16 [M, K] -> (codes u8, scales u8, x_exp int32) in the layout of
-    include/qgemm.h (three E2M1 terms per row with the weight format's block scales)."""
+    include/qgemm.h (three E2M1 terms per row for MXFP4 / NVFP4, two E4M3 terms for FP8, with the
+    MMA's block scales)."""
     assert x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous() and x.dim() == 2
     M, K = x.shape
     nc, ns, ne = bs_split_size(fmt, M, K)
@@ -264,7 +265,7 @@ def bs_workspace_size(fmt: int, N: int, K: int, M: int) -> int:
 
 def bs_run(x: torch.Tensor, pw: PackedWeight, y: torch.Tensor | None = None, y_dtype=torch.float32,
            workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """qgemm_bs_run: the block-scaled path (MXFP4 or NVFP4 weights): x bf16 [M, K] -> y [M, N]."""
+    """qgemm_bs_run: the block-scaled path (MXFP4, NVFP4 or FP8 weights): x bf16 [M, K] -> y [M, N]."""
     assert x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous() and x.dim() == 2
     M, K = x.shape
     assert K == pw.K
