@@ -958,6 +958,20 @@ __global__ void __launch_bounds__(kBdThreads, 1) qgemm_bs_dec_kernel(const __gri
     griddep_wait();  // x_exp comes from the split kernel
     const size_t MN = (size_t)p.M * p.N;
     const float tsv = kTs ? __ldg(p.ts) : 1.0f;  // tensor scale, applied before 2^x_exp
+    // 2^x_exp of token column b = lane + 32 j held by lane `lane` as fac[j] (M <= 128); when
+    // every column's exponent is in the normal range the restore is one multiply by a factor
+    // fetched with a shuffle, otherwise bs_scale_pow2 per element
+    float fac[4];
+    bool fast = true;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int b = lane + 32 * j;
+      const int e = (b < p.M) ? __ldg(p.x_exp + b) : 0;
+      const bool f = e >= -126 && e <= 127;
+      fast = fast && f;
+      fac[j] = __int_as_float(((f ? e : 0) + 127) << 23);
+    }
+    const bool all_fast = __all_sync(0xffffffffu, fast);
     int ti = 0;
     for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++ti) {
       int t, s, c0, c1;
@@ -980,18 +994,29 @@ __global__ void __launch_bounds__(kBdThreads, 1) qgemm_bs_dec_kernel(const __gri
 #pragma unroll
           for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) + __uint_as_float(w[i]));
         }
+        // the factors of columns cb .. cb+15 (all lanes take part in the shuffles)
+        const int jb = cb >> 5;
+        const float fr = jb == 0 ? fac[0] : jb == 1 ? fac[1] : jb == 2 ? fac[2] : fac[3];
+        float fv[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) fv[i] = __shfl_sync(0xffffffffu, fr, (cb & 16) + i);
         if (n64 < p.N) {
           const int n = (int)n64;
+          auto put = [&](int b, float val) {
+            if (p.S > 1) p.ws[(size_t)s * MN + (size_t)b * p.N + n] = val;
+            else if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)b * p.N + n] = __float2bfloat16_rn(val);
+            else reinterpret_cast<float*>(p.out)[(size_t)b * p.N + n] = val;
+          };
+          if (all_fast) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int b = cb + i;
-            if (b < p.M) {
-              const float acc = kTs ? __uint_as_float(v[i]) * tsv : __uint_as_float(v[i]);
-              const float val = bs_scale_pow2(acc, __ldg(p.x_exp + b));
-              if (p.S > 1) p.ws[(size_t)s * MN + (size_t)b * p.N + n] = val;
-              else if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)b * p.N + n] = __float2bfloat16_rn(val);
-              else reinterpret_cast<float*>(p.out)[(size_t)b * p.N + n] = val;
-            }
+            for (int i = 0; i < 16; ++i)
+              if (cb + i < p.M) put(cb + i, (kTs ? __uint_as_float(v[i]) * tsv : __uint_as_float(v[i])) * fv[i]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              if (cb + i < p.M)
+                put(cb + i, bs_scale_pow2(kTs ? __uint_as_float(v[i]) * tsv : __uint_as_float(v[i]),
+                                          __ldg(p.x_exp + cb + i)));
           }
         }
       }
